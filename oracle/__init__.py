@@ -1,0 +1,11 @@
+"""Float64 CPU oracle of the MoE layer forward pass (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference legs may import this package; the CUDA product path never does.
+"""
+from .moe_oracle import (  # noqa: F401
+    LayerConfig, Routing, Dispatch, Forward, RELU, SWIGLU,
+    gate_logits, normalise_logits, softmax, top_k, route, capacity, dispatch,
+    expert_hidden, expert_ffn, expert_segments, combine, forward, forward_tokens,
+    brute_force,
+)
