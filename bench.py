@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Forward throughput of the top-k gated MoE FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl moe|reference]
+
+A step is one moe_layer_forward (gate GEMM + normalisation/top-k, permutation
+with capacity, both grouped expert GEMMs, combine) over one batch of
+synthetic tokens already resident in HBM; by default it is replayed from a
+CUDA graph.  Between timed steps a 512 MiB memset flushes the 126 MB L2, and
+each step is bracketed by its own CUDA events (the flush is outside them).
+Under torchrun each rank runs an independent replica on its own token shard
+(weak scaling; no collective on the data path) and the reported time is the
+maximum over ranks.
+
+One JSON line is printed by rank 0.  ``--impl reference`` times the float64
+CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import moe_workloads as mw  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (GEMM), % HBM BW (permute)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 6   # route, scan, scatter, grouped GEMM x2, combine
+L2_FLUSH_BYTES = 512 << 20
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "tc_grouped_gemm_fastmoe_txl.md")
+GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc", "gemm_tc.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=mw.BENCH_WORKLOAD, choices=sorted(mw.WORKLOADS))
+    ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
+    ap.add_argument("--no-graph", action="store_true", help="launch the C ABI call directly instead of a graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget for cpu_baseline")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w: mw.Workload, n_gpus: int, graph: bool):
+    return {"workload": w.name, "tokens_per_gpu": w.T, "global_batch": w.T * n_gpus, "d_model": w.d,
+            "experts": w.E, "ffn_hidden": w.F, "top_k": w.k, "activation": w.act,
+            "capacity_factor": w.capacity_factor if w.capacity_factor > 0 else "dropless",
+            "lambda": w.lam, "gate_bias": "zipf1.2" if w.zipf_bias else None,
+            "parallelism": "replicas" if n_gpus == 1 else f"dp{n_gpus} replicas",
+            "l2": "flushed between steps (512 MiB memset outside the timed events)",
+            "cuda_graph": graph}
+
+
+# ------------------------------------------------------------ CPU oracle
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        return int(n[0]) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_forward_fn(w: mw.Workload, inp: mw.Inputs, T_sample: int):
+    import oracle
+    from oracle import moe_oracle as om
+    cfg = oracle.LayerConfig.from_workload(w, T_sample)
+    x = mw.to_f64(inp.x[:T_sample])
+    wg = mw.to_f64(inp.wg)
+    w1, w2 = mw.F64Experts(inp.w1), mw.F64Experts(inp.w2)
+    return lambda: om.forward(x, wg, inp.bias, w1, w2, cfg)
+
+
+def reference_sample_tokens(w: mw.Workload) -> int:
+    # full batch where one float64 forward takes about a second on the host
+    flop_per_tok = (6 if w.act == mw.SWIGLU else 4) * w.d * w.F * w.k + 2 * w.d * w.E
+    return int(max(64, min(w.T, 2.0e10 // flop_per_tok)))
+
+
+def cpu_baseline(w: mw.Workload, inp: mw.Inputs, budget_s: float):
+    Ts = reference_sample_tokens(w)
+    fwd = oracle_forward_fn(w, inp, Ts)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fwd()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": n * Ts / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} float64 oracle forwards of the first {Ts} of {w.T} tokens ({el:.1f} s, "
+                      f"numpy/OpenBLAS on {blas_threads()} threads)"}
+
+
+def run_reference(a):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    w = mw.WORKLOADS[a.workload]
+    inp = mw.generate(w)
+    Ts = reference_sample_tokens(w)
+    fwd = oracle_forward_fn(w, inp, Ts)
+    for _ in range(a.warmup):
+        fwd()
+    times = []
+    for _ in range(a.steps):
+        t0 = time.perf_counter()
+        fwd()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = Ts / (ms / 1e3)
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, 1, False),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"each step: float64 oracle forward of the first {Ts} of {w.T} tokens"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ clock sampling
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    p = [s.strip() for s in line.split(",")]
+                    if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                        rows.append(p)
+            os.unlink(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------------- roofline
+def step_bytes(w: mw.Workload, offsets: np.ndarray):
+    """Algorithmic bytes (and FLOPs for the experts) of one forward's steps."""
+    b = 2 if w.dtype == mw.BF16 else 4
+    T, d, F, k, E = w.T, w.d, w.F, w.k, w.E
+    A = T * k
+    kept = int(offsets[-1])
+    F1 = F if w.act == mw.RELU else 2 * F
+    touched = int(np.sum(np.diff(offsets) > 0))
+    return {
+        "route": T * d * b + E * d * b + A * 8 + T * 4,
+        "permute": (T * d + kept * d) * b + 4 * (2 * A + kept),
+        "expert_ffn": touched * (F1 + F) * d * b + kept * (2 * d + 2 * F) * b,
+        "combine": (kept * d + T * d) * b + 8 * A,
+        "expert_flops": 2 * kept * d * (F1 + F),
+        "weight_bytes": touched * (F1 + F) * d * b,
+    }
+
+
+def committed_traffic():
+    """DRAM bytes per grouped-GEMM launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    try:
+        src = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()[:16]
+        txt = open(GEMM_PROFILE).read()
+        m_hash = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+        m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+        if m_hash and m_tr and m_hash.group(1) == src:
+            return float(m_tr.group(1))
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ main
+def main():
+    a = parse_args()
+    if a.impl == "reference":
+        return run_reference(a)
+
+    import torch
+    import torch.distributed as dist
+    import mixture_experts_layer_logit_b200 as moe
+    from mixture_experts_layer_logit_b200 import build as moe_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        print(f"warning: --gpus {a.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        moe_build.build()
+    if world > 1:
+        dist.barrier()
+    moe.lib()
+
+    w = mw.WORKLOADS[a.workload]
+    inp = mw.generate(w, shard=rank)
+    cfg = moe.make_config(w.T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam)
+    tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
+    x = mw.to_device(inp.x, dev)
+    wg, bias = mw.to_device(inp.wg, dev), mw.to_device(inp.bias, dev)
+    w1, w2 = mw.to_device(inp.w1, dev), mw.to_device(inp.w2, dev)
+    nbytes, lay = moe.moe_workspace_size(cfg)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.T, w.d), dtype=tdt, device=dev)
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        moe.moe_layer_forward(cfg, x, wg, bias, w1, w2, out, stats, ws)
+
+    fwd()
+    torch.cuda.synchronize()
+    graph = None
+    run = fwd
+    if not a.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fwd()
+        run = graph.replay
+
+    def timed(fn, steps, flush_between=True):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            if flush_between:
+                flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------- headline
+    timed(run, a.warmup)
+    barrier()
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    barrier()
+    times = timed(run, a.steps)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(sum(times))
+    ms = total_ms / a.steps
+    value = world * w.T / (ms / 1e3)
+    st = moe.read_stats(stats)
+    offsets = ws[lay.offsets:lay.offsets + 4 * (w.E + 1)].view(torch.int32).cpu().numpy()
+    assert st["status"] == 0, f"device status {st['status']}"
+
+    # ------------------------------------------- per-step breakdown (rank-local)
+    pk, pk_src = peaks()
+    sb = step_bytes(w, offsets)
+    breakdown = None
+    roofline = None
+    if not a.no_breakdown:
+        A = w.T * w.k
+        L = lay
+        sv = lambda off, n, dt: ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)  # noqa: E731
+        idx, tw, gap = sv(L.topk_idx, A, torch.int32), sv(L.topk_w, A, torch.float32), sv(L.gap, w.T, torch.float32)
+        counts, kept, offs = sv(L.counts, w.E, torch.int32), sv(L.kept, w.E, torch.int32), sv(L.offsets, w.E + 1, torch.int32)
+        row_of, src_tok = sv(L.row_of, A, torch.int32), sv(L.src_tok, A, torch.int32)
+        xp, h, yp = sv(L.xp, A * w.d, tdt), sv(L.h, A * w.F, tdt), sv(L.yp, A * w.d, tdt)
+        scr = ws[L.scratch:]
+        pm = torch.empty(w.E, dtype=torch.float32, device=dev)
+        names = ["route", "permute", "expert_ffn", "combine"]
+        acc = {n: 0.0 for n in names}
+        for i in range(a.warmup + a.steps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            ev[0].record()
+            moe.moe_route(cfg, x, wg, bias, idx, tw, gap, pm, scr)
+            ev[1].record()
+            moe.moe_permute(cfg, x, idx, gap, pm, counts, kept, offs, row_of, src_tok, xp, stats, scr)
+            ev[2].record()
+            moe.moe_expert_ffn(cfg, xp, offs, w1, w2, h, yp, stats, scr)
+            ev[3].record()
+            moe.moe_combine(cfg, yp, row_of, tw, out)
+            ev[4].record()
+            torch.cuda.synchronize()
+            if i >= a.warmup:
+                for j, n in enumerate(names):
+                    acc[n] += ev[j].elapsed_time(ev[j + 1])
+        breakdown = {n: acc[n] / a.steps for n in names}
+        rl = {}
+        for n in ["route", "permute", "combine"]:
+            gbs = sb[n] / (breakdown[n] * 1e-3) / 1e9
+            rl[n] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / pk["hbm_gbs"], "bytes": sb[n]}
+        t_ffn = breakdown["expert_ffn"] * 1e-3
+        tflops = sb["expert_flops"] / t_ffn / 1e12
+        gbs = sb["expert_ffn"] / t_ffn / 1e9
+        t_hbm = sb["expert_ffn"] / (pk["hbm_gbs"] * 1e9)
+        t_tc = sb["expert_flops"] / (pk["bf16_tflops"] * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        traffic = committed_traffic() if a.workload == mw.BENCH_WORKLOAD else None
+        if bound == "hbm":
+            roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / pk["hbm_gbs"], "traffic": traffic}
+        else:
+            roofline = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": tflops / pk["bf16_tflops"], "traffic": traffic}
+        roofline.update({
+            "kernel": "tc_grouped_gemm (expert FFN step: 2 launches, layer 1 + layer 2)",
+            "launches_per_step": 2, "algorithmic_bytes_per_launch": sb["expert_ffn"] / 2,
+            "algorithmic_flops_per_launch": sb["expert_flops"] / 2, "launch_ms": breakdown["expert_ffn"] / 2,
+            "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"], "hbm_gbs": gbs,
+            "hbm_frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured"
+            else "fallback (recipe)", "other_steps": rl})
+
+    # ------------------------------------------------------------------ e2e
+    e2e = None
+    if not a.no_e2e:
+        x_host = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        x_host.copy_(x.cpu())
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        st_host = torch.empty(stats.shape, dtype=stats.dtype).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            run()
+            out_host.copy_(out, non_blocking=True)
+            st_host.copy_(stats, non_blocking=True)
+
+        timed(e2e_step, a.warmup)
+        barrier()
+        et = timed(e2e_step, a.steps)
+        barrier()
+        e_ms = max_over_ranks(sum(et)) / a.steps
+        e2e = {"value": world * w.T / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": x.numel() * x.element_size(),
+               "d2h_bytes_per_step": out.numel() * out.element_size() + stats.numel()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, a.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.dtype == mw.BF16 else "f32", "data": "synthetic",
+                "config": workload_config(w, world, graph is not None),
+                "gpu_launches": LAUNCHES_PER_STEP * a.steps,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+                "breakdown_ms": breakdown,
+                "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "rows_kept": st["rows_kept"],
+                          "capacity": st["capacity"], "near_tie_count": st["near_tie_count"]}}
+        print(json.dumps(line), flush=True)
+    if graph is not None:
+        del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,217 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) top-k gated Mixture-of-Experts FFN
+ * layer, forward pass, on one GPU.
+ *
+ * The layer (FastMoE announcement "智源x清华开源FastMoE", section
+ * "1. MoE 设计", Figure 1): a gating network scores E experts for each token,
+ * the k best are activated, and the token's output is the gate-weighted sum of
+ * those k experts' outputs.  Five steps, each a hand-written CUDA kernel:
+ *
+ *   1. gate GEMM            z = x W_gate^T (+ b)
+ *   2. normalise + top-k    optional z_hat = lambda (z - mean_e z) / std_e z,
+ *                           p = softmax, top-k (lowest expert index wins ties),
+ *                           weights = p of the selected experts / their sum
+ *   3. permute              per-expert histogram + prefix sums group the
+ *                           (token, slot) assignments by expert in ascending
+ *                           token order; each expert keeps its first C
+ *                           assignments (capacity mode) or all (dropless)
+ *   4. expert FFN           grouped GEMMs over the variable-length expert
+ *                           segments: ReLU MLP or SwiGLU
+ *   5. combine              out[t] = sum over kept slots of w * expert output
+ *
+ * Conventions shared by every entry point:
+ *   - Every data pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned.  The library allocates no memory and never synchronises: work
+ *     is enqueued on `stream` (NULL = legacy default stream) and returns.
+ *   - Row-major layouts.  Weights use the nn.Linear [out, in] layout:
+ *     W_gate[E, d]; W1[E, F1, d] with F1 = F (ReLU) or 2F (SwiGLU: rows [0, F)
+ *     are the gate projection, rows [F, 2F) the up projection -- the order of
+ *     the merged pair matters, Megatron-Core best-practice page, section
+ *     "从HuggingFace到Megatron的权重转换要点"); W2[E, d, F].
+ *   - Element type of x, weights, xp, h, yp and out: bf16 (MOE_DTYPE_BF16,
+ *     fp32 accumulation, tcgen05 tensor cores) or fp32 (MOE_DTYPE_F32, CUDA-core
+ *     FFMA throughout).  Gate bias, gate weights (topk_w), gap and prob_mean are
+ *     fp32; indices are int32.
+ *   - Errors a host can see (bad arguments, unsupported shapes, too small a
+ *     workspace, a failed launch) are returned synchronously and nothing is
+ *     enqueued.  Errors only the device can see (an index out of range, a
+ *     bounded wait that gave up) are OR-ed into moe_stats.status (device
+ *     memory), which the caller reads after synchronising.
+ *   - A = T*k assignments.  Buffers indexed by permuted row (src_tok, xp, h,
+ *     yp) are sized for A rows (the dropless worst case); the rows in use are
+ *     [0, offsets[E]).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so that callers need no CUDA header. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,         /* null or misaligned pointer, negative size, k > E, bad enum */
+  MOE_ERR_UNSUPPORTED = 2, /* shape outside the supported set (see moe_config) or no sm_100 device */
+  MOE_ERR_WORKSPACE = 3,   /* ws is NULL, misaligned (256 B) or smaller than required */
+  MOE_ERR_CUDA = 4         /* a CUDA runtime/driver call failed (launch, tensor-map encoding) */
+} moe_status;
+
+enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+
+/* Device-detected error bits in moe_stats.status. */
+#define MOE_DEV_TIMEOUT 1u   /* a bounded wait inside a kernel gave up (~2 s); the kernel returned early */
+#define MOE_DEV_BOUNDS  2u   /* an expert index outside [0, E) was seen and skipped */
+
+/* Near-tie threshold: tokens whose k-th and (k+1)-th scores differ by less
+ * than this are counted in moe_stats.near_tie_count. */
+#define MOE_NEAR_TIE_GAP 1e-4f
+
+/*
+ * Layer shape and mode.
+ *   T >= 0 tokens, d >= 1 model width, 1 <= E <= 256 experts, F >= 1 expert
+ *   hidden width, 1 <= k <= E experts per token.
+ *   bf16: d and F multiples of 16.  fp32: d and F multiples of 4.
+ *   capacity_factor <= 0: dropless.  Otherwise the per-expert capacity is
+ *     C = ceil((double)capacity_factor * (double)(T*k) / (double)E), computed on
+ *     the host in that order from the float32 factor (Switch/GShard capacity;
+ *     Megatron-Core best-practice page, section "MoE负载均衡的挑战与应对";
+ *     Skywork-MoE slides, slide 4 "Preliminaries": based on Switch).
+ *   lambda <= 0: plain softmax gating.  lambda > 0: gating-logit
+ *     normalisation z_hat = lambda * (z - mean) / std over the E logits of a
+ *     token (population std; zero spread gives z_hat = 0) before softmax and
+ *     top-k (Skywork-MoE release, section "Gating Logits归一化操作"; slides,
+ *     slide 6, "lambda = 1 seems to be the best value").
+ */
+typedef struct moe_config {
+  int32_t T, d, E, F, k;
+  int32_t act;               /* MOE_ACT_RELU | MOE_ACT_SWIGLU */
+  int32_t dtype;             /* MOE_DTYPE_BF16 | MOE_DTYPE_F32 */
+  float capacity_factor;     /* <= 0: dropless */
+  float lambda;              /* <= 0: plain softmax */
+} moe_config;
+
+/* Per-forward statistics, in DEVICE memory, written by moe_permute (and by
+ * moe_layer_forward).  Drop-token rate and load balance are the quantities the
+ * Skywork-MoE adaptive aux-loss controller monitors (Skywork-MoE release,
+ * section "2.自适应的Aux Loss"). */
+typedef struct moe_stats {
+  int32_t drop_count;        /* assignments dropped by the capacity */
+  int32_t rows_kept;         /* offsets[E] = T*k - drop_count */
+  int32_t capacity;          /* C, or -1 in dropless mode */
+  int32_t near_tie_count;    /* tokens with gap < MOE_NEAR_TIE_GAP; -1 if gap was not given */
+  float drop_rate;           /* drop_count / (T*k); 0 when T == 0 */
+  float aux_loss;            /* E * sum_e (counts_e/(T*k)) * P_e (pre-drop counts); NaN if P not given or T == 0 */
+  uint32_t status;           /* MOE_DEV_* bits; cleared by moe_permute, OR-ed by later steps */
+  int32_t reserved;
+} moe_stats;
+
+/* Byte offsets of the intermediates inside a moe_layer_forward workspace
+ * (each 256-byte aligned), so that a caller can read them after a forward. */
+typedef struct moe_ws_layout {
+  size_t topk_idx, topk_w, gap, counts, kept, offsets, row_of, src_tok;
+  size_t xp, h, yp, scratch, total;
+} moe_ws_layout;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status s);
+
+/* Scratch bytes the step calls (moe_route, moe_permute, moe_expert_ffn) need
+ * in `ws`; 0 when cfg is invalid. */
+size_t moe_scratch_size(const moe_config* cfg);
+
+/* Workspace bytes moe_layer_forward needs (all intermediates + scratch); 0
+ * when cfg is invalid.  Fills *layout when it is not NULL. */
+size_t moe_workspace_size(const moe_config* cfg, moe_ws_layout* layout);
+
+/*
+ * Steps 1-2: gate GEMM, optional normalisation, softmax, top-k.
+ * FastMoE announcement, "特色二" (the gate is one fully-connected layer) and
+ * "图4" (top-2 gate: the two highest-scoring experts are activated).
+ *   x[T, d], Wg[E, d] (cfg dtype); bg[E] fp32 or NULL (no bias).
+ *   topk_idx[T, k] int32: selected experts, best first; equal scores resolve
+ *     to the lower expert index.
+ *   topk_w[T, k] fp32: softmax probabilities of the selected experts divided
+ *     by their sum (they sum to 1).
+ *   gap[T] fp32: k-th minus (k+1)-th largest score (z_hat or z), +inf if k == E.
+ *   prob_mean[E] fp32 or NULL: P_e = mean over tokens of the full softmax
+ *     probability of expert e (input of the aux loss).
+ *   ws: at least moe_scratch_size(cfg) bytes.
+ */
+moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Step 3: histogram, prefix sums, stable ranks, capacity drop, gather.
+ * Megatron-Core best-practice page, sections "MoE负载均衡的挑战与应对" (expert
+ * capacity; overflow tokens are dropped and carried by the residual; dropless
+ * alternative) and "Megatron-Core MoE的关键特性" (token permutation kernels).
+ *   topk_idx[T, k] int32 (an index outside [0, E) sets MOE_DEV_BOUNDS and the
+ *     slot is treated as dropped).
+ *   gap[T] fp32 or NULL: only used for near_tie_count.
+ *   prob_mean[E] fp32 or NULL: only used for aux_loss.
+ *   counts[E]: assignments per expert; kept[E]: after the capacity;
+ *   offsets[E+1]: exclusive prefix sum of kept (expert e owns permuted rows
+ *     [offsets[e], offsets[e+1]) in ascending token order).
+ *   row_of[T, k]: permuted row of slot (t, j), -1 if dropped.
+ *   src_tok[A]: token of each permuted row (rows >= offsets[E] untouched).
+ *   xp[A, d]: xp[row] = x[src_tok[row]].
+ *   stats: device moe_stats (required).
+ */
+moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                       const float* gap, const float* prob_mean,
+                       int32_t* counts, int32_t* kept, int32_t* offsets,
+                       int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Step 4: the experts over their row segments, one grouped GEMM per layer.
+ * Megatron-Core best-practice page, "Megatron-Core MoE的关键特性"
+ * (GroupedGEMM merges the experts' small GEMMs into one kernel); FastMoE
+ * announcement, Transformer-XL experiment (two-layer ReLU MLP experts).
+ *   ReLU:   h = relu(xp W1[e]^T);  SwiGLU: h = silu(xp Wg_e^T) * (xp Wu_e^T),
+ *           silu(u) = u / (1 + exp(-u));   then yp = h W2[e]^T.
+ *   xp[A, d], offsets[E+1] (device, from moe_permute), W1[E, F1, d],
+ *   W2[E, d, F]; h[A, F] and yp[A, d] are written for rows [0, offsets[E]).
+ *   bf16: h is rounded to bf16 after the fp32 activation; yp is bf16.
+ *   stats: device moe_stats; a kernel timeout ORs MOE_DEV_TIMEOUT into status.
+ *   ws: at least moe_scratch_size(cfg) bytes.
+ */
+moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                          const void* W1, const void* W2, void* h, void* yp,
+                          moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Step 5: un-permute and combine.  out[t] = sum over j = 0..k-1 with
+ * row_of[t, j] >= 0 of topk_w[t, j] * yp[row_of[t, j]], accumulated in fp32 in
+ * slot order; 0 for a token whose slots were all dropped (the residual path
+ * outside the layer carries it: Megatron-Core best-practice page, section
+ * "MoE负载均衡的挑战与应对").
+ *   yp[A, d], row_of[T, k], topk_w[T, k] -> out[T, d].
+ */
+moe_status moe_combine(const moe_config* cfg, const void* yp, const int32_t* row_of,
+                       const float* topk_w, void* out, moe_stream_t stream);
+
+/*
+ * The whole layer: steps 1-5 back to back on `stream`, intermediates inside
+ * `ws` (layout from moe_workspace_size).  No host synchronisation and no
+ * device-to-host copy, so it may be captured in a CUDA graph.
+ *   x[T, d], Wg[E, d], bg[E] or NULL, W1[E, F1, d], W2[E, d, F] -> out[T, d];
+ *   stats: device moe_stats (required).
+ */
+moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                             const void* W1, const void* W2, void* out, moe_stats* stats,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

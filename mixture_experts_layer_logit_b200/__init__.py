@@ -1,0 +1,178 @@
+"""Python binding of libmoe, the sm_100a MoE-layer forward library.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libmoe.so`` behind the C ABI declared in ``include/moe.h``.  PyTorch is used
+for device memory and streams; tensors are passed as raw device pointers and
+the current torch stream is used unless another one is given.  There is no
+CPU fallback: if the library is missing, loading it raises.
+
+Python names match the C entry points: ``moe_route``, ``moe_permute``,
+``moe_expert_ffn``, ``moe_combine``, ``moe_layer_forward``, plus
+``moe_scratch_size``, ``moe_workspace_size`` and ``moe_status_string``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "LIB_PATH", "MoeError", "moe_config", "moe_stats", "moe_ws_layout", "lib", "make_config",
+    "moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route", "moe_permute",
+    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "MOE_ACT_RELU", "MOE_ACT_SWIGLU",
+    "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+MOE_DEV_TIMEOUT, MOE_DEV_BOUNDS = 1, 2
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA"}
+
+EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route",
+                    "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"]
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("lambda_", ctypes.c_float)]
+
+
+class moe_stats(ctypes.Structure):
+    _fields_ = [("drop_count", ctypes.c_int32), ("rows_kept", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("near_tie_count", ctypes.c_int32), ("drop_rate", ctypes.c_float), ("aux_loss", ctypes.c_float),
+                ("status", ctypes.c_uint32), ("reserved", ctypes.c_int32)]
+
+
+class moe_ws_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ["topk_idx", "topk_w", "gap", "counts", "kept", "offsets", "row_of", "src_tok",
+                 "xp", "h", "yp", "scratch", "total"]]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)} ({moe_status_string(code)})")
+        self.code = code
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: run `python -m mixture_experts_layer_logit_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    cfgp = ctypes.POINTER(moe_config)
+    st = ctypes.c_int
+    L.moe_status_string.argtypes = [st]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_scratch_size.argtypes = [cfgp]
+    L.moe_scratch_size.restype = ctypes.c_size_t
+    L.moe_workspace_size.argtypes = [cfgp, ctypes.POINTER(moe_ws_layout)]
+    L.moe_workspace_size.restype = ctypes.c_size_t
+    L.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_permute.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_combine.argtypes = [cfgp, P, P, P, P, P]
+    L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"]:
+        getattr(L, n).restype = st
+    _lib = L
+    return L
+
+
+def make_config(T: int, d: int, E: int, F: int, k: int, act: str = "relu", dtype: str = "bf16",
+                capacity_factor: float = 0.0, lam: float = 0.0) -> moe_config:
+    return moe_config(T, d, E, F, k, MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_RELU,
+                      MOE_DTYPE_BF16 if dtype == "bf16" else MOE_DTYPE_F32, capacity_factor, lam)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a tensor (None -> NULL); also accepts raw ints."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MoeError(fn, code)
+
+
+def moe_status_string(code: int) -> str:
+    return lib().moe_status_string(code).decode()
+
+
+def moe_scratch_size(cfg: moe_config) -> int:
+    return lib().moe_scratch_size(ctypes.byref(cfg))
+
+
+def moe_workspace_size(cfg: moe_config):
+    """(bytes, moe_ws_layout) of the moe_layer_forward workspace."""
+    L = moe_ws_layout()
+    n = lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(L))
+    return n, L
+
+
+def moe_route(cfg, x, Wg, bg, topk_idx, topk_w, gap, prob_mean, ws, stream=None):
+    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg), _ptr(topk_idx),
+                                        _ptr(topk_w), _ptr(gap), _ptr(prob_mean), _ptr(ws), _nbytes(ws),
+                                        _stream(stream)))
+
+
+def moe_permute(cfg, x, topk_idx, gap, prob_mean, counts, kept, offsets, row_of, src_tok, xp, stats, ws,
+                stream=None):
+    _check("moe_permute", lib().moe_permute(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(gap),
+                                            _ptr(prob_mean), _ptr(counts), _ptr(kept), _ptr(offsets),
+                                            _ptr(row_of), _ptr(src_tok), _ptr(xp), _ptr(stats), _ptr(ws),
+                                            _nbytes(ws), _stream(stream)))
+
+
+def moe_expert_ffn(cfg, xp, offsets, W1, W2, h, yp, stats, ws, stream=None):
+    _check("moe_expert_ffn", lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(xp), _ptr(offsets), _ptr(W1),
+                                                  _ptr(W2), _ptr(h), _ptr(yp), _ptr(stats), _ptr(ws),
+                                                  _nbytes(ws), _stream(stream)))
+
+
+def moe_combine(cfg, yp, row_of, topk_w, out, stream=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(yp), _ptr(row_of), _ptr(topk_w),
+                                            _ptr(out), _stream(stream)))
+
+
+def moe_layer_forward(cfg, x, Wg, bg, W1, W2, out, stats, ws, stream=None):
+    _check("moe_layer_forward", lib().moe_layer_forward(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg),
+                                                        _ptr(W1), _ptr(W2), _ptr(out), _ptr(stats), _ptr(ws),
+                                                        _nbytes(ws), _stream(stream)))
+
+
+def read_stats(stats_tensor) -> dict:
+    """Copy a device moe_stats (a uint8 tensor of sizeof(moe_stats) bytes) to a dict (synchronises)."""
+    raw = bytes(stats_tensor.cpu().numpy().tobytes())
+    s = moe_stats.from_buffer_copy(raw[:ctypes.sizeof(moe_stats)])
+    return {f: getattr(s, f) for f, _ in moe_stats._fields_}
+
+
+STATS_BYTES = ctypes.sizeof(moe_stats)

@@ -1,0 +1,291 @@
+// C ABI of libmoe: argument checks, workspace layout and the order of the
+// kernels of each step.  See include/moe.h for the contract of every entry.
+#include "internal.cuh"
+
+#include <math.h>
+#include <mutex>
+
+namespace moe {
+
+cudaError_t device_info(DeviceInfo* out) {
+  constexpr int kMaxDev = 64;
+  static DeviceInfo cache[kMaxDev];
+  static std::once_flag once[kMaxDev];
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  cudaError_t res = cudaSuccess;
+  std::call_once(once[dev], [&] {
+    DeviceInfo d;
+    int v = 0;
+    if ((res = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return;
+    d.sms = v;
+    if ((res = cudaDeviceGetAttribute(&v, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return;
+    d.major = v;
+    if ((res = cudaDeviceGetAttribute(&v, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return;
+    d.minor = v;
+    if ((res = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return;
+    d.smem_optin = (size_t)v;
+    cache[dev] = d;
+  });
+  if (res != cudaSuccess) return res;
+  if (cache[dev].sms == 0) return cudaErrorUnknown;
+  *out = cache[dev];
+  return cudaSuccess;
+}
+
+Scratch scratch_layout(const moe_config& c) {
+  const size_t nch = (size_t)num_chunks(c.T);
+  Scratch s;
+  size_t off = 0;
+  s.hist = off;  off = align256(off + sizeof(int32_t) * (size_t)c.E * nch);
+  s.choff = off; off = align256(off + sizeof(int32_t) * (size_t)c.E * nch);
+  s.psum = off;  off = align256(off + sizeof(float) * (size_t)c.E * nch);
+  s.ntie = off;  off = align256(off + sizeof(int32_t) * nch);
+  s.total = off > 0 ? off : 256;
+  return s;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+moe_status check_config(const moe_config* c) {
+  if (c == nullptr) return MOE_ERR_ARG;
+  if (c->T < 0 || c->d < 1 || c->E < 1 || c->F < 1 || c->k < 1) return MOE_ERR_ARG;
+  if (c->k > c->E) return MOE_ERR_ARG;
+  if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
+  if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32) return MOE_ERR_ARG;
+  if (!isfinite(c->capacity_factor) || !isfinite(c->lambda)) return MOE_ERR_ARG;
+  if (c->E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  const int mult = (c->dtype == MOE_DTYPE_BF16) ? 16 : 4;
+  if (c->d % mult != 0 || c->F % mult != 0) return MOE_ERR_UNSUPPORTED;
+  // index arithmetic stays in int32 for T*k rows and 64-bit for elements
+  if ((long long)c->T * c->k > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c->E * (c->act == MOE_ACT_SWIGLU ? 2 : 1) * c->F > (1LL << 31) - 1) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Capacity in assignments; -1 in dropless mode.  Evaluated in double in the
+// order the header states; saturates at INT32_MAX (any C >= T keeps everything).
+int capacity_of(const moe_config& c) {
+  if (!(c.capacity_factor > 0.f)) return -1;
+  const double C = ceil((double)c.capacity_factor * (double)((long long)c.T * c.k) / (double)c.E);
+  if (C >= 2147483647.0) return 2147483647;
+  return (int)C;
+}
+
+moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status check_device(bool need_tc) {
+  DeviceInfo di;
+  if (device_info(&di) != cudaSuccess) return MOE_ERR_CUDA;
+  if (need_tc && di.major != 10) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+size_t elem_size(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+moe_ws_layout layout_of(const moe_config& c) {
+  moe_ws_layout L{};
+  const size_t T = (size_t)c.T, k = (size_t)c.k, E = (size_t)c.E, A = T * k, es = elem_size(c);
+  size_t off = 0;
+  L.topk_idx = off;  off = align256(off + 4 * A);
+  L.topk_w = off;    off = align256(off + 4 * A);
+  L.gap = off;       off = align256(off + 4 * T);
+  L.counts = off;    off = align256(off + 4 * E);
+  L.kept = off;      off = align256(off + 4 * E);
+  L.offsets = off;   off = align256(off + 4 * (E + 1));
+  L.row_of = off;    off = align256(off + 4 * A);
+  L.src_tok = off;   off = align256(off + 4 * A);
+  L.xp = off;        off = align256(off + es * A * (size_t)c.d);
+  L.h = off;         off = align256(off + es * A * (size_t)c.F);
+  L.yp = off;        off = align256(off + es * A * (size_t)c.d);
+  L.scratch = off;   off = align256(off + scratch_layout(c).total);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(base) + off); }
+
+// step 3 given the histogram already in scratch
+moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* topk_idx,
+                             const float* prob_mean, const float* psum, const int32_t* ntie,
+                             int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
+                             int32_t* src_tok, void* xp, moe_stats* stats, const Scratch& sc, void* ws,
+                             cudaStream_t s) {
+  const int cap = capacity_of(c);
+  cudaError_t e = launch_scan(c, cap, at<int32_t>(ws, sc.hist), at<int32_t>(ws, sc.choff), prob_mean, psum,
+                              ntie, counts, kept, offsets, stats, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_scatter(c, cap, x, topk_idx, at<int32_t>(ws, sc.choff), offsets, row_of, src_tok, xp,
+                     &stats->status, s);
+  return cuda_status(e);
+}
+
+moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
+                      const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s) {
+  if (c.dtype == MOE_DTYPE_BF16)
+    return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
+  return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_ARG: return "MOE_ERR_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape or device not supported";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+  }
+  return "unknown moe_status";
+}
+
+size_t moe_scratch_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return scratch_layout(*cfg).total;
+}
+
+size_t moe_workspace_size(const moe_config* cfg, moe_ws_layout* layout) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  const moe_ws_layout L = layout_of(*cfg);
+  if (layout != nullptr) *layout = L;
+  return L.total;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean,
+                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T > 0 && (x == nullptr || Wg == nullptr || topk_idx == nullptr || topk_w == nullptr || gap == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned4(bg) || !aligned4(topk_idx) || !aligned4(topk_w) ||
+      !aligned4(gap) || !aligned4(prob_mean))
+    return MOE_ERR_ARG;
+  const Scratch sc = scratch_layout(c);
+  if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
+  if ((st = check_device(false)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_route(c, x, Wg, bg, topk_idx, topk_w, gap, at<int32_t>(ws, sc.hist),
+                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (prob_mean != nullptr) e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s);
+  return cuda_status(e);
+}
+
+moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                       const float* gap, const float* prob_mean,
+                       int32_t* counts, int32_t* kept, int32_t* offsets,
+                       int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (counts == nullptr || kept == nullptr || offsets == nullptr || stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (x == nullptr || topk_idx == nullptr || row_of == nullptr || src_tok == nullptr || xp == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(xp) || !aligned4(topk_idx) || !aligned4(gap) || !aligned4(prob_mean) ||
+      !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) || !aligned4(row_of) || !aligned4(src_tok) ||
+      !aligned4(stats))
+    return MOE_ERR_ARG;
+  const Scratch sc = scratch_layout(c);
+  if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
+  if ((st = check_device(false)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = launch_hist(c, topk_idx, gap, at<int32_t>(ws, sc.hist), at<int32_t>(ws, sc.ntie),
+                              &stats->status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return permute_from_hist(c, x, topk_idx, prob_mean, nullptr,
+                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, counts, kept,
+                           offsets, row_of, src_tok, xp, stats, sc, ws, s);
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                          const void* W1, const void* W2, void* h, void* yp,
+                          moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (offsets == nullptr || stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (xp == nullptr || W1 == nullptr || W2 == nullptr || h == nullptr || yp == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(xp) || !aligned16(W1) || !aligned16(W2) || !aligned16(h) || !aligned16(yp) ||
+      !aligned4(offsets) || !aligned4(stats))
+    return MOE_ERR_ARG;
+  const Scratch sc = scratch_layout(c);
+  if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
+  if ((st = check_device(c.dtype == MOE_DTYPE_BF16)) != MOE_OK) return st;
+  return expert_ffn(c, xp, offsets, W1, W2, h, yp, stats, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* yp, const int32_t* row_of,
+                       const float* topk_w, void* out, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T > 0 && (yp == nullptr || row_of == nullptr || topk_w == nullptr || out == nullptr)) return MOE_ERR_ARG;
+  if (!aligned16(yp) || !aligned16(out) || !aligned4(row_of) || !aligned4(topk_w)) return MOE_ERR_ARG;
+  if ((st = check_device(false)) != MOE_OK) return st;
+  return cuda_status(launch_combine(c, yp, row_of, topk_w, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                             const void* W1, const void* W2, void* out, moe_stats* stats,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (x == nullptr || Wg == nullptr || W1 == nullptr || W2 == nullptr || out == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned4(bg) || !aligned16(W1) || !aligned16(W2) ||
+      !aligned16(out) || !aligned4(stats))
+    return MOE_ERR_ARG;
+  const moe_ws_layout L = layout_of(c);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return st;
+  if ((st = check_device(c.dtype == MOE_DTYPE_BF16)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scr = at<char>(ws, L.scratch);
+  const Scratch sc = scratch_layout(c);
+  int32_t* idx = at<int32_t>(ws, L.topk_idx);
+  float* w = at<float>(ws, L.topk_w);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  void* yp = at<char>(ws, L.yp);
+
+  if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  // steps 1-2: the route kernel also leaves the histogram, probability sums and
+  // near-tie counts of every chunk in scratch, so step 3 starts at the scan
+  cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
+                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
+                         c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, at<int32_t>(ws, L.counts),
+                         at<int32_t>(ws, L.kept), offsets, row_of, at<int32_t>(ws, L.src_tok),
+                         at<char>(ws, L.xp), stats, sc, scr, s);
+  if (st != MOE_OK) return st;
+  st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_combine(c, yp, row_of, w, out, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+// Step 5 of the layer: un-permute and combine.
+//
+// out[t] = sum over kept slots j (slot order, fp32 accumulation) of
+// w[t, j] * yp[row_of[t, j]]; a token whose slots were all dropped gets 0, the
+// residual path outside the layer carrying it (Megatron-Core best-practice
+// page, "MoE负载均衡的挑战与应对").  The sum itself is the definition of the
+// layer output (FastMoE announcement, "1. MoE 设计").
+//
+// One warp per token; each lane owns 16-byte column vectors of the row and
+// issues the k row reads of a vector back to back.
+#include "internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTokPerBlock = kThreads / 32;
+
+template <typename TX> struct Pack;
+template <> struct Pack<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void acc(const uint4& v, float w, float* a) {
+    a[0] = fmaf(w, __uint_as_float(v.x), a[0]);
+    a[1] = fmaf(w, __uint_as_float(v.y), a[1]);
+    a[2] = fmaf(w, __uint_as_float(v.z), a[2]);
+    a[3] = fmaf(w, __uint_as_float(v.w), a[3]);
+  }
+  __device__ __forceinline__ static uint4 store(const float* a) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+template <> struct Pack<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void acc(const uint4& v, float w, float* a) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      a[2 * i] = fmaf(w, f.x, a[2 * i]);
+      a[2 * i + 1] = fmaf(w, f.y, a[2 * i + 1]);
+    }
+  }
+  __device__ __forceinline__ static uint4 store(const float* a) {
+    uint4 r;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+    return r;
+  }
+};
+
+template <typename TX, int KB>
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
+               const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
+  constexpr int N = Pack<TX>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTokPerBlock + warp;
+  if (t >= T) return;
+  int rows[KB];
+  float ws[KB];
+  const int A = T * k;
+#pragma unroll
+  for (int j = 0; j < KB; ++j) {
+    rows[j] = (j < k) ? __ldg(row_of + (size_t)t * k + j) : -1;
+    if (rows[j] >= A) rows[j] = -1;   // outside the permuted buffer: treated as dropped
+    ws[j] = (j < k) ? __ldg(topk_w + (size_t)t * k + j) : 0.f;
+  }
+  const int nvec = d / N;
+  uint4* o = reinterpret_cast<uint4*>(out + (size_t)t * d);
+  for (int v = lane; v < nvec; v += 32) {
+    uint4 in[KB];
+#pragma unroll
+    for (int j = 0; j < KB; ++j)
+      if (rows[j] >= 0) in[j] = __ldg(reinterpret_cast<const uint4*>(yp + (size_t)rows[j] * d) + v);
+    float a[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) a[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KB; ++j)
+      if (rows[j] >= 0) Pack<TX>::acc(in[j], ws[j], a);
+    o[v] = Pack<TX>::store(a);
+  }
+}
+
+// any k: rows read slot by slot
+template <typename TX>
+__global__ void __launch_bounds__(kThreads)
+combine_generic_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
+                       const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
+  constexpr int N = Pack<TX>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTokPerBlock + warp;
+  if (t >= T) return;
+  const int nvec = d / N;
+  uint4* o = reinterpret_cast<uint4*>(out + (size_t)t * d);
+  for (int v = lane; v < nvec; v += 32) {
+    float a[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) a[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int r = row_of[(size_t)t * k + j];
+      if (r < 0 || r >= T * k) continue;
+      Pack<TX>::acc(__ldg(reinterpret_cast<const uint4*>(yp + (size_t)r * d) + v), topk_w[(size_t)t * k + j], a);
+    }
+    o[v] = Pack<TX>::store(a);
+  }
+}
+
+template <typename TX>
+cudaError_t launch_t(const moe_config& c, const void* yp, const int32_t* row_of, const float* w,
+                     void* out, cudaStream_t s) {
+  const int grid = (c.T + kTokPerBlock - 1) / kTokPerBlock;
+  const TX* y = static_cast<const TX*>(yp);
+  TX* o = static_cast<TX*>(out);
+  if (c.k <= 1) combine_kernel<TX, 1><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
+  else if (c.k <= 2) combine_kernel<TX, 2><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
+  else if (c.k <= 4) combine_kernel<TX, 4><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
+  else if (c.k <= 8) combine_kernel<TX, 8><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
+  else combine_generic_kernel<TX><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_config& c, const void* yp, const int32_t* row_of,
+                           const float* topk_w, void* out, cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  if (c.dtype == MOE_DTYPE_BF16) return launch_t<__nv_bfloat16>(c, yp, row_of, topk_w, out, s);
+  return launch_t<float>(c, yp, row_of, topk_w, out, s);
+}
+
+}  // namespace moe

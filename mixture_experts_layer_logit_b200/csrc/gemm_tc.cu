@@ -1,0 +1,448 @@
+// Step 4 on the 5th-generation tensor cores (sm_100a): the experts' two
+// layers as grouped GEMMs over the variable-length expert segments.
+//
+// Megatron-Core best-practice page, "Megatron-Core MoE的关键特性": GroupedGEMM
+// merges the experts' many small GEMMs into one kernel to keep the SMs busy.
+// Experts: two-layer ReLU MLP (FastMoE announcement, Transformer-XL
+// experiment) or SwiGLU whose W1 holds the gate rows before the up rows
+// (Megatron-Core page, "从HuggingFace到Megatron的权重转换要点").
+//
+// Design (one CTA per SM, persistent):
+//   * A = expert-grouped rows (xp or h), B = one expert's weight rows; both
+//     K-major bf16, staged by TMA (128-byte swizzle) into a STAGES-deep ring.
+//   * warp 0 lane 0 issues the TMA loads, warp 1 lane 0 issues
+//     tcgen05.mma.cta_group::1.kind::f16 (128 x 256 x 16, fp32 accumulators in
+//     TMEM), warps 2-5 drain TMEM with tcgen05.ld, apply the activation
+//     (ReLU, or silu(gate) * up for SwiGLU) and store bf16 rows.
+//   * two 256-column TMEM accumulators let the epilogue of one tile overlap
+//     the main loop of the next.
+//   * the tile table (ceil(M_e / 128) * n-tiles per expert) is built on the
+//     device from offsets[], so nothing is read back to the host; within an
+//     expert the m-tiles of one n-tile are consecutive, so the CTAs working at
+//     the same time share the same weight tile in L2.
+//   * a tile that runs past its expert's segment computes rows of the next
+//     expert (or zero rows past the buffer) and masks them at the store.
+//   * every mbarrier wait is bounded (~2 s); on timeout the kernel sets
+//     MOE_DEV_TIMEOUT, tells the other roles to stop, waits for its own TMA
+//     loads and MMAs, frees TMEM and returns.
+#include "internal.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;              // 16 KB
+constexpr int B_BYTES = BN * BK * 2;              // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 2000000000ull;    // bounded waits: 2 s
+constexpr unsigned long long kDrainNs = 200000000ull;    // teardown waits: 0.2 s
+enum { kPlain = 0, kRelu = 1, kSwiglu = 2 };
+
+// instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B bf16,
+// both K-major, M = 128, N = 256
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+struct Tail {
+  unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int tstart[kMaxExperts + 1];
+};
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Tail);
+
+struct Params {
+  const int32_t* offsets;
+  __nv_bfloat16* out;   // [rows][Nout]
+  int E, K, Nout;
+  int b_rows;           // B rows per expert
+  int up_off;           // SwiGLU: first up row inside an expert's B block
+  int rows_alloc;       // rows of the A and output buffers (T*k); stores stop there
+  uint32_t* status;
+};
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of `parity` to complete.  Gives up (false) after `limit`
+// ns or, when `abort_flag` is given, once another role has given up.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                       unsigned long long limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0) {
+      if (abort_flag != nullptr && *abort_flag) return false;
+      if (now_ns() - t0 > limit) return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns; thread i of the warp gets its lane's row
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), descriptor version 1.  The start address advances by
+// 32 bytes per K = 16 step inside the 128-byte swizzle row.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;               // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
+  d |= (uint64_t)1 << 46;               // version
+  d |= (uint64_t)2 << 61;               // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+struct TileCoord {
+  int e, row0, rows, n0;
+};
+
+template <int MODE>
+__device__ __forceinline__ TileCoord decode_tile(const int* tstart, const int32_t* offsets, int E, int L) {
+  TileCoord c;
+  c.e = tile_expert(tstart, E, L);
+  const int seg0 = offsets[c.e];
+  const int M = offsets[c.e + 1] - seg0;
+  const int mt = (M + BM - 1) / BM;
+  const int local = L - tstart[c.e];
+  const int nti = local / mt, mti = local - nti * mt;
+  c.row0 = seg0 + mti * BM;
+  c.rows = min(BM, M - mti * BM);
+  c.n0 = nti * (MODE == kSwiglu ? BN / 2 : BN);
+  return c;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  Tail* tail = reinterpret_cast<Tail*>(smem_raw + (base - raw) + (size_t)STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nt = (MODE == kSwiglu) ? (p.Nout + BN / 2 - 1) / (BN / 2) : (p.Nout + BN - 1) / BN;
+  const int nkb = (p.K + BK - 1) / BK;
+
+  const uint32_t full0 = smem_u32(&tail->full[0]), empty0 = smem_u32(&tail->empty[0]);
+  const uint32_t tfull0 = smem_u32(&tail->tfull[0]), tempty0 = smem_u32(&tail->tempty[0]);
+  const uint32_t drain = smem_u32(&tail->drain);
+  const volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 4);
+    }
+    mbar_init(drain, 1);
+    tail->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tile_table_warp(p.offsets, p.E, BM, nt, tail->tstart, lane);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&tail->tmem_base)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+  const int total = tail->tstart[p.E];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+      int it = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+        const TileCoord c = decode_tile<MODE>(tail->tstart, p.offsets, p.E, L);
+        const int b0 = c.e * p.b_rows + c.n0;
+        const int b1 = (MODE == kSwiglu) ? b0 + p.up_off : b0 + BN / 2;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+          const uint32_t sa = base + (uint32_t)(s * STAGE_BYTES);
+          mbar_expect_tx(full0 + 8 * s, STAGE_BYTES);
+          tma_load_2d(sa, &tmA, full0 + 8 * s, kb * BK, c.row0);
+          tma_load_2d(sa + A_BYTES, &tmB, full0 + 8 * s, kb * BK, b0);
+          tma_load_2d(sa + A_BYTES + B_BYTES / 2, &tmB, full0 + 8 * s, kb * BK, b1);
+          ++it;
+        }
+      }
+      if (!ok) {
+        atomicOr(p.status, MOE_DEV_TIMEOUT);
+        tail->abort_flag = 1;
+      }
+      // wait for the loads still in flight before the CTA may exit
+      for (int i = max(0, it - STAGES); i < it; ++i)
+        mbar_wait(full0 + 8 * (i % STAGES), (uint32_t)(i / STAGES) & 1u, nullptr, kDrainNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kWaitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + (uint32_t)(s * STAGE_BYTES);
+          const uint64_t ad = sdesc(sa), bd = sdesc(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), kIdesc, (kb | kk) != 0);
+          tc_commit(empty0 + 8 * s);   // frees the stage once these MMAs have read it
+          ++it;
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);   // accumulator ready for the epilogue
+      }
+      if (!ok) {
+        atomicOr(p.status, MOE_DEV_TIMEOUT);
+        tail->abort_flag = 1;
+      }
+      tc_commit(drain);                 // every MMA issued above has completed
+      mbar_wait(drain, 0, nullptr, kDrainNs);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;              // TMEM lanes 32q..32q+31 belong to this warp
+    int tl = 0;
+    bool ok = true;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tl) {
+      const TileCoord c = decode_tile<MODE>(tail->tstart, p.offsets, p.E, L);
+      const int acc = tl & 1;
+      const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
+      ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int r = q * 32 + lane;
+      bool rv = r < c.rows;
+      if (rv && c.row0 + r >= p.rows_alloc) {   // offsets[] beyond the buffers: skip and flag
+        atomicOr(p.status, MOE_DEV_BOUNDS);
+        rv = false;
+      }
+      __nv_bfloat16* orow = p.out + (size_t)(c.row0 + (rv ? r : 0)) * p.Nout;
+      if (MODE == kSwiglu) {
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 64; ++ch) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tb + ch * 32, g);
+          tmem_ld32(tb + BN / 2 + ch * 32, u);
+          tmem_wait_ld();
+          const int col = c.n0 + ch * 32;
+          if (rv) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + 8 * v >= p.Nout) break;
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float g0 = __uint_as_float(g[8 * v + 2 * i]), g1 = __uint_as_float(g[8 * v + 2 * i + 1]);
+                const float u0 = __uint_as_float(u[8 * v + 2 * i]), u1 = __uint_as_float(u[8 * v + 2 * i + 1]);
+                pk[i] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+              }
+              *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t a[32];
+          tmem_ld32(tb + ch * 32, a);
+          tmem_wait_ld();
+          const int col = c.n0 + ch * 32;
+          if (rv) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + 8 * v >= p.Nout) break;
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                float a0 = __uint_as_float(a[8 * v + 2 * i]), a1 = __uint_as_float(a[8 * v + 2 * i + 1]);
+                if (MODE == kRelu) { a0 = fmaxf(a0, 0.f); a1 = fmaxf(a1, 0.f); }
+                pk[i] = pack_bf16x2(a0, a1);
+              }
+              *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);   // accumulator free again
+    }
+    if (!ok && lane == 0) {
+      atomicOr(p.status, MOE_DEV_TIMEOUT);
+      tail->abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix; box = 64 columns
+// (128 bytes) x 128 rows, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid, cudaStream_t s) {
+  cudaError_t err = set_smem_once<tc_grouped_gemm<MODE>>(kSmemBytes);
+  if (err != cudaSuccess) return err;
+  tc_grouped_gemm<MODE><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
+                                 const void* w1, const void* w2, void* h, void* yp,
+                                 uint32_t* status, cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
+  const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
+  const long long mt_max = (long long)(rows / BM) + c.E;
+  CUtensorMap ma, mb;
+
+  // layer 1: h = act(xp W1[e]^T)
+  if (!make_map(&ma, xp, rows, (uint64_t)c.d) || !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d))
+    return cudaErrorInvalidValue;
+  Params p1{offsets, static_cast<__nv_bfloat16*>(h), c.E, c.d, c.F, F1, c.F, (int)rows, status};
+  if (c.act == MOE_ACT_SWIGLU) {
+    const long long nt = (c.F + BN / 2 - 1) / (BN / 2);
+    err = launch_one<kSwiglu>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, di.sms), s);
+  } else {
+    const long long nt = (c.F + BN - 1) / BN;
+    err = launch_one<kRelu>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, di.sms), s);
+  }
+  if (err != cudaSuccess) return err;
+
+  // layer 2: yp = h W2[e]^T
+  if (!make_map(&ma, h, rows, (uint64_t)c.F) || !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F))
+    return cudaErrorInvalidValue;
+  Params p2{offsets, static_cast<__nv_bfloat16*>(yp), c.E, c.F, c.d, c.d, 0, (int)rows, status};
+  const long long nt2 = (c.d + BN - 1) / BN;
+  return launch_one<kPlain>(ma, mb, p2, (int)std::min<long long>(mt_max * nt2, di.sms), s);
+}
+
+}  // namespace moe

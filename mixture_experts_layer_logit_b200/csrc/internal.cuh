@@ -1,0 +1,160 @@
+// Internal declarations shared by the CUDA translation units of libmoe.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Tokens per routing / permutation chunk.  The route kernel, the histogram and
+// the scatter kernel all cut the token axis into chunks of this size, and the
+// per-chunk histograms and prefix sums live in the scratch workspace.
+constexpr int kChunk = 64;
+constexpr int kMaxExperts = 256;
+
+// Scratch layout (byte offsets into the step workspace).
+struct Scratch {
+  size_t hist;      // int32 [E][nchunks]   assignments per (expert, chunk)
+  size_t choff;     // int32 [E][nchunks]   exclusive prefix over chunks
+  size_t psum;      // float [nchunks][E]   per-chunk sums of softmax probabilities
+  size_t ntie;      // int32 [nchunks]      near-tie tokens per chunk
+  size_t total;
+};
+
+inline int num_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+Scratch scratch_layout(const moe_config& c);
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------------ launchers
+// Every launcher enqueues on `s` and returns cudaGetLastError().
+
+// Route: logits, normalisation, softmax, top-k; per-chunk histogram, probability
+// sums and near-tie counts into scratch.  TX = float or __nv_bfloat16.
+cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
+                         int32_t* topk_idx, float* topk_w, float* gap,
+                         int32_t* hist, float* psum, int32_t* ntie, cudaStream_t s);
+// prob_mean[e] = sum over chunks of psum / T (fixed order).
+cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
+// Histogram of topk_idx per chunk (+ near ties from gap when given).
+cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const float* gap,
+                        int32_t* hist, int32_t* ntie, uint32_t* status, cudaStream_t s);
+// Scan: counts, kept, offsets, per-chunk offsets, stats.  Either prob_mean
+// (standalone) or psum (fused forward) or neither supplies P_e for the aux loss.
+cudaError_t launch_scan(const moe_config& c, int capacity, const int32_t* hist, int32_t* choff,
+                        const float* prob_mean, const float* psum, const int32_t* ntie,
+                        int32_t* counts, int32_t* kept, int32_t* offsets, moe_stats* stats,
+                        cudaStream_t s);
+// Stable ranks, capacity test, row_of/src_tok, and the gather xp[row] = x[t].
+cudaError_t launch_scatter(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
+                           const int32_t* choff, const int32_t* offsets, int32_t* row_of,
+                           int32_t* src_tok, void* xp, uint32_t* status, cudaStream_t s);
+// Expert FFN on CUDA cores (fp32 path).
+cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
+                                   const void* w1, const void* w2, void* h, void* yp, cudaStream_t s);
+// Expert FFN on tcgen05 tensor cores (bf16 path).
+cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
+                                 const void* w1, const void* w2, void* h, void* yp,
+                                 uint32_t* status, cudaStream_t s);
+// Combine.
+cudaError_t launch_combine(const moe_config& c, const void* yp, const int32_t* row_of,
+                           const float* topk_w, void* out, cudaStream_t s);
+
+// Device properties cached per device (SM count, compute capability).
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  size_t smem_optin = 0;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+}  // namespace moe
+
+namespace moe {
+
+// Tile table of a grouped GEMM over expert segments: expert e owns rows
+// [offsets[e], offsets[e+1]) and ceil(M_e / BM) * nt tiles, numbered from
+// tstart[e]; tstart[E] is the total.  Run by the 32 lanes of one warp
+// (E <= 256, 8 experts per lane).
+__device__ __forceinline__ void tile_table_warp(const int32_t* __restrict__ offsets, int E, int BM,
+                                                int nt, int* tstart, int lane) {
+  constexpr int PER = kMaxExperts / 32;
+  int loc[PER];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    int m = (e < E) ? offsets[e + 1] - offsets[e] : 0;
+    m = m > 0 ? m : 0;
+    loc[i] = ((m + BM - 1) / BM) * nt;
+    sum += loc[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    if (e < E) tstart[e] = run;
+    run += loc[i];
+  }
+  if (lane == 31) tstart[E] = incl;
+}
+
+// Expert owning tile L: the largest e with tstart[e] <= L (empty experts have
+// tstart[e] == tstart[e+1] and are skipped by taking the largest).
+__device__ __forceinline__ int tile_expert(const int* tstart, int E, int L) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tstart[mid] <= L) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace moe
+
+#include <atomic>
+
+namespace moe {
+
+// Raises a kernel's dynamic shared-memory limit once per device (the first
+// call, made before any stream capture, does the work; later calls only read
+// an atomic), so launches stay free of attribute calls.
+template <auto Kernel>
+cudaError_t set_smem_once(size_t bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+}  // namespace moe

@@ -216,6 +216,16 @@ def generate(w: Workload, shard: int = 0, threads: int = 8) -> Inputs:
     return Inputs(w, gen_x(w, shard), gen_wg(w), gen_bias(w), gen_w1(w, threads), gen_w2(w, threads))
 
 
+def to_device(a: Optional[np.ndarray], device="cuda"):
+    """Upload a stored input to a torch tensor (bf16 bit patterns -> torch.bfloat16)."""
+    if a is None:
+        return None
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
 class F64Experts:
     """Lazy float64 view of a stacked [E, ...] bf16/fp32 weight array: ``a[e]``
     returns expert e's matrix as exact float64, one expert at a time."""

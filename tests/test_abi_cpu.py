@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute call made).
+
+The library must load, export every function include/moe.h declares, size its
+workspaces consistently, and reject bad arguments synchronously -- before any
+CUDA call -- with the documented status codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_layer_logit_b200 as moe
+from mixture_experts_layer_logit_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|size_t|moe_status)\s+(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"]:
+        assert name in fns
+    assert sorted(moe.EXPORTED_SYMBOLS) == fns
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_functions():
+        assert hasattr(L, name), name
+    # and nothing is linked against libcuda / libtorch: check the dynamic deps
+    import subprocess
+    out = subprocess.run(["ldd", moe.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libtorch" not in out and "libcudart.so" not in out
+
+
+def test_struct_sizes_match_header(L):
+    assert ctypes.sizeof(moe.moe_config) == 9 * 4
+    assert ctypes.sizeof(moe.moe_stats) == 8 * 4
+    assert ctypes.sizeof(moe.moe_ws_layout) == 13 * 8
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert moe.moe_status_string(code).startswith(moe.STATUS_NAMES[code])
+    assert moe.moe_status_string(99) == "unknown moe_status"
+
+
+def cfg(**kw):
+    base = dict(T=100, d=64, E=8, F=128, k=2, act="relu", dtype="bf16", capacity_factor=1.0, lam=0.0)
+    base.update(kw)
+    return moe.make_config(**base)
+
+
+@pytest.mark.parametrize("bad", [dict(k=9), dict(k=0), dict(T=-1), dict(d=0), dict(E=0), dict(F=0),
+                                 dict(capacity_factor=float("nan")), dict(lam=float("inf"))])
+def test_invalid_config_sizes_zero(L, bad):
+    assert moe.moe_scratch_size(cfg(**bad)) == 0
+    assert moe.moe_workspace_size(cfg(**bad))[0] == 0
+
+
+@pytest.mark.parametrize("bad", [dict(E=257), dict(d=72), dict(F=40), dict(dtype="f32", d=66)])
+def test_unsupported_config(L, bad):
+    c = cfg(**bad)
+    assert moe.moe_scratch_size(c) == 0
+    # a step call reports the reason synchronously, before touching the device
+    code = L.moe_combine(ctypes.byref(c), None, None, None, None, None)
+    assert code == 2
+
+
+def test_bad_enum_is_arg_error(L):
+    c = cfg()
+    c.act = 7
+    assert L.moe_combine(ctypes.byref(c), None, None, None, None, None) == 1
+    c = cfg()
+    c.dtype = 5
+    assert L.moe_layer_forward(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None) == 1
+    assert L.moe_route(None, None, None, None, None, None, None, None, None, 0, None) == 1
+
+
+def test_null_and_misaligned_pointers(L):
+    c = cfg()
+    P = 1 << 20  # an aligned non-null stand-in: never dereferenced, the calls fail earlier
+    # required pointers missing
+    assert L.moe_route(ctypes.byref(c), None, P, None, P, P, P, None, P, 1 << 20, None) == 1
+    assert L.moe_permute(ctypes.byref(c), P, P, None, None, P, P, P, P, P, P, None, P, 1 << 20, None) == 1
+    assert L.moe_expert_ffn(ctypes.byref(c), P, None, P, P, P, P, P, P, 1 << 20, None) == 1
+    # misaligned activations (TMA and 16-byte vectors need 16-byte alignment)
+    assert L.moe_route(ctypes.byref(c), P + 8, P, None, P, P, P, None, P, 1 << 20, None) == 1
+    assert L.moe_combine(ctypes.byref(c), P + 4, P, P, P, None) == 1
+
+
+def test_workspace_checks(L):
+    c = cfg()
+    need = moe.moe_scratch_size(c)
+    P = 1 << 20
+    assert L.moe_route(ctypes.byref(c), P, P, None, P, P, P, None, None, need, None) == 3
+    assert L.moe_route(ctypes.byref(c), P, P, None, P, P, P, None, P, need - 1, None) == 3
+    assert L.moe_route(ctypes.byref(c), P, P, None, P, P, P, None, P + 16, need, None) == 3   # not 256-aligned
+    full, layout = moe.moe_workspace_size(c)
+    assert L.moe_layer_forward(ctypes.byref(c), P, P, None, P, P, P, P, P, full - 1, None) == 3
+
+
+def test_workspace_layout_is_disjoint_and_aligned(L):
+    for kw in [dict(), dict(T=32768, d=2048, E=64, F=1408, k=6, act="swiglu"), dict(T=1, E=1, k=1),
+               dict(dtype="f32", d=64, F=96, T=300, E=5)]:
+        c = cfg(**kw)
+        total, lay = moe.moe_workspace_size(c)
+        T, k, E, d, F = c.T, c.k, c.E, c.d, c.F
+        es = 2 if c.dtype == moe.MOE_DTYPE_BF16 else 4
+        A = T * k
+        regions = [("topk_idx", 4 * A), ("topk_w", 4 * A), ("gap", 4 * T), ("counts", 4 * E), ("kept", 4 * E),
+                   ("offsets", 4 * (E + 1)), ("row_of", 4 * A), ("src_tok", 4 * A), ("xp", es * A * d),
+                   ("h", es * A * F), ("yp", es * A * d), ("scratch", moe.moe_scratch_size(c))]
+        spans = sorted((getattr(lay, n), getattr(lay, n) + sz, n) for n, sz in regions)
+        for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
+            assert a1 <= b0, (an, bn)
+        for a0, a1, n in spans:
+            assert a0 % 256 == 0, n
+            assert a1 <= total
+        assert lay.total == total
+
+
+def test_scratch_grows_with_tokens(L):
+    assert moe.moe_scratch_size(cfg(T=64)) < moe.moe_scratch_size(cfg(T=64 * 100))
+    assert moe.moe_scratch_size(cfg(T=0)) > 0

@@ -1,0 +1,104 @@
+"""Whole-layer parity of moe_layer_forward against the float64 oracle.
+
+* small/medium layers and the decode-sized workloads: every output element;
+* the full-size workloads (FastMoE 8192 x 512, Skywork 4096 x 4096, Mixtral
+  16384 x 4096, fine-grained 32768 x 2048): routing, counts, permutation and
+  drop mask over all tokens, outputs on sampled tokens the oracle evaluates one
+  by one (the FastMoE layer is small enough to check in full);
+* edge cases: no tokens, one token, k = E, one expert, determinism."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as mw
+import mixture_experts_layer_logit_b200 as moe
+from oracle import moe_oracle as om
+from tests.gpu_harness import DeviceLayer, check_routing, check_dispatch_exact, check_out, lcfg_of, to_np64
+
+pytestmark = pytest.mark.gpu
+
+W = mw.Workload
+
+
+def run_and_check(L: DeviceLayer, sample: int = 0, seed: int = 0):
+    res = L.forward()
+    x = mw.to_f64(L.inp.x)
+    wg = mw.to_f64(L.inp.wg)
+    w1, w2 = mw.F64Experts(L.inp.w1), mw.F64Experts(L.inp.w2)
+    cfg = lcfg_of(L.w, L.T)
+    r0 = om.route(x, wg, L.inp.bias, cfg)
+    forced, n_tie = check_routing(res["topk_idx"], r0)
+    # near-tie tokens take the device's selection; everything downstream exact
+    r = om.route(x, wg, L.inp.bias, cfg, forced, res["topk_idx"]) if n_tie else r0
+    d = om.dispatch(r.idx, cfg, r.prob_mean)
+    check_dispatch_exact(res, d, r, res["topk_idx"])
+    st = res["stats"]
+    assert st["status"] == 0
+    assert st["drop_count"] == d.drop_count and st["rows_kept"] == int(d.offsets[-1])
+    assert st["capacity"] == (-1 if d.C is None else d.C)
+    if L.T > 0:
+        assert abs(st["aux_loss"] - d.aux) <= 1e-4 * max(1.0, abs(d.aux))
+        assert abs(st["drop_rate"] - d.drop_rate) <= 1e-6
+    out = res["out"]
+    if sample and sample < L.T:
+        toks = np.sort(np.random.default_rng(seed).choice(L.T, size=sample, replace=False))
+        toks = np.unique(np.concatenate([toks, [0, L.T - 1]]))
+        ref = om.forward_tokens(x, w1, w2, cfg, r, d, toks)
+        rel = check_out(to_np64(out[torch.from_numpy(toks).cuda()]), ref, L.w.dtype)
+    else:
+        ref = om.combine(om.expert_segments(x[d.src_tok], d.offsets, w1, w2, cfg)[1], d.row_of, r.w, L.T, L.w.d)
+        rel = check_out(to_np64(out), ref, L.w.dtype)
+    return res, rel, n_tie
+
+
+MEDIUM = [
+    W("m_relu_cap", T=777, d=256, E=12, F=320, k=3, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.1, seed=21),
+    W("m_swiglu_lam", T=1000, d=192, E=8, F=208, k=2, act=mw.SWIGLU, dtype=mw.BF16, capacity_factor=0.9, lam=1.0,
+      zipf_bias=True, seed=22),
+    W("m_fp32", T=300, d=64, E=5, F=96, k=2, act=mw.RELU, dtype=mw.F32, seed=23),
+    W("m_fine", T=700, d=128, E=64, F=176, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True, capacity_factor=1.0,
+      seed=24),
+    W("m_kE", T=150, d=64, E=4, F=64, k=4, act=mw.SWIGLU, dtype=mw.BF16, lam=1.0, seed=25),
+    W("m_one", T=1, d=64, E=8, F=64, k=2, act=mw.RELU, dtype=mw.BF16, seed=26),
+    W("m_E1", T=200, d=64, E=1, F=128, k=1, act=mw.SWIGLU, dtype=mw.BF16, seed=27),
+    W("m_long_k", T=333, d=64, E=40, F=48, k=12, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.2, seed=28),
+    W("m_multi_tile", T=3000, d=512, E=4, F=640, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=29),
+]
+
+
+@pytest.mark.parametrize("w", MEDIUM, ids=[w.name for w in MEDIUM])
+def test_layer_medium(w):
+    run_and_check(DeviceLayer(w))
+
+
+def test_layer_empty_tokens():
+    w = W("empty", T=0, d=64, E=4, F=64, k=2, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.0)
+    L = DeviceLayer(w)
+    res = L.forward()
+    assert res["out"].numel() == 0
+    assert res["stats"]["rows_kept"] == 0 and res["stats"]["drop_count"] == 0
+    assert np.all(res["offsets"] == 0) and np.all(res["counts"] == 0)
+    assert res["stats"]["drop_rate"] == 0.0 and np.isnan(res["stats"]["aux_loss"])
+
+
+def test_layer_deterministic():
+    L = DeviceLayer(MEDIUM[1])
+    a = L.forward()
+    b = L.forward()
+    assert torch.equal(a["out"].view(torch.int16), b["out"].view(torch.int16))
+    assert a["stats"] == b["stats"]
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "fastmoe_txl", "fine_decode_dropless", "fine_decode_cap"])
+def test_layer_named_full(name):
+    _, rel, _ = run_and_check(DeviceLayer(mw.WORKLOADS[name]))
+    assert rel < 1.0
+
+
+@pytest.mark.parametrize("name", ["skywork_lambda1", "mixtral_8x7b", "fine_large_dropless", "fine_large_cap"])
+def test_layer_named_full_size_sampled(name):
+    L = DeviceLayer(mw.WORKLOADS[name])
+    _, rel, n_tie = run_and_check(L, sample=192, seed=1)
+    assert rel < 1.0
+    del L
+    torch.cuda.empty_cache()

@@ -1,0 +1,219 @@
+"""Per-step parity of the CUDA path (through the C ABI) against the float64
+oracle, at sizes the oracle runs in seconds that still span several tiles and
+leave ragged tails (T not a multiple of the 64-token chunk, segments not a
+multiple of the 128-row tile, F not a multiple of the 128/256-column tile)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as mw
+import mixture_experts_layer_logit_b200 as moe
+from oracle import moe_oracle as om
+from tests.gpu_harness import (DeviceLayer, check_routing, check_dispatch_exact, check_out, lcfg_of, to_np64,
+                               NEAR_TIE)
+
+pytestmark = pytest.mark.gpu
+
+W = mw.Workload
+MEDIUM = {
+    "relu_cap_ragged": W("relu_cap_ragged", T=777, d=256, E=12, F=320, k=3, act=mw.RELU, dtype=mw.BF16,
+                         capacity_factor=1.1, seed=11),
+    "swiglu_lambda_bias": W("swiglu_lambda_bias", T=1000, d=192, E=8, F=208, k=2, act=mw.SWIGLU, dtype=mw.BF16,
+                            capacity_factor=0.9, lam=1.0, zipf_bias=True, seed=12),
+    "fp32_relu": W("fp32_relu", T=300, d=64, E=5, F=96, k=2, act=mw.RELU, dtype=mw.F32, seed=13),
+    "fp32_swiglu_cap": W("fp32_swiglu_cap", T=257, d=32, E=6, F=40, k=3, act=mw.SWIGLU, dtype=mw.F32,
+                         capacity_factor=1.0, lam=0.5, seed=14),
+    "fine_top6": W("fine_top6", T=500, d=128, E=64, F=176, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True,
+                   seed=15),
+    "dense_E1": W("dense_E1", T=130, d=64, E=1, F=64, k=1, act=mw.RELU, dtype=mw.BF16, seed=16),
+    "big_k10": W("big_k10", T=200, d=64, E=16, F=64, k=10, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.0,
+                 seed=17),
+    "E256": W("E256", T=300, d=64, E=256, F=32, k=4, act=mw.RELU, dtype=mw.BF16, seed=18),
+}
+
+
+@pytest.fixture(scope="module", params=sorted(MEDIUM))
+def layer(request):
+    w = MEDIUM[request.param]
+    return DeviceLayer(w)
+
+
+def oracle_inputs(L: DeviceLayer):
+    x = mw.to_f64(L.inp.x)
+    return x, mw.to_f64(L.inp.wg), L.inp.bias, mw.F64Experts(L.inp.w1), mw.F64Experts(L.inp.w2)
+
+
+def test_route(layer):
+    L = layer
+    idx, wt, gap, pm = L.route()
+    torch.cuda.synchronize()
+    x, wg, b, _, _ = oracle_inputs(L)
+    r = om.route(x, wg, b, lcfg_of(L.w, L.T))
+    di = idx.cpu().numpy()
+    nt, _ = check_routing(di, r)
+    # weights / gaps / probability means against float64
+    dw = wt.cpu().numpy()
+    ok = ~nt
+    ref_w = np.take_along_axis(r.p, di, axis=1)
+    ref_w = ref_w / ref_w.sum(axis=1, keepdims=True)
+    assert np.max(np.abs(dw[ok] - ref_w[ok])) < 2e-5
+    assert np.allclose(dw.sum(axis=1), 1.0, atol=1e-5)
+    dg = gap.cpu().numpy()
+    fin = np.isfinite(r.gap)
+    assert np.array_equal(np.isfinite(dg), fin)
+    assert np.max(np.abs(dg[fin] - r.gap[fin]), initial=0.0) < 1e-4
+    assert np.allclose(pm.cpu().numpy(), r.prob_mean, rtol=1e-5, atol=1e-7)
+
+
+def test_permute_exact(layer):
+    """Permutation from the oracle's own selection: everything bit-exact."""
+    L = layer
+    x, wg, b, _, _ = oracle_inputs(L)
+    cfg = lcfg_of(L.w, L.T)
+    r = om.route(x, wg, b, cfg)
+    d = om.dispatch(r.idx, cfg, r.prob_mean)
+    idx = torch.from_numpy(r.idx.astype(np.int32)).cuda()
+    gap = torch.from_numpy(r.gap.astype(np.float32)).cuda()
+    pm = torch.from_numpy(r.prob_mean.astype(np.float32)).cuda()
+    res = L.permute(idx, gap, pm)
+    torch.cuda.synchronize()
+    dev = {k: v.cpu().numpy() for k, v in res.items() if k not in ("xp", "stats")}
+    check_dispatch_exact(dev, d, r, r.idx)
+    assert np.array_equal(dev["row_of"], d.row_of)
+    n = int(d.offsets[-1])
+    # the gather is a bit copy of x rows
+    xp = res["xp"][:n].cpu()
+    ref = L.x.cpu()[torch.from_numpy(d.src_tok)]
+    assert torch.equal(xp.view(torch.int16) if xp.dtype == torch.bfloat16 else xp,
+                       ref.view(torch.int16) if ref.dtype == torch.bfloat16 else ref)
+    st = moe.read_stats(res["stats"])
+    assert st["drop_count"] == d.drop_count and st["rows_kept"] == n
+    assert st["capacity"] == (-1 if d.C is None else d.C)
+    assert st["status"] == 0
+    assert abs(st["drop_rate"] - d.drop_rate) <= 1e-7
+    assert abs(st["aux_loss"] - d.aux) <= 1e-5 * max(1.0, abs(d.aux))
+    assert st["near_tie_count"] == int(np.sum(r.gap.astype(np.float32) < np.float32(NEAR_TIE)))
+
+
+def test_expert_ffn(layer):
+    """Grouped GEMMs on the oracle's permuted rows."""
+    L = layer
+    x, wg, b, w1, w2 = oracle_inputs(L)
+    cfg = lcfg_of(L.w, L.T)
+    r = om.route(x, wg, b, cfg)
+    d = om.dispatch(r.idx, cfg, r.prob_mean)
+    n = int(d.offsets[-1])
+    A = max(L.T * L.w.k, 1)
+    xp = torch.zeros((A, L.w.d), dtype=L.tdt, device="cuda")
+    xp[:n] = L.x[torch.from_numpy(d.src_tok).cuda()]
+    # poison the unused rows: results must not depend on them
+    if n < A:
+        xp[n:] = float("nan")
+    off = torch.from_numpy(d.offsets.astype(np.int32)).cuda()
+    h, yp, stats = L.expert_ffn(xp, off)
+    torch.cuda.synchronize()
+    assert moe.read_stats(stats)["status"] == 0
+    h_ref, yp_ref = om.expert_segments(x[d.src_tok], d.offsets, w1, w2, cfg, want_hidden=True)
+    check_out(to_np64(h[:n]), h_ref, L.w.dtype)
+    check_out(to_np64(yp[:n]), yp_ref, L.w.dtype)
+
+
+def test_combine(layer):
+    L = layer
+    x, wg, b, w1, w2 = oracle_inputs(L)
+    cfg = lcfg_of(L.w, L.T)
+    r = om.route(x, wg, b, cfg)
+    d = om.dispatch(r.idx, cfg, r.prob_mean)
+    n = int(d.offsets[-1])
+    A = max(L.T * L.w.k, 1)
+    g = torch.Generator().manual_seed(5)
+    yp = torch.randn((A, L.w.d), generator=g).to(L.tdt).cuda()
+    row_of = torch.from_numpy(d.row_of.astype(np.int32)).cuda()
+    tw = torch.from_numpy(r.w.astype(np.float32)).cuda()
+    out = L.combine(yp, row_of, tw)
+    torch.cuda.synchronize()
+    ref = om.combine(to_np64(yp[:max(n, 1)]), d.row_of, r.w.astype(np.float32).astype(np.float64), L.T, L.w.d)
+    o = to_np64(out)
+    # fp32 accumulation, one rounding to the output type
+    tol = (2.0 ** -8 if L.w.dtype == mw.BF16 else 1e-6) * np.abs(ref) + 1e-6
+    assert np.all(np.abs(o - ref) <= tol)
+
+
+# ------------------------------------------------------ adversarial permutes
+def _small(T, E, k, cf, dtype=mw.BF16, d=32):
+    return DeviceLayer(W("adv", T=T, d=d, E=E, F=32, k=k, act=mw.RELU, dtype=dtype, capacity_factor=cf, seed=3))
+
+
+def _run_permute(L, idx_np, cf_cfg):
+    idx = torch.from_numpy(idx_np.astype(np.int32)).cuda()
+    res = L.permute(idx)
+    torch.cuda.synchronize()
+    return {k: (v.cpu().numpy() if k != "stats" else moe.read_stats(v)) for k, v in res.items() if k != "xp"}
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(300, 4, 2, 0.5), (129, 8, 1, 0.1), (1000, 16, 8, 1.0), (64, 3, 3, 0.0),
+                                       (333, 20, 10, 0.7)])
+def test_permute_all_to_few_experts(T, E, k, cf):
+    """Every token picks experts 0..k-1 (maximal imbalance, heavy dropping)."""
+    L = _small(T, E, k, cf)
+    idx = np.tile(np.arange(k), (T, 1))
+    idx[1::2] = idx[1::2, ::-1]    # vary slot order
+    got = _run_permute(L, idx, cf)
+    cfg = lcfg_of(L.w, T)
+    d = om.dispatch(idx, cfg, None)
+    assert np.array_equal(got["counts"], d.counts) and np.array_equal(got["kept"], d.kept)
+    assert np.array_equal(got["offsets"], d.offsets) and np.array_equal(got["row_of"], d.row_of)
+    assert np.array_equal(got["src_tok"][:int(d.offsets[-1])], d.src_tok)
+    assert got["stats"]["drop_count"] == d.drop_count
+
+
+def test_permute_random_indices_exact():
+    """Uniformly random (distinct per token) selections over many chunks."""
+    rng = np.random.default_rng(9)
+    T, E, k = 4097, 37, 5
+    L = _small(T, E, k, 1.3)
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    got = _run_permute(L, idx, 1.3)
+    d = om.dispatch(idx, lcfg_of(L.w, T), None)
+    assert np.array_equal(got["row_of"], d.row_of) and np.array_equal(got["offsets"], d.offsets)
+    assert np.array_equal(got["src_tok"][:int(d.offsets[-1])], d.src_tok)
+
+
+def test_permute_repeated_expert_in_token():
+    """A caller-made selection naming one expert twice is ordered by slot."""
+    T, E, k = 70, 4, 2
+    L = _small(T, E, k, 0.0)
+    idx = np.array([[t % E, t % E] if t % 3 == 0 else [t % E, (t + 1) % E] for t in range(T)])
+    got = _run_permute(L, idx, 0.0)
+    d = om.dispatch(idx, lcfg_of(L.w, T), None)
+    assert np.array_equal(got["row_of"], d.row_of)
+    assert np.array_equal(got["src_tok"][:int(d.offsets[-1])], d.src_tok)
+
+
+def test_permute_out_of_range_index_flags_and_drops():
+    T, E, k = 40, 4, 2
+    L = _small(T, E, k, 0.0)
+    idx = np.array([[t % E, (t + 1) % E] for t in range(T)])
+    idx[5, 1] = 9
+    idx[17, 0] = -1
+    got = _run_permute(L, idx, 0.0)
+    assert got["stats"]["status"] & moe.MOE_DEV_BOUNDS
+    assert got["row_of"][5, 1] == -1 and got["row_of"][17, 0] == -1
+    # the valid slots are grouped exactly as if the bad slots did not exist
+    valid = (idx >= 0) & (idx < E)
+    assert int(got["offsets"][-1]) == int(valid.sum())
+    for e in range(E):
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        seg = got["src_tok"][got["offsets"][e]:got["offsets"][e + 1]]
+        assert np.array_equal(seg, toks)
+
+
+def test_bad_arguments_rejected_on_gpu():
+    L = _small(64, 4, 2, 0.0)
+    idx, wt, gap, pm = L.route()
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_route(L.cfg, L.x, L.wg, None, idx, wt, gap, pm, torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert ei.value.code == 3
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_combine(L.cfg, None, idx, wt, torch.empty_like(L.x))
+    assert ei.value.code == 1
