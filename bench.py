@@ -76,6 +76,7 @@ def workload_config(w: mw.Workload, n_gpus: int, graph: bool):
             "experts": w.E, "ffn_hidden": w.F, "top_k": w.k, "activation": w.act,
             "capacity_factor": w.capacity_factor if w.capacity_factor > 0 else "dropless",
             "lambda": w.lam, "gate_bias": "zipf1.2" if w.zipf_bias else None,
+            "hidden_dtype": "f16" if w.dtype == mw.BF16 else "f32", "out_dtype": "f32",
             "parallelism": "replicas" if n_gpus == 1 else f"dp{n_gpus} replicas",
             "l2": "flushed between steps (512 MiB memset outside the timed events)",
             "cuda_graph": graph}
@@ -210,11 +211,14 @@ def step_bytes(w: mw.Workload, offsets: np.ndarray):
     kept = int(offsets[-1])
     F1 = F if w.act == mw.RELU else 2 * F
     touched = int(np.sum(np.diff(offsets) > 0))
+    # h is 2-byte (bf16/fp16) on the bf16 path; yp and out are fp32 on both paths
+    hb = 2 if w.dtype == mw.BF16 else 4
     return {
         "route": T * d * b + E * d * b + A * 8 + T * 4,
         "permute": (T * d + kept * d) * b + 4 * (2 * A + kept),
-        "expert_ffn": touched * (F1 + F) * d * b + kept * (2 * d + 2 * F) * b,
-        "combine": (kept * d + T * d) * b + 8 * A,
+        # weights of the experts that received rows, xp read, h written and read, yp written
+        "expert_ffn": touched * (F1 + F) * d * b + kept * (d * b + 2 * F * hb + d * 4),
+        "combine": (kept * d + T * d) * 4 + 8 * A,
         "expert_flops": 2 * kept * d * (F1 + F),
         "weight_bytes": touched * (F1 + F) * d * b,
     }
@@ -268,10 +272,12 @@ def main():
     tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
     x = mw.to_device(inp.x, dev)
     wg, bias = mw.to_device(inp.wg, dev), mw.to_device(inp.bias, dev)
-    w1, w2 = mw.to_device(inp.w1, dev), mw.to_device(inp.w2, dev)
+    w1 = mw.to_device(inp.w1, dev)
+    # weight preparation at load time (not part of a step): W2 in the hidden type
+    w2 = moe.prepare_w2(cfg, mw.to_device(inp.w2, dev))
     nbytes, lay = moe.moe_workspace_size(cfg)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    out = torch.empty((w.T, w.d), dtype=tdt, device=dev)
+    out = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
     stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -345,7 +351,7 @@ def main():
         idx, tw, gap = sv(L.topk_idx, A, torch.int32), sv(L.topk_w, A, torch.float32), sv(L.gap, w.T, torch.float32)
         counts, kept, offs = sv(L.counts, w.E, torch.int32), sv(L.kept, w.E, torch.int32), sv(L.offsets, w.E + 1, torch.int32)
         row_of, src_tok = sv(L.row_of, A, torch.int32), sv(L.src_tok, A, torch.int32)
-        xp, h, yp = sv(L.xp, A * w.d, tdt), sv(L.h, A * w.F, tdt), sv(L.yp, A * w.d, tdt)
+        xp, h, yp = sv(L.xp, A * w.d, tdt), sv(L.h, A * w.F, tdt), sv(L.yp, A * w.d, torch.float32)
         scr = ws[L.scratch:]
         pm = torch.empty(w.E, dtype=torch.float32, device=dev)
         names = ["route", "permute", "expert_ffn", "combine"]

@@ -28,10 +28,15 @@
  *     are the gate projection, rows [F, 2F) the up projection -- the order of
  *     the merged pair matters, Megatron-Core best-practice page, section
  *     "从HuggingFace到Megatron的权重转换要点"); W2[E, d, F].
- *   - Element type of x, weights, xp, h, yp and out: bf16 (MOE_DTYPE_BF16,
- *     fp32 accumulation, tcgen05 tensor cores) or fp32 (MOE_DTYPE_F32, CUDA-core
- *     FFMA throughout).  Gate bias, gate weights (topk_w), gap and prob_mean are
- *     fp32; indices are int32.
+ *   - Element type of x, W_gate, W1 and xp: bf16 (MOE_DTYPE_BF16, fp32
+ *     accumulation, tcgen05 tensor cores) or fp32 (MOE_DTYPE_F32, CUDA-core
+ *     FFMA throughout).  On the bf16 path the expert hidden activation h and
+ *     W2 share moe_config.hidden_dtype: bf16, or fp16 (10-bit mantissa, 8x
+ *     finer rounding of h; W2 then has to be given in fp16, see
+ *     moe_convert_bf16_to_f16).  The expert outputs yp and the layer output out
+ *     are fp32 for both paths (rounding them to bf16 would by itself use up
+ *     most of the output tolerance on the largest elements).  Gate bias, gate
+ *     weights (topk_w), gap and prob_mean are fp32; indices are int32.
  *   - Errors a host can see (bad arguments, unsupported shapes, too small a
  *     workspace, a failed launch) are returned synchronously and nothing is
  *     enqueued.  Errors only the device can see (an index out of range, a
@@ -63,11 +68,12 @@ typedef enum moe_status {
 } moe_status;
 
 enum { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 };
-enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1, MOE_DTYPE_F16 = 2 };
 
 /* Device-detected error bits in moe_stats.status. */
 #define MOE_DEV_TIMEOUT 1u   /* a bounded wait inside a kernel gave up (~2 s); the kernel returned early */
-#define MOE_DEV_BOUNDS  2u   /* an expert index outside [0, E) was seen and skipped */
+#define MOE_DEV_BOUNDS  2u   /* an expert index or a row outside its buffer was seen and skipped */
+#define MOE_DEV_RANGE   4u   /* an fp16 hidden activation exceeded +-65504 and was saturated */
 
 /* Near-tie threshold: tokens whose k-th and (k+1)-th scores differ by less
  * than this are counted in moe_stats.near_tie_count. */
@@ -95,6 +101,8 @@ typedef struct moe_config {
   int32_t dtype;             /* MOE_DTYPE_BF16 | MOE_DTYPE_F32 */
   float capacity_factor;     /* <= 0: dropless */
   float lambda;              /* <= 0: plain softmax */
+  int32_t hidden_dtype;      /* element type of h and W2: MOE_DTYPE_BF16 | MOE_DTYPE_F16 on the
+                                bf16 path, MOE_DTYPE_F32 on the fp32 path */
 } moe_config;
 
 /* Per-forward statistics, in DEVICE memory, written by moe_permute (and by
@@ -179,8 +187,11 @@ moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk
  *   ReLU:   h = relu(xp W1[e]^T);  SwiGLU: h = silu(xp Wg_e^T) * (xp Wu_e^T),
  *           silu(u) = u / (1 + exp(-u));   then yp = h W2[e]^T.
  *   xp[A, d], offsets[E+1] (device, from moe_permute), W1[E, F1, d],
- *   W2[E, d, F]; h[A, F] and yp[A, d] are written for rows [0, offsets[E]).
- *   bf16: h is rounded to bf16 after the fp32 activation; yp is bf16.
+ *   W2[E, d, F] (hidden_dtype); h[A, F] (hidden_dtype) and yp[A, d] fp32 are
+ *   written for rows [0, offsets[E]).
+ *   bf16 path: the activation is computed in fp32 from the fp32 accumulator and
+ *   h is rounded once to hidden_dtype (it is the tensor-core operand of the
+ *   second layer); fp16 h saturates at +-65504 and sets MOE_DEV_RANGE.
  *   stats: device moe_stats; a kernel timeout ORs MOE_DEV_TIMEOUT into status.
  *   ws: at least moe_scratch_size(cfg) bytes.
  */
@@ -194,7 +205,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* 
  * slot order; 0 for a token whose slots were all dropped (the residual path
  * outside the layer carries it: Megatron-Core best-practice page, section
  * "MoE负载均衡的挑战与应对").
- *   yp[A, d], row_of[T, k], topk_w[T, k] -> out[T, d].
+ *   yp[A, d] fp32, row_of[T, k], topk_w[T, k] -> out[T, d] fp32.
  */
 moe_status moe_combine(const moe_config* cfg, const void* yp, const int32_t* row_of,
                        const float* topk_w, void* out, moe_stream_t stream);
@@ -203,12 +214,23 @@ moe_status moe_combine(const moe_config* cfg, const void* yp, const int32_t* row
  * The whole layer: steps 1-5 back to back on `stream`, intermediates inside
  * `ws` (layout from moe_workspace_size).  No host synchronisation and no
  * device-to-host copy, so it may be captured in a CUDA graph.
- *   x[T, d], Wg[E, d], bg[E] or NULL, W1[E, F1, d], W2[E, d, F] -> out[T, d];
+ *   x[T, d], Wg[E, d], bg[E] or NULL, W1[E, F1, d], W2[E, d, F] -> out[T, d] fp32;
  *   stats: device moe_stats (required).
  */
 moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
                              const void* W1, const void* W2, void* out, moe_stats* stats,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Weight preparation (run once when the weights are loaded, not per forward):
+ * dst[i] = fp16(src[i]) for n bf16 values, round to nearest even; values
+ * beyond the fp16 range saturate to +-65504.  Every bf16 value of magnitude in
+ * [2^-17, 65504] converts exactly; smaller ones round to fp16 subnormals.
+ * Used to give W2 to the layer when hidden_dtype is MOE_DTYPE_F16.
+ * src and dst: device, 16-byte aligned, not overlapping.  No counterpart on
+ * the pages: it prepares the storage format of the second expert layer.
+ */
+moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,25 +19,28 @@ from typing import Optional
 __all__ = [
     "LIB_PATH", "MoeError", "moe_config", "moe_stats", "moe_ws_layout", "lib", "make_config",
     "moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route", "moe_permute",
-    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "MOE_ACT_RELU", "MOE_ACT_SWIGLU",
-    "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "EXPORTED_SYMBOLS",
+    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "prepare_w2",
+    "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
+    "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
-MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
-MOE_DEV_TIMEOUT, MOE_DEV_BOUNDS = 1, 2
+MOE_DTYPE_F32, MOE_DTYPE_BF16, MOE_DTYPE_F16 = 0, 1, 2
+MOE_DEV_TIMEOUT, MOE_DEV_BOUNDS, MOE_DEV_RANGE = 1, 2, 4
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA"}
 
 EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route",
-                    "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"]
+                    "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+                    "moe_convert_bf16_to_f16"]
 
 
 class moe_config(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("capacity_factor", ctypes.c_float), ("lambda_", ctypes.c_float)]
+                ("capacity_factor", ctypes.c_float), ("lambda_", ctypes.c_float),
+                ("hidden_dtype", ctypes.c_int32)]
 
 
 class moe_stats(ctypes.Structure):
@@ -83,16 +86,25 @@ def lib() -> ctypes.CDLL:
     L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_combine.argtypes = [cfgp, P, P, P, P, P]
     L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
-    for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"]:
+    L.moe_convert_bf16_to_f16.argtypes = [P, P, ctypes.c_size_t, P]
+    for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+              "moe_convert_bf16_to_f16"]:
         getattr(L, n).restype = st
     _lib = L
     return L
 
 
+_DTYPES = {"f32": MOE_DTYPE_F32, "bf16": MOE_DTYPE_BF16, "f16": MOE_DTYPE_F16}
+
+
 def make_config(T: int, d: int, E: int, F: int, k: int, act: str = "relu", dtype: str = "bf16",
-                capacity_factor: float = 0.0, lam: float = 0.0) -> moe_config:
-    return moe_config(T, d, E, F, k, MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_RELU,
-                      MOE_DTYPE_BF16 if dtype == "bf16" else MOE_DTYPE_F32, capacity_factor, lam)
+                capacity_factor: float = 0.0, lam: float = 0.0, hidden: Optional[str] = None) -> moe_config:
+    """hidden: element type of the expert hidden activation and of W2 on the bf16
+    path ("f16", the default, or "bf16"); always "f32" on the fp32 path."""
+    if hidden is None:
+        hidden = "f16" if dtype == "bf16" else "f32"
+    return moe_config(T, d, E, F, k, MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_RELU, _DTYPES[dtype],
+                      capacity_factor, lam, _DTYPES[hidden])
 
 
 def _ptr(t) -> Optional[int]:
@@ -166,6 +178,23 @@ def moe_layer_forward(cfg, x, Wg, bg, W1, W2, out, stats, ws, stream=None):
     _check("moe_layer_forward", lib().moe_layer_forward(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg),
                                                         _ptr(W1), _ptr(W2), _ptr(out), _ptr(stats), _ptr(ws),
                                                         _nbytes(ws), _stream(stream)))
+
+
+def moe_convert_bf16_to_f16(src, dst, n: Optional[int] = None, stream=None):
+    """Weight preparation: dst = fp16(src) for bf16 src (device tensors)."""
+    n = src.numel() if n is None else n
+    _check("moe_convert_bf16_to_f16", lib().moe_convert_bf16_to_f16(_ptr(src), _ptr(dst), n, _stream(stream)))
+
+
+def prepare_w2(cfg: moe_config, w2):
+    """W2 in the storage type the layer expects (a new fp16 tensor when the
+    hidden activation is fp16, else w2 itself).  Run once at load time."""
+    if cfg.hidden_dtype != MOE_DTYPE_F16:
+        return w2
+    import torch
+    out = torch.empty(w2.shape, dtype=torch.float16, device=w2.device)
+    moe_convert_bf16_to_f16(w2, out)
+    return out
 
 
 def read_stats(stats_tensor) -> dict:

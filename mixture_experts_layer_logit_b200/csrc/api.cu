@@ -62,6 +62,9 @@ moe_status check_config(const moe_config* c) {
   if (c->k > c->E) return MOE_ERR_ARG;
   if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
   if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32) return MOE_ERR_ARG;
+  if (c->dtype == MOE_DTYPE_BF16 && c->hidden_dtype != MOE_DTYPE_BF16 && c->hidden_dtype != MOE_DTYPE_F16)
+    return MOE_ERR_ARG;
+  if (c->dtype == MOE_DTYPE_F32 && c->hidden_dtype != MOE_DTYPE_F32) return MOE_ERR_ARG;
   if (!isfinite(c->capacity_factor) || !isfinite(c->lambda)) return MOE_ERR_ARG;
   if (c->E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
   const int mult = (c->dtype == MOE_DTYPE_BF16) ? 16 : 4;
@@ -111,7 +114,7 @@ moe_ws_layout layout_of(const moe_config& c) {
   L.src_tok = off;   off = align256(off + 4 * A);
   L.xp = off;        off = align256(off + es * A * (size_t)c.d);
   L.h = off;         off = align256(off + es * A * (size_t)c.F);
-  L.yp = off;        off = align256(off + es * A * (size_t)c.d);
+  L.yp = off;        off = align256(off + 4 * A * (size_t)c.d);   // fp32 for both element types
   L.scratch = off;   off = align256(off + scratch_layout(c).total);
   L.total = off;
   return L;

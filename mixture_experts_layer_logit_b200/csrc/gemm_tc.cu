@@ -45,10 +45,12 @@ constexpr unsigned long long kWaitNs = 2000000000ull;    // bounded waits: 2 s
 constexpr unsigned long long kDrainNs = 200000000ull;    // teardown waits: 0.2 s
 enum { kPlain = 0, kRelu = 1, kSwiglu = 2 };
 
-// instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B bf16,
-// both K-major, M = 128, N = 256
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B of one
+// type (format 1 = bf16, 0 = fp16), both K-major, M = 128, N = 256
+constexpr uint32_t idesc_for(bool f16_operands) {
+  return (1u << 4) | ((f16_operands ? 0u : 1u) << 7) | ((f16_operands ? 0u : 1u) << 10) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 
 struct Tail {
   unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -60,7 +62,7 @@ constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Tail)
 
 struct Params {
   const int32_t* offsets;
-  __nv_bfloat16* out;   // [rows][Nout]
+  void* out;            // [rows][Nout]: bf16 h (layer 1) or fp32 yp (layer 2)
   int E, K, Nout;
   int b_rows;           // B rows per expert
   int up_off;           // SwiGLU: first up row inside an expert's B block
@@ -158,9 +160,21 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
+// Two fp32 values -> one 32-bit pair of the hidden type (round to nearest
+// even).  fp16 saturates at +-65504 (NaN passes through) and notes it in `over`.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_hidden(float a, float b, bool& over) {
+  if constexpr (F16) {
+    const bool oa = fabsf(a) > 65504.f, ob = fabsf(b) > 65504.f;
+    over |= oa | ob;
+    a = oa ? copysignf(65504.f, a) : a;
+    b = ob ? copysignf(65504.f, b) : b;
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
 }
 
 struct TileCoord {
@@ -182,10 +196,13 @@ __device__ __forceinline__ TileCoord decode_tile(const int* tstart, const int32_
   return c;
 }
 
-template <int MODE>
+// F16: the hidden activation (layer-1 output, layer-2 A operand) and W2 are
+// fp16 instead of bf16.
+template <int MODE, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
+  constexpr uint32_t kIdesc = idesc_for(MODE == kPlain && F16);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -309,7 +326,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         atomicOr(p.status, MOE_DEV_BOUNDS);
         rv = false;
       }
-      __nv_bfloat16* orow = p.out + (size_t)(c.row0 + (rv ? r : 0)) * p.Nout;
+      const size_t orow_off = (size_t)(c.row0 + (rv ? r : 0)) * p.Nout;
+      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off;   // layer 1: h (bf16 or fp16)
+      float* orow32 = static_cast<float*>(p.out) + orow_off;       // layer 2: fp32 yp
+      bool over = false;
       if (MODE == kSwiglu) {
 #pragma unroll 1
         for (int ch = 0; ch < BN / 64; ++ch) {
@@ -327,7 +347,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
               for (int i = 0; i < 4; ++i) {
                 const float g0 = __uint_as_float(g[8 * v + 2 * i]), g1 = __uint_as_float(g[8 * v + 2 * i + 1]);
                 const float u0 = __uint_as_float(u[8 * v + 2 * i]), u1 = __uint_as_float(u[8 * v + 2 * i + 1]);
-                pk[i] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+                pk[i] = pack_hidden<F16>(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1, over);
               }
               *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
@@ -340,7 +360,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           tmem_ld32(tb + ch * 32, a);
           tmem_wait_ld();
           const int col = c.n0 + ch * 32;
-          if (rv) {
+          if (rv && MODE == kPlain) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (col + 4 * v >= p.Nout) break;
+              *reinterpret_cast<uint4*>(orow32 + col + 4 * v) =
+                  make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
+            }
+          } else if (rv) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               if (col + 8 * v >= p.Nout) break;
@@ -349,13 +376,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
               for (int i = 0; i < 4; ++i) {
                 float a0 = __uint_as_float(a[8 * v + 2 * i]), a1 = __uint_as_float(a[8 * v + 2 * i + 1]);
                 if (MODE == kRelu) { a0 = fmaxf(a0, 0.f); a1 = fmaxf(a1, 0.f); }
-                pk[i] = pack_bf16x2(a0, a1);
+                pk[i] = pack_hidden<F16>(a0, a1, over);
               }
               *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
         }
       }
+      if (F16 && over) atomicOr(p.status, MOE_DEV_RANGE);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);   // accumulator free again
@@ -388,26 +416,59 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix; box = 64 columns
-// (128 bytes) x 128 rows, 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+// 2-D tensor map over a row-major [rows, cols] matrix of 16-bit elements
+// (bf16 or fp16); box = 64 columns (128 bytes) x 128 rows, 128-byte swizzle,
+// zero fill outside.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, bool f16) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {BK, BM};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool F16>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_grouped_gemm<MODE>>(kSmemBytes);
+  cudaError_t err = set_smem_once<tc_grouped_gemm<MODE, F16>>(kSmemBytes);
   if (err != cudaSuccess) return err;
-  tc_grouped_gemm<MODE><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, p);
+  tc_grouped_gemm<MODE, F16><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, p);
   return cudaGetLastError();
+}
+
+template <bool F16>
+cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
+                          const void* w2, void* h, void* yp, uint32_t* status, int sms, cudaStream_t s) {
+  const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
+  const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
+  const long long mt_max = (long long)(rows / BM) + c.E;
+  CUtensorMap ma, mb;
+  cudaError_t err;
+
+  // layer 1: h = act(xp W1[e]^T)
+  if (!make_map(&ma, xp, rows, (uint64_t)c.d, false) || !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false))
+    return cudaErrorInvalidValue;
+  Params p1{offsets, h, c.E, c.d, c.F, F1, c.F, (int)rows, status};
+  if (c.act == MOE_ACT_SWIGLU) {
+    const long long nt = (c.F + BN / 2 - 1) / (BN / 2);
+    err = launch_one<kSwiglu, F16>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, sms), s);
+  } else {
+    const long long nt = (c.F + BN - 1) / BN;
+    err = launch_one<kRelu, F16>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, sms), s);
+  }
+  if (err != cudaSuccess) return err;
+
+  // layer 2: yp = h W2[e]^T, kept in fp32 so that the combine adds unrounded
+  // expert outputs
+  if (!make_map(&ma, h, rows, (uint64_t)c.F, F16) || !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F, F16))
+    return cudaErrorInvalidValue;
+  Params p2{offsets, yp, c.E, c.F, c.d, c.d, 0, (int)rows, status};
+  const long long nt2 = (c.d + BN - 1) / BN;
+  return launch_one<kPlain, F16>(ma, mb, p2, (int)std::min<long long>(mt_max * nt2, sms), s);
 }
 
 }  // namespace
@@ -419,30 +480,9 @@ cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int3
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
-  const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
-  const long long mt_max = (long long)(rows / BM) + c.E;
-  CUtensorMap ma, mb;
-
-  // layer 1: h = act(xp W1[e]^T)
-  if (!make_map(&ma, xp, rows, (uint64_t)c.d) || !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d))
-    return cudaErrorInvalidValue;
-  Params p1{offsets, static_cast<__nv_bfloat16*>(h), c.E, c.d, c.F, F1, c.F, (int)rows, status};
-  if (c.act == MOE_ACT_SWIGLU) {
-    const long long nt = (c.F + BN / 2 - 1) / (BN / 2);
-    err = launch_one<kSwiglu>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, di.sms), s);
-  } else {
-    const long long nt = (c.F + BN - 1) / BN;
-    err = launch_one<kRelu>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, di.sms), s);
-  }
-  if (err != cudaSuccess) return err;
-
-  // layer 2: yp = h W2[e]^T
-  if (!make_map(&ma, h, rows, (uint64_t)c.F) || !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F))
-    return cudaErrorInvalidValue;
-  Params p2{offsets, static_cast<__nv_bfloat16*>(yp), c.E, c.F, c.d, c.d, 0, (int)rows, status};
-  const long long nt2 = (c.d + BN - 1) / BN;
-  return launch_one<kPlain>(ma, mb, p2, (int)std::min<long long>(mt_max * nt2, di.sms), s);
+  if (c.hidden_dtype == MOE_DTYPE_F16)
+    return launch_layers<true>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s);
+  return launch_layers<false>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s);
 }
 
 }  // namespace moe

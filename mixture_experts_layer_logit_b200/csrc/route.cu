@@ -260,13 +260,17 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
   if (tid == 0) ntie_out[chunk] = misc[0];
 }
 
+// One warp per expert: lanes stride over the chunks, then a fixed-order
+// butterfly sum (deterministic).
 __global__ void prob_mean_kernel(const float* __restrict__ psum, int nch, int E, int T,
                                  float* __restrict__ prob_mean) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float s = 0.f;
-    for (int c = 0; c < nch; ++c) s += psum[(size_t)c * E + e];
-    prob_mean[e] = s / (float)T;
-  }
+  const int e = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (e >= E) return;
+  float s = 0.f;
+  for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
+  s = warp_sum(s);
+  if (lane == 0) prob_mean[e] = s / (float)T;
 }
 
 template <int NJ, typename TX>
@@ -306,7 +310,7 @@ cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, con
 }
 
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s) {
-  prob_mean_kernel<<<1, 256, 0, s>>>(psum, num_chunks(c.T), c.E, c.T, prob_mean);
+  prob_mean_kernel<<<(c.E + 7) / 8, 256, 0, s>>>(psum, num_chunks(c.T), c.E, c.T, prob_mean);
   return cudaGetLastError();
 }
 

@@ -25,8 +25,9 @@ BF16_TOL = 2e-2     # x RMS(out)
 F32_TOL = 1e-4      # relative to max |out|
 
 
-def cfg_of(w: mw.Workload, T=None):
-    return moe.make_config(w.T if T is None else T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam)
+def cfg_of(w: mw.Workload, T=None, hidden=None):
+    return moe.make_config(w.T if T is None else T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam,
+                           hidden)
 
 
 def lcfg_of(w: mw.Workload, T=None):
@@ -45,24 +46,26 @@ def view(ws, off, n, dtype):
 class DeviceLayer:
     """One workload's inputs on the device plus the outputs of a forward."""
 
-    def __init__(self, w: mw.Workload, inp: mw.Inputs = None):
+    def __init__(self, w: mw.Workload, inp: mw.Inputs = None, hidden=None):
         self.w = w
         self.inp = inp if inp is not None else mw.generate(w)
-        self.cfg = cfg_of(w, self.inp.x.shape[0])
+        self.cfg = cfg_of(w, self.inp.x.shape[0], hidden)
+        self.hidden = {moe.MOE_DTYPE_F16: "f16", moe.MOE_DTYPE_BF16: "bf16"}.get(self.cfg.hidden_dtype, "f32")
         self.T = self.inp.x.shape[0]
         self.x = mw.to_device(self.inp.x)
         self.wg = mw.to_device(self.inp.wg)
         self.bias = mw.to_device(self.inp.bias)
         self.w1 = mw.to_device(self.inp.w1)
-        self.w2 = mw.to_device(self.inp.w2)
+        self.w2 = moe.prepare_w2(self.cfg, mw.to_device(self.inp.w2))   # weight preparation, once
         self.tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
+        self.hdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[self.hidden]
 
     # ---------------------------------------------------------- whole layer
     def forward(self):
         n, L = moe.moe_workspace_size(self.cfg)
         assert n > 0
         ws = dev_bytes(n)
-        out = torch.empty((self.T, self.w.d), dtype=self.tdt, device="cuda")
+        out = torch.empty((self.T, self.w.d), dtype=torch.float32, device="cuda")
         stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
         moe.moe_layer_forward(self.cfg, self.x, self.wg, self.bias, self.w1, self.w2, out, stats, ws)
         torch.cuda.synchronize()
@@ -108,14 +111,14 @@ class DeviceLayer:
 
     def expert_ffn(self, xp, offsets):
         A = max(self.T * self.w.k, 1)
-        h = torch.empty((A, self.w.F), dtype=self.tdt, device="cuda")
-        yp = torch.empty((A, self.w.d), dtype=self.tdt, device="cuda")
+        h = torch.empty((A, self.w.F), dtype=self.hdt, device="cuda")
+        yp = torch.empty((A, self.w.d), dtype=torch.float32, device="cuda")
         stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
         moe.moe_expert_ffn(self.cfg, xp, offsets, self.w1, self.w2, h, yp, stats, self.scratch())
         return h, yp, stats
 
     def combine(self, yp, row_of, topk_w):
-        out = torch.empty((self.T, self.w.d), dtype=self.tdt, device="cuda")
+        out = torch.empty((self.T, self.w.d), dtype=torch.float32, device="cuda")
         moe.moe_combine(self.cfg, yp, row_of, topk_w, out)
         return out
 

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_struct_sizes_match_header(L):
-    assert ctypes.sizeof(moe.moe_config) == 9 * 4
+    assert ctypes.sizeof(moe.moe_config) == 10 * 4
     assert ctypes.sizeof(moe.moe_stats) == 8 * 4
     assert ctypes.sizeof(moe.moe_ws_layout) == 13 * 8
 
@@ -82,6 +82,12 @@ def test_bad_enum_is_arg_error(L):
     c = cfg()
     c.act = 7
     assert L.moe_combine(ctypes.byref(c), None, None, None, None, None) == 1
+    for dtype, hidden in [("bf16", "f32"), ("f32", "bf16"), ("f32", "f16")]:
+        c = cfg(dtype=dtype, hidden=hidden)
+        assert moe.moe_scratch_size(c) == 0
+        assert L.moe_combine(ctypes.byref(c), None, None, None, None, None) == 1
+    for hidden in ["bf16", "f16"]:
+        assert moe.moe_scratch_size(cfg(hidden=hidden)) > 0
     c = cfg()
     c.dtype = 5
     assert L.moe_layer_forward(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None) == 1
@@ -98,6 +104,14 @@ def test_null_and_misaligned_pointers(L):
     # misaligned activations (TMA and 16-byte vectors need 16-byte alignment)
     assert L.moe_route(ctypes.byref(c), P + 8, P, None, P, P, P, None, P, 1 << 20, None) == 1
     assert L.moe_combine(ctypes.byref(c), P + 4, P, P, P, None) == 1
+
+
+def test_convert_rejects_bad_pointers(L):
+    P = 1 << 20
+    assert L.moe_convert_bf16_to_f16(None, P, 8, None) == 1
+    assert L.moe_convert_bf16_to_f16(P + 2, P + 4096, 8, None) == 1   # misaligned
+    assert L.moe_convert_bf16_to_f16(P, P + 8, 64, None) == 1         # overlapping
+    assert L.moe_convert_bf16_to_f16(None, None, 0, None) == 0        # nothing to do
 
 
 def test_workspace_checks(L):
@@ -121,7 +135,7 @@ def test_workspace_layout_is_disjoint_and_aligned(L):
         A = T * k
         regions = [("topk_idx", 4 * A), ("topk_w", 4 * A), ("gap", 4 * T), ("counts", 4 * E), ("kept", 4 * E),
                    ("offsets", 4 * (E + 1)), ("row_of", 4 * A), ("src_tok", 4 * A), ("xp", es * A * d),
-                   ("h", es * A * F), ("yp", es * A * d), ("scratch", moe.moe_scratch_size(c))]
+                   ("h", es * A * F), ("yp", 4 * A * d), ("scratch", moe.moe_scratch_size(c))]
         spans = sorted((getattr(lay, n), getattr(lay, n) + sz, n) for n, sz in regions)
         for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
             assert a1 <= b0, (an, bn)

@@ -81,11 +81,23 @@ def test_layer_empty_tokens():
     assert res["stats"]["drop_rate"] == 0.0 and np.isnan(res["stats"]["aux_loss"])
 
 
+@pytest.mark.parametrize("name", ["fastmoe_txl", "m_relu_cap", "m_multi_tile"])
+def test_layer_bf16_hidden(name):
+    """The bf16 hidden activation (h and W2 in bf16) also meets the output
+    tolerance on these layers; on the capacity-mode fine-grained layers its
+    single rounding of h reaches ~0.026 RMS, above 2e-2, which is why fp16 is
+    the default hidden type."""
+    w = mw.WORKLOADS.get(name) or next(m for m in MEDIUM if m.name == name)
+    L = DeviceLayer(w, hidden="bf16")
+    assert L.hidden == "bf16"
+    run_and_check(L)
+
+
 def test_layer_deterministic():
     L = DeviceLayer(MEDIUM[1])
     a = L.forward()
     b = L.forward()
-    assert torch.equal(a["out"].view(torch.int16), b["out"].view(torch.int16))
+    assert torch.equal(a["out"], b["out"])
     assert a["stats"] == b["stats"]
 
 
