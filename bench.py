@@ -239,6 +239,30 @@ def committed_traffic():
     return None
 
 
+# ------------------------------------------------------- data-parallel plumbing
+def replica_inputs(w: mw.Workload, rank: int) -> mw.Inputs:
+    """Each rank is an independent replica: the same expert and gate weights,
+    its own shard of tokens (x drawn with shard index = rank)."""
+    return mw.generate(w, shard=rank)
+
+
+def reduce_max_over_ranks(v: float, world: int, device) -> float:
+    """The slowest rank's time (only collective of the benchmark, never on the
+    data path)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_second(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------ main
 def main():
     a = parse_args()
@@ -267,7 +291,7 @@ def main():
     moe.lib()
 
     w = mw.WORKLOADS[a.workload]
-    inp = mw.generate(w, shard=rank)
+    inp = replica_inputs(w, rank)
     cfg = moe.make_config(w.T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam)
     tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
     x = mw.to_device(inp.x, dev)
@@ -312,11 +336,7 @@ def main():
         torch.cuda.synchronize()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(v, world, dev)
 
     # ---------------------------------------------------------- headline
     timed(run, a.warmup)
@@ -334,7 +354,7 @@ def main():
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(times))
     ms = total_ms / a.steps
-    value = world * w.T / (ms / 1e3)
+    value = job_tokens_per_second(world, w.T, ms)
     st = moe.read_stats(stats)
     offsets = ws[lay.offsets:lay.offsets + 4 * (w.E + 1)].view(torch.int32).cpu().numpy()
     assert st["status"] == 0, f"device status {st['status']}"

@@ -43,6 +43,7 @@ Scratch scratch_layout(const moe_config& c) {
   s.choff = off; off = align256(off + sizeof(int32_t) * (size_t)c.E * nch);
   s.psum = off;  off = align256(off + sizeof(float) * (size_t)c.E * nch);
   s.ntie = off;  off = align256(off + sizeof(int32_t) * nch);
+  s.status = off; off = align256(off + sizeof(uint32_t));
   s.total = off > 0 ? off : 256;
   return s;
 }
@@ -90,6 +91,9 @@ moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 moe_status check_device(bool need_tc) {
+  // A non-sticky error left by an earlier, unrelated runtime call would
+  // otherwise be picked up by the launch checks below and reported as ours.
+  (void)cudaGetLastError();
   DeviceInfo di;
   if (device_info(&di) != cudaSuccess) return MOE_ERR_CUDA;
   if (need_tc && di.major != 10) return MOE_ERR_UNSUPPORTED;
@@ -142,7 +146,7 @@ moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offset
                       const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s) {
   if (c.dtype == MOE_DTYPE_BF16)
     return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
-  return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, s));
+  return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
 }
 
 }  // namespace
@@ -188,7 +192,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const
   if ((st = check_device(false)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(c, x, Wg, bg, topk_idx, topk_w, gap, at<int32_t>(ws, sc.hist),
-                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), s);
+                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<uint32_t>(ws, sc.status), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (prob_mean != nullptr) e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s);
   return cuda_status(e);
@@ -279,7 +283,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
   // near-tie counts of every chunk in scratch, so step 3 starts at the scan
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
-                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), s);
+                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
                          c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, at<int32_t>(ws, L.counts),

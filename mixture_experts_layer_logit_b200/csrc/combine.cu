@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
                const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
   constexpr int N = Pack<TX>::N;
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTokPerBlock + warp;
   if (t >= T) return;
@@ -70,6 +72,8 @@ __global__ void __launch_bounds__(kThreads)
 combine_generic_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
                        const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
   constexpr int N = Pack<TX>::N;
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTokPerBlock + warp;
   if (t >= T) return;
@@ -94,12 +98,12 @@ cudaError_t launch_t(const moe_config& c, const void* yp, const int32_t* row_of,
   const int grid = (c.T + kTokPerBlock - 1) / kTokPerBlock;
   const TX* y = static_cast<const TX*>(yp);
   TX* o = static_cast<TX*>(out);
-  if (c.k <= 1) combine_kernel<TX, 1><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
-  else if (c.k <= 2) combine_kernel<TX, 2><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
-  else if (c.k <= 4) combine_kernel<TX, 4><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
-  else if (c.k <= 8) combine_kernel<TX, 8><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
-  else combine_generic_kernel<TX><<<grid, kThreads, 0, s>>>(y, row_of, w, o, c.T, c.d, c.k);
-  return cudaGetLastError();
+  const dim3 g(grid), b(kThreads);
+  if (c.k <= 1) return launch_pdl(combine_kernel<TX, 1>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
+  if (c.k <= 2) return launch_pdl(combine_kernel<TX, 2>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
+  if (c.k <= 4) return launch_pdl(combine_kernel<TX, 4>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
+  if (c.k <= 8) return launch_pdl(combine_kernel<TX, 8>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
+  return launch_pdl(combine_generic_kernel<TX>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
 }
 
 }  // namespace

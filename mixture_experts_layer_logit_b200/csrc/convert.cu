@@ -36,6 +36,7 @@ extern "C" moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t
   if ((reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(dst) & 15u)) return MOE_ERR_ARG;
   const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
   if (s0 < d0 + 2 * n && d0 < s0 + 2 * n) return MOE_ERR_ARG;   // overlap
+  (void)cudaGetLastError();   // do not report an earlier caller's stale error as ours
   moe::DeviceInfo di;
   if (moe::device_info(&di) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t nvec = n / 8;

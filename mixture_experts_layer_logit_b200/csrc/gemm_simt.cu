@@ -20,14 +20,18 @@ enum { kPlain = 0, kRelu = 1, kSwiglu = 2 };
 template <int MODE>
 __global__ void __launch_bounds__(kThreads)
 simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, float* __restrict__ C,
-                  const int32_t* __restrict__ offsets, int E, int K, int Nout, int NB, int F, int rows_alloc) {
+                  const int32_t* __restrict__ offsets, int E, int K, int Nout, int NB, int F, int rows_alloc,
+                  uint32_t* __restrict__ status) {
   __shared__ int tstart[kMaxExperts + 1];
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Bs[kBK][kBN + 4];
   __shared__ float Bu[MODE == kSwiglu ? kBK : 1][kBN + 4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = (Nout + kBN - 1) / kBN;
-  if (warp == 0) tile_table_warp(offsets, E, kBM, nt, tstart, lane);
+  if (warp == 0) {
+    if (!tile_table_warp(offsets, E, kBM, nt, rows_alloc, tstart, lane) && lane == 0 && blockIdx.x == 0)
+      atomicOr(status, MOE_DEV_BOUNDS);   // offsets[] unusable: no tile is scheduled
+  }
   __syncthreads();
   const int total = tstart[E];
   const int ty = tid >> 4, tx = tid & 15;
@@ -96,7 +100,8 @@ simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, floa
 }  // namespace
 
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
-                                   const void* w1, const void* w2, void* h, void* yp, cudaStream_t s) {
+                                   const void* w1, const void* w2, void* h, void* yp, uint32_t* status,
+                                   cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
@@ -111,15 +116,16 @@ cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const in
   float* H = static_cast<float*>(h);
   if (c.act == MOE_ACT_SWIGLU)
     simt_grouped_gemm<kSwiglu><<<grid_for(c.F), kThreads, 0, s>>>(X, static_cast<const float*>(w1), H,
-                                                                   offsets, c.E, c.d, c.F, 2 * c.F, c.F, (int)A);
+                                                                   offsets, c.E, c.d, c.F, 2 * c.F, c.F, (int)A,
+                                                                   status);
   else
     simt_grouped_gemm<kRelu><<<grid_for(c.F), kThreads, 0, s>>>(X, static_cast<const float*>(w1), H,
-                                                                 offsets, c.E, c.d, c.F, c.F, 0, (int)A);
+                                                                 offsets, c.E, c.d, c.F, c.F, 0, (int)A, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   simt_grouped_gemm<kPlain><<<grid_for(c.d), kThreads, 0, s>>>(H, static_cast<const float*>(w2),
                                                                 static_cast<float*>(yp), offsets, c.E,
-                                                                c.F, c.d, c.d, 0, (int)A);
+                                                                c.F, c.d, c.d, 0, (int)A, status);
   return cudaGetLastError();
 }
 

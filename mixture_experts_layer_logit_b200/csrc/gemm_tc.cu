@@ -25,14 +25,12 @@
 //   * every mbarrier wait is bounded (~2 s); on timeout the kernel sets
 //     MOE_DEV_TIMEOUT, tells the other roles to stop, waits for its own TMA
 //     loads and MMAs, frees TMEM and returns.
-#include "internal.cuh"
-
-#include <cuda.h>
-#include <cudaTypedefs.h>
-#include <mutex>
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int STAGES = 4;
@@ -41,24 +39,21 @@ constexpr int B_BYTES = BN * BK * 2;              // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr unsigned long long kWaitNs = 2000000000ull;    // bounded waits: 2 s
-constexpr unsigned long long kDrainNs = 200000000ull;    // teardown waits: 0.2 s
 enum { kPlain = 0, kRelu = 1, kSwiglu = 2 };
 
-// instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B of one
-// type (format 1 = bf16, 0 = fp16), both K-major, M = 128, N = 256
-constexpr uint32_t idesc_for(bool f16_operands) {
-  return (1u << 4) | ((f16_operands ? 0u : 1u) << 7) | ((f16_operands ? 0u : 1u) << 10) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
 
 struct Tail {
   unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int tstart[kMaxExperts + 1];
+  int seg[kMaxExperts + 1];     // copy of offsets[]: tiles are decoded without global loads
 };
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Tail);
+// Epilogue staging: each epilogue warp turns its 32 rows x 128 bytes of output
+// around in shared memory so that the global stores write whole 128-byte lines.
+constexpr int kStageWarpBytes = 32 * 128;
+constexpr size_t kStagingBytes = 4 * kStageWarpBytes;
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + kStagingBytes + sizeof(Tail);
 
 struct Params {
   const int32_t* offsets;
@@ -69,96 +64,6 @@ struct Params {
   int rows_alloc;       // rows of the A and output buffers (T*k); stores stop there
   uint32_t* status;
 };
-
-// ------------------------------------------------------------------ PTX
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Waits for the phase of `parity` to complete.  Gives up (false) after `limit`
-// ns or, when `abort_flag` is given, once another role has given up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
-                                       unsigned long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = now_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (now_ns() - t0 > limit) return false;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 32 lanes x 32 consecutive fp32 columns; thread i of the warp gets its lane's row
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), descriptor version 1.  The start address advances by
-// 32 bytes per K = 16 step inside the 128-byte swizzle row.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;               // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset
-  d |= (uint64_t)1 << 46;               // version
-  d |= (uint64_t)2 << 61;               // SWIZZLE_128B
-  return d;
-}
 
 // Two fp32 values -> one 32-bit pair of the hidden type (round to nearest
 // even).  fp16 saturates at +-65504 (NaN passes through) and notes it in `over`.
@@ -202,11 +107,12 @@ template <int MODE, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
-  constexpr uint32_t kIdesc = idesc_for(MODE == kPlain && F16);
+  constexpr uint32_t kIdesc = idesc_f16kind(BM, BN, MODE == kPlain && F16);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  Tail* tail = reinterpret_cast<Tail*>(smem_raw + (base - raw) + (size_t)STAGES * STAGE_BYTES);
+  unsigned char* staging = smem_raw + (base - raw) + (size_t)STAGES * STAGE_BYTES;
+  Tail* tail = reinterpret_cast<Tail*>(staging + kStagingBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = (MODE == kSwiglu) ? (p.Nout + BN / 2 - 1) / (BN / 2) : (p.Nout + BN - 1) / BN;
   const int nkb = (p.K + BK - 1) / BK;
@@ -229,12 +135,23 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     tail->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) tile_table_warp(p.offsets, p.E, BM, nt, tail->tstart, lane);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(&tail->tmem_base)), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  pdl_wait();                  // offsets[] and the A rows come from earlier kernels
+  pdl_launch_dependents();
+  if (warp == 0) {
+    if (!tile_table_warp(p.offsets, p.E, BM, nt, p.rows_alloc, tail->tstart, lane) && lane == 0 &&
+        blockIdx.x == 0)
+      atomicOr(p.status, MOE_DEV_BOUNDS);   // offsets[] unusable: no tile is scheduled
+  }
+  for (int e = threadIdx.x; e <= p.E; e += kThreads) tail->seg[e] = p.offsets[e];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -244,12 +161,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
       int it = 0;
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        const TileCoord c = decode_tile<MODE>(tail->tstart, p.offsets, p.E, L);
+        const TileCoord c = decode_tile<MODE>(tail->tstart, tail->seg, p.E, L);
         const int b0 = c.e * p.b_rows + c.n0;
         const int b1 = (MODE == kSwiglu) ? b0 + p.up_off : b0 + BN / 2;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -309,10 +224,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;              // TMEM lanes 32q..32q+31 belong to this warp
+    uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)(warp - 2) * kStageWarpBytes);
     int tl = 0;
     bool ok = true;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tl) {
-      const TileCoord c = decode_tile<MODE>(tail->tstart, p.offsets, p.E, L);
+      const TileCoord c = decode_tile<MODE>(tail->tstart, tail->seg, p.E, L);
       const int acc = tl & 1;
       const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
       ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kWaitNs);
@@ -320,66 +236,75 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       if (!ok) break;
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int r = q * 32 + lane;
-      bool rv = r < c.rows;
-      if (rv && c.row0 + r >= p.rows_alloc) {   // offsets[] beyond the buffers: skip and flag
-        atomicOr(p.status, MOE_DEV_BOUNDS);
-        rv = false;
+      // rows of this warp that may be stored: inside the segment and the buffers
+      const int wrow0 = c.row0 + q * 32;
+      int nrows = min(32, c.rows - q * 32);
+      if (nrows > 0 && wrow0 + nrows > p.rows_alloc) {   // offsets[] beyond the buffers: skip and flag
+        if (lane == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
+        nrows = p.rows_alloc - wrow0;
       }
-      const size_t orow_off = (size_t)(c.row0 + (rv ? r : 0)) * p.Nout;
-      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off;   // layer 1: h (bf16 or fp16)
-      float* orow32 = static_cast<float*>(p.out) + orow_off;       // layer 2: fp32 yp
       bool over = false;
-      if (MODE == kSwiglu) {
+      // One block = 128 bytes of output per row: 32 fp32 columns (layer 2) or
+      // 64 16-bit hidden columns (layer 1).  Thread `lane` owns TMEM row
+      // wrow0 + lane; the block is turned around in shared memory (16-byte
+      // chunk i of row r at slot i ^ (r & 7), conflict-free both ways) and
+      // written as 4 rows x 128 contiguous bytes per store instruction.
+      constexpr int kBlocks = (MODE == kPlain) ? BN / 32 : (MODE == kRelu ? BN / 64 : BN / 128);
+      constexpr int kPer16 = (MODE == kPlain) ? 4 : 8;
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 64; ++ch) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tb + ch * 32, g);
-          tmem_ld32(tb + BN / 2 + ch * 32, u);
+      for (int blk = 0; blk < kBlocks; ++blk) {
+        uint4 v[8];
+        if (MODE == kPlain) {
+          uint32_t a[32];
+          tmem_ld32(tb + blk * 32, a);
           tmem_wait_ld();
-          const int col = c.n0 + ch * 32;
-          if (rv) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col + 8 * v >= p.Nout) break;
+          for (int i = 0; i < 8; ++i) v[i] = make_uint4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t a[32], u[32];
+            if (MODE == kRelu) {
+              tmem_ld32(tb + blk * 64 + hf * 32, a);
+            } else {   // SwiGLU: gate columns, then the up columns BN/2 further
+              tmem_ld32(tb + blk * 64 + hf * 32, a);
+              tmem_ld32(tb + BN / 2 + blk * 64 + hf * 32, u);
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
               uint32_t pk[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float g0 = __uint_as_float(g[8 * v + 2 * i]), g1 = __uint_as_float(g[8 * v + 2 * i + 1]);
-                const float u0 = __uint_as_float(u[8 * v + 2 * i]), u1 = __uint_as_float(u[8 * v + 2 * i + 1]);
-                pk[i] = pack_hidden<F16>(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1, over);
+              for (int j = 0; j < 4; ++j) {
+                float a0 = __uint_as_float(a[8 * i + 2 * j]), a1 = __uint_as_float(a[8 * i + 2 * j + 1]);
+                if (MODE == kRelu) {
+                  a0 = fmaxf(a0, 0.f);
+                  a1 = fmaxf(a1, 0.f);
+                } else {
+                  const float u0 = __uint_as_float(u[8 * i + 2 * j]), u1 = __uint_as_float(u[8 * i + 2 * j + 1]);
+                  a0 = a0 / (1.f + __expf(-a0)) * u0;
+                  a1 = a1 / (1.f + __expf(-a1)) * u1;
+                }
+                pk[j] = pack_hidden<F16>(a0, a1, over);
               }
-              *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              v[hf * 4 + i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
         }
-      } else {
-#pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t a[32];
-          tmem_ld32(tb + ch * 32, a);
-          tmem_wait_ld();
-          const int col = c.n0 + ch * 32;
-          if (rv && MODE == kPlain) {
+        __syncwarp();
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              if (col + 4 * v >= p.Nout) break;
-              *reinterpret_cast<uint4*>(orow32 + col + 4 * v) =
-                  make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
-            }
-          } else if (rv) {
+        for (int i = 0; i < 8; ++i) stg[lane * 8 + (i ^ (lane & 7))] = v[i];
+        __syncwarp();
+        const int col0 = c.n0 + blk * 8 * kPer16;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col + 8 * v >= p.Nout) break;
-              uint32_t pk[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                float a0 = __uint_as_float(a[8 * v + 2 * i]), a1 = __uint_as_float(a[8 * v + 2 * i + 1]);
-                if (MODE == kRelu) { a0 = fmaxf(a0, 0.f); a1 = fmaxf(a1, 0.f); }
-                pk[i] = pack_hidden<F16>(a0, a1, over);
-              }
-              *reinterpret_cast<uint4*>(orow + col + 8 * v) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + (lane >> 3), cc = lane & 7;
+          const uint4 val = stg[rr * 8 + (cc ^ (rr & 7))];
+          const int col = col0 + cc * kPer16;
+          if (rr < nrows && col < p.Nout) {
+            const size_t off = (size_t)(wrow0 + rr) * p.Nout + col;
+            if (MODE == kPlain) *reinterpret_cast<uint4*>(static_cast<float*>(p.out) + off) = val;
+            else *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + off) = val;
           }
         }
       }
@@ -436,8 +361,7 @@ template <int MODE, bool F16>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid, cudaStream_t s) {
   cudaError_t err = set_smem_once<tc_grouped_gemm<MODE, F16>>(kSmemBytes);
   if (err != cudaSuccess) return err;
-  tc_grouped_gemm<MODE, F16><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, p);
-  return cudaGetLastError();
+  return launch_pdl(tc_grouped_gemm<MODE, F16>, dim3(grid), dim3(kThreads), kSmemBytes, s, ma, mb, p);
 }
 
 template <bool F16>

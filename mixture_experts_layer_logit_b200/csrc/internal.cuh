@@ -7,14 +7,14 @@
 #include <stdint.h>
 #include <stddef.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 
 namespace moe {
 
 // Tokens per routing / permutation chunk.  The route kernel, the histogram and
 // the scatter kernel all cut the token axis into chunks of this size, and the
 // per-chunk histograms and prefix sums live in the scratch workspace.
-constexpr int kChunk = 64;
+constexpr int kChunk = 128;
 constexpr int kMaxExperts = 256;
 
 // Scratch layout (byte offsets into the step workspace).
@@ -23,6 +23,7 @@ struct Scratch {
   size_t choff;     // int32 [E][nchunks]   exclusive prefix over chunks
   size_t psum;      // float [nchunks][E]   per-chunk sums of softmax probabilities
   size_t ntie;      // int32 [nchunks]      near-tie tokens per chunk
+  size_t status;    // uint32               device error bits of a standalone moe_route
   size_t total;
 };
 
@@ -38,7 +39,12 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // sums and near-tie counts into scratch.  TX = float or __nv_bfloat16.
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
-                         int32_t* hist, float* psum, int32_t* ntie, cudaStream_t s);
+                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, cudaStream_t s);
+// The same on tcgen05 tensor cores (bf16, k <= 8).
+bool route_tc_supported(const moe_config& c);
+cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
+                            int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
+                            int32_t* ntie, uint32_t* status, cudaStream_t s);
 // prob_mean[e] = sum over chunks of psum / T (fixed order).
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
 // Histogram of topk_idx per chunk (+ near ties from gap when given).
@@ -56,7 +62,8 @@ cudaError_t launch_scatter(const moe_config& c, int capacity, const void* x, con
                            int32_t* src_tok, void* xp, uint32_t* status, cudaStream_t s);
 // Expert FFN on CUDA cores (fp32 path).
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
-                                   const void* w1, const void* w2, void* h, void* yp, cudaStream_t s);
+                                   const void* w1, const void* w2, void* h, void* yp, uint32_t* status,
+                                   cudaStream_t s);
 // Expert FFN on tcgen05 tensor cores (bf16 path).
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
@@ -95,18 +102,38 @@ namespace moe {
 // Tile table of a grouped GEMM over expert segments: expert e owns rows
 // [offsets[e], offsets[e+1]) and ceil(M_e / BM) * nt tiles, numbered from
 // tstart[e]; tstart[E] is the total.  Run by the 32 lanes of one warp
-// (E <= 256, 8 experts per lane).
-__device__ __forceinline__ void tile_table_warp(const int32_t* __restrict__ offsets, int E, int BM,
-                                                int nt, int* tstart, int lane) {
+// (E <= 256, 8 experts per lane).  offsets[] must be non-decreasing inside
+// [0, rows_alloc] with at most 2^30 tiles in all; otherwise the table is
+// left empty (no tile runs, nothing is written) and false is returned.
+__device__ __forceinline__ bool tile_table_warp(const int32_t* __restrict__ offsets, int E, int BM,
+                                                int nt, int rows_alloc, int* tstart, int lane) {
   constexpr int PER = kMaxExperts / 32;
   int loc[PER];
-  int sum = 0;
+  long long sum64 = 0;
+  bool ok = true;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane * PER + i;
-    int m = (e < E) ? offsets[e + 1] - offsets[e] : 0;
-    m = m > 0 ? m : 0;
-    loc[i] = ((m + BM - 1) / BM) * nt;
+    long long m = 0;
+    if (e < E) {
+      const int a = offsets[e], b = offsets[e + 1];
+      ok &= (a >= 0) && (b >= a) && (b <= rows_alloc);
+      m = (long long)b - a;
+    }
+    const long long tiles = ((m + BM - 1) / BM) * (long long)nt;
+    ok &= tiles <= (1LL << 30);
+    loc[i] = (int)(tiles > (1LL << 30) ? 0 : tiles);
+    sum64 += loc[i];
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  long long tot = sum64;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  ok = ok && tot <= (1LL << 30);
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    if (!ok) loc[i] = 0;
     sum += loc[i];
   }
   int incl = sum;
@@ -123,6 +150,7 @@ __device__ __forceinline__ void tile_table_warp(const int32_t* __restrict__ offs
     run += loc[i];
   }
   if (lane == 31) tstart[E] = incl;
+  return ok;
 }
 
 // Expert owning tile L: the largest e with tstart[e] <= L (empty experts have
@@ -139,8 +167,37 @@ __device__ __forceinline__ int tile_expert(const int* tstart, int E, int L) {
 }  // namespace moe
 
 #include <atomic>
+#include <utility>
 
 namespace moe {
+
+// Programmatic dependent launch.  Every kernel of the layer is launched with
+// the programmatic-serialization attribute, so it may start while the kernel
+// before it in the stream drains.  A kernel does only work that touches no
+// global memory before pdl_wait() (barrier set-up, TMEM allocation,
+// tensor-map prefetch); pdl_wait() returns once the previous grid has
+// completed and its writes are visible, which by induction covers every
+// earlier kernel.  Without a programmatic predecessor both calls are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Raises a kernel's dynamic shared-memory limit once per device (the first
 // call, made before any stream capture, does the work; later calls only read
@@ -155,6 +212,7 @@ cudaError_t set_smem_once(size_t bytes) {
   if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
   e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  else (void)cudaGetLastError();   // report it here, do not leave it for the next launch check
   return e;
 }
 

@@ -30,6 +30,8 @@ hist_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ gap,
   __shared__ int nt;
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
   if (threadIdx.x == 0) nt = 0;
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
   const int t = blockIdx.x * kChunk + threadIdx.x;
   if (t < T) {
@@ -61,21 +63,34 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
   __shared__ int s_ntie;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = kScanThreads / 32;
+  pdl_wait();
+  pdl_launch_dependents();
 
-  // per-expert exclusive scan over chunks (expert-major hist, coalesced)
+  // per-expert exclusive scan over chunks (expert-major hist, coalesced); the
+  // loads of four 32-chunk groups are issued before any of them is scanned
+  constexpr int kBatch = 4;
   for (int e = warp; e < E; e += nwarps) {
     int running = 0;
-    for (int c0 = 0; c0 < nch; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = (c < nch) ? hist[(size_t)e * nch + c] : 0;
-      int incl = v;
+    const int32_t* hrow = hist + (size_t)e * nch;
+    for (int c0 = 0; c0 < nch; c0 += 32 * kBatch) {
+      int v[kBatch];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += u;
+      for (int b = 0; b < kBatch; ++b) {
+        const int c = c0 + 32 * b + lane;
+        v[b] = (c < nch) ? hrow[c] : 0;
       }
-      if (c < nch) choff[(size_t)e * nch + c] = running + incl - v;
-      running += __shfl_sync(kFull, incl, 31);
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int c = c0 + 32 * b + lane;
+        int incl = v[b];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(kFull, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (c < nch) choff[(size_t)e * nch + c] = running + incl - v[b];
+        running += __shfl_sync(kFull, incl, 31);
+      }
     }
     // P_e for the aux loss
     float P = NAN;
@@ -83,6 +98,7 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
       P = prob_mean[e];
     } else if (psum != nullptr) {
       float s = 0.f;
+#pragma unroll 4
       for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
       P = warp_sum(s) / (float)T;
     }
@@ -154,7 +170,7 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
 }
 
 // ------------------------------------------------------------------ scatter
-constexpr int kScatterThreads = 256;
+constexpr int kScatterThreads = 512;   // 4 rank warps, then 16 warps copying rows
 
 template <typename TX>
 __device__ __forceinline__ void copy_rows(const TX* __restrict__ x, TX* __restrict__ xp, int d,
@@ -181,16 +197,20 @@ scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
                const int32_t* __restrict__ choff, const int32_t* __restrict__ offsets,
                int T, int d, int E, int k, int nch, int capacity,
                int32_t* __restrict__ row_of, int32_t* __restrict__ src_tok, TX* __restrict__ xp) {
-  __shared__ int wcnt[2][kMaxExperts];
+  constexpr int kRankWarps = kChunk / 32;
+  static_assert(kRankWarps <= kScatterThreads / 32, "one rank warp per 32 tokens of a chunk");
+  __shared__ int wcnt[kRankWarps][kMaxExperts];
   __shared__ int rows_sm[kChunk][KB];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
-  for (int i = threadIdx.x; i < 2 * kMaxExperts; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < kRankWarps * kMaxExperts; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
 
   int val[KB], rank_w[KB];
   const int t = chunk * kChunk + warp * 32 + lane;
-  if (warp < 2) {
+  if (warp < kRankWarps) {
     const bool tv = t < T;
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
@@ -227,13 +247,15 @@ scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
     }
   }
   __syncthreads();
-  if (warp < 2) {
+  if (warp < kRankWarps) {
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
       const int e = val[j];
       int row = -1;
       if (e < E) {
-        const int r = choff[(size_t)e * nch + chunk] + (warp == 1 ? wcnt[0][e] : 0) + rank_w[j];
+        int before = 0;   // assignments of expert e in the earlier warps of this chunk
+        for (int w = 0; w < warp; ++w) before += wcnt[w][e];
+        const int r = choff[(size_t)e * nch + chunk] + before + rank_w[j];
         if (capacity < 0 || r < capacity) {
           row = offsets[e] + r;
           src_tok[row] = t;
@@ -260,16 +282,17 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
                        const int32_t* __restrict__ choff, const int32_t* __restrict__ offsets,
                        int T, int d, int E, int k, int nch, int capacity,
                        int32_t* __restrict__ row_of, int32_t* __restrict__ src_tok, TX* __restrict__ xp) {
-  extern __shared__ int dyn[];
-  int* idx_sm = dyn;                  // [kChunk * k]
-  int* rows_sm = dyn + kChunk * k;    // [kChunk * k]
+  extern __shared__ int idx_sm[];     // [kChunk * k] expert of each assignment, -1 if invalid
+  pdl_wait();
+  pdl_launch_dependents();
   const int chunk = blockIdx.x;
   const int t0 = chunk * kChunk;
   const int n = min(kChunk, T - t0) * k;
+  int32_t* rows = row_of + (size_t)t0 * k;
   for (int i = threadIdx.x; i < n; i += kScatterThreads) {
     int e = topk_idx[(size_t)t0 * k + i];
     idx_sm[i] = (e < 0 || e >= E) ? -1 : e;
-    rows_sm[i] = -1;
+    rows[i] = -1;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kScatterThreads) {
@@ -278,19 +301,18 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
       if (idx_sm[i] != e) continue;
       if (capacity < 0 || r < capacity) {
         const int row = offsets[e] + r;
-        rows_sm[i] = row;
+        rows[i] = row;
         src_tok[row] = t0 + i / k;
       }
       ++r;
     }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kScatterThreads) row_of[(size_t)t0 * k + i] = rows_sm[i];
+  __syncthreads();   // the row numbers written above are visible to the whole block
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = warp; i < kChunk; i += kScatterThreads / 32) {
     const int tt = t0 + i;
     if (tt >= T) break;
-    copy_rows<TX>(x, xp, d, tt, rows_sm + i * k, k, lane);
+    copy_rows<TX>(x, xp, d, tt, rows + (size_t)i * k, k, lane);
   }
 }
 
@@ -301,23 +323,20 @@ cudaError_t launch_scatter_t(const moe_config& c, int cap, const void* x, const 
   const int nch = num_chunks(c.T);
   const TX* xx = static_cast<const TX*>(x);
   TX* pp = static_cast<TX*>(xp);
-#define MOE_SCATTER(KB)                                                                       \
-  scatter_kernel<KB, TX><<<nch, kScatterThreads, 0, s>>>(xx, idx, choff, off, c.T, c.d, c.E, \
-                                                         c.k, nch, cap, row_of, src_tok, pp)
+  const dim3 g(nch), b(kScatterThreads);
+#define MOE_SCATTER(KB) \
+  return launch_pdl(scatter_kernel<KB, TX>, g, b, 0, s, xx, idx, choff, off, c.T, c.d, c.E, c.k, nch, cap, \
+                    row_of, src_tok, pp)
   if (c.k <= 1) MOE_SCATTER(1);
-  else if (c.k <= 2) MOE_SCATTER(2);
-  else if (c.k <= 4) MOE_SCATTER(4);
-  else if (c.k <= 8) MOE_SCATTER(8);
-  else {
-    const size_t smem = sizeof(int) * 2 * kChunk * (size_t)c.k;
-    auto kern = scatter_generic_kernel<TX>;
-    cudaError_t err = set_smem_once<scatter_generic_kernel<TX>>(sizeof(int) * 2 * kChunk * kMaxExperts);
-    if (err != cudaSuccess) return err;
-    kern<<<nch, kScatterThreads, smem, s>>>(xx, idx, choff, off, c.T, c.d, c.E, c.k, nch, cap,
-                                            row_of, src_tok, pp);
-  }
+  if (c.k <= 2) MOE_SCATTER(2);
+  if (c.k <= 4) MOE_SCATTER(4);
+  if (c.k <= 8) MOE_SCATTER(8);
 #undef MOE_SCATTER
-  return cudaGetLastError();
+  const size_t smem = sizeof(int) * kChunk * (size_t)c.k;
+  cudaError_t err = set_smem_once<scatter_generic_kernel<TX>>(sizeof(int) * kChunk * kMaxExperts);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(scatter_generic_kernel<TX>, g, b, smem, s, xx, idx, choff, off, c.T, c.d, c.E, c.k, nch, cap,
+                    row_of, src_tok, pp);
 }
 
 }  // namespace
@@ -325,18 +344,16 @@ cudaError_t launch_scatter_t(const moe_config& c, int cap, const void* x, const 
 cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const float* gap,
                         int32_t* hist, int32_t* ntie, uint32_t* status, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
-  hist_kernel<<<num_chunks(c.T), kChunk, 0, s>>>(topk_idx, gap, c.T, c.E, c.k, num_chunks(c.T), hist,
-                                                 gap != nullptr ? ntie : nullptr, status);
-  return cudaGetLastError();
+  return launch_pdl(hist_kernel, dim3(num_chunks(c.T)), dim3(kChunk), 0, s, topk_idx, gap, c.T, c.E, c.k,
+                    num_chunks(c.T), hist, gap != nullptr ? ntie : nullptr, status);
 }
 
 cudaError_t launch_scan(const moe_config& c, int capacity, const int32_t* hist, int32_t* choff,
                         const float* prob_mean, const float* psum, const int32_t* ntie,
                         int32_t* counts, int32_t* kept, int32_t* offsets, moe_stats* stats,
                         cudaStream_t s) {
-  scan_kernel<<<1, kScanThreads, 0, s>>>(hist, choff, num_chunks(c.T), c.T, c.E, c.k, capacity,
-                                         prob_mean, psum, ntie, counts, kept, offsets, stats);
-  return cudaGetLastError();
+  return launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, hist, choff, num_chunks(c.T), c.T, c.E, c.k,
+                    capacity, prob_mean, psum, ntie, counts, kept, offsets, stats);
 }
 
 cudaError_t launch_scatter(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,

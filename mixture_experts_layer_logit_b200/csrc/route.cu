@@ -47,8 +47,8 @@ template <> struct VecLoad<__nv_bfloat16> {
 template <int NJ>
 struct RouteSmem {
   static constexpr int EP = 16 * NJ;
-  static constexpr size_t xs = 0;                                          // float [kChunk][kKC+1]
-  static constexpr size_t ws = xs + sizeof(float) * kChunk * (kKC + 1);    // float [EP][kKC+1]
+  static constexpr size_t xs = 0;                                          // float [64][kKC+1]
+  static constexpr size_t ws = xs + sizeof(float) * 64 * (kKC + 1);        // float [EP][kKC+1]
   static constexpr size_t zs = ws + sizeof(float) * EP * (kKC + 1);        // float [kChunk][EP+1]
   static constexpr size_t selp = zs + sizeof(float) * kChunk * (EP + 1);   // float [8][EP]
   static constexpr size_t seli = selp + sizeof(float) * 8 * EP;            // int   [8][EP]
@@ -87,8 +87,9 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
   for (int e = tid; e < EP; e += kThreads) shist[e] = 0;
   if (tid == 0) misc[0] = 0;
 
-  // ---- gate GEMM: z[64][EP] = x[64][d] . wg[EP][d]^T, fp32 accumulation
+  // ---- gate GEMM: z[kChunk][EP] = x . wg^T in fp32, 64 token rows at a time
   const int ty = tid >> 4, tx = tid & 15;
+  for (int half = 0; half < kChunk / 64; ++half) {
   float acc[4][NJ];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -96,12 +97,12 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
     for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
 
   for (int k0 = 0; k0 < d; k0 += kKC) {
-    // stage x: kChunk rows x kKC columns
-    for (int v = tid; v < kChunk * (kKC / V); v += kThreads) {
+    // stage x: 64 rows x kKC columns
+    for (int v = tid; v < 64 * (kKC / V); v += kThreads) {
       const int r = v / (kKC / V), c = (v % (kKC / V)) * V;
       float f[V];
-      if (r < rows && k0 + c < d) {
-        VecLoad<TX>::load(x + (size_t)(t0 + r) * d + k0 + c, f);
+      if (half * 64 + r < rows && k0 + c < d) {
+        VecLoad<TX>::load(x + (size_t)(t0 + half * 64 + r) * d + k0 + c, f);
       } else {
 #pragma unroll
         for (int q = 0; q < V; ++q) f[q] = 0.f;
@@ -141,8 +142,9 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int e = tx + 16 * j;
-      zs[ty * 4 + i][e] = acc[i][j] + ((bg != nullptr && e < E) ? bg[e] : 0.f);
+      zs[half * 64 + ty * 4 + i][e] = acc[i][j] + ((bg != nullptr && e < E) ? bg[e] : 0.f);
     }
+  }
   __syncthreads();
 
   // ---- routing epilogue: one warp per token, lane holds experts lane + 32 i
@@ -302,8 +304,10 @@ cudaError_t launch_route_t(const moe_config& c, const void* x, const void* wg, c
 
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
-                         int32_t* hist, float* psum, int32_t* ntie, cudaStream_t s) {
+                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
+  if (route_tc_supported(c))
+    return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, s);
   if (c.dtype == MOE_DTYPE_BF16)
     return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, s);
   return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, s);

@@ -1,0 +1,344 @@
+// Steps 1-2 on the tensor cores for the bf16 layer: the gate GEMM as one
+// tcgen05 tile of 128 tokens x E experts per CTA, followed by the gating
+// epilogue (normalisation, softmax, top-k, renormalised weights, near-tie
+// gap) on the token rows of logits.
+//
+// Gate: one fully-connected layer z = x W_gate^T (+ b) (FastMoE announcement,
+// "特色二"); the gating network activates the k best experts of each input
+// (FastMoE announcement, "1. MoE 设计" and "图4").  Normalisation
+// (Skywork-MoE release, "Gating Logits归一化操作"; slides, slide 6):
+// z_hat = lambda (z - mean) / std over the experts, population std, zero
+// spread -> 0.  Equal scores: the lower expert index wins.
+//
+// Layout: x [T, d] and W_gate [E, d] are K-major bf16 and go through TMA
+// (128-byte swizzle) into a ring of up to 8 stages (enough for the whole
+// d = 512 reduction to be in flight at once); tcgen05.mma kind::f16 with
+// M = 128, N = E rounded up to 16 (rows of W_gate past E load as zeros)
+// accumulates the 128 x N logits in fp32 in TMEM.  The epilogue copies them to
+// shared memory and gives every token two threads, each owning half of the
+// experts: partial sums, maxima and top-(k+1) lists are merged through shared
+// memory.  Each CTA is one routing chunk of 128 tokens: it also writes the
+// chunk's per-expert histogram, per-expert sum of softmax probabilities
+// (summed in a fixed order) and near-tie count for the permutation step.
+#include "tc_ptx.cuh"
+
+#include <math.h>
+
+namespace moe {
+namespace {
+
+using namespace tc;
+
+constexpr int RM = 128;            // tokens per CTA = routing chunk
+constexpr int RK = 64;             // model-width slice per stage (128 bytes of bf16)
+constexpr int kMaxStages = 8;
+constexpr int kRingBytes = 192 * 1024;
+constexpr int kSplit = 2;          // threads per token in the epilogue
+constexpr int kThreads = RM * kSplit;
+constexpr int kMaxKeep = 9;        // top-(k+1) list length for k <= 8
+static_assert(RM == kChunk, "one CTA per routing chunk");
+
+struct RTail {
+  unsigned long long full[kMaxStages], empty[kMaxStages], done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ntie;
+  int hist[kMaxExperts];
+  float bias[kMaxExperts];
+  float part[kSplit][4][RM];       // per half: sum, squares, max, exp-sum of each row
+  float lv[kMaxKeep][RM];          // the upper half's top list of each row
+  int li[kMaxKeep][RM];
+};
+
+__host__ __device__ constexpr int stage_bytes(int EP) { return RM * RK * 2 + EP * RK * 2; }
+inline int num_stages(int EP) { return std::min(kMaxStages, kRingBytes / stage_bytes(EP)); }
+inline size_t smem_bytes(int EP) { return 1024 + (size_t)num_stages(EP) * stage_bytes(EP) + sizeof(RTail); }
+__host__ __device__ constexpr uint32_t tmem_cols(int EP) { return EP <= 32 ? 32 : EP <= 64 ? 64 : EP <= 128 ? 128 : 256; }
+
+// Keeps the n <= KB + 1 best (score, expert) pairs, best first, in registers
+// (every index is a compile-time constant).  Pairs arrive in ascending expert
+// order, so a new pair goes behind every kept pair whose score is >= its own:
+// equal scores stay in ascending index order.
+template <int KB>
+struct TopList {
+  static constexpr int kEmpty = 0x7fffffff;
+  float v[KB + 1];
+  int i[KB + 1];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j <= KB; ++j) { v[j] = -INFINITY; i[j] = kEmpty; }
+  }
+  __device__ __forceinline__ void insert(float s, int e, int n) {
+    int pos = 0;   // kept pairs that stay ahead (a prefix of the sorted list)
+#pragma unroll
+    for (int j = 0; j <= KB; ++j)
+      if (j < n && i[j] != kEmpty && !(s > v[j])) pos = j + 1;
+    if (pos >= n) return;
+#pragma unroll
+    for (int j = KB; j >= 1; --j)
+      if (j < n && j > pos) { v[j] = v[j - 1]; i[j] = i[j - 1]; }
+#pragma unroll
+    for (int j = 0; j <= KB; ++j)
+      if (j == pos) { v[j] = s; i[j] = e; }
+  }
+};
+
+// Score the top-k is taken on: the biased logit, or its normalised value.
+__device__ __forceinline__ float gate_score(float zb, float lam, float mu, float sd) {
+  return lam > 0.f ? (sd > 0.f ? lam * (zb - mu) / sd : 0.f) : zb;
+}
+
+// KB is the exact number of experts per token, so that every index into the
+// top-k registers is a compile-time constant.
+template <int KB>
+__global__ void __launch_bounds__(kThreads, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
+                int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
+                int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
+                int nch, uint32_t* __restrict__ status) {
+  constexpr int k = KB;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sbase = smem_raw + (base - raw);
+  const int SB = stage_bytes(EP);
+  RTail* tail = reinterpret_cast<RTail*>(sbase + (size_t)nst * SB);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x, t0 = chunk * RM;
+  const int nkb = (d + RK - 1) / RK;
+  const uint32_t full0 = smem_u32(&tail->full[0]), empty0 = smem_u32(&tail->empty[0]);
+  const uint32_t done = smem_u32(&tail->done);
+  const volatile int* abort_flag = &tail->abort_flag;
+  const uint32_t ncols = tmem_cols(EP);
+
+  if (tid == 0) {
+    for (int s = 0; s < nst; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done, 1);
+    tail->abort_flag = 0;
+    tail->ntie = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int e = tid; e < E; e += kThreads) tail->hist[e] = 0;
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&tail->tmem_base)), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+  }
+  pdl_wait();                  // x, W_gate and b may come from the previous kernel
+  pdl_launch_dependents();
+  for (int e = tid; e < E; e += kThreads) tail->bias[e] = (bg != nullptr) ? bg[e] : 0.f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+
+  // ------------------------------------------------- gate GEMM main loop
+  if (warp == 0 && lane == 0) {
+    int issued = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % nst;
+      const uint32_t ph = (uint32_t)(kb / nst) & 1u;
+      if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kWaitNs)) {
+        atomicOr(status, MOE_DEV_TIMEOUT);
+        tail->abort_flag = 1;
+        break;
+      }
+      const uint32_t sa = base + (uint32_t)(s * SB);
+      mbar_expect_tx(full0 + 8 * s, (uint32_t)SB);
+      tma_load_2d(sa, &tmX, full0 + 8 * s, kb * RK, t0);
+      tma_load_2d(sa + RM * RK * 2, &tmW, full0 + 8 * s, kb * RK, 0);
+      ++issued;
+    }
+    for (int i = max(0, issued - nst); i < issued; ++i)   // loads still in flight
+      mbar_wait(full0 + 8 * (i % nst), (uint32_t)(i / nst) & 1u, nullptr, kDrainNs);
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_f16kind(RM, EP, false);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % nst;
+      const uint32_t ph = (uint32_t)(kb / nst) & 1u;
+      if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kWaitNs)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = base + (uint32_t)(s * SB);
+      const uint64_t ad = sdesc(sa), bd = sdesc(sa + RM * RK * 2);
+#pragma unroll
+      for (int kk = 0; kk < RK / 16; ++kk)
+        tc_mma(tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kb | kk) != 0);
+      tc_commit(empty0 + 8 * s);
+    }
+    if (!ok) {
+      atomicOr(status, MOE_DEV_TIMEOUT);
+      tail->abort_flag = 1;
+    }
+    tc_commit(done);   // arrives once every MMA above has completed
+  }
+  __syncwarp();
+  bool ok = mbar_wait(done, 0, nullptr, kWaitNs) && !*abort_flag;
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+
+  // ------------------------------------------------- gating epilogue
+  // The logits of each row go from TMEM to a padded shared-memory row (the
+  // stage ring is free now; the odd row stride keeps a warp's column accesses
+  // conflict-free).  Warps q and q + 4 read the same TMEM lanes 32q..32q+31:
+  // half 0 owns experts [0, E0), half 1 owns [E0, E).
+  const int q = warp & 3, half = warp >> 2;
+  const int row = q * 32 + lane;
+  const int t = t0 + row;
+  const bool valid = ok && t < T;
+  const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16);
+  const int ldz = E | 1;
+  float* Zall = reinterpret_cast<float*>(sbase);   // [RM][ldz]
+  float* Z = Zall + (size_t)row * ldz;
+  const int nch32 = (E + 31) / 32;
+  for (int c = half; c < nch32; c += kSplit) {
+    uint32_t r[32];
+    tmem_ld32(tb + c * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = c * 32 + i;
+      if (e < E) Z[e] = __uint_as_float(r[i]) + tail->bias[e];
+    }
+  }
+  __syncthreads();
+  const int E0 = (E + 1) / 2;
+  const int lo = half ? E0 : 0, hi = half ? E : E0;
+  float (*part)[4][RM] = tail->part;
+  if (lam > 0.f) {   // z_hat = lambda (z - mean) / std, written over z
+    float s = 0.f;
+#pragma unroll 4
+    for (int e = lo; e < hi; ++e) s += Z[e];
+    part[half][0][row] = s;
+    __syncthreads();
+    const float mu = (part[0][0][row] + part[1][0][row]) / (float)E;
+    float qq = 0.f;
+#pragma unroll 4
+    for (int e = lo; e < hi; ++e) {
+      const float dv = Z[e] - mu;
+      qq += dv * dv;
+    }
+    part[half][1][row] = qq;
+    __syncthreads();
+    const float sd = sqrtf((part[0][1][row] + part[1][1][row]) / (float)E);
+#pragma unroll 4
+    for (int e = lo; e < hi; ++e) Z[e] = gate_score(Z[e], lam, mu, sd);
+  }
+  const int nkeep = (k < E) ? k + 1 : k;
+  TopList<KB> top;
+  top.init();
+  float mh = -INFINITY;
+#pragma unroll 4
+  for (int e = lo; e < hi; ++e) {
+    const float sc = Z[e];
+    mh = fmaxf(mh, sc);
+    top.insert(sc, e, nkeep);
+  }
+  part[half][2][row] = mh;
+  if (half == 1) {
+#pragma unroll
+    for (int j = 0; j <= KB; ++j) {
+      tail->lv[j][row] = top.v[j];
+      tail->li[j][row] = top.i[j];
+    }
+  }
+  __syncthreads();
+  const float m = fmaxf(part[0][2][row], part[1][2][row]);
+  float Sh = 0.f;
+#pragma unroll 4
+  for (int e = lo; e < hi; ++e) Sh += __expf(Z[e] - m);
+  part[half][3][row] = Sh;
+  __syncthreads();
+  const float S = part[0][3][row] + part[1][3][row];
+  const float invS = 1.f / S;
+  if (half == 0) {
+    // merge: the upper half's experts all have higher indices, so inserting
+    // its list (best first) keeps the lowest-index-wins order on equal scores
+#pragma unroll
+    for (int j = 0; j <= KB; ++j) {
+      const int ie = tail->li[j][row];
+      if (ie != TopList<KB>::kEmpty) top.insert(tail->lv[j][row], ie, nkeep);
+    }
+    float psel[KB], sel = 0.f;
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      psel[j] = __expf(top.v[j] - m) * invS;
+      sel += psel[j];                     // slot order
+    }
+    const float rs = 1.f / sel;
+    const float gap = (k < E) ? top.v[k - 1] - top.v[k] : INFINITY;
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < KB; ++j) {
+        topk_idx[(size_t)t * k + j] = top.i[j];
+        topk_w[(size_t)t * k + j] = psel[j] * rs;
+        atomicAdd(&tail->hist[top.i[j]], 1);
+      }
+      gap_out[t] = gap;
+      if (gap < MOE_NEAR_TIE_GAP) atomicAdd(&tail->ntie, 1);
+    }
+  }
+
+  // per-expert probability sums of the chunk: probabilities over the scores
+  // in shared memory, then one thread per expert adds its column in row order
+#pragma unroll 4
+  for (int e = lo; e < hi; ++e) Z[e] = valid ? __expf(Z[e] - m) * invS : 0.f;
+  tc_fence_before();
+  __syncthreads();
+  for (int e = tid; e < E; e += kThreads) {
+    float s = 0.f;
+    for (int rr = 0; rr < RM; ++rr) s += Zall[(size_t)rr * ldz + e];
+    psum_out[(size_t)chunk * E + e] = s;
+    hist_out[(size_t)e * nch + chunk] = tail->hist[e];
+  }
+  if (tid == 0) ntie_out[chunk] = tail->ntie;
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+  }
+}
+
+template <int KB>
+cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
+                      int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
+                      uint32_t* status, cudaStream_t s) {
+  // the ring never exceeds kRingBytes, whatever E is
+  cudaError_t err = set_smem_once<route_tc_kernel<KB>>(1024 + (size_t)kRingBytes + sizeof(RTail));
+  if (err != cudaSuccess) return err;
+  const int nch = num_chunks(c.T);
+  return launch_pdl(route_tc_kernel<KB>, dim3(nch), dim3(kThreads), smem_bytes(EP), s, mx, mw, bg, c.T, c.d, c.E,
+                    EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status);
+}
+
+}  // namespace
+
+bool route_tc_supported(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.k <= 8; }
+
+cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
+                            int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
+                            int32_t* ntie, uint32_t* status, cudaStream_t s) {
+  if (c.T == 0) return cudaSuccess;
+  const int EP = ((c.E + 15) / 16) * 16;
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, (uint64_t)c.T, (uint64_t)c.d, false, RM) ||
+      !make_map(&mw, wg, (uint64_t)c.E, (uint64_t)c.d, false, (uint32_t)EP))
+    return cudaErrorInvalidValue;
+#define MOE_ROUTE_K(K) \
+  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, s)
+  switch (c.k) {
+    MOE_ROUTE_K(1); MOE_ROUTE_K(2); MOE_ROUTE_K(3); MOE_ROUTE_K(4);
+    MOE_ROUTE_K(5); MOE_ROUTE_K(6); MOE_ROUTE_K(7); MOE_ROUTE_K(8);
+    default: return cudaErrorInvalidValue;
+  }
+#undef MOE_ROUTE_K
+}
+
+}  // namespace moe

@@ -245,3 +245,25 @@ def test_convert_bf16_to_f16_matches_numpy():
     # every value in [2^-17, 65504] survives exactly
     exact = (np.abs(f) >= 2.0 ** -17) & (np.abs(f) <= 65504)
     assert np.array_equal(got[exact].astype(np.float32), f[exact])
+
+
+@pytest.mark.parametrize("dtype", [mw.BF16, mw.F32])
+@pytest.mark.parametrize("case", ["negative", "decreasing", "past_buffer"])
+def test_expert_ffn_rejects_corrupt_offsets(dtype, case):
+    """offsets[] that are not a non-decreasing sequence inside [0, T*k] make the
+    grouped GEMMs schedule no tile: nothing is written and MOE_DEV_BOUNDS is set."""
+    w = W("corrupt", T=200, d=64, E=4, F=64, k=2, act=mw.SWIGLU, dtype=dtype, seed=5)
+    L = DeviceLayer(w)
+    A = L.T * w.k
+    off = {"negative": [-256, 0, 100, 200, 400], "decreasing": [0, 150, 90, 300, 400],
+           "past_buffer": [0, 100, 200, 300, A + 128]}[case]
+    xp = torch.zeros((A, w.d), dtype=L.tdt, device="cuda")
+    h0 = torch.full((A, w.F), 7.0, dtype=L.hdt, device="cuda")
+    yp0 = torch.full((A, w.d), 7.0, dtype=torch.float32, device="cuda")
+    h, yp = h0.clone(), yp0.clone()
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
+    moe.moe_expert_ffn(L.cfg, xp, torch.tensor(off, dtype=torch.int32, device="cuda"), L.w1, L.w2, h, yp, stats,
+                       L.scratch())
+    torch.cuda.synchronize()
+    assert moe.read_stats(stats)["status"] & moe.MOE_DEV_BOUNDS
+    assert torch.equal(h, h0) and torch.equal(yp, yp0)
