@@ -55,10 +55,12 @@ inline int num_stages(int EP) { return std::min(kMaxStages, kRingBytes / stage_b
 inline size_t smem_bytes(int EP) { return 1024 + (size_t)num_stages(EP) * stage_bytes(EP) + sizeof(RTail); }
 __host__ __device__ constexpr uint32_t tmem_cols(int EP) { return EP <= 32 ? 32 : EP <= 64 ? 64 : EP <= 128 ? 128 : 256; }
 
-// Keeps the n <= KB + 1 best (score, expert) pairs, best first, in registers
+// Keeps the N <= KB + 1 best (score, expert) pairs, best first, in registers
 // (every index is a compile-time constant).  Pairs arrive in ascending expert
 // order, so a new pair goes behind every kept pair whose score is >= its own:
-// equal scores stay in ascending index order.
+// equal scores stay in ascending index order.  Empty slots hold -inf, so a
+// NaN or -inf score is never kept.  The insertion is branch-free: slot j only
+// looks at the old contents of slots j - 1 and j.
 template <int KB>
 struct TopList {
   static constexpr int kEmpty = 0x7fffffff;
@@ -68,20 +70,40 @@ struct TopList {
 #pragma unroll
     for (int j = 0; j <= KB; ++j) { v[j] = -INFINITY; i[j] = kEmpty; }
   }
-  __device__ __forceinline__ void insert(float s, int e, int n) {
-    int pos = 0;   // kept pairs that stay ahead (a prefix of the sorted list)
+  template <int N>
+  __device__ __forceinline__ void insert(float s, int e) {
 #pragma unroll
-    for (int j = 0; j <= KB; ++j)
-      if (j < n && i[j] != kEmpty && !(s > v[j])) pos = j + 1;
-    if (pos >= n) return;
-#pragma unroll
-    for (int j = KB; j >= 1; --j)
-      if (j < n && j > pos) { v[j] = v[j - 1]; i[j] = i[j - 1]; }
-#pragma unroll
-    for (int j = 0; j <= KB; ++j)
-      if (j == pos) { v[j] = s; i[j] = e; }
+    for (int j = N - 1; j >= 1; --j) {
+      const bool up = s > v[j - 1];            // s ranks above slot j - 1: slot j takes j - 1
+      const bool here = !up && s > v[j];       // s lands in slot j
+      v[j] = up ? v[j - 1] : (here ? s : v[j]);
+      i[j] = up ? i[j - 1] : (here ? e : i[j]);
+    }
+    const bool top = s > v[0];
+    v[0] = top ? s : v[0];
+    i[0] = top ? e : i[0];
   }
 };
+
+// Top-N over the scores Z[lo, hi) of one row (and their maximum), then, for
+// the lower half, the upper half's list merged in: its experts all have higher
+// indices, so inserting them (best first) keeps lowest-index-wins order.
+template <int N, int KB>
+__device__ __forceinline__ float topk_range(TopList<KB>& top, const float* Z, int lo, int hi) {
+  float mh = -INFINITY;
+#pragma unroll 4
+  for (int e = lo; e < hi; ++e) {
+    const float sc = Z[e];
+    mh = fmaxf(mh, sc);
+    top.template insert<N>(sc, e);
+  }
+  return mh;
+}
+template <int N, int KB>
+__device__ __forceinline__ void topk_merge(TopList<KB>& top, const float (*lv)[RM], const int (*li)[RM], int row) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) top.template insert<N>(lv[j][row], li[j][row]);
+}
 
 // Score the top-k is taken on: the biased logit, or its normalised value.
 __device__ __forceinline__ float gate_score(float zb, float lam, float mu, float sd) {
@@ -232,16 +254,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll 4
     for (int e = lo; e < hi; ++e) Z[e] = gate_score(Z[e], lam, mu, sd);
   }
-  const int nkeep = (k < E) ? k + 1 : k;
+  // the (k+1)-th score is only needed for the gap, which does not exist when k == E
   TopList<KB> top;
   top.init();
-  float mh = -INFINITY;
-#pragma unroll 4
-  for (int e = lo; e < hi; ++e) {
-    const float sc = Z[e];
-    mh = fmaxf(mh, sc);
-    top.insert(sc, e, nkeep);
-  }
+  const float mh = (k < E) ? topk_range<KB + 1>(top, Z, lo, hi) : topk_range<KB>(top, Z, lo, hi);
   part[half][2][row] = mh;
   if (half == 1) {
 #pragma unroll
@@ -254,19 +270,18 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   const float m = fmaxf(part[0][2][row], part[1][2][row]);
   float Sh = 0.f;
 #pragma unroll 4
-  for (int e = lo; e < hi; ++e) Sh += __expf(Z[e] - m);
+  for (int e = lo; e < hi; ++e) {   // unnormalised probabilities over the scores
+    const float pe = __expf(Z[e] - m);
+    Z[e] = pe;
+    Sh += pe;
+  }
   part[half][3][row] = Sh;
   __syncthreads();
   const float S = part[0][3][row] + part[1][3][row];
   const float invS = 1.f / S;
   if (half == 0) {
-    // merge: the upper half's experts all have higher indices, so inserting
-    // its list (best first) keeps the lowest-index-wins order on equal scores
-#pragma unroll
-    for (int j = 0; j <= KB; ++j) {
-      const int ie = tail->li[j][row];
-      if (ie != TopList<KB>::kEmpty) top.insert(tail->lv[j][row], ie, nkeep);
-    }
+    if (k < E) topk_merge<KB + 1>(top, tail->lv, tail->li, row);
+    else topk_merge<KB>(top, tail->lv, tail->li, row);
     float psel[KB], sel = 0.f;
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
@@ -287,15 +302,27 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     }
   }
 
-  // per-expert probability sums of the chunk: probabilities over the scores
-  // in shared memory, then one thread per expert adds its column in row order
+  // per-expert probability sums of the chunk: the probabilities of each row in
+  // shared memory, columns summed by nG groups of threads over row ranges, the
+  // group partials added in group order (fixed order, deterministic)
 #pragma unroll 4
-  for (int e = lo; e < hi; ++e) Z[e] = valid ? __expf(Z[e] - m) * invS : 0.f;
+  for (int e = lo; e < hi; ++e) Z[e] = valid ? Z[e] * invS : 0.f;
   tc_fence_before();
+  __syncthreads();
+  float* colpart = &part[0][0][0];               // [nG][E]; part is free again
+  const int nG = kThreads / E;                   // >= 1 since E <= 256 = kThreads
+  const int R = (RM + nG - 1) / nG;
+  if (tid < nG * E) {
+    const int e = tid % E, g = tid / E;
+    float s = 0.f;
+    const int r1 = min(RM, (g + 1) * R);
+    for (int rr = g * R; rr < r1; ++rr) s += Zall[(size_t)rr * ldz + e];
+    colpart[g * E + e] = s;
+  }
   __syncthreads();
   for (int e = tid; e < E; e += kThreads) {
     float s = 0.f;
-    for (int rr = 0; rr < RM; ++rr) s += Zall[(size_t)rr * ldz + e];
+    for (int g = 0; g < nG; ++g) s += colpart[g * E + e];
     psum_out[(size_t)chunk * E + e] = s;
     hist_out[(size_t)e * nch + chunk] = tail->hist[e];
   }
