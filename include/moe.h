@@ -232,6 +232,34 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
  */
 moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_stream_t stream);
 
+/* Size of the library's fixed device scratch array used by moe_permute_static. */
+#define MOE_STATIC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * moe_permute without a caller workspace: the same kernels and results, with
+ * their scratch (per-chunk histograms, chunk offsets, near-tie counts) in one
+ * fixed device array of MOE_STATIC_SCRATCH_BYTES bytes that the library owns,
+ * one per device.  It allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.  No counterpart on the pages: it is a calling
+ * convention for users that cannot hand out device memory.
+ *   Arguments, layout, ownership and results: as moe_permute, minus ws.
+ *   Limit: moe_scratch_size(cfg) <= MOE_STATIC_SCRATCH_BYTES, else
+ *     MOE_ERR_UNSUPPORTED before any device work (e.g. E = 64 experts allows
+ *     T up to about 347k tokens).
+ *   The first call on a device looks up the array's address (that device
+ *     must be current) and returns MOE_ERR_CUDA if the lookup fails.
+ *   Every scratch word the kernels read is written earlier in the same call;
+ *     the one value that must start at zero, stats->status, is cleared by the
+ *     call on `stream`.
+ *   Calls that overlap in time on one device (several streams or host
+ *     threads) share the array and race: the caller must serialise them.
+ */
+moe_status moe_permute_static(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                              const float* gap, const float* prob_mean,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                              moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

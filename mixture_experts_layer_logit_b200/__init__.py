@@ -19,7 +19,8 @@ from typing import Optional
 __all__ = [
     "LIB_PATH", "MoeError", "moe_config", "moe_stats", "moe_ws_layout", "lib", "make_config",
     "moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route", "moe_permute",
-    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "prepare_w2",
+    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "moe_permute_static",
+    "MOE_STATIC_SCRATCH_BYTES", "prepare_w2",
     "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
     "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
@@ -33,7 +34,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE
 
 EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route",
                     "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-                    "moe_convert_bf16_to_f16"]
+                    "moe_convert_bf16_to_f16", "moe_permute_static"]
+MOE_STATIC_SCRATCH_BYTES = 2 << 20
 
 
 class moe_config(ctypes.Structure):
@@ -87,8 +89,9 @@ def lib() -> ctypes.CDLL:
     L.moe_combine.argtypes = [cfgp, P, P, P, P, P]
     L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_convert_bf16_to_f16.argtypes = [P, P, ctypes.c_size_t, P]
+    L.moe_permute_static.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P]
     for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-              "moe_convert_bf16_to_f16"]:
+              "moe_convert_bf16_to_f16", "moe_permute_static"]:
         getattr(L, n).restype = st
     _lib = L
     return L
@@ -161,6 +164,16 @@ def moe_permute(cfg, x, topk_idx, gap, prob_mean, counts, kept, offsets, row_of,
                                             _ptr(prob_mean), _ptr(counts), _ptr(kept), _ptr(offsets),
                                             _ptr(row_of), _ptr(src_tok), _ptr(xp), _ptr(stats), _ptr(ws),
                                             _nbytes(ws), _stream(stream)))
+
+
+def moe_permute_static(cfg, x, topk_idx, gap, prob_mean, counts, kept, offsets, row_of, src_tok, xp, stats,
+                       stream=None):
+    """moe_permute with its scratch in the library's fixed device array (no
+    workspace argument; calls that overlap in time race on that array)."""
+    _check("moe_permute_static", lib().moe_permute_static(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(gap),
+                                                          _ptr(prob_mean), _ptr(counts), _ptr(kept),
+                                                          _ptr(offsets), _ptr(row_of), _ptr(src_tok), _ptr(xp),
+                                                          _ptr(stats), _stream(stream)))
 
 
 def moe_expert_ffn(cfg, xp, offsets, W1, W2, h, yp, stats, ws, stream=None):

@@ -295,4 +295,35 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));
 }
 
+moe_status moe_permute_static(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                              const float* gap, const float* prob_mean,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                              moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (counts == nullptr || kept == nullptr || offsets == nullptr || stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (x == nullptr || topk_idx == nullptr || row_of == nullptr || src_tok == nullptr || xp == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(xp) || !aligned4(topk_idx) || !aligned4(gap) || !aligned4(prob_mean) ||
+      !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) || !aligned4(row_of) || !aligned4(src_tok) ||
+      !aligned4(stats))
+    return MOE_ERR_ARG;
+  const Scratch sc = scratch_layout(c);
+  if (sc.total > (size_t)MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;   // beyond the fixed array
+  if ((st = check_device(false)) != MOE_OK) return st;
+  void* ws = nullptr;
+  if (static_scratch_address(&ws) != cudaSuccess) return MOE_ERR_CUDA;
+  // the kernels of moe_permute, in the same order, on the library's array
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = launch_hist(c, topk_idx, gap, at<int32_t>(ws, sc.hist), at<int32_t>(ws, sc.ntie),
+                              &stats->status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return permute_from_hist(c, x, topk_idx, prob_mean, nullptr,
+                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, counts, kept,
+                           offsets, row_of, src_tok, xp, stats, sc, ws, s);
+}
+
 }  // extern "C"

@@ -80,6 +80,10 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// Address of the library's fixed scratch array (MOE_STATIC_SCRATCH_BYTES) on
+// the current device; looked up once per device.
+cudaError_t static_scratch_address(void** out);
+
 // ------------------------------------------------------------ device helpers
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
