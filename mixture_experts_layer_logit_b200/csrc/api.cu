@@ -133,13 +133,9 @@ moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* 
                              int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                              int32_t* src_tok, void* xp, moe_stats* stats, const Scratch& sc, void* ws,
                              cudaStream_t s) {
-  const int cap = capacity_of(c);
-  cudaError_t e = launch_scan(c, cap, at<int32_t>(ws, sc.hist), at<int32_t>(ws, sc.choff), prob_mean, psum,
-                              ntie, counts, kept, offsets, stats, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_scatter(c, cap, x, topk_idx, at<int32_t>(ws, sc.choff), offsets, row_of, src_tok, xp,
-                     &stats->status, s);
-  return cuda_status(e);
+  return cuda_status(launch_permute(c, capacity_of(c), x, topk_idx, at<int32_t>(ws, sc.hist),
+                                    at<int32_t>(ws, sc.choff), prob_mean, psum, ntie, counts, kept, offsets,
+                                    row_of, src_tok, xp, stats, s));
 }
 
 moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,

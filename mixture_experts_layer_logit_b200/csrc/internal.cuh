@@ -50,16 +50,15 @@ cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob
 // Histogram of topk_idx per chunk (+ near ties from gap when given).
 cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const float* gap,
                         int32_t* hist, int32_t* ntie, uint32_t* status, cudaStream_t s);
-// Scan: counts, kept, offsets, per-chunk offsets, stats.  Either prob_mean
-// (standalone) or psum (fused forward) or neither supplies P_e for the aux loss.
-cudaError_t launch_scan(const moe_config& c, int capacity, const int32_t* hist, int32_t* choff,
-                        const float* prob_mean, const float* psum, const int32_t* ntie,
-                        int32_t* counts, int32_t* kept, int32_t* offsets, moe_stats* stats,
-                        cudaStream_t s);
-// Stable ranks, capacity test, row_of/src_tok, and the gather xp[row] = x[t].
-cudaError_t launch_scatter(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
-                           const int32_t* choff, const int32_t* offsets, int32_t* row_of,
-                           int32_t* src_tok, void* xp, uint32_t* status, cudaStream_t s);
+// Step 3 after the histograms: counts, kept, offsets, statistics, stable
+// ranks, the capacity test, row_of/src_tok and the gather xp[row] = x[t].
+// Either prob_mean (standalone) or psum (fused forward) or neither supplies
+// P_e for the aux loss; choff is scratch for the chunk offsets when the scan
+// runs as its own kernel.
+cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
+                           const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
+                           const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
+                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s);
 // Expert FFN on CUDA cores (fp32 path).
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
                                    const void* w1, const void* w2, void* h, void* yp, uint32_t* status,

@@ -17,6 +17,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 namespace moe {
 namespace {
 
@@ -53,6 +55,123 @@ hist_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ gap,
 // --------------------------------------------------------------------- scan
 constexpr int kScanThreads = 1024;
 
+// Expert totals of one warp's experts: the total over all chunks and the
+// prefix over the chunks before `chunk` (hist is expert-major, so a warp reads
+// each expert's chunk counts coalesced; four 32-chunk loads are in flight at
+// once).  P_e (aux loss input) and the chunk offsets are optional.
+__device__ __forceinline__ void expert_totals(const int32_t* __restrict__ hist, int e, int nch, int chunk,
+                                              int32_t* __restrict__ choff, int lane, int* total, int* prefix) {
+  constexpr int kBatch = 4;
+  int running = 0, pre = 0;
+  const int32_t* hrow = hist + (size_t)e * nch;
+  for (int c0 = 0; c0 < nch; c0 += 32 * kBatch) {
+    int v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int c = c0 + 32 * b + lane;
+      v[b] = (c < nch) ? hrow[c] : 0;
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int c = c0 + 32 * b + lane;
+      int incl = v[b];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (choff != nullptr && c < nch) choff[(size_t)e * nch + c] = running + incl - v[b];
+      if (c < chunk) pre += v[b];
+      running += __shfl_sync(kFull, incl, 31);
+    }
+  }
+  *total = running;
+  *prefix = warp_sum(pre);
+}
+
+__device__ __forceinline__ float expert_prob_mean(const float* __restrict__ prob_mean, const float* __restrict__ psum,
+                                                  int e, int E, int nch, int T, int lane) {
+  if (prob_mean != nullptr) return prob_mean[e];
+  if (psum == nullptr) return NAN;
+  float s = 0.f;
+#pragma unroll 4
+  for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
+  return warp_sum(s) / (float)T;
+}
+
+__device__ __forceinline__ int chunk_ties(const int32_t* __restrict__ ntie, int nch, int lane) {
+  int s = 0;
+  if (ntie != nullptr)
+    for (int c = lane; c < nch; c += 32) s += ntie[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+  return (ntie != nullptr) ? s : -1;
+}
+
+// One warp: kept = min(count, C) (all in dropless mode), offsets = exclusive
+// scan of kept over the experts (8 experts per lane), the drop count and the
+// Switch aux loss E * sum_e (count_e / (T k)) * P_e in double.  Writes the
+// offsets to s_off when given and the global results when `out` is set.
+__device__ __forceinline__ void expert_offsets(const int* s_counts, const float* s_p, int s_ntie, int E, int T,
+                                               int k, int capacity, int* s_off, bool out, int32_t* counts,
+                                               int32_t* kept, int32_t* offsets, moe_stats* stats, int lane) {
+  constexpr int PER = kMaxExperts / 32;
+  int kv[PER];
+  int local = 0, drop = 0;
+  double aux = 0.0;
+  const double A = (double)T * (double)k;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    int cnt = 0, kp = 0;
+    if (e < E) {
+      cnt = s_counts[e];
+      kp = (capacity < 0) ? cnt : min(cnt, capacity);
+      if (out) aux += ((double)cnt / A) * (double)s_p[e];
+    }
+    kv[i] = kp;
+    local += kp;
+    drop += cnt - kp;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += u;
+  }
+  int run = incl - local;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    if (e < E) {
+      if (s_off != nullptr) s_off[e] = run;
+      if (out) {
+        offsets[e] = run;
+        counts[e] = s_counts[e];
+        kept[e] = kv[i];
+      }
+    }
+    run += kv[i];
+  }
+  if (!out) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    drop += __shfl_xor_sync(kFull, drop, o);
+    aux += __shfl_xor_sync(kFull, aux, o);
+  }
+  const int total = __shfl_sync(kFull, incl, 31);
+  if (lane == 0) {
+    offsets[E] = total;
+    stats->drop_count = drop;
+    stats->rows_kept = total;
+    stats->capacity = capacity;
+    stats->near_tie_count = s_ntie;
+    stats->drop_rate = (T > 0) ? (float)((double)drop / A) : 0.f;
+    stats->aux_loss = (T > 0) ? (float)((double)E * aux) : NAN;
+  }
+}
+
+// Standalone scan (one CTA): chunk offsets for the scatter, and the results.
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int nch, int T, int E, int k,
             int capacity, const float* __restrict__ prob_mean, const float* __restrict__ psum,
@@ -65,112 +184,22 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
   const int nwarps = kScanThreads / 32;
   pdl_wait();
   pdl_launch_dependents();
-
-  // per-expert exclusive scan over chunks (expert-major hist, coalesced); the
-  // loads of four 32-chunk groups are issued before any of them is scanned
-  constexpr int kBatch = 4;
   for (int e = warp; e < E; e += nwarps) {
-    int running = 0;
-    const int32_t* hrow = hist + (size_t)e * nch;
-    for (int c0 = 0; c0 < nch; c0 += 32 * kBatch) {
-      int v[kBatch];
-#pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int c = c0 + 32 * b + lane;
-        v[b] = (c < nch) ? hrow[c] : 0;
-      }
-#pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int c = c0 + 32 * b + lane;
-        int incl = v[b];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int u = __shfl_up_sync(kFull, incl, o);
-          if (lane >= o) incl += u;
-        }
-        if (c < nch) choff[(size_t)e * nch + c] = running + incl - v[b];
-        running += __shfl_sync(kFull, incl, 31);
-      }
-    }
-    // P_e for the aux loss
-    float P = NAN;
-    if (prob_mean != nullptr) {
-      P = prob_mean[e];
-    } else if (psum != nullptr) {
-      float s = 0.f;
-#pragma unroll 4
-      for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
-      P = warp_sum(s) / (float)T;
-    }
-    if (lane == 0) { s_counts[e] = running; s_p[e] = P; }
+    int tot, pre;
+    expert_totals(hist, e, nch, 0, choff, lane, &tot, &pre);
+    const float P = expert_prob_mean(prob_mean, psum, e, E, nch, T, lane);
+    if (lane == 0) { s_counts[e] = tot; s_p[e] = P; }
   }
   if (warp == nwarps - 1) {
-    int s = 0;
-    if (ntie != nullptr)
-      for (int c = lane; c < nch; c += 32) s += ntie[c];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-    if (lane == 0) s_ntie = (ntie != nullptr) ? s : -1;
+    const int nt = chunk_ties(ntie, nch, lane);
+    if (lane == 0) s_ntie = nt;
   }
   __syncthreads();
-
-  // offsets = exclusive scan of kept over experts (one warp, 8 experts per lane)
-  if (warp == 0) {
-    constexpr int PER = kMaxExperts / 32;
-    int kv[PER];
-    int local = 0, drop = 0;
-    double aux = 0.0;
-    const double A = (double)T * (double)k;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = lane * PER + i;
-      int cnt = 0, kp = 0;
-      if (e < E) {
-        cnt = s_counts[e];
-        kp = (capacity < 0) ? cnt : min(cnt, capacity);
-        aux += ((double)cnt / A) * (double)s_p[e];
-      }
-      kv[i] = kp;
-      local += kp;
-      drop += cnt - kp;
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += u;
-    }
-    int run = incl - local;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = lane * PER + i;
-      if (e < E) {
-        offsets[e] = run;
-        counts[e] = s_counts[e];
-        kept[e] = kv[i];
-      }
-      run += kv[i];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      drop += __shfl_xor_sync(kFull, drop, o);
-      aux += __shfl_xor_sync(kFull, aux, o);
-    }
-    const int total = __shfl_sync(kFull, incl, 31);
-    if (lane == 0) {
-      offsets[E] = total;
-      stats->drop_count = drop;
-      stats->rows_kept = total;
-      stats->capacity = capacity;
-      stats->near_tie_count = s_ntie;
-      stats->drop_rate = (T > 0) ? (float)((double)drop / A) : 0.f;
-      stats->aux_loss = (T > 0) ? (float)((double)E * aux) : NAN;
-    }
-  }
+  if (warp == 0) expert_offsets(s_counts, s_p, s_ntie, E, T, k, capacity, nullptr, true, counts, kept, offsets, stats, lane);
 }
 
 // ------------------------------------------------------------------ scatter
-constexpr int kScatterThreads = 512;   // 4 rank warps, then 16 warps copying rows
+constexpr int kScatterThreads = 512;   // 4 rank warps, then all 16 warps copy
 
 template <typename TX>
 __device__ __forceinline__ void copy_rows(const TX* __restrict__ x, TX* __restrict__ xp, int d,
@@ -186,26 +215,74 @@ __device__ __forceinline__ void copy_rows(const TX* __restrict__ x, TX* __restri
   }
 }
 
+struct ScatterArgs {
+  const int32_t* topk_idx;
+  const int32_t* hist;        // FUSED: per-chunk histograms [E][nch]
+  int32_t* choff;             // separate scan: chunk offsets [E][nch]
+  const float* prob_mean;     // FUSED, lead block: P_e given, or
+  const float* psum;          //   summed from the per-chunk probability sums
+  const int32_t* ntie;
+  int32_t* counts;
+  int32_t* kept;
+  int32_t* offsets;           // read (separate scan) or written by the lead block (FUSED)
+  moe_stats* stats;
+  int32_t* row_of;
+  int32_t* src_tok;
+  int T, d, E, k, nch, capacity;
+  int slice_vec;              // 16-byte vectors of a row per column slice (gridDim.y slices)
+};
+
 // Ranks with warp ballots (k <= KB <= 8).  Lane l of rank warp w owns token
-// t = chunk*64 + 32 w + l.  For each slot j' the 9 ballots of the bits of the
-// slot-j' expert ids let every lane count, for each of its own experts e, the
-// lanes below it that also chose e (in any slot): that count is the rank of
-// (t, e) inside the warp.  Expert ids are < 256, so bit 8 marks "no expert".
-template <int KB, typename TX>
+// t = chunk*128 + 32 w + l.  For each slot j' the 9 ballots of the bits of
+// the slot-j' expert ids let every lane count, for each of its own experts e,
+// the lanes below it that also chose e (in any slot): that count is the rank
+// of (t, e) inside the warp.  Expert ids are < 256, so bit 8 marks "no expert".
+//
+// FUSED: the block first derives its chunk's offsets from the histograms
+// itself (every block reads all E x nch counts from L2 and scans them), so no
+// separate scan kernel runs; block (0, 0) also writes counts, kept, offsets
+// and the statistics.  The grid's y dimension splits each token row into
+// column slices, so that layers with few chunks and wide rows still spread
+// the gather over all SMs; the ranks are recomputed by every slice.
+template <int KB, typename TX, bool FUSED>
 __global__ void __launch_bounds__(kScatterThreads)
-scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
-               const int32_t* __restrict__ choff, const int32_t* __restrict__ offsets,
-               int T, int d, int E, int k, int nch, int capacity,
-               int32_t* __restrict__ row_of, int32_t* __restrict__ src_tok, TX* __restrict__ xp) {
+scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs a) {
   constexpr int kRankWarps = kChunk / 32;
-  static_assert(kRankWarps <= kScatterThreads / 32, "one rank warp per 32 tokens of a chunk");
+  constexpr int kWarps = kScatterThreads / 32;
+  static_assert(kRankWarps <= kWarps, "one rank warp per 32 tokens of a chunk");
   __shared__ int wcnt[kRankWarps][kMaxExperts];
   __shared__ int rows_sm[kChunk][KB];
+  __shared__ int s_pre[kMaxExperts], s_off[kMaxExperts], s_counts[kMaxExperts];
+  __shared__ float s_p[kMaxExperts];
+  __shared__ int s_ntie;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
+  const bool lead = FUSED && chunk == 0 && blockIdx.y == 0;
+  const int E = a.E, k = a.k, T = a.T;
   for (int i = threadIdx.x; i < kRankWarps * kMaxExperts; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
   pdl_wait();
   pdl_launch_dependents();
+  if (FUSED) {
+    for (int e = warp; e < E; e += kWarps) {
+      int tot, pre;
+      expert_totals(a.hist, e, a.nch, chunk, nullptr, lane, &tot, &pre);
+      const float P = lead ? expert_prob_mean(a.prob_mean, a.psum, e, E, a.nch, T, lane) : 0.f;
+      if (lane == 0) { s_counts[e] = tot; s_pre[e] = pre; s_p[e] = P; }
+    }
+    if (lead && warp == kWarps - 1) {
+      const int nt = chunk_ties(a.ntie, a.nch, lane);
+      if (lane == 0) s_ntie = nt;
+    }
+    __syncthreads();
+    if (warp == 0)
+      expert_offsets(s_counts, s_p, s_ntie, E, T, k, a.capacity, s_off, lead, a.counts, a.kept, a.offsets,
+                     a.stats, lane);
+  } else {
+    for (int e = threadIdx.x; e < E; e += kScatterThreads) {
+      s_pre[e] = a.choff[(size_t)e * a.nch + chunk];
+      s_off[e] = a.offsets[e];
+    }
+  }
   __syncthreads();
 
   int val[KB], rank_w[KB];
@@ -216,7 +293,7 @@ scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
     for (int j = 0; j < KB; ++j) {
       int e = 0x1ff;
       if (tv && j < k) {
-        e = topk_idx[(size_t)t * k + j];
+        e = a.topk_idx[(size_t)t * k + j];
         if (e < 0 || e >= E) e = 0x1ff;
       }
       val[j] = e;
@@ -248,6 +325,7 @@ scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
   }
   __syncthreads();
   if (warp < kRankWarps) {
+    const bool writer = blockIdx.y == 0;   // one slice writes the index outputs
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
       const int e = val[j];
@@ -255,22 +333,47 @@ scatter_kernel(const TX* __restrict__ x, const int32_t* __restrict__ topk_idx,
       if (e < E) {
         int before = 0;   // assignments of expert e in the earlier warps of this chunk
         for (int w = 0; w < warp; ++w) before += wcnt[w][e];
-        const int r = choff[(size_t)e * nch + chunk] + before + rank_w[j];
-        if (capacity < 0 || r < capacity) {
-          row = offsets[e] + r;
-          src_tok[row] = t;
+        const int r = s_pre[e] + before + rank_w[j];
+        if (a.capacity < 0 || r < a.capacity) {
+          row = s_off[e] + r;
+          if (writer) a.src_tok[row] = t;
         }
       }
-      if (t < T && j < k) row_of[(size_t)t * k + j] = row;
+      if (writer && t < T && j < k) a.row_of[(size_t)t * k + j] = row;
       rows_sm[warp * 32 + lane][j] = row;
     }
   }
   __syncthreads();
-  // gather: each warp copies whole token rows to their kept destinations
-  for (int i = warp; i < kChunk; i += kScatterThreads / 32) {
-    const int tt = chunk * kChunk + i;
-    if (tt >= T) break;
-    copy_rows<TX>(x, xp, d, tt, rows_sm[i], k, lane);
+
+  // gather: this block's column slice [v0, v0 + W) of every token row of the
+  // chunk, 16-byte vectors, four loads in flight per thread
+  const int nvec = a.d * (int)sizeof(TX) / 16;
+  const int v0 = blockIdx.y * a.slice_vec;
+  const int W = min(nvec, v0 + a.slice_vec) - v0;
+  const int t0 = chunk * kChunk;
+  const int units = (W > 0) ? min(kChunk, T - t0) * W : 0;
+  for (int u0 = threadIdx.x; u0 < units; u0 += 4 * kScatterThreads) {
+    uint4 v[4];
+    int tok[4], col[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int u = u0 + q * kScatterThreads;
+      tok[q] = -1;
+      if (u < units) {
+        tok[q] = u / W;
+        col[q] = v0 + (u - tok[q] * W);
+        v[q] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok[q]) * a.d) + col[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (tok[q] < 0) continue;
+#pragma unroll
+      for (int j = 0; j < KB; ++j) {
+        const int r = rows_sm[tok[q]][j];
+        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[col[q]] = v[q];
+      }
+    }
   }
 }
 
@@ -316,27 +419,57 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
   }
 }
 
+// Column slices per chunk: enough blocks for about two per SM, each slice at
+// least 32 vectors (512 bytes) of a row.
+inline int scatter_slices(int nch, int nvec, int* slice_vec) {
+  DeviceInfo di;
+  const int sms = (device_info(&di) == cudaSuccess) ? di.sms : 148;
+  int S = (2 * sms + nch - 1) / nch;
+  S = std::max(1, std::min(S, nvec / 32));
+  *slice_vec = (nvec + S - 1) / S;
+  return (nvec + *slice_vec - 1) / *slice_vec;
+}
+
+template <typename TX, bool FUSED>
+cudaError_t launch_scatter_t(const moe_config& c, const TX* x, TX* xp, const ScatterArgs& a, cudaStream_t s) {
+  int slice_vec = 0;
+  const int S = scatter_slices(a.nch, c.d * (int)sizeof(TX) / 16, &slice_vec);
+  ScatterArgs b = a;
+  b.slice_vec = slice_vec;
+  const dim3 g(a.nch, S), blk(kScatterThreads);
+  if (c.k <= 1) return launch_pdl(scatter_kernel<1, TX, FUSED>, g, blk, 0, s, x, xp, b);
+  if (c.k <= 2) return launch_pdl(scatter_kernel<2, TX, FUSED>, g, blk, 0, s, x, xp, b);
+  if (c.k <= 4) return launch_pdl(scatter_kernel<4, TX, FUSED>, g, blk, 0, s, x, xp, b);
+  return launch_pdl(scatter_kernel<8, TX, FUSED>, g, blk, 0, s, x, xp, b);
+}
+
 template <typename TX>
-cudaError_t launch_scatter_t(const moe_config& c, int cap, const void* x, const int32_t* idx,
-                             const int32_t* choff, const int32_t* off, int32_t* row_of,
-                             int32_t* src_tok, void* xp, cudaStream_t s) {
-  const int nch = num_chunks(c.T);
-  const TX* xx = static_cast<const TX*>(x);
-  TX* pp = static_cast<TX*>(xp);
-  const dim3 g(nch), b(kScatterThreads);
-#define MOE_SCATTER(KB) \
-  return launch_pdl(scatter_kernel<KB, TX>, g, b, 0, s, xx, idx, choff, off, c.T, c.d, c.E, c.k, nch, cap, \
-                    row_of, src_tok, pp)
-  if (c.k <= 1) MOE_SCATTER(1);
-  if (c.k <= 2) MOE_SCATTER(2);
-  if (c.k <= 4) MOE_SCATTER(4);
-  if (c.k <= 8) MOE_SCATTER(8);
-#undef MOE_SCATTER
+cudaError_t launch_generic_t(const moe_config& c, const TX* xx, TX* pp, const ScatterArgs& a, cudaStream_t s) {
+  const dim3 g(a.nch), b(kScatterThreads);
   const size_t smem = sizeof(int) * kChunk * (size_t)c.k;
   cudaError_t err = set_smem_once<scatter_generic_kernel<TX>>(sizeof(int) * kChunk * kMaxExperts);
   if (err != cudaSuccess) return err;
-  return launch_pdl(scatter_generic_kernel<TX>, g, b, smem, s, xx, idx, choff, off, c.T, c.d, c.E, c.k, nch, cap,
-                    row_of, src_tok, pp);
+  return launch_pdl(scatter_generic_kernel<TX>, g, b, smem, s, xx, a.topk_idx, a.choff, a.offsets, c.T, c.d, c.E,
+                    c.k, a.nch, a.capacity, a.row_of, a.src_tok, pp);
+}
+
+// The scan is fused into the scatter while the histograms every block reads
+// stay small (64 KB); otherwise, and for k > 8 or no tokens, one scan block
+// runs first and the scatter reads its chunk offsets.
+constexpr long long kFusedHistMax = 16384;
+
+template <typename TX>
+cudaError_t launch_permute_t(const moe_config& c, const void* x, void* xp, ScatterArgs a, cudaStream_t s) {
+  const TX* xx = static_cast<const TX*>(x);
+  TX* pp = static_cast<TX*>(xp);
+  if (c.T > 0 && c.k <= 8 && (long long)c.E * a.nch <= kFusedHistMax)
+    return launch_scatter_t<TX, true>(c, xx, pp, a, s);
+  cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, a.hist, a.choff,
+                             a.nch, c.T, c.E, c.k, a.capacity, a.prob_mean, a.psum, a.ntie, a.counts, a.kept,
+                             a.offsets, a.stats);
+  if (e != cudaSuccess || c.T == 0) return e;
+  if (c.k <= 8) return launch_scatter_t<TX, false>(c, xx, pp, a, s);
+  return launch_generic_t<TX>(c, xx, pp, a, s);
 }
 
 }  // namespace
@@ -348,22 +481,31 @@ cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const floa
                     num_chunks(c.T), hist, gap != nullptr ? ntie : nullptr, status);
 }
 
-cudaError_t launch_scan(const moe_config& c, int capacity, const int32_t* hist, int32_t* choff,
-                        const float* prob_mean, const float* psum, const int32_t* ntie,
-                        int32_t* counts, int32_t* kept, int32_t* offsets, moe_stats* stats,
-                        cudaStream_t s) {
-  return launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, hist, choff, num_chunks(c.T), c.T, c.E, c.k,
-                    capacity, prob_mean, psum, ntie, counts, kept, offsets, stats);
-}
-
-cudaError_t launch_scatter(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
-                           const int32_t* choff, const int32_t* offsets, int32_t* row_of,
-                           int32_t* src_tok, void* xp, uint32_t* status, cudaStream_t s) {
-  (void)status;
-  if (c.T == 0) return cudaSuccess;
-  if (c.dtype == MOE_DTYPE_BF16)
-    return launch_scatter_t<__nv_bfloat16>(c, capacity, x, topk_idx, choff, offsets, row_of, src_tok, xp, s);
-  return launch_scatter_t<float>(c, capacity, x, topk_idx, choff, offsets, row_of, src_tok, xp, s);
+cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
+                           const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
+                           const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
+                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s) {
+  ScatterArgs a{};
+  a.topk_idx = topk_idx;
+  a.hist = hist;
+  a.choff = choff;
+  a.prob_mean = prob_mean;
+  a.psum = psum;
+  a.ntie = ntie;
+  a.counts = counts;
+  a.kept = kept;
+  a.offsets = offsets;
+  a.stats = stats;
+  a.row_of = row_of;
+  a.src_tok = src_tok;
+  a.T = c.T;
+  a.d = c.d;
+  a.E = c.E;
+  a.k = c.k;
+  a.nch = num_chunks(c.T);
+  a.capacity = capacity;
+  if (c.dtype == MOE_DTYPE_BF16) return launch_permute_t<__nv_bfloat16>(c, x, xp, a, s);
+  return launch_permute_t<float>(c, x, xp, a, s);
 }
 
 }  // namespace moe
