@@ -38,7 +38,6 @@ import moe_workloads as mw  # noqa: E402
 METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (GEMM), % HBM BW (permute)"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 6   # route, scan, scatter, grouped GEMM x2, combine
 L2_FLUSH_BYTES = 512 << 20
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "tc_grouped_gemm_fastmoe_txl.md")
 GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc", "gemm_tc.cu")
@@ -69,6 +68,18 @@ def peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def graph_kernel_nodes(graph) -> int:
+    """Kernel nodes of a captured CUDA graph (kept un-instantiated by keep_graph)."""
+    from cuda.bindings import runtime as rt
+    g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(g, 0)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    err, nodes, n = rt.cudaGraphGetNodes(g, n)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
 
 
 def workload_config(w: mw.Workload, n_gpus: int, graph: bool):
@@ -310,12 +321,16 @@ def main():
 
     fwd()
     torch.cuda.synchronize()
-    graph = None
+    # one step captured as a CUDA graph; its kernel nodes are the launches of a step
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(graph):
+        fwd()
+    launches_per_step = graph_kernel_nodes(graph)
     run = fwd
-    if not a.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            fwd()
+    if a.no_graph:
+        graph.reset()
+        graph = None
+    else:
         run = graph.replay
 
     def timed(fn, steps, flush_between=True):
@@ -451,7 +466,7 @@ def main():
                 "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == mw.BF16 else "f32", "data": "synthetic",
                 "config": workload_config(w, world, graph is not None),
-                "gpu_launches": LAUNCHES_PER_STEP * a.steps,
+                "gpu_launches": launches_per_step * a.steps,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "breakdown_ms": breakdown,
                 "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "rows_kept": st["rows_kept"],

@@ -121,9 +121,12 @@ typedef struct moe_stats {
 } moe_stats;
 
 /* Byte offsets of the intermediates inside a moe_layer_forward workspace
- * (each 256-byte aligned), so that a caller can read them after a forward. */
+ * (each 256-byte aligned), so that a caller can read them after a forward.
+ * row_w[A] fp32 holds the gate weight of each kept permuted row.  On the bf16
+ * path with k <= 2 the forward fuses step 5 into the second expert GEMM: it
+ * writes row_w and leaves yp unwritten; otherwise it writes yp and not row_w. */
 typedef struct moe_ws_layout {
-  size_t topk_idx, topk_w, gap, counts, kept, offsets, row_of, src_tok;
+  size_t topk_idx, topk_w, gap, counts, kept, offsets, row_of, src_tok, row_w;
   size_t xp, h, yp, scratch, total;
 } moe_ws_layout;
 

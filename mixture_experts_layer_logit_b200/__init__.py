@@ -53,7 +53,7 @@ class moe_stats(ctypes.Structure):
 
 class moe_ws_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ["topk_idx", "topk_w", "gap", "counts", "kept", "offsets", "row_of", "src_tok",
+                ["topk_idx", "topk_w", "gap", "counts", "kept", "offsets", "row_of", "src_tok", "row_w",
                  "xp", "h", "yp", "scratch", "total"]]
 
 

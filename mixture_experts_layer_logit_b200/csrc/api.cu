@@ -116,6 +116,7 @@ moe_ws_layout layout_of(const moe_config& c) {
   L.offsets = off;   off = align256(off + 4 * (E + 1));
   L.row_of = off;    off = align256(off + 4 * A);
   L.src_tok = off;   off = align256(off + 4 * A);
+  L.row_w = off;     off = align256(off + 4 * A);
   L.xp = off;        off = align256(off + es * A * (size_t)c.d);
   L.h = off;         off = align256(off + es * A * (size_t)c.F);
   L.yp = off;        off = align256(off + 4 * A * (size_t)c.d);   // fp32 for both element types
@@ -132,18 +133,33 @@ moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* 
                              const float* prob_mean, const float* psum, const int32_t* ntie,
                              int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                              int32_t* src_tok, void* xp, moe_stats* stats, const Scratch& sc, void* ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, const float* topk_w = nullptr, float* row_w = nullptr,
+                             float* out = nullptr) {
   return cuda_status(launch_permute(c, capacity_of(c), x, topk_idx, at<int32_t>(ws, sc.hist),
                                     at<int32_t>(ws, sc.choff), prob_mean, psum, ntie, counts, kept, offsets,
-                                    row_of, src_tok, xp, stats, s));
+                                    row_of, src_tok, xp, stats, s, topk_w, row_w, out));
 }
 
+// Mean assignments per expert from which the expert GEMMs use 2-SM tiles.
+constexpr long long kPairRowsPerExpert = 512;
+
 moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
-                      const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s) {
-  if (c.dtype == MOE_DTYPE_BF16)
-    return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
+                      const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s,
+                      const CombineOut* comb = nullptr) {
+  if (c.dtype == MOE_DTYPE_BF16) {
+    // 2-SM pair tiles (256 rows) pay off once the expert segments hold a few
+    // hundred rows on average; short segments waste half a pair tile.
+    if ((long long)c.T * c.k >= (long long)kPairRowsPerExpert * c.E)
+      return cuda_status(launch_expert_ffn_tc_pair(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
+    return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
+  }
   return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
 }
+
+// The forward fuses step 5 into the second expert GEMM when a token has at
+// most two expert outputs to add (then the sum does not depend on the order
+// the additions arrive in) and the tensor-core path runs.
+bool fused_combine(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.k <= 2 && c.T > 0; }
 
 }  // namespace
 
@@ -281,11 +297,20 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
                                at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const bool fuse = fused_combine(c);
+  float* row_w = at<float>(ws, L.row_w);
+  float* out_f = static_cast<float*>(out);
   st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
                          c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, at<int32_t>(ws, L.counts),
                          at<int32_t>(ws, L.kept), offsets, row_of, at<int32_t>(ws, L.src_tok),
-                         at<char>(ws, L.xp), stats, sc, scr, s);
+                         at<char>(ws, L.xp), stats, sc, scr, s, fuse ? w : nullptr, fuse ? row_w : nullptr,
+                         fuse ? out_f : nullptr);
   if (st != MOE_OK) return st;
+  if (fuse) {
+    // steps 4-5: the second GEMM adds the gate-weighted expert outputs into out
+    const CombineOut comb{at<int32_t>(ws, L.src_tok), row_w, out_f, c.T};
+    return expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s, &comb);
+  }
   st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));

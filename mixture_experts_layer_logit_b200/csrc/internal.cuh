@@ -54,19 +54,34 @@ cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const floa
 // ranks, the capacity test, row_of/src_tok and the gather xp[row] = x[t].
 // Either prob_mean (standalone) or psum (fused forward) or neither supplies
 // P_e for the aux loss; choff is scratch for the chunk offsets when the scan
-// runs as its own kernel.
+// runs as its own kernel.  With row_w and out (fused combine, k <= 8 path):
+// row_w[row] = topk_w of each kept assignment and out is zeroed.
 cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
                            const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
-                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s);
+                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
+                           const float* topk_w = nullptr, float* row_w = nullptr, float* out = nullptr);
 // Expert FFN on CUDA cores (fp32 path).
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
                                    const void* w1, const void* w2, void* h, void* yp, uint32_t* status,
                                    cudaStream_t s);
+// Fused step 5 for the bf16 path with k <= 2: layer 2 adds row_w[row] * y of
+// every permuted row into out[src_tok[row]] (out zeroed beforehand) instead
+// of writing yp.
+struct CombineOut {
+  const int32_t* src_tok;
+  const float* row_w;
+  float* out;
+  int T;
+};
 // Expert FFN on tcgen05 tensor cores (bf16 path).
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
-                                 uint32_t* status, cudaStream_t s);
+                                 uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
+// The same with 2-SM pair tiles (tcgen05.mma.cta_group::2, 256 x 256).
+cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
+                                      const void* w1, const void* w2, void* h, void* yp,
+                                      uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
 // Combine.
 cudaError_t launch_combine(const moe_config& c, const void* yp, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s);

@@ -13,7 +13,7 @@
 //   scatter : one CTA per chunk; stable rank of every assignment inside its
 //             expert from warp ballots, the capacity test, row_of / src_tok,
 //             and the 16-byte-vector gather xp[row] = x[token]
-#include "internal.cuh"
+#include "tc_ptx.cuh"
 
 #include <math.h>
 
@@ -58,7 +58,7 @@ constexpr int kScanThreads = 1024;
 // Expert totals of one warp's experts: the total over all chunks and the
 // prefix over the chunks before `chunk` (hist is expert-major, so a warp reads
 // each expert's chunk counts coalesced; four 32-chunk loads are in flight at
-// once).  P_e (aux loss input) and the chunk offsets are optional.
+// once), and optionally the exclusive chunk offsets.
 __device__ __forceinline__ void expert_totals(const int32_t* __restrict__ hist, int e, int nch, int chunk,
                                               int32_t* __restrict__ choff, int lane, int* total, int* prefix) {
   constexpr int kBatch = 4;
@@ -89,16 +89,6 @@ __device__ __forceinline__ void expert_totals(const int32_t* __restrict__ hist, 
   *prefix = warp_sum(pre);
 }
 
-__device__ __forceinline__ float expert_prob_mean(const float* __restrict__ prob_mean, const float* __restrict__ psum,
-                                                  int e, int E, int nch, int T, int lane) {
-  if (prob_mean != nullptr) return prob_mean[e];
-  if (psum == nullptr) return NAN;
-  float s = 0.f;
-#pragma unroll 4
-  for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
-  return warp_sum(s) / (float)T;
-}
-
 __device__ __forceinline__ int chunk_ties(const int32_t* __restrict__ ntie, int nch, int lane) {
   int s = 0;
   if (ntie != nullptr)
@@ -106,6 +96,52 @@ __device__ __forceinline__ int chunk_ties(const int32_t* __restrict__ ntie, int 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
   return (ntie != nullptr) ? s : -1;
+}
+
+// Expert totals for the whole block at once: thread (e, s), s < 8, sums the
+// counts of chunks c = s, s + 8, ... of expert e (all its loads independent,
+// so one round trip to L2 serves the block), the total and the part before
+// `chunk`; the 8 partials of an expert meet by shuffles in a fixed order.
+// With want_p it also forms P_e the same way from the per-chunk probability
+// sums (or takes prob_mean), so P does not depend on the block size.
+constexpr int kTotGroup = 8;
+
+template <int kBlock>
+__device__ __forceinline__ void block_expert_totals(const int32_t* __restrict__ hist, const float* __restrict__ psum,
+                                                    const float* __restrict__ prob_mean, int E, int nch, int chunk,
+                                                    int T, bool want_p, int* s_counts, int* s_pre, float* s_p) {
+  static_assert(kBlock % 32 == 0, "whole warps");
+  for (int i0 = 0; i0 < E * kTotGroup; i0 += kBlock) {
+    const int idx = i0 + (int)threadIdx.x;
+    const bool active = idx < E * kTotGroup;
+    const int e = idx / kTotGroup, sub = idx % kTotGroup;
+    int tot = 0, pre = 0;
+    float ps = 0.f;
+    if (active) {
+      const int32_t* h = hist + (size_t)e * nch;
+#pragma unroll 8
+      for (int c = sub; c < nch; c += kTotGroup) {
+        const int v = h[c];
+        tot += v;
+        pre += (c < chunk) ? v : 0;
+      }
+      if (want_p && prob_mean == nullptr && psum != nullptr) {
+#pragma unroll 8
+        for (int c = sub; c < nch; c += kTotGroup) ps += psum[(size_t)c * E + e];
+      }
+    }
+#pragma unroll
+    for (int o = kTotGroup / 2; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(kFull, tot, o);
+      pre += __shfl_xor_sync(kFull, pre, o);
+      ps += __shfl_xor_sync(kFull, ps, o);
+    }
+    if (active && sub == 0) {
+      s_counts[e] = tot;
+      if (s_pre != nullptr) s_pre[e] = pre;
+      if (want_p) s_p[e] = (prob_mean != nullptr) ? prob_mean[e] : (psum != nullptr ? ps / (float)T : NAN);
+    }
+  }
 }
 
 // One warp: kept = min(count, C) (all in dropless mode), offsets = exclusive
@@ -184,12 +220,11 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
   const int nwarps = kScanThreads / 32;
   pdl_wait();
   pdl_launch_dependents();
-  for (int e = warp; e < E; e += nwarps) {
+  for (int e = warp; e < E; e += nwarps) {   // chunk offsets for the scatter
     int tot, pre;
     expert_totals(hist, e, nch, 0, choff, lane, &tot, &pre);
-    const float P = expert_prob_mean(prob_mean, psum, e, E, nch, T, lane);
-    if (lane == 0) { s_counts[e] = tot; s_p[e] = P; }
   }
+  block_expert_totals<kScanThreads>(hist, psum, prob_mean, E, nch, 0, T, true, s_counts, nullptr, s_p);
   if (warp == nwarps - 1) {
     const int nt = chunk_ties(ntie, nch, lane);
     if (lane == 0) s_ntie = nt;
@@ -228,6 +263,10 @@ struct ScatterArgs {
   moe_stats* stats;
   int32_t* row_of;
   int32_t* src_tok;
+  const float* topk_w;        // with row_w: the gate weight of each kept row is
+  float* row_w;               //   copied to row_w[row] (fused combine)
+  float* out;                 // fused combine: the layer output, zeroed here
+  uint32_t* status;           // device error bits (a bounded wait that gave up)
   int T, d, E, k, nch, capacity;
   int slice_vec;              // 16-byte vectors of a row per column slice (gridDim.y slices)
 };
@@ -250,6 +289,8 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   constexpr int kRankWarps = kChunk / 32;
   constexpr int kWarps = kScatterThreads / 32;
   static_assert(kRankWarps <= kWarps, "one rank warp per 32 tokens of a chunk");
+  extern __shared__ __align__(128) uint4 xs[];    // [tokens][W]: this block's slice of the chunk's x rows
+  __shared__ __align__(8) unsigned long long xbar;
   __shared__ int wcnt[kRankWarps][kMaxExperts];
   __shared__ int rows_sm[kChunk][KB];
   __shared__ int s_pre[kMaxExperts], s_off[kMaxExperts], s_counts[kMaxExperts];
@@ -259,16 +300,58 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   const int chunk = blockIdx.x;
   const bool lead = FUSED && chunk == 0 && blockIdx.y == 0;
   const int E = a.E, k = a.k, T = a.T;
+  const int nvec = a.d * (int)sizeof(TX) / 16;
+  const int v0 = blockIdx.y * a.slice_vec;
+  const int W = max(0, min(nvec, v0 + a.slice_vec) - v0);
+  const int t0 = chunk * kChunk;
+  const int ntok = min(kChunk, T - t0);
+  const uint32_t bar = tc::smem_u32(&xbar);
   for (int i = threadIdx.x; i < kRankWarps * kMaxExperts; i += kScatterThreads) (&wcnt[0][0])[i] = 0;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // Before the wait on the routing kernel: x and out are not touched by it
+  // (it starts only after everything earlier on the stream has finished), so
+  // the slice of the chunk's x rows is brought into shared memory by TMA bulk
+  // copies and the fused-combine output rows are zeroed while it runs.
+  if (warp == 0 && W > 0) {
+    if (lane == 0) tc::mbar_expect_tx(bar, (uint32_t)(ntok * W * 16));
+    __syncwarp();
+    const char* src = reinterpret_cast<const char*>(x) + ((size_t)t0 * nvec + v0) * 16;
+    for (int i = lane; i < ntok; i += 32)
+      tc::bulk_load(tc::smem_u32(xs + (size_t)i * W), src + (size_t)i * nvec * 16, (uint32_t)(W * 16), bar);
+  }
+  if (a.out != nullptr) {
+    constexpr int kOutVec = 16 / (int)sizeof(TX) / 4;   // float4 of out per 16-byte vector of x
+    const int wo = W * kOutVec;
+    for (int u = threadIdx.x; u < ntok * wo; u += kScatterThreads) {
+      const int tok = u / wo;
+      reinterpret_cast<float4*>(a.out + (size_t)(t0 + tok) * a.d)[v0 * kOutVec + (u - tok * wo)] =
+          make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   pdl_wait();
   pdl_launch_dependents();
-  if (FUSED) {
-    for (int e = warp; e < E; e += kWarps) {
-      int tot, pre;
-      expert_totals(a.hist, e, a.nch, chunk, nullptr, lane, &tot, &pre);
-      const float P = lead ? expert_prob_mean(a.prob_mean, a.psum, e, E, a.nch, T, lane) : 0.f;
-      if (lane == 0) { s_counts[e] = tot; s_pre[e] = pre; s_p[e] = P; }
+  // the rank warps' expert ids first: their loads overlap the histogram reads
+  int val[KB], rank_w[KB];
+  const int t = chunk * kChunk + warp * 32 + lane;
+  if (warp < kRankWarps) {
+    const bool tv = t < T;
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      int e = 0x1ff;
+      if (tv && j < k) {
+        e = a.topk_idx[(size_t)t * k + j];
+        if (e < 0 || e >= E) e = 0x1ff;
+      }
+      val[j] = e;
     }
+  }
+  if (FUSED) {
+    block_expert_totals<kScatterThreads>(a.hist, a.psum, a.prob_mean, E, a.nch, chunk, T, lead, s_counts, s_pre,
+                                         s_p);
     if (lead && warp == kWarps - 1) {
       const int nt = chunk_ties(a.ntie, a.nch, lane);
       if (lane == 0) s_ntie = nt;
@@ -285,19 +368,7 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   }
   __syncthreads();
 
-  int val[KB], rank_w[KB];
-  const int t = chunk * kChunk + warp * 32 + lane;
   if (warp < kRankWarps) {
-    const bool tv = t < T;
-#pragma unroll
-    for (int j = 0; j < KB; ++j) {
-      int e = 0x1ff;
-      if (tv && j < k) {
-        e = a.topk_idx[(size_t)t * k + j];
-        if (e < 0 || e >= E) e = 0x1ff;
-      }
-      val[j] = e;
-    }
     unsigned B[KB][9];
 #pragma unroll
     for (int j = 0; j < KB; ++j)
@@ -336,7 +407,10 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
         const int r = s_pre[e] + before + rank_w[j];
         if (a.capacity < 0 || r < a.capacity) {
           row = s_off[e] + r;
-          if (writer) a.src_tok[row] = t;
+          if (writer) {
+            a.src_tok[row] = t;
+            if (a.row_w != nullptr) a.row_w[row] = a.topk_w[(size_t)t * k + j];
+          }
         }
       }
       if (writer && t < T && j < k) a.row_of[(size_t)t * k + j] = row;
@@ -345,34 +419,20 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   }
   __syncthreads();
 
-  // gather: this block's column slice [v0, v0 + W) of every token row of the
-  // chunk, 16-byte vectors, four loads in flight per thread
-  const int nvec = a.d * (int)sizeof(TX) / 16;
-  const int v0 = blockIdx.y * a.slice_vec;
-  const int W = min(nvec, v0 + a.slice_vec) - v0;
-  const int t0 = chunk * kChunk;
-  const int units = (W > 0) ? min(kChunk, T - t0) * W : 0;
-  for (int u0 = threadIdx.x; u0 < units; u0 += 4 * kScatterThreads) {
-    uint4 v[4];
-    int tok[4], col[4];
+  // gather: the block's column slice [v0, v0 + W) of every token row of the
+  // chunk, from shared memory to the kept destination rows
+  if (W > 0 && !tc::mbar_wait(bar, 0, nullptr, tc::kWaitNs)) {
+    if (threadIdx.x == 0) atomicOr(a.status, MOE_DEV_TIMEOUT);
+    return;
+  }
+  const int units = ntok * W;
+  for (int u = threadIdx.x; u < units; u += kScatterThreads) {
+    const int tok = u / W, col = u - tok * W;
+    const uint4 v = xs[u];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int u = u0 + q * kScatterThreads;
-      tok[q] = -1;
-      if (u < units) {
-        tok[q] = u / W;
-        col[q] = v0 + (u - tok[q] * W);
-        v[q] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok[q]) * a.d) + col[q]);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (tok[q] < 0) continue;
-#pragma unroll
-      for (int j = 0; j < KB; ++j) {
-        const int r = rows_sm[tok[q]][j];
-        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[col[q]] = v[q];
-      }
+    for (int j = 0; j < KB; ++j) {
+      const int r = rows_sm[tok][j];
+      if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[v0 + col] = v;
     }
   }
 }
@@ -419,15 +479,30 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
   }
 }
 
-// Column slices per chunk: enough blocks for about two per SM, each slice at
-// least 32 vectors (512 bytes) of a row.
+// Column slices per chunk: a slice is at most kSliceVec 16-byte vectors of a
+// row (its x rows are staged in shared memory: 64 KB for a 128-token chunk),
+// and rows are cut finer, down to 8 vectors, until there are about two blocks
+// per SM.
+constexpr int kSliceVec = 32;
+
 inline int scatter_slices(int nch, int nvec, int* slice_vec) {
   DeviceInfo di;
   const int sms = (device_info(&di) == cudaSuccess) ? di.sms : 148;
-  int S = (2 * sms + nch - 1) / nch;
-  S = std::max(1, std::min(S, nvec / 32));
+  int S = (nvec + kSliceVec - 1) / kSliceVec;
+  const int want = (2 * sms + nch - 1) / nch;
+  if (S < want) S = std::max(S, std::min(want, nvec / 8));
+  S = std::max(S, 1);
   *slice_vec = (nvec + S - 1) / S;
   return (nvec + *slice_vec - 1) / *slice_vec;
+}
+
+template <typename TX, bool FUSED, int KB>
+cudaError_t launch_scatter_kb(const dim3& g, const TX* x, TX* xp, const ScatterArgs& b, cudaStream_t s) {
+  constexpr size_t kMaxSmem = (size_t)kChunk * kSliceVec * 16;
+  cudaError_t err = set_smem_once<scatter_kernel<KB, TX, FUSED>>(kMaxSmem);
+  if (err != cudaSuccess) return err;
+  const size_t smem = (size_t)kChunk * b.slice_vec * 16;
+  return launch_pdl(scatter_kernel<KB, TX, FUSED>, g, dim3(kScatterThreads), smem, s, x, xp, b);
 }
 
 template <typename TX, bool FUSED>
@@ -436,11 +511,11 @@ cudaError_t launch_scatter_t(const moe_config& c, const TX* x, TX* xp, const Sca
   const int S = scatter_slices(a.nch, c.d * (int)sizeof(TX) / 16, &slice_vec);
   ScatterArgs b = a;
   b.slice_vec = slice_vec;
-  const dim3 g(a.nch, S), blk(kScatterThreads);
-  if (c.k <= 1) return launch_pdl(scatter_kernel<1, TX, FUSED>, g, blk, 0, s, x, xp, b);
-  if (c.k <= 2) return launch_pdl(scatter_kernel<2, TX, FUSED>, g, blk, 0, s, x, xp, b);
-  if (c.k <= 4) return launch_pdl(scatter_kernel<4, TX, FUSED>, g, blk, 0, s, x, xp, b);
-  return launch_pdl(scatter_kernel<8, TX, FUSED>, g, blk, 0, s, x, xp, b);
+  const dim3 g(a.nch, S);
+  if (c.k <= 1) return launch_scatter_kb<TX, FUSED, 1>(g, x, xp, b, s);
+  if (c.k <= 2) return launch_scatter_kb<TX, FUSED, 2>(g, x, xp, b, s);
+  if (c.k <= 4) return launch_scatter_kb<TX, FUSED, 4>(g, x, xp, b, s);
+  return launch_scatter_kb<TX, FUSED, 8>(g, x, xp, b, s);
 }
 
 template <typename TX>
@@ -484,7 +559,8 @@ cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const floa
 cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
                            const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
-                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s) {
+                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
+                           const float* topk_w, float* row_w, float* out) {
   ScatterArgs a{};
   a.topk_idx = topk_idx;
   a.hist = hist;
@@ -498,6 +574,10 @@ cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, con
   a.stats = stats;
   a.row_of = row_of;
   a.src_tok = src_tok;
+  a.topk_w = topk_w;
+  a.row_w = row_w;
+  a.out = out;
+  a.status = &stats->status;
   a.T = c.T;
   a.d = c.d;
   a.E = c.E;

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 def test_struct_sizes_match_header(L):
     assert ctypes.sizeof(moe.moe_config) == 10 * 4
     assert ctypes.sizeof(moe.moe_stats) == 8 * 4
-    assert ctypes.sizeof(moe.moe_ws_layout) == 13 * 8
+    assert ctypes.sizeof(moe.moe_ws_layout) == 14 * 8
 
 
 def test_status_strings(L):
@@ -134,7 +134,8 @@ def test_workspace_layout_is_disjoint_and_aligned(L):
         es = 2 if c.dtype == moe.MOE_DTYPE_BF16 else 4
         A = T * k
         regions = [("topk_idx", 4 * A), ("topk_w", 4 * A), ("gap", 4 * T), ("counts", 4 * E), ("kept", 4 * E),
-                   ("offsets", 4 * (E + 1)), ("row_of", 4 * A), ("src_tok", 4 * A), ("xp", es * A * d),
+                   ("offsets", 4 * (E + 1)), ("row_of", 4 * A), ("src_tok", 4 * A), ("row_w", 4 * A),
+                   ("xp", es * A * d),
                    ("h", es * A * F), ("yp", 4 * A * d), ("scratch", moe.moe_scratch_size(c))]
         spans = sorted((getattr(lay, n), getattr(lay, n) + sz, n) for n, sz in regions)
         for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):

@@ -62,7 +62,9 @@ MEDIUM = [
     W("m_one", T=1, d=64, E=8, F=64, k=2, act=mw.RELU, dtype=mw.BF16, seed=26),
     W("m_E1", T=200, d=64, E=1, F=128, k=1, act=mw.SWIGLU, dtype=mw.BF16, seed=27),
     W("m_long_k", T=333, d=64, E=40, F=48, k=12, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.2, seed=28),
-    W("m_multi_tile", T=3000, d=512, E=4, F=640, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=29),
+    W("m_multi_tile", T=3000, d=512, E=4, F=640, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=29),   # 2-SM tiles
+    W("m_pair_relu_cap", T=2600, d=128, E=8, F=192, k=2, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.1,
+      seed=30),                                                                                  # 2-SM tiles
 ]
 
 
@@ -114,3 +116,26 @@ def test_layer_named_full_size_sampled(name):
     assert rel < 1.0
     del L
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["m_swiglu_lam", "m_E1", "m_one", "m_pair_relu_cap", "fastmoe_txl"])
+def test_fused_combine_matches_the_steps(name):
+    """bf16 layers with k <= 2: the forward adds the gate-weighted expert
+    outputs inside the second GEMM (out zeroed by the permutation) instead of
+    writing yp and running the combine kernel.  It must agree with the four
+    step calls to fp32 rounding (w*y rounded, then one addition, against one
+    fused multiply-add), and it must leave a token whose slots were all
+    dropped at exactly zero."""
+    w = mw.WORKLOADS.get(name) or next(m for m in MEDIUM if m.name == name)
+    assert w.dtype == mw.BF16 and w.k <= 2
+    L = DeviceLayer(w)
+    fused = L.forward()["out"]
+    idx, wt, gap, pm = L.route()
+    perm = L.permute(idx, gap, pm)
+    _, yp, _ = L.expert_ffn(perm["xp"], perm["offsets"])
+    steps = L.combine(yp, perm["row_of"], wt)
+    torch.cuda.synchronize()
+    scale = float(steps.abs().max())
+    assert float((fused - steps).abs().max()) <= 1e-6 * max(scale, 1e-30)
+    dropped = (perm["row_of"] < 0).all(dim=1)
+    assert torch.equal(fused[dropped], torch.zeros_like(fused[dropped]))

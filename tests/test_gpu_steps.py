@@ -29,6 +29,12 @@ MEDIUM = {
     "big_k10": W("big_k10", T=200, d=64, E=16, F=64, k=10, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.0,
                  seed=17),
     "E256": W("E256", T=300, d=64, E=256, F=32, k=4, act=mw.RELU, dtype=mw.BF16, seed=18),
+    # T*k >= 512*E: the expert GEMMs run on 2-SM pair tiles (256 rows); ragged
+    # segment ends, a ragged last n-tile (F = 320) and both activations
+    "pair_relu_ragged": W("pair_relu_ragged", T=1100, d=256, E=4, F=320, k=2, act=mw.RELU, dtype=mw.BF16,
+                          capacity_factor=1.25, seed=19),
+    "pair_swiglu_lambda": W("pair_swiglu_lambda", T=1500, d=192, E=3, F=208, k=2, act=mw.SWIGLU, dtype=mw.BF16,
+                            lam=1.0, seed=20),
 }
 
 
