@@ -283,7 +283,7 @@ struct ScatterArgs {
 // and the statistics.  The grid's y dimension splits each token row into
 // column slices, so that layers with few chunks and wide rows still spread
 // the gather over all SMs; the ranks are recomputed by every slice.
-template <int KB, typename TX, bool FUSED>
+template <int KB, typename TX, bool FUSED, bool STAGED>
 __global__ void __launch_bounds__(kScatterThreads)
 scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs a) {
   constexpr int kRankWarps = kChunk / 32;
@@ -316,7 +316,7 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   // (it starts only after everything earlier on the stream has finished), so
   // the slice of the chunk's x rows is brought into shared memory by TMA bulk
   // copies and the fused-combine output rows are zeroed while it runs.
-  if (warp == 0 && W > 0) {
+  if (STAGED && warp == 0 && W > 0) {
     if (lane == 0) tc::mbar_expect_tx(bar, (uint32_t)(ntok * W * 16));
     __syncwarp();
     const char* src = reinterpret_cast<const char*>(x) + ((size_t)t0 * nvec + v0) * 16;
@@ -420,19 +420,46 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   __syncthreads();
 
   // gather: the block's column slice [v0, v0 + W) of every token row of the
-  // chunk, from shared memory to the kept destination rows
-  if (W > 0 && !tc::mbar_wait(bar, 0, nullptr, tc::kWaitNs)) {
-    if (threadIdx.x == 0) atomicOr(a.status, MOE_DEV_TIMEOUT);
+  // chunk to the kept destination rows, from shared memory (STAGED) or
+  // straight from x with four 16-byte loads in flight per thread
+  const int units = ntok * W;
+  if (STAGED) {
+    if (W > 0 && !tc::mbar_wait(bar, 0, nullptr, tc::kWaitNs)) {
+      if (threadIdx.x == 0) atomicOr(a.status, MOE_DEV_TIMEOUT);
+      return;
+    }
+    for (int u = threadIdx.x; u < units; u += kScatterThreads) {
+      const int tok = u / W, col = u - tok * W;
+      const uint4 v = xs[u];
+#pragma unroll
+      for (int j = 0; j < KB; ++j) {
+        const int r = rows_sm[tok][j];
+        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[v0 + col] = v;
+      }
+    }
     return;
   }
-  const int units = ntok * W;
-  for (int u = threadIdx.x; u < units; u += kScatterThreads) {
-    const int tok = u / W, col = u - tok * W;
-    const uint4 v = xs[u];
+  for (int u0 = threadIdx.x; u0 < units; u0 += 4 * kScatterThreads) {
+    uint4 v[4];
+    int tok[4], col[4];
 #pragma unroll
-    for (int j = 0; j < KB; ++j) {
-      const int r = rows_sm[tok][j];
-      if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[v0 + col] = v;
+    for (int q = 0; q < 4; ++q) {
+      const int u = u0 + q * kScatterThreads;
+      tok[q] = -1;
+      if (u < units) {
+        tok[q] = u / W;
+        col[q] = v0 + (u - tok[q] * W);
+        v[q] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tok[q]) * a.d) + col[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (tok[q] < 0) continue;
+#pragma unroll
+      for (int j = 0; j < KB; ++j) {
+        const int r = rows_sm[tok[q]][j];
+        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[col[q]] = v[q];
+      }
     }
   }
 }
@@ -479,43 +506,62 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
   }
 }
 
-// Column slices per chunk: a slice is at most kSliceVec 16-byte vectors of a
-// row (its x rows are staged in shared memory: 64 KB for a 128-token chunk),
-// and rows are cut finer, down to 8 vectors, until there are about two blocks
-// per SM.
+// Column slices per chunk.  When the whole grid fits in about one wave (two
+// blocks per SM), every block stages its slice of x in shared memory before
+// it waits for the routing kernel (slices of up to kSliceVec 16-byte vectors,
+// 64 KB for a 128-token chunk), so the reads overlap that kernel.  Otherwise
+// blocks read x directly, and rows are cut into slices of at least 32 vectors
+// until there are about two blocks per SM.
 constexpr int kSliceVec = 32;
 
-inline int scatter_slices(int nch, int nvec, int* slice_vec) {
-  DeviceInfo di;
-  const int sms = (device_info(&di) == cudaSuccess) ? di.sms : 148;
-  int S = (nvec + kSliceVec - 1) / kSliceVec;
-  const int want = (2 * sms + nch - 1) / nch;
-  if (S < want) S = std::max(S, std::min(want, nvec / 8));
+inline bool scatter_staged(int nch, int nvec, int sms) {
+  return (long long)nch * ((nvec + kSliceVec - 1) / kSliceVec) <= 2LL * sms;
+}
+
+inline int scatter_slices(int nch, int nvec, bool staged, int sms, int* slice_vec) {
+  int S;
+  if (staged) {
+    S = (nvec + kSliceVec - 1) / kSliceVec;
+  } else {
+    S = (2 * sms + nch - 1) / nch;
+    S = std::min(S, nvec / 32);
+  }
   S = std::max(S, 1);
   *slice_vec = (nvec + S - 1) / S;
   return (nvec + *slice_vec - 1) / *slice_vec;
 }
 
-template <typename TX, bool FUSED, int KB>
+template <typename TX, bool FUSED, bool STAGED, int KB>
 cudaError_t launch_scatter_kb(const dim3& g, const TX* x, TX* xp, const ScatterArgs& b, cudaStream_t s) {
-  constexpr size_t kMaxSmem = (size_t)kChunk * kSliceVec * 16;
-  cudaError_t err = set_smem_once<scatter_kernel<KB, TX, FUSED>>(kMaxSmem);
-  if (err != cudaSuccess) return err;
-  const size_t smem = (size_t)kChunk * b.slice_vec * 16;
-  return launch_pdl(scatter_kernel<KB, TX, FUSED>, g, dim3(kScatterThreads), smem, s, x, xp, b);
+  size_t smem = 0;
+  if (STAGED) {
+    constexpr size_t kMaxSmem = (size_t)kChunk * kSliceVec * 16;
+    cudaError_t err = set_smem_once<scatter_kernel<KB, TX, FUSED, STAGED>>(kMaxSmem);
+    if (err != cudaSuccess) return err;
+    smem = (size_t)kChunk * b.slice_vec * 16;
+  }
+  return launch_pdl(scatter_kernel<KB, TX, FUSED, STAGED>, g, dim3(kScatterThreads), smem, s, x, xp, b);
+}
+
+template <typename TX, bool FUSED, bool STAGED>
+cudaError_t launch_scatter_s(const moe_config& c, const TX* x, TX* xp, ScatterArgs b, int sms, cudaStream_t s) {
+  int slice_vec = 0;
+  const int S = scatter_slices(b.nch, c.d * (int)sizeof(TX) / 16, STAGED, sms, &slice_vec);
+  b.slice_vec = slice_vec;
+  const dim3 g(b.nch, S);
+  if (c.k <= 1) return launch_scatter_kb<TX, FUSED, STAGED, 1>(g, x, xp, b, s);
+  if (c.k <= 2) return launch_scatter_kb<TX, FUSED, STAGED, 2>(g, x, xp, b, s);
+  if (c.k <= 4) return launch_scatter_kb<TX, FUSED, STAGED, 4>(g, x, xp, b, s);
+  return launch_scatter_kb<TX, FUSED, STAGED, 8>(g, x, xp, b, s);
 }
 
 template <typename TX, bool FUSED>
 cudaError_t launch_scatter_t(const moe_config& c, const TX* x, TX* xp, const ScatterArgs& a, cudaStream_t s) {
-  int slice_vec = 0;
-  const int S = scatter_slices(a.nch, c.d * (int)sizeof(TX) / 16, &slice_vec);
-  ScatterArgs b = a;
-  b.slice_vec = slice_vec;
-  const dim3 g(a.nch, S);
-  if (c.k <= 1) return launch_scatter_kb<TX, FUSED, 1>(g, x, xp, b, s);
-  if (c.k <= 2) return launch_scatter_kb<TX, FUSED, 2>(g, x, xp, b, s);
-  if (c.k <= 4) return launch_scatter_kb<TX, FUSED, 4>(g, x, xp, b, s);
-  return launch_scatter_kb<TX, FUSED, 8>(g, x, xp, b, s);
+  DeviceInfo di;
+  const int sms = (device_info(&di) == cudaSuccess) ? di.sms : 148;
+  if (scatter_staged(a.nch, c.d * (int)sizeof(TX) / 16, sms))
+    return launch_scatter_s<TX, FUSED, true>(c, x, xp, a, sms, s);
+  return launch_scatter_s<TX, FUSED, false>(c, x, xp, a, sms, s);
 }
 
 template <typename TX>
