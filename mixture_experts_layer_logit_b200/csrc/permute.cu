@@ -146,7 +146,8 @@ __device__ __forceinline__ void block_expert_totals(const int32_t* __restrict__ 
 
 // One warp: kept = min(count, C) (all in dropless mode), offsets = exclusive
 // scan of kept over the experts (8 experts per lane), the drop count and the
-// Switch aux loss E * sum_e (count_e / (T k)) * P_e in double.  Writes the
+// Switch aux loss E * sum_e (count_e / (T k)) * P_e in double (the sum of
+// count_e * P_e is divided by T k once: double divisions are slow).  Writes the
 // offsets to s_off when given and the global results when `out` is set.
 __device__ __forceinline__ void expert_offsets(const int* s_counts, const float* s_p, int s_ntie, int E, int T,
                                                int k, int capacity, int* s_off, bool out, int32_t* counts,
@@ -163,7 +164,7 @@ __device__ __forceinline__ void expert_offsets(const int* s_counts, const float*
     if (e < E) {
       cnt = s_counts[e];
       kp = (capacity < 0) ? cnt : min(cnt, capacity);
-      if (out) aux += ((double)cnt / A) * (double)s_p[e];
+      if (out) aux += (double)cnt * (double)s_p[e];   // divided by T k once, below
     }
     kv[i] = kp;
     local += kp;
@@ -203,7 +204,7 @@ __device__ __forceinline__ void expert_offsets(const int* s_counts, const float*
     stats->capacity = capacity;
     stats->near_tie_count = s_ntie;
     stats->drop_rate = (T > 0) ? (float)((double)drop / A) : 0.f;
-    stats->aux_loss = (T > 0) ? (float)((double)E * aux) : NAN;
+    stats->aux_loss = (T > 0) ? (float)((double)E * aux / A) : NAN;
   }
 }
 
