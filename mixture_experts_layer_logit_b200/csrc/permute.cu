@@ -255,12 +255,12 @@ struct ScatterArgs {
   const int32_t* topk_idx;
   const int32_t* hist;        // FUSED: per-chunk histograms [E][nch]
   int32_t* choff;             // separate scan: chunk offsets [E][nch]
-  const float* prob_mean;     // FUSED, lead block: P_e given, or
+  const float* prob_mean;     // FUSED, statistics block: P_e given, or
   const float* psum;          //   summed from the per-chunk probability sums
   const int32_t* ntie;
   int32_t* counts;
   int32_t* kept;
-  int32_t* offsets;           // read (separate scan) or written by the lead block (FUSED)
+  int32_t* offsets;           // read (separate scan) or written by the statistics block (FUSED)
   moe_stats* stats;
   int32_t* row_of;
   int32_t* src_tok;
@@ -280,8 +280,8 @@ struct ScatterArgs {
 //
 // FUSED: the block first derives its chunk's offsets from the histograms
 // itself (every block reads all E x nch counts from L2 and scans them), so no
-// separate scan kernel runs; block (0, 0) also writes counts, kept, offsets
-// and the statistics.  The grid's y dimension splits each token row into
+// separate scan kernel runs; one extra block, (nch, 0), writes counts, kept,
+// offsets and the statistics.  The grid's y dimension splits each token row into
 // column slices, so that layers with few chunks and wide rows still spread
 // the gather over all SMs; the ranks are recomputed by every slice.
 template <int KB, typename TX, bool FUSED, bool STAGED>
@@ -299,8 +299,25 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   __shared__ int s_ntie;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
-  const bool lead = FUSED && chunk == 0 && blockIdx.y == 0;
   const int E = a.E, k = a.k, T = a.T;
+  if (FUSED && chunk == a.nch) {
+    // One extra block (x = nch, y = 0) writes the layer's counts, kept,
+    // offsets and statistics, so that no chunk block carries that work.
+    if (blockIdx.y != 0) return;
+    pdl_wait();
+    pdl_launch_dependents();
+    block_expert_totals<kScatterThreads>(a.hist, a.psum, a.prob_mean, E, a.nch, a.nch, T, true, s_counts, nullptr,
+                                         s_p);
+    if (warp == kWarps - 1) {
+      const int nt = chunk_ties(a.ntie, a.nch, lane);
+      if (lane == 0) s_ntie = nt;
+    }
+    __syncthreads();
+    if (warp == 0)
+      expert_offsets(s_counts, s_p, s_ntie, E, T, k, a.capacity, nullptr, true, a.counts, a.kept, a.offsets,
+                     a.stats, lane);
+    return;
+  }
   const int nvec = a.d * (int)sizeof(TX) / 16;
   const int v0 = blockIdx.y * a.slice_vec;
   const int W = max(0, min(nvec, v0 + a.slice_vec) - v0);
@@ -335,32 +352,32 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   }
   pdl_wait();
   pdl_launch_dependents();
-  // the rank warps' expert ids first: their loads overlap the histogram reads
+  // the rank warps' expert ids (and gate weights) first: their loads overlap
+  // the histogram reads
   int val[KB], rank_w[KB];
+  float wsel[KB];
   const int t = chunk * kChunk + warp * 32 + lane;
   if (warp < kRankWarps) {
     const bool tv = t < T;
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
       int e = 0x1ff;
+      wsel[j] = 0.f;
       if (tv && j < k) {
         e = a.topk_idx[(size_t)t * k + j];
         if (e < 0 || e >= E) e = 0x1ff;
+        if (a.row_w != nullptr) wsel[j] = a.topk_w[(size_t)t * k + j];
       }
       val[j] = e;
     }
   }
   if (FUSED) {
-    block_expert_totals<kScatterThreads>(a.hist, a.psum, a.prob_mean, E, a.nch, chunk, T, lead, s_counts, s_pre,
-                                         s_p);
-    if (lead && warp == kWarps - 1) {
-      const int nt = chunk_ties(a.ntie, a.nch, lane);
-      if (lane == 0) s_ntie = nt;
-    }
+    block_expert_totals<kScatterThreads>(a.hist, nullptr, nullptr, E, a.nch, chunk, T, false, s_counts, s_pre,
+                                         nullptr);
     __syncthreads();
     if (warp == 0)
-      expert_offsets(s_counts, s_p, s_ntie, E, T, k, a.capacity, s_off, lead, a.counts, a.kept, a.offsets,
-                     a.stats, lane);
+      expert_offsets(s_counts, nullptr, 0, E, T, k, a.capacity, s_off, false, nullptr, nullptr, nullptr, nullptr,
+                     lane);
   } else {
     for (int e = threadIdx.x; e < E; e += kScatterThreads) {
       s_pre[e] = a.choff[(size_t)e * a.nch + chunk];
@@ -410,7 +427,7 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
           row = s_off[e] + r;
           if (writer) {
             a.src_tok[row] = t;
-            if (a.row_w != nullptr) a.row_w[row] = a.topk_w[(size_t)t * k + j];
+            if (a.row_w != nullptr) a.row_w[row] = wsel[j];
           }
         }
       }
@@ -429,15 +446,18 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
       if (threadIdx.x == 0) atomicOr(a.status, MOE_DEV_TIMEOUT);
       return;
     }
-    for (int u = threadIdx.x; u < units; u += kScatterThreads) {
-      const int tok = u / W, col = u - tok * W;
-      const uint4 v = xs[u];
-#pragma unroll
-      for (int j = 0; j < KB; ++j) {
-        const int r = rows_sm[tok][j];
-        if (r >= 0) reinterpret_cast<uint4*>(xp + (size_t)r * a.d)[v0 + col] = v;
+    // one bulk copy of the slice per kept (token, slot), shared memory -> xp row
+    bool issued = false;
+    for (int u = threadIdx.x; u < ntok * KB && W > 0; u += kScatterThreads) {
+      const int tok = u / KB, j = u - tok * KB;
+      const int r = rows_sm[tok][j];
+      if (r >= 0) {
+        tc::bulk_store(reinterpret_cast<char*>(xp) + ((size_t)r * nvec + v0) * 16, tc::smem_u32(xs + (size_t)tok * W),
+                       (uint32_t)(W * 16));
+        issued = true;
       }
     }
+    if (issued) tc::bulk_store_drain();
     return;
   }
   for (int u0 = threadIdx.x; u0 < units; u0 += 4 * kScatterThreads) {
@@ -549,7 +569,7 @@ cudaError_t launch_scatter_s(const moe_config& c, const TX* x, TX* xp, ScatterAr
   int slice_vec = 0;
   const int S = scatter_slices(b.nch, c.d * (int)sizeof(TX) / 16, STAGED, sms, &slice_vec);
   b.slice_vec = slice_vec;
-  const dim3 g(b.nch, S);
+  const dim3 g(b.nch + (FUSED ? 1 : 0), S);   // FUSED: one more block row for the statistics
   if (c.k <= 1) return launch_scatter_kb<TX, FUSED, STAGED, 1>(g, x, xp, b, s);
   if (c.k <= 2) return launch_scatter_kb<TX, FUSED, STAGED, 2>(g, x, xp, b, s);
   if (c.k <= 4) return launch_scatter_kb<TX, FUSED, STAGED, 4>(g, x, xp, b, s);
