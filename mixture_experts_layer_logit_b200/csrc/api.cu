@@ -142,6 +142,7 @@ moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* 
 
 // Mean assignments per expert from which the expert GEMMs use 2-SM tiles.
 constexpr long long kPairRowsPerExpert = 512;
+bool pair_tiles(const moe_config& c) { return (long long)c.T * c.k >= kPairRowsPerExpert * c.E; }
 
 moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                       const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s,
@@ -149,7 +150,7 @@ moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offset
   if (c.dtype == MOE_DTYPE_BF16) {
     // 2-SM pair tiles (256 rows) pay off once the expert segments hold a few
     // hundred rows on average; short segments waste half a pair tile.
-    if ((long long)c.T * c.k >= (long long)kPairRowsPerExpert * c.E)
+    if (pair_tiles(c))
       return cuda_status(launch_expert_ffn_tc_pair(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
     return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
   }
@@ -291,13 +292,21 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   void* yp = at<char>(ws, L.yp);
 
+  const bool fuse = fused_combine(c);
+  // k <= 2 on the 1-SM tiles: both expert layers and the combine in one launch
+  // with a dynamic tile queue; its counters use the yp region, which the fused
+  // combine leaves unwritten
+  const bool one_launch = fuse && !pair_tiles(c) &&
+                          sizeof(int) * expert_mlp_counters(c) <= sizeof(float) * (size_t)c.T * c.k * c.d;
+  int* counters = at<int>(ws, L.yp);
   if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (one_launch && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
   // near-tie counts of every chunk in scratch, so step 3 starts at the scan
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
                                at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  const bool fuse = fused_combine(c);
   float* row_w = at<float>(ws, L.row_w);
   float* out_f = static_cast<float*>(out);
   st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
@@ -309,6 +318,9 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   if (fuse) {
     // steps 4-5: the second GEMM adds the gate-weighted expert outputs into out
     const CombineOut comb{at<int32_t>(ws, L.src_tok), row_w, out_f, c.T};
+    if (one_launch)
+      return cuda_status(launch_expert_mlp(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), comb,
+                                           counters, &stats->status, s));
     return expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s, &comb);
   }
   st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);

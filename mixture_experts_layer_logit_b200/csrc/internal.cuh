@@ -78,6 +78,13 @@ struct CombineOut {
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
                                  uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
+// Steps 4-5 in one launch for the bf16 path with k <= 2: both expert layers
+// and the fused combine from one dynamic tile queue.  `counters` holds
+// expert_mlp_counters(c) ints, zeroed before the launch.
+size_t expert_mlp_counters(const moe_config& c);
+cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
+                              const void* w2, void* h, const CombineOut& comb, int* counters, uint32_t* status,
+                              cudaStream_t s);
 // The same with 2-SM pair tiles (tcgen05.mma.cta_group::2, 256 x 256).
 cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
                                       const void* w1, const void* w2, void* h, void* yp,

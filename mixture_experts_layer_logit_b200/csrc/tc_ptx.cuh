@@ -109,6 +109,36 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// ---- flags between CTAs of one grid (global memory, GPU scope)
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// orders this thread's earlier generic-proxy accesses (e.g. the acquire of a
+// flag) before its later async-proxy (TMA) accesses of global memory
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Waits until *p >= target (acquire).  Gives up (false) after `limit` ns or
+// once `abort_flag` is raised.
+static __device__ __noinline__ bool wait_flag_geq(const int* p, int target, const volatile int* abort_flag,
+                                                  unsigned long long limit) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const unsigned long long t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (abort_flag != nullptr && *abort_flag) return false;
+      if (now_ns() - t0 > limit) return false;
+    }
+  }
+}
+
 // ---- CTA pairs (a cluster of two CTAs sharing one tcgen05 MMA, cta_group::2)
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
