@@ -39,8 +39,8 @@ METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (GEMM), % HBM BW 
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
-GEMM_PROFILE = os.path.join(ROOT, "profiles", "tc_grouped_gemm_fastmoe_txl.md")
-GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc", "gemm_tc.cu")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "tc_expert_mlp_fastmoe_txl.md")
+GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc", "gemm_mlp.cu")
 
 
 def parse_args():
@@ -230,9 +230,16 @@ def step_bytes(w: mw.Workload, offsets: np.ndarray):
         # weights of the experts that received rows, xp read, h written and read, yp written
         "expert_ffn": touched * (F1 + F) * d * b + kept * (d * b + 2 * F * hb + d * 4),
         "combine": (kept * d + T * d) * 4 + 8 * A,
+        # the fused steps 4-5: as expert_ffn, but out (T x d fp32) written instead of yp
+        "experts_combine": touched * (F1 + F) * d * b + kept * (d * b + 2 * F * hb) + T * d * 4 + 8 * kept,
         "expert_flops": 2 * kept * d * (F1 + F),
         "weight_bytes": touched * (F1 + F) * d * b,
     }
+
+
+def fused_combine(w: mw.Workload) -> bool:
+    """The forward fuses step 5 into the expert kernel for bf16 layers with k <= 2."""
+    return w.dtype == mw.BF16 and w.k <= 2
 
 
 def committed_traffic():
@@ -408,28 +415,55 @@ def main():
                 for j, n in enumerate(names):
                     acc[n] += ev[j].elapsed_time(ev[j + 1])
         breakdown = {n: acc[n] / a.steps for n in names}
+        # The forward's own steps 4-5 on bf16 layers with k <= 2: the expert
+        # kernel with the combine fused in, fed the forward's permuted rows and
+        # row weights; out is zeroed before each call, outside the events.
+        fused = fused_combine(w)
+        one_launch = fused and w.T * w.k < 512 * w.E
+        if fused:
+            row_w = sv(L.row_w, A, torch.float32)
+            out_fc = torch.empty_like(out)
+            t_fc = 0.0
+            for i in range(a.warmup + a.steps):
+                flush.zero_()
+                out_fc.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                moe.moe_expert_ffn_combine(cfg, xp, offs, src_tok, row_w, w1, w2, h, out_fc, stats, ws)
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= a.warmup:
+                    t_fc += e0.elapsed_time(e1)
+            breakdown["experts_combine"] = t_fc / a.steps
         rl = {}
         for n in ["route", "permute", "combine"]:
             gbs = sb[n] / (breakdown[n] * 1e-3) / 1e9
             rl[n] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / pk["hbm_gbs"], "bytes": sb[n]}
-        t_ffn = breakdown["expert_ffn"] * 1e-3
+        step = "experts_combine" if fused else "expert_ffn"
+        t_ffn = breakdown[step] * 1e-3
         tflops = sb["expert_flops"] / t_ffn / 1e12
-        gbs = sb["expert_ffn"] / t_ffn / 1e9
-        t_hbm = sb["expert_ffn"] / (pk["hbm_gbs"] * 1e9)
+        gbs = sb[step] / t_ffn / 1e9
+        t_hbm = sb[step] / (pk["hbm_gbs"] * 1e9)
         t_tc = sb["expert_flops"] / (pk["bf16_tflops"] * 1e12)
         bound = "hbm" if t_hbm >= t_tc else "tensor"
-        traffic = committed_traffic() if a.workload == mw.BENCH_WORKLOAD else None
+        traffic = committed_traffic() if (a.workload == mw.BENCH_WORKLOAD and one_launch) else None
         if bound == "hbm":
             roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic}
         else:
             roofline = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": tflops / pk["bf16_tflops"], "traffic": traffic}
+        if one_launch:
+            kname, nl = "tc_expert_mlp (steps 4-5 in one launch: both expert layers + the combine)", 1
+        elif fused:
+            kname, nl = "tc_grouped_gemm(_pair) (layer 1, then layer 2 with the combine fused: 2 launches)", 2
+        else:
+            kname, nl = "tc_grouped_gemm(_pair) (expert FFN step: 2 launches, layer 1 + layer 2)", 2
         roofline.update({
-            "kernel": "tc_grouped_gemm (expert FFN step: 2 launches, layer 1 + layer 2)",
-            "launches_per_step": 2, "algorithmic_bytes_per_launch": sb["expert_ffn"] / 2,
-            "algorithmic_flops_per_launch": sb["expert_flops"] / 2, "launch_ms": breakdown["expert_ffn"] / 2,
+            "kernel": kname,
+            "launches_per_step": nl, "algorithmic_bytes_per_launch": sb[step] / nl,
+            "algorithmic_flops_per_launch": sb["expert_flops"] / nl, "launch_ms": breakdown[step] / nl,
             "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"], "hbm_gbs": gbs,
             "hbm_frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured"
             else "fallback (recipe)", "other_steps": rl})

@@ -203,6 +203,29 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* 
                           moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Steps 4-5 fused, as moe_layer_forward runs them on the bf16 path with
+ * k <= 2: the expert FFNs of moe_expert_ffn, each kept row's output added,
+ * times its gate weight, straight into the token's row of out.  No yp is
+ * formed.  Megatron-Core best-practice page, "Megatron-Core MoE的关键特性"
+ * (GroupedGEMM); FastMoE announcement, "1. MoE 设计" (the output is the
+ * gate-weighted sum of the selected experts' outputs).
+ *   xp[A, d], offsets[E+1], W1, W2, h: as moe_expert_ffn.
+ *   src_tok[A]: token of each permuted row (from moe_permute).
+ *   row_w[A] fp32: gate weight of each kept row (the row_w region of a
+ *     moe_layer_forward workspace holds it after a forward).
+ *   out[T, d] fp32: must hold zeros on entry; each element receives at most
+ *     two additions (k <= 2) onto that exact zero, so the result does not
+ *     depend on their order.
+ *   ws: a moe_layer_forward workspace (moe_workspace_size bytes); its yp
+ *     region is used for the tile scheduler's counters.
+ *   MOE_ERR_UNSUPPORTED unless dtype is bf16 and k <= 2.
+ */
+moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                                  const int32_t* src_tok, const float* row_w, const void* W1, const void* W2,
+                                  void* h, void* out, moe_stats* stats, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
+/*
  * Step 5: un-permute and combine.  out[t] = sum over j = 0..k-1 with
  * row_of[t, j] >= 0 of topk_w[t, j] * yp[row_of[t, j]], accumulated in fp32 in
  * slot order; 0 for a token whose slots were all dropped (the residual path

@@ -20,7 +20,7 @@ __all__ = [
     "LIB_PATH", "MoeError", "moe_config", "moe_stats", "moe_ws_layout", "lib", "make_config",
     "moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "moe_permute_static",
-    "MOE_STATIC_SCRATCH_BYTES", "prepare_w2",
+    "moe_expert_ffn_combine", "MOE_STATIC_SCRATCH_BYTES", "prepare_w2",
     "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
     "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE
 
 EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route",
                     "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-                    "moe_convert_bf16_to_f16", "moe_permute_static"]
+                    "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine"]
 MOE_STATIC_SCRATCH_BYTES = 2 << 20
 
 
@@ -90,8 +90,9 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_convert_bf16_to_f16.argtypes = [P, P, ctypes.c_size_t, P]
     L.moe_permute_static.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P]
+    L.moe_expert_ffn_combine.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-              "moe_convert_bf16_to_f16", "moe_permute_static"]:
+              "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine"]:
         getattr(L, n).restype = st
     _lib = L
     return L
@@ -180,6 +181,15 @@ def moe_expert_ffn(cfg, xp, offsets, W1, W2, h, yp, stats, ws, stream=None):
     _check("moe_expert_ffn", lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(xp), _ptr(offsets), _ptr(W1),
                                                   _ptr(W2), _ptr(h), _ptr(yp), _ptr(stats), _ptr(ws),
                                                   _nbytes(ws), _stream(stream)))
+
+
+def moe_expert_ffn_combine(cfg, xp, offsets, src_tok, row_w, W1, W2, h, out, stats, ws, stream=None):
+    """Steps 4-5 fused (bf16, k <= 2): out (zeroed by the caller) += gate-weighted expert outputs.
+    ws is a moe_layer_forward workspace."""
+    _check("moe_expert_ffn_combine",
+           lib().moe_expert_ffn_combine(ctypes.byref(cfg), _ptr(xp), _ptr(offsets), _ptr(src_tok), _ptr(row_w),
+                                        _ptr(W1), _ptr(W2), _ptr(h), _ptr(out), _ptr(stats), _ptr(ws), _nbytes(ws),
+                                        _stream(stream)))
 
 
 def moe_combine(cfg, yp, row_of, topk_w, out, stream=None):

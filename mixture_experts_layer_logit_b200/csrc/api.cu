@@ -162,6 +162,27 @@ moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offset
 // the additions arrive in) and the tensor-core path runs.
 bool fused_combine(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.k <= 2 && c.T > 0; }
 
+// On the 1-SM tiles both expert layers and the combine run as one launch
+// with a dynamic tile queue; its counters use the yp region of the forward
+// workspace, which the fused combine leaves unwritten.
+bool one_launch(const moe_config& c) {
+  return fused_combine(c) && !pair_tiles(c) &&
+         sizeof(int) * expert_mlp_counters(c) <= sizeof(float) * (size_t)c.T * c.k * c.d;
+}
+
+// Steps 4-5 fused (out zeroed beforehand); counters: the yp region.
+moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* offsets, const int32_t* src_tok,
+                           const float* row_w, const void* w1, const void* w2, void* h, float* out, int* counters,
+                           void* yp, moe_stats* stats, bool counters_zeroed, cudaStream_t s) {
+  const CombineOut comb{src_tok, row_w, out, c.T};
+  if (one_launch(c)) {
+    if (!counters_zeroed && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, comb, counters, &stats->status, s));
+  }
+  return expert_ffn(c, xp, offsets, w1, w2, h, yp, stats, s, &comb);
+}
+
 }  // namespace
 
 extern "C" {
@@ -257,6 +278,29 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* 
   return expert_ffn(c, xp, offsets, W1, W2, h, yp, stats, reinterpret_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                                  const int32_t* src_tok, const float* row_w, const void* W1, const void* W2,
+                                  void* h, void* out, moe_stats* stats, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DTYPE_BF16 || c.k > 2) return MOE_ERR_UNSUPPORTED;
+  if (offsets == nullptr || stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (xp == nullptr || src_tok == nullptr || row_w == nullptr || W1 == nullptr || W2 == nullptr ||
+                  h == nullptr || out == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(xp) || !aligned16(W1) || !aligned16(W2) || !aligned16(h) || !aligned16(out) ||
+      !aligned4(offsets) || !aligned4(src_tok) || !aligned4(row_w) || !aligned4(stats))
+    return MOE_ERR_ARG;
+  const moe_ws_layout L = layout_of(c);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return st;
+  if ((st = check_device(true)) != MOE_OK) return st;
+  if (c.T == 0) return MOE_OK;
+  return experts_combine(c, xp, offsets, src_tok, row_w, W1, W2, h, static_cast<float*>(out), at<int>(ws, L.yp),
+                         at<char>(ws, L.yp), stats, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_combine(const moe_config* cfg, const void* yp, const int32_t* row_of,
                        const float* topk_w, void* out, moe_stream_t stream) {
   moe_status st = check_config(cfg);
@@ -293,14 +337,10 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   void* yp = at<char>(ws, L.yp);
 
   const bool fuse = fused_combine(c);
-  // k <= 2 on the 1-SM tiles: both expert layers and the combine in one launch
-  // with a dynamic tile queue; its counters use the yp region, which the fused
-  // combine leaves unwritten
-  const bool one_launch = fuse && !pair_tiles(c) &&
-                          sizeof(int) * expert_mlp_counters(c) <= sizeof(float) * (size_t)c.T * c.k * c.d;
   int* counters = at<int>(ws, L.yp);
   if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (one_launch && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
+  // the tile-queue counters are zeroed here, ahead of the kernel chain
+  if (one_launch(c) && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
   // near-tie counts of every chunk in scratch, so step 3 starts at the scan
@@ -315,14 +355,9 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
                          at<char>(ws, L.xp), stats, sc, scr, s, fuse ? w : nullptr, fuse ? row_w : nullptr,
                          fuse ? out_f : nullptr);
   if (st != MOE_OK) return st;
-  if (fuse) {
-    // steps 4-5: the second GEMM adds the gate-weighted expert outputs into out
-    const CombineOut comb{at<int32_t>(ws, L.src_tok), row_w, out_f, c.T};
-    if (one_launch)
-      return cuda_status(launch_expert_mlp(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), comb,
-                                           counters, &stats->status, s));
-    return expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s, &comb);
-  }
+  if (fuse)   // steps 4-5: the second layer adds the gate-weighted expert outputs into out
+    return experts_combine(c, at<char>(ws, L.xp), offsets, at<int32_t>(ws, L.src_tok), row_w, W1, W2,
+                           at<char>(ws, L.h), out_f, counters, yp, stats, true, s);
   st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));

@@ -94,6 +94,10 @@ __device__ __forceinline__ void store_tile(const Params& p, uint32_t tb, int wro
   constexpr bool kF32Out = (MODE == kPlain || MODE == kCombine);
   constexpr int kBlocks = kF32Out ? BN / 32 : (MODE == kRelu ? BN / 64 : BN / 128);
   constexpr int kPer16 = kF32Out ? 4 : 8;
+  // rows past the segment (the next expert's rows, or unwritten rows past
+  // the kept ones) are computed but never stored: only stored rows may
+  // report an fp16 overflow
+  bool row_over = false;
   int tok = 0;
   float wgt = 0.f;
   if (MODE == kCombine && lane < nrows) {
@@ -135,7 +139,7 @@ __device__ __forceinline__ void store_tile(const Params& p, uint32_t tb, int wro
               a0 = a0 / (1.f + __expf(-a0)) * u0;
               a1 = a1 / (1.f + __expf(-a1)) * u1;
             }
-            pk[j] = pack_hidden<F16>(a0, a1, over);
+            pk[j] = pack_hidden<F16>(a0, a1, row_over);
           }
           v[hf * 4 + i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
@@ -170,6 +174,7 @@ __device__ __forceinline__ void store_tile(const Params& p, uint32_t tb, int wro
       }
     }
   }
+  over |= row_over && lane < nrows;
 }
 
 // Layer-2 modes read fp16 operands when the hidden type is fp16.

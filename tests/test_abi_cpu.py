@@ -106,6 +106,17 @@ def test_null_and_misaligned_pointers(L):
     assert L.moe_combine(ctypes.byref(c), P + 4, P, P, P, None) == 1
 
 
+def test_fused_expert_combine_limits(L):
+    P = 1 << 20
+    for bad in [cfg(k=3, E=8), cfg(dtype="f32", d=64, F=128)]:
+        full, _ = moe.moe_workspace_size(bad)
+        assert L.moe_expert_ffn_combine(ctypes.byref(bad), P, P, P, P, P, P, P, P, P, P, full, None) == 2
+    c = cfg(k=2)
+    full, _ = moe.moe_workspace_size(c)
+    assert L.moe_expert_ffn_combine(ctypes.byref(c), P, P, P, None, P, P, P, P, P, P, full, None) == 1   # no row_w
+    assert L.moe_expert_ffn_combine(ctypes.byref(c), P, P, P, P, P, P, P, P, P, P, full - 1, None) == 3
+
+
 def test_convert_rejects_bad_pointers(L):
     P = 1 << 20
     assert L.moe_convert_bf16_to_f16(None, P, 8, None) == 1

@@ -139,3 +139,31 @@ def test_fused_combine_matches_the_steps(name):
     assert float((fused - steps).abs().max()) <= 1e-6 * max(scale, 1e-30)
     dropped = (perm["row_of"] < 0).all(dim=1)
     assert torch.equal(fused[dropped], torch.zeros_like(fused[dropped]))
+
+
+@pytest.mark.parametrize("name", ["fastmoe_txl", "m_swiglu_lam", "m_pair_relu_cap", "m_one", "m_E1"])
+def test_expert_ffn_combine_entry_matches_forward(name):
+    """moe_expert_ffn_combine runs steps 4-5 exactly as the forward does
+    (one-launch kernel on 1-SM tiles, pair tiles otherwise): given the
+    forward's permuted rows, tokens and row weights, and a zeroed out, it
+    must reproduce the forward's output bit for bit, on two calls in a row."""
+    w = mw.WORKLOADS.get(name) or next(m for m in MEDIUM if m.name == name)
+    L = DeviceLayer(w)
+    res = L.forward()
+    ws, lay = res["ws"], res["layout"]
+    T, k, d, F, E = L.T, w.k, w.d, w.F, w.E
+    A = T * k
+
+    def v(off, n, dt):
+        return ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)
+
+    xp = v(lay.xp, A * d, L.tdt)
+    offsets, src_tok, row_w = v(lay.offsets, E + 1, torch.int32), v(lay.src_tok, A, torch.int32), v(lay.row_w, A, torch.float32)
+    h = torch.empty((A, F), dtype=L.hdt, device="cuda")
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        out = torch.zeros((T, d), dtype=torch.float32, device="cuda")
+        moe.moe_expert_ffn_combine(L.cfg, xp, offsets, src_tok, row_w, L.w1, L.w2, h, out, stats, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out, res["out"]), name
+    assert moe.read_stats(stats)["status"] == 0
