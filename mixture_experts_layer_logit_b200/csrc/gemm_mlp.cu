@@ -16,7 +16,7 @@
 // for the token of each row; at most two additions per output, k <= 2).  A
 // layer-2 tile needs the h rows of its m-tile from all layer-1 n-tiles: each
 // epilogue warp of a finished layer-1 tile adds 1 to the m-tile's counter
-// (fence, then release, after its h stores), and the TMA producer of a
+// (a release after its h stores), and the TMA producer of a
 // layer-2 tile waits for the counter to reach 4 x the layer-1 n-tile count
 // (acquire, then a proxy fence so that its TMA reads see those stores).  Tiles are claimed in increasing
 // order, so a claimed layer-2 tile only waits for layer-1 tiles already
@@ -286,7 +286,8 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         const int nrows = warp_rows(p1, wrow0, t.c.rows - qw * 32, lane);
         if (nrows > 0) store_tile<ACT, F16>(p1, tb, wrow0, nrows, t.c.n0, stg, lane, over);
         // this warp's h rows of the tile are written: count them for the m-tile
-        __threadfence();
+        // (__syncwarp orders the lanes' stores before lane 0's release, which
+        // carries them to GPU scope)
         __syncwarp();
         if (lane == 0) red_release_gpu_add(p.dep + t.m, 1);
       } else {

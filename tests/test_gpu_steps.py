@@ -273,3 +273,29 @@ def test_expert_ffn_rejects_corrupt_offsets(dtype, case):
     torch.cuda.synchronize()
     assert moe.read_stats(stats)["status"] & moe.MOE_DEV_BOUNDS
     assert torch.equal(h, h0) and torch.equal(yp, yp0)
+
+
+def test_fp16_hidden_saturates_and_flags():
+    """fp16 hidden activations beyond +-65504 saturate and set MOE_DEV_RANGE;
+    rows that are computed but not stored never raise it (the rows past the
+    kept ones hold NaN here)."""
+    w = W("sat", T=256, d=64, E=4, F=64, k=2, act=mw.RELU, dtype=mw.BF16, seed=31)
+    L = DeviceLayer(w)
+    assert L.hidden == "f16"
+    idx, _, gap, pm = L.route()
+    perm = L.permute(idx, gap, pm)
+    torch.cuda.synchronize()
+    n = int(perm["offsets"][w.E].item())
+    xp = perm["xp"].clone()
+    xp[n:] = float("nan")
+    _, _, st0 = L.expert_ffn(xp, perm["offsets"])
+    torch.cuda.synchronize()
+    assert moe.read_stats(st0)["status"] == 0
+    L.w1.mul_(2.0 ** 17)                 # exact in bf16: pre-activations of ~1e5
+    h, yp, st = L.expert_ffn(xp, perm["offsets"])
+    torch.cuda.synchronize()
+    assert moe.read_stats(st)["status"] & moe.MOE_DEV_RANGE
+    hk = h[:n].float()
+    assert torch.isfinite(hk).all()
+    assert float(hk.abs().max()) == 65504.0
+    assert bool((hk >= 0).all())         # ReLU, saturated to +65504, never wrapped
