@@ -343,7 +343,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   if (one_launch(c) && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
-  // near-tie counts of every chunk in scratch, so step 3 starts at the scan
+  // near-tie counts of every chunk in scratch, so step 3 starts from the
+  // histograms (the scatter scans them itself)
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
                                at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;

@@ -9,11 +9,14 @@
 //
 // Design (one CTA per SM, persistent):
 //   * A = expert-grouped rows (xp or h), B = one expert's weight rows; both
-//     K-major bf16, staged by TMA (128-byte swizzle) into a STAGES-deep ring.
+//     K-major 16-bit (bf16 for layer 1; the hidden type, fp16 or bf16, for
+//     layer 2), staged by TMA (128-byte swizzle) into a STAGES-deep ring.
 //   * warp 0 lane 0 issues the TMA loads, warp 1 lane 0 issues
 //     tcgen05.mma.cta_group::1.kind::f16 (128 x 256 x 16, fp32 accumulators in
-//     TMEM), warps 2-5 drain TMEM with tcgen05.ld, apply the activation
-//     (ReLU, or silu(gate) * up for SwiGLU) and store bf16 rows.
+//     TMEM), warps 2-5 drain TMEM with tcgen05.ld and run the epilogue of
+//     gemm_common.cuh: layer 1 applies the activation (ReLU, or
+//     silu(gate) * up for SwiGLU) and stores h; layer 2 stores fp32 yp or
+//     adds the gate-weighted rows into out (fused combine).
 //   * two 256-column TMEM accumulators let the epilogue of one tile overlap
 //     the main loop of the next.
 //   * the tile table (ceil(M_e / 128) * n-tiles per expert) is built on the
