@@ -15,9 +15,9 @@
 // d = 512 reduction to be in flight at once); tcgen05.mma kind::f16 with
 // M = 128, N = E rounded up to 16 (rows of W_gate past E load as zeros)
 // accumulates the 128 x N logits in fp32 in TMEM.  The epilogue copies them to
-// shared memory and gives every token two threads, each owning half of the
-// experts: partial sums, maxima and top-(k+1) lists are merged through shared
-// memory.  Each CTA is one routing chunk of 128 tokens: it also writes the
+// shared memory and gives every token four threads, each owning a quarter
+// of the experts: partial sums, maxima and top-(k+1) lists are merged through
+// shared memory in quarter order.  Each CTA is one routing chunk of 128 tokens: it also writes the
 // chunk's per-expert histogram, per-expert sum of softmax probabilities
 // (summed in a fixed order) and near-tie count for the permutation step.
 #include "tc_ptx.cuh"
@@ -33,7 +33,7 @@ constexpr int RM = 128;            // tokens per CTA = routing chunk
 constexpr int RK = 64;             // model-width slice per stage (128 bytes of bf16)
 constexpr int kMaxStages = 8;
 constexpr int kRingBytes = 192 * 1024;
-constexpr int kSplit = 2;          // threads per token in the epilogue
+constexpr int kSplit = 4;          // threads per token in the epilogue, each owning a quarter of the experts
 constexpr int kThreads = RM * kSplit;
 constexpr int kMaxKeep = 9;        // top-(k+1) list length for k <= 8
 static_assert(RM == kChunk, "one CTA per routing chunk");
@@ -45,14 +45,30 @@ struct RTail {
   int ntie;
   int hist[kMaxExperts];
   float bias[kMaxExperts];
-  float part[kSplit][4][RM];       // per half: sum, squares, max, exp-sum of each row
-  float lv[kMaxKeep][RM];          // the upper half's top list of each row
-  int li[kMaxKeep][RM];
+  float part[kSplit][4][RM];       // per quarter: sum, squares, max, exp-sum of each row
+};
+
+// The top lists of quarters 1..3 of each row: (score, expert) pairs.  They
+// live in the stage ring after the logits when there is room (the ring is
+// free by then), else after the tail.
+struct RLists {
+  float v[kSplit - 1][kMaxKeep][RM];
+  int i[kSplit - 1][kMaxKeep][RM];
 };
 
 __host__ __device__ constexpr int stage_bytes(int EP) { return RM * RK * 2 + EP * RK * 2; }
 inline int num_stages(int EP) { return std::min(kMaxStages, kRingBytes / stage_bytes(EP)); }
-inline size_t smem_bytes(int EP) { return 1024 + (size_t)num_stages(EP) * stage_bytes(EP) + sizeof(RTail); }
+inline size_t logits_bytes(int E) { return ((size_t)RM * (size_t)(E | 1) * sizeof(float) + 15) & ~(size_t)15; }
+inline bool lists_in_ring(int E, int EP) {
+  return logits_bytes(E) + sizeof(RLists) <= (size_t)num_stages(EP) * stage_bytes(EP);
+}
+// byte offset of the lists from the 1024-aligned base of shared memory
+inline size_t lists_offset(int E, int EP) {
+  return lists_in_ring(E, EP) ? logits_bytes(E) : (size_t)num_stages(EP) * stage_bytes(EP) + sizeof(RTail);
+}
+inline size_t smem_bytes(int E, int EP) {
+  return 1024 + (size_t)num_stages(EP) * stage_bytes(EP) + sizeof(RTail) + (lists_in_ring(E, EP) ? 0 : sizeof(RLists));
+}
 __host__ __device__ constexpr uint32_t tmem_cols(int EP) { return EP <= 32 ? 32 : EP <= 64 ? 64 : EP <= 128 ? 128 : 256; }
 
 // Keeps the N <= KB + 1 best (score, expert) pairs, best first, in registers
@@ -85,9 +101,9 @@ struct TopList {
   }
 };
 
-// Top-N over the scores Z[lo, hi) of one row (and their maximum), then, for
-// the lower half, the upper half's list merged in: its experts all have higher
-// indices, so inserting them (best first) keeps lowest-index-wins order.
+// Top-N over the scores Z[lo, hi) of one row (and their maximum); a later
+// quarter's list is merged in by inserting its pairs best first: its experts
+// all have higher indices, so lowest-index-wins order is kept.
 template <int N, int KB>
 __device__ __forceinline__ float topk_range(TopList<KB>& top, const float* Z, int lo, int hi) {
   float mh = -INFINITY;
@@ -118,7 +134,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
                 int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-                int nch, uint32_t* __restrict__ status) {
+                int nch, uint32_t* __restrict__ status, int lists_off) {
   constexpr int k = KB;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -126,6 +142,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   unsigned char* sbase = smem_raw + (base - raw);
   const int SB = stage_bytes(EP);
   RTail* tail = reinterpret_cast<RTail*>(sbase + (size_t)nst * SB);
+  RLists* lists = reinterpret_cast<RLists*>(sbase + lists_off);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, t0 = chunk * RM;
   const int nkb = (d + RK - 1) / RK;
@@ -210,9 +227,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   // ------------------------------------------------- gating epilogue
   // The logits of each row go from TMEM to a padded shared-memory row (the
   // stage ring is free now; the odd row stride keeps a warp's column accesses
-  // conflict-free).  Warps q and q + 4 read the same TMEM lanes 32q..32q+31:
-  // half 0 owns experts [0, E0), half 1 owns [E0, E).
-  const int q = warp & 3, half = warp >> 2;
+  // conflict-free).  Warps q, q + 4, q + 8 and q + 12 read the same TMEM lanes
+  // 32q..32q+31: quarter p (= warp / 4) owns experts [E p / 4, E (p + 1) / 4).
+  // Partial sums, maxima and top lists of the four quarters meet in shared
+  // memory, always combined in quarter order.
+  const int q = warp & 3, qtr = warp >> 2;
   const int row = q * 32 + lane;
   const int t = t0 + row;
   const bool valid = ok && t < T;
@@ -221,7 +240,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   float* Zall = reinterpret_cast<float*>(sbase);   // [RM][ldz]
   float* Z = Zall + (size_t)row * ldz;
   const int nch32 = (E + 31) / 32;
-  for (int c = half; c < nch32; c += kSplit) {
+  for (int c = qtr; c < nch32; c += kSplit) {
     uint32_t r[32];
     tmem_ld32(tb + c * 32, r);
     tmem_wait_ld();
@@ -232,25 +251,25 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     }
   }
   __syncthreads();
-  const int E0 = (E + 1) / 2;
-  const int lo = half ? E0 : 0, hi = half ? E : E0;
+  const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
   float (*part)[4][RM] = tail->part;
   if (lam > 0.f) {   // z_hat = lambda (z - mean) / std, written over z
     float s = 0.f;
 #pragma unroll 4
     for (int e = lo; e < hi; ++e) s += Z[e];
-    part[half][0][row] = s;
+    part[qtr][0][row] = s;
     __syncthreads();
-    const float mu = (part[0][0][row] + part[1][0][row]) / (float)E;
+    const float mu = (((part[0][0][row] + part[1][0][row]) + part[2][0][row]) + part[3][0][row]) / (float)E;
     float qq = 0.f;
 #pragma unroll 4
     for (int e = lo; e < hi; ++e) {
       const float dv = Z[e] - mu;
       qq += dv * dv;
     }
-    part[half][1][row] = qq;
+    part[qtr][1][row] = qq;
     __syncthreads();
-    const float sd = sqrtf((part[0][1][row] + part[1][1][row]) / (float)E);
+    const float sd =
+        sqrtf((((part[0][1][row] + part[1][1][row]) + part[2][1][row]) + part[3][1][row]) / (float)E);
 #pragma unroll 4
     for (int e = lo; e < hi; ++e) Z[e] = gate_score(Z[e], lam, mu, sd);
   }
@@ -258,16 +277,16 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   TopList<KB> top;
   top.init();
   const float mh = (k < E) ? topk_range<KB + 1>(top, Z, lo, hi) : topk_range<KB>(top, Z, lo, hi);
-  part[half][2][row] = mh;
-  if (half == 1) {
+  part[qtr][2][row] = mh;
+  if (qtr > 0) {
 #pragma unroll
     for (int j = 0; j <= KB; ++j) {
-      tail->lv[j][row] = top.v[j];
-      tail->li[j][row] = top.i[j];
+      lists->v[qtr - 1][j][row] = top.v[j];
+      lists->i[qtr - 1][j][row] = top.i[j];
     }
   }
   __syncthreads();
-  const float m = fmaxf(part[0][2][row], part[1][2][row]);
+  const float m = fmaxf(fmaxf(part[0][2][row], part[1][2][row]), fmaxf(part[2][2][row], part[3][2][row]));
   float Sh = 0.f;
 #pragma unroll 4
   for (int e = lo; e < hi; ++e) {   // unnormalised probabilities over the scores
@@ -275,13 +294,18 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     Z[e] = pe;
     Sh += pe;
   }
-  part[half][3][row] = Sh;
+  part[qtr][3][row] = Sh;
   __syncthreads();
-  const float S = part[0][3][row] + part[1][3][row];
+  const float S = ((part[0][3][row] + part[1][3][row]) + part[2][3][row]) + part[3][3][row];
   const float invS = 1.f / S;
-  if (half == 0) {
-    if (k < E) topk_merge<KB + 1>(top, tail->lv, tail->li, row);
-    else topk_merge<KB>(top, tail->lv, tail->li, row);
+  if (qtr == 0) {
+    // the other quarters' lists, in quarter order: their experts all have
+    // higher indices, so inserting them keeps lowest-index-wins order
+#pragma unroll
+    for (int p = 0; p < kSplit - 1; ++p) {
+      if (k < E) topk_merge<KB + 1>(top, lists->v[p], lists->i[p], row);
+      else topk_merge<KB>(top, lists->v[p], lists->i[p], row);
+    }
     float psel[KB], sel = 0.f;
 #pragma unroll
     for (int j = 0; j < KB; ++j) {
@@ -337,12 +361,18 @@ template <int KB>
 cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
                       int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
                       uint32_t* status, cudaStream_t s) {
-  // the ring never exceeds kRingBytes, whatever E is
-  cudaError_t err = set_smem_once<route_tc_kernel<KB>>(1024 + (size_t)kRingBytes + sizeof(RTail));
+  // the most any E <= kMaxExperts needs, so one attribute serves every launch
+  static const size_t kMaxSmem = [] {
+    size_t m = 0;
+    for (int e = 1; e <= kMaxExperts; ++e) m = std::max(m, smem_bytes(e, ((e + 15) / 16) * 16));
+    return m;
+  }();
+  cudaError_t err = set_smem_once<route_tc_kernel<KB>>(kMaxSmem);
   if (err != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
-  return launch_pdl(route_tc_kernel<KB>, dim3(nch), dim3(kThreads), smem_bytes(EP), s, mx, mw, bg, c.T, c.d, c.E,
-                    EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status);
+  return launch_pdl(route_tc_kernel<KB>, dim3(nch), dim3(kThreads), smem_bytes(c.E, EP), s, mx, mw, bg, c.T, c.d,
+                    c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status,
+                    (int)lists_offset(c.E, EP));
 }
 
 }  // namespace
