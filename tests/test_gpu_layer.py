@@ -65,6 +65,10 @@ MEDIUM = [
     W("m_multi_tile", T=3000, d=512, E=4, F=640, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=29),   # 2-SM tiles
     W("m_pair_relu_cap", T=2600, d=128, E=8, F=192, k=2, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.1,
       seed=30),                                                                                  # 2-SM tiles
+    # one-launch expert kernel with the largest expert count: 256 tile-table
+    # entries and dependency counters, many experts with no rows
+    W("m_E256_k2", T=900, d=64, E=256, F=64, k=2, act=mw.SWIGLU, dtype=mw.BF16, capacity_factor=1.5, lam=1.0,
+      zipf_bias=True, seed=32),
 ]
 
 
@@ -118,7 +122,7 @@ def test_layer_named_full_size_sampled(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", ["m_swiglu_lam", "m_E1", "m_one", "m_pair_relu_cap", "fastmoe_txl"])
+@pytest.mark.parametrize("name", ["m_swiglu_lam", "m_E1", "m_one", "m_pair_relu_cap", "m_E256_k2", "fastmoe_txl"])
 def test_fused_combine_matches_the_steps(name):
     """bf16 layers with k <= 2: the forward adds the gate-weighted expert
     outputs inside the second GEMM (out zeroed by the permutation) instead of
