@@ -299,3 +299,25 @@ def test_fp16_hidden_saturates_and_flags():
     assert torch.isfinite(hk).all()
     assert float(hk.abs().max()) == 65504.0
     assert bool((hk >= 0).all())         # ReLU, saturated to +65504, never wrapped
+
+
+@pytest.mark.parametrize("offsets", [[0, 100, 130, 150, 160], [0, 0, 64, 65, 65], [0, 63, 64, 128, 160]])
+def test_expert_ffn_short_layer_any_segment(offsets):
+    """Caller-made expert segments on a small layer: longer than the layer's
+    token count (an expert repeated inside a token), empty, or ending on and
+    just past tile edges; every row must match the oracle's experts."""
+    w = W("short", T=40, d=64, E=4, F=64, k=4, act=mw.SWIGLU, dtype=mw.BF16, seed=33)
+    L = DeviceLayer(w)
+    _, _, _, w1, w2 = oracle_inputs(L)
+    cfg = lcfg_of(w, L.T)
+    A = L.T * w.k
+    g = torch.Generator().manual_seed(7)
+    xp = torch.randn((A, w.d), generator=g).to(torch.bfloat16).cuda()
+    off = torch.tensor(offsets, dtype=torch.int32).cuda()
+    h, yp, stats = L.expert_ffn(xp, off)
+    torch.cuda.synchronize()
+    assert moe.read_stats(stats)["status"] == 0
+    n = offsets[-1]
+    xp64 = xp.float().cpu().numpy().astype(np.float64)
+    _, yp_ref = om.expert_segments(xp64[:n], np.array(offsets), w1, w2, cfg)
+    check_out(to_np64(yp[:n]), yp_ref, w.dtype)
