@@ -44,6 +44,7 @@ Scratch scratch_layout(const moe_config& c) {
   s.psum = off;  off = align256(off + sizeof(float) * (size_t)c.E * nch);
   s.ntie = off;  off = align256(off + sizeof(int32_t) * nch);
   s.status = off; off = align256(off + sizeof(uint32_t));
+  s.kslice = off; off = align256(off + route_tc_scratch_bytes(c));
   s.total = off > 0 ? off : 256;
   return s;
 }
@@ -226,7 +227,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const
   if ((st = check_device(false)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(c, x, Wg, bg, topk_idx, topk_w, gap, at<int32_t>(ws, sc.hist),
-                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<uint32_t>(ws, sc.status), s);
+                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<uint32_t>(ws, sc.status),
+                               at<char>(ws, sc.kslice), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (prob_mean != nullptr) e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s);
   return cuda_status(e);
@@ -346,7 +348,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   // near-tie counts of every chunk in scratch, so step 3 starts from the
   // histograms (the scatter scans them itself)
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
-                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status, s);
+                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status,
+                               at<char>(scr, sc.kslice), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   float* row_w = at<float>(ws, L.row_w);
   float* out_f = static_cast<float*>(out);

@@ -6,8 +6,12 @@
 // page, "MoE负载均衡的挑战与应对").  The sum itself is the definition of the
 // layer output (FastMoE announcement, "1. MoE 设计").
 //
-// One warp per token; each lane owns 16-byte column vectors of the row and
-// issues the k row reads of a vector back to back.
+// One warp per (token, column slice).  A token's row of 16-byte vectors is
+// dealt to `nslice` warps: slice s takes vectors s*32 + lane, then every
+// 32*nslice after that.  Each lane issues the k row reads of a vector back to
+// back.  A large batch keeps nslice = 1 (one warp walks the whole row).  A
+// small one (decode) splits its rows so that enough warps keep reads in
+// flight: otherwise each warp would wait on d/128 serial read latencies.
 #include "internal.cuh"
 
 namespace moe {
@@ -33,12 +37,13 @@ template <> struct Pack<float> {
 template <typename TX, int KB>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
-               const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
+               const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k, int nslice) {
   constexpr int N = Pack<TX>::N;
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kTokPerBlock + warp;
+  const int g = blockIdx.x * kTokPerBlock + warp;
+  const int t = g / nslice, sl = g - t * nslice;
   if (t >= T) return;
   int rows[KB];
   float ws[KB];
@@ -51,7 +56,7 @@ combine_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
   }
   const int nvec = d / N;
   uint4* o = reinterpret_cast<uint4*>(out + (size_t)t * d);
-  for (int v = lane; v < nvec; v += 32) {
+  for (int v = sl * 32 + lane; v < nvec; v += 32 * nslice) {
     uint4 in[KB];
 #pragma unroll
     for (int j = 0; j < KB; ++j)
@@ -70,16 +75,18 @@ combine_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
 template <typename TX>
 __global__ void __launch_bounds__(kThreads)
 combine_generic_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ row_of,
-                       const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k) {
+                       const float* __restrict__ topk_w, TX* __restrict__ out, int T, int d, int k,
+                       int nslice) {
   constexpr int N = Pack<TX>::N;
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kTokPerBlock + warp;
+  const int g = blockIdx.x * kTokPerBlock + warp;
+  const int t = g / nslice, sl = g - t * nslice;
   if (t >= T) return;
   const int nvec = d / N;
   uint4* o = reinterpret_cast<uint4*>(out + (size_t)t * d);
-  for (int v = lane; v < nvec; v += 32) {
+  for (int v = sl * 32 + lane; v < nvec; v += 32 * nslice) {
     float a[N];
 #pragma unroll
     for (int i = 0; i < N; ++i) a[i] = 0.f;
@@ -92,18 +99,33 @@ combine_generic_kernel(const TX* __restrict__ yp, const int32_t* __restrict__ ro
   }
 }
 
+// Column slices per token: doubled while the batch gives fewer than 32 warps
+// per SM, and never more than one 32-vector group per slice.
+int num_slices(const moe_config& c, int N, int sms) {
+  const int groups = (c.d / N + 31) / 32;
+  const long long want = 32LL * sms;
+  int ns = 1;
+  while (ns < groups && (long long)c.T * ns < want) ns *= 2;
+  return ns < groups ? ns : (groups > 0 ? groups : 1);
+}
+
 template <typename TX>
 cudaError_t launch_t(const moe_config& c, const void* yp, const int32_t* row_of, const float* w,
                      void* out, cudaStream_t s) {
-  const int grid = (c.T + kTokPerBlock - 1) / kTokPerBlock;
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const int ns = num_slices(c, Pack<TX>::N, di.sms);
+  const long long grid = ((long long)c.T * ns + kTokPerBlock - 1) / kTokPerBlock;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const TX* y = static_cast<const TX*>(yp);
   TX* o = static_cast<TX*>(out);
-  const dim3 g(grid), b(kThreads);
-  if (c.k <= 1) return launch_pdl(combine_kernel<TX, 1>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
-  if (c.k <= 2) return launch_pdl(combine_kernel<TX, 2>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
-  if (c.k <= 4) return launch_pdl(combine_kernel<TX, 4>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
-  if (c.k <= 8) return launch_pdl(combine_kernel<TX, 8>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
-  return launch_pdl(combine_generic_kernel<TX>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k);
+  const dim3 g((unsigned)grid), b(kThreads);
+  if (c.k <= 1) return launch_pdl(combine_kernel<TX, 1>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k, ns);
+  if (c.k <= 2) return launch_pdl(combine_kernel<TX, 2>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k, ns);
+  if (c.k <= 4) return launch_pdl(combine_kernel<TX, 4>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k, ns);
+  if (c.k <= 8) return launch_pdl(combine_kernel<TX, 8>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k, ns);
+  return launch_pdl(combine_generic_kernel<TX>, g, b, 0, s, y, row_of, w, o, c.T, c.d, c.k, ns);
 }
 
 }  // namespace

@@ -24,6 +24,7 @@ struct Scratch {
   size_t psum;      // float [nchunks][E]   per-chunk sums of softmax probabilities
   size_t ntie;      // int32 [nchunks]      near-tie tokens per chunk
   size_t status;    // uint32               device error bits of a standalone moe_route
+  size_t kslice;    // the route's K-slice arrival counters and partial logits (may be empty); last
   size_t total;
 };
 
@@ -37,14 +38,19 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Route: logits, normalisation, softmax, top-k; per-chunk histogram, probability
 // sums and near-tie counts into scratch.  TX = float or __nv_bfloat16.
+// kscratch: route_tc_scratch_bytes(c) bytes (or NULL: no K-slice split).
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
-                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, cudaStream_t s);
+                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, void* kscratch,
+                         cudaStream_t s);
 // The same on tcgen05 tensor cores (bf16, k <= 8).
 bool route_tc_supported(const moe_config& c);
+// Scratch bytes of the tensor-core route's model-width split (0 when it never
+// splits this layer): per-chunk arrival counters, then the partial logits.
+size_t route_tc_scratch_bytes(const moe_config& c);
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, uint32_t* status, cudaStream_t s);
+                            int32_t* ntie, uint32_t* status, void* kscratch, cudaStream_t s);
 // prob_mean[e] = sum over chunks of psum / T (fixed order).
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
 // Histogram of topk_idx per chunk (+ near ties from gap when given).

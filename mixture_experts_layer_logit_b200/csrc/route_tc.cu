@@ -20,6 +20,14 @@
 // shared memory in quarter order.  Each CTA is one routing chunk of 128 tokens: it also writes the
 // chunk's per-expert histogram, per-expert sum of softmax probabilities
 // (summed in a fixed order) and near-tie count for the permutation step.
+//
+// A small batch with a wide model (decode: one chunk, d = 2048) would leave
+// the reduction to one SM, one ring of loads after another.  There the model
+// width is cut into up to 8 slices, one CTA each.  Every CTA writes its
+// partial logits to the scratch workspace and takes a ticket.  The last CTA
+// of the chunk to arrive adds the partials in slice order (the same sum
+// whichever CTA comes last) and runs the epilogue.  Nothing waits on another
+// CTA, so the split cannot stall.
 #include "tc_ptx.cuh"
 
 #include <math.h>
@@ -36,6 +44,9 @@ constexpr int kRingBytes = 192 * 1024;
 constexpr int kSplit = 4;          // threads per token in the epilogue, each owning a quarter of the experts
 constexpr int kThreads = RM * kSplit;
 constexpr int kMaxKeep = 9;        // top-(k+1) list length for k <= 8
+constexpr int kMaxKSlices = 8;     // CTAs that may share one chunk's model width
+constexpr int kKSliceMaxChunks = 74;           // only batches of at most this many chunks split
+constexpr size_t kKSliceBudget = 1u << 20;     // bytes of partial logits at most
 static_assert(RM == kChunk, "one CTA per routing chunk");
 
 struct RTail {
@@ -43,6 +54,7 @@ struct RTail {
   uint32_t tmem_base;
   int abort_flag;
   int ntie;
+  int ticket;                      // arrival order of this CTA among its chunk's slices
   int hist[kMaxExperts];
   float bias[kMaxExperts];
   float part[kSplit][4][RM];       // per quarter: sum, squares, max, exp-sum of each row
@@ -134,7 +146,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
                 int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-                int nch, uint32_t* __restrict__ status, int lists_off) {
+                int nch, uint32_t* __restrict__ status, int lists_off, float* __restrict__ kpart,
+                int* __restrict__ karrive, int nks) {
   constexpr int k = KB;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -144,8 +157,9 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   RTail* tail = reinterpret_cast<RTail*>(sbase + (size_t)nst * SB);
   RLists* lists = reinterpret_cast<RLists*>(sbase + lists_off);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, t0 = chunk * RM;
-  const int nkb = (d + RK - 1) / RK;
+  const int chunk = blockIdx.x / nks, ks = blockIdx.x - chunk * nks, t0 = chunk * RM;
+  const int nkb_all = (d + RK - 1) / RK;   // the host keeps nks <= nkb_all
+  const int kb0 = (nkb_all * ks) / nks, nkb = (nkb_all * (ks + 1)) / nks - kb0;
   const uint32_t full0 = smem_u32(&tail->full[0]), empty0 = smem_u32(&tail->empty[0]);
   const uint32_t done = smem_u32(&tail->done);
   const volatile int* abort_flag = &tail->abort_flag;
@@ -192,8 +206,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       }
       const uint32_t sa = base + (uint32_t)(s * SB);
       mbar_expect_tx(full0 + 8 * s, (uint32_t)SB);
-      tma_load_2d(sa, &tmX, full0 + 8 * s, kb * RK, t0);
-      tma_load_2d(sa + RM * RK * 2, &tmW, full0 + 8 * s, kb * RK, 0);
+      tma_load_2d(sa, &tmX, full0 + 8 * s, (kb0 + kb) * RK, t0);
+      tma_load_2d(sa + RM * RK * 2, &tmW, full0 + 8 * s, (kb0 + kb) * RK, 0);
       ++issued;
     }
     for (int i = max(0, issued - nst); i < issued; ++i)   // loads still in flight
@@ -247,120 +261,187 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int e = c * 32 + i;
-      if (e < E) Z[e] = __uint_as_float(r[i]) + tail->bias[e];
+      if (e < E) Z[e] = __uint_as_float(r[i]) + (nks == 1 ? tail->bias[e] : 0.f);
     }
   }
-  __syncthreads();
-  const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
-  float (*part)[4][RM] = tail->part;
-  if (lam > 0.f) {   // z_hat = lambda (z - mean) / std, written over z
-    float s = 0.f;
-#pragma unroll 4
-    for (int e = lo; e < hi; ++e) s += Z[e];
-    part[qtr][0][row] = s;
-    __syncthreads();
-    const float mu = (((part[0][0][row] + part[1][0][row]) + part[2][0][row]) + part[3][0][row]) / (float)E;
-    float qq = 0.f;
-#pragma unroll 4
-    for (int e = lo; e < hi; ++e) {
-      const float dv = Z[e] - mu;
-      qq += dv * dv;
-    }
-    part[qtr][1][row] = qq;
-    __syncthreads();
-    const float sd =
-        sqrtf((((part[0][1][row] + part[1][1][row]) + part[2][1][row]) + part[3][1][row]) / (float)E);
-#pragma unroll 4
-    for (int e = lo; e < hi; ++e) Z[e] = gate_score(Z[e], lam, mu, sd);
-  }
-  // the (k+1)-th score is only needed for the gap, which does not exist when k == E
-  TopList<KB> top;
-  top.init();
-  const float mh = (k < E) ? topk_range<KB + 1>(top, Z, lo, hi) : topk_range<KB>(top, Z, lo, hi);
-  part[qtr][2][row] = mh;
-  if (qtr > 0) {
-#pragma unroll
-    for (int j = 0; j <= KB; ++j) {
-      lists->v[qtr - 1][j][row] = top.v[j];
-      lists->i[qtr - 1][j][row] = top.i[j];
-    }
-  }
-  __syncthreads();
-  const float m = fmaxf(fmaxf(part[0][2][row], part[1][2][row]), fmaxf(part[2][2][row], part[3][2][row]));
-  float Sh = 0.f;
-#pragma unroll 4
-  for (int e = lo; e < hi; ++e) {   // unnormalised probabilities over the scores
-    const float pe = __expf(Z[e] - m);
-    Z[e] = pe;
-    Sh += pe;
-  }
-  part[qtr][3][row] = Sh;
-  __syncthreads();
-  const float S = ((part[0][3][row] + part[1][3][row]) + part[2][3][row]) + part[3][3][row];
-  const float invS = 1.f / S;
-  if (qtr == 0) {
-    // the other quarters' lists, in quarter order: their experts all have
-    // higher indices, so inserting them keeps lowest-index-wins order
-#pragma unroll
-    for (int p = 0; p < kSplit - 1; ++p) {
-      if (k < E) topk_merge<KB + 1>(top, lists->v[p], lists->i[p], row);
-      else topk_merge<KB>(top, lists->v[p], lists->i[p], row);
-    }
-    float psel[KB], sel = 0.f;
-#pragma unroll
-    for (int j = 0; j < KB; ++j) {
-      psel[j] = __expf(top.v[j] - m) * invS;
-      sel += psel[j];                     // slot order
-    }
-    const float rs = 1.f / sel;
-    const float gap = (k < E) ? top.v[k - 1] - top.v[k] : INFINITY;
-    if (valid) {
-#pragma unroll
-      for (int j = 0; j < KB; ++j) {
-        topk_idx[(size_t)t * k + j] = top.i[j];
-        topk_w[(size_t)t * k + j] = psel[j] * rs;
-        atomicAdd(&tail->hist[top.i[j]], 1);
-      }
-      gap_out[t] = gap;
-      if (gap < MOE_NEAR_TIE_GAP) atomicAdd(&tail->ntie, 1);
-    }
-  }
-
-  // per-expert probability sums of the chunk: the probabilities of each row in
-  // shared memory, columns summed by nG groups of threads over row ranges, the
-  // group partials added in group order (fixed order, deterministic)
-#pragma unroll 4
-  for (int e = lo; e < hi; ++e) Z[e] = valid ? Z[e] * invS : 0.f;
   tc_fence_before();
   __syncthreads();
-  float* colpart = &part[0][0][0];               // [nG][E]; part is free again
-  const int nG = kThreads / E;                   // >= 1 since E <= 256 = kThreads
-  const int R = (RM + nG - 1) / nG;
-  if (tid < nG * E) {
-    const int e = tid % E, g = tid / E;
-    float s = 0.f;
-    const int r1 = min(RM, (g + 1) * R);
-    for (int rr = g * R; rr < r1; ++rr) s += Zall[(size_t)rr * ldz + e];
-    colpart[g * E + e] = s;
+  bool lead = true;   // this CTA finishes the chunk
+  if (nks > 1) {
+    // partials [chunk][slice][row][expert] in fp32 (RM * E is a multiple of 4:
+    // 16-byte vectors); fence, then the ticket
+    const int nv = RM * E / 4;
+    float4* mine = reinterpret_cast<float4*>(kpart + ((size_t)chunk * nks + ks) * RM * E);
+    for (int v = tid; v < nv; v += kThreads) {
+      float z[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = 4 * v + u, r = i / E;
+        z[u] = Zall[(size_t)r * ldz + (i - r * E)];
+      }
+      mine[v] = make_float4(z[0], z[1], z[2], z[3]);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) tail->ticket = atomicAdd(&karrive[chunk], 1);
+    __syncthreads();
+    lead = tail->ticket == nks - 1;
+    if (lead) {
+      __threadfence();
+      // every slice's vector is loaded before any is added, so the loads
+      // overlap; the additions run in slice order
+      const float4* c0 = reinterpret_cast<const float4*>(kpart + (size_t)chunk * nks * RM * E);
+      for (int v = tid; v < nv; v += kThreads) {
+        float4 p[kMaxKSlices];
+#pragma unroll
+        for (int sl = 0; sl < kMaxKSlices; ++sl)
+          if (sl < nks) p[sl] = __ldcg(c0 + (size_t)sl * nv + v);
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int sl = 0; sl < kMaxKSlices; ++sl)
+          if (sl < nks) {
+            z[0] += p[sl].x;
+            z[1] += p[sl].y;
+            z[2] += p[sl].z;
+            z[3] += p[sl].w;
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * v + u, r = i / E, e = i - r * E;
+          Zall[(size_t)r * ldz + e] = z[u] + tail->bias[e];
+        }
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int e = tid; e < E; e += kThreads) {
-    float s = 0.f;
-    for (int g = 0; g < nG; ++g) s += colpart[g * E + e];
-    psum_out[(size_t)chunk * E + e] = s;
-    hist_out[(size_t)e * nch + chunk] = tail->hist[e];
-  }
-  if (tid == 0) ntie_out[chunk] = tail->ntie;
+  if (lead) {
+    const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
+    float (*part)[4][RM] = tail->part;
+    if (lam > 0.f) {   // z_hat = lambda (z - mean) / std, written over z
+      float s = 0.f;
+#pragma unroll 4
+      for (int e = lo; e < hi; ++e) s += Z[e];
+      part[qtr][0][row] = s;
+      __syncthreads();
+      const float mu = (((part[0][0][row] + part[1][0][row]) + part[2][0][row]) + part[3][0][row]) / (float)E;
+      float qq = 0.f;
+#pragma unroll 4
+      for (int e = lo; e < hi; ++e) {
+        const float dv = Z[e] - mu;
+        qq += dv * dv;
+      }
+      part[qtr][1][row] = qq;
+      __syncthreads();
+      const float sd =
+          sqrtf((((part[0][1][row] + part[1][1][row]) + part[2][1][row]) + part[3][1][row]) / (float)E);
+#pragma unroll 4
+      for (int e = lo; e < hi; ++e) Z[e] = gate_score(Z[e], lam, mu, sd);
+    }
+    // the (k+1)-th score is only needed for the gap, which does not exist when k == E
+    TopList<KB> top;
+    top.init();
+    const float mh = (k < E) ? topk_range<KB + 1>(top, Z, lo, hi) : topk_range<KB>(top, Z, lo, hi);
+    part[qtr][2][row] = mh;
+    if (qtr > 0) {
+#pragma unroll
+      for (int j = 0; j <= KB; ++j) {
+        lists->v[qtr - 1][j][row] = top.v[j];
+        lists->i[qtr - 1][j][row] = top.i[j];
+      }
+    }
+    __syncthreads();
+    const float m = fmaxf(fmaxf(part[0][2][row], part[1][2][row]), fmaxf(part[2][2][row], part[3][2][row]));
+    float Sh = 0.f;
+#pragma unroll 4
+    for (int e = lo; e < hi; ++e) {   // unnormalised probabilities over the scores
+      const float pe = __expf(Z[e] - m);
+      Z[e] = pe;
+      Sh += pe;
+    }
+    part[qtr][3][row] = Sh;
+    __syncthreads();
+    const float S = ((part[0][3][row] + part[1][3][row]) + part[2][3][row]) + part[3][3][row];
+    const float invS = 1.f / S;
+    if (qtr == 0) {
+      // the other quarters' lists, in quarter order: their experts all have
+      // higher indices, so inserting them keeps lowest-index-wins order
+#pragma unroll
+      for (int p = 0; p < kSplit - 1; ++p) {
+        if (k < E) topk_merge<KB + 1>(top, lists->v[p], lists->i[p], row);
+        else topk_merge<KB>(top, lists->v[p], lists->i[p], row);
+      }
+      float psel[KB], sel = 0.f;
+#pragma unroll
+      for (int j = 0; j < KB; ++j) {
+        psel[j] = __expf(top.v[j] - m) * invS;
+        sel += psel[j];                     // slot order
+      }
+      const float rs = 1.f / sel;
+      const float gap = (k < E) ? top.v[k - 1] - top.v[k] : INFINITY;
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+          topk_idx[(size_t)t * k + j] = top.i[j];
+          topk_w[(size_t)t * k + j] = psel[j] * rs;
+          atomicAdd(&tail->hist[top.i[j]], 1);
+        }
+        gap_out[t] = gap;
+        if (gap < MOE_NEAR_TIE_GAP) atomicAdd(&tail->ntie, 1);
+      }
+    }
+
+    // per-expert probability sums of the chunk: the probabilities of each row in
+    // shared memory, columns summed by nG groups of threads over row ranges, the
+    // group partials added in group order (fixed order, deterministic)
+#pragma unroll 4
+    for (int e = lo; e < hi; ++e) Z[e] = valid ? Z[e] * invS : 0.f;
+    tc_fence_before();
+    __syncthreads();
+    float* colpart = &part[0][0][0];               // [nG][E]; part is free again
+    const int nG = kThreads / E;                   // >= 1 since E <= 256 = kThreads
+    const int R = (RM + nG - 1) / nG;
+    if (tid < nG * E) {
+      const int e = tid % E, g = tid / E;
+      float s = 0.f;
+      const int r1 = min(RM, (g + 1) * R);
+      for (int rr = g * R; rr < r1; ++rr) s += Zall[(size_t)rr * ldz + e];
+      colpart[g * E + e] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kThreads) {
+      float s = 0.f;
+      for (int g = 0; g < nG; ++g) s += colpart[g * E + e];
+      psum_out[(size_t)chunk * E + e] = s;
+      hist_out[(size_t)e * nch + chunk] = tail->hist[e];
+    }
+    if (tid == 0) ntie_out[chunk] = tail->ntie;
+  }   // lead
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
   }
 }
 
+// Slices of the model width per chunk: doubled while the reduction takes more
+// than one round of the stage ring, each slice keeps at least half a ring of
+// k-blocks, the grid stays within one CTA per SM and the partials within the
+// budget.
+int kslices(const moe_config& c, long long sms) {
+  const int EP = ((c.E + 15) / 16) * 16;
+  const int nch = num_chunks(c.T), nkb = (c.d + RK - 1) / RK, nst = num_stages(EP);
+  if (nkb <= nst || nch > kKSliceMaxChunks) return 1;
+  int n = 1;
+  while (n < kMaxKSlices && (long long)nch * n * 2 <= sms && nkb / (n * 2) >= nst / 2 &&
+         (size_t)nch * n * 2 * RM * c.E * sizeof(float) <= kKSliceBudget)
+    n *= 2;
+  return n;
+}
+size_t karrive_bytes(int nch) { return ((size_t)nch * sizeof(int) + 255) & ~(size_t)255; }
+
 template <int KB>
 cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
                       int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
-                      uint32_t* status, cudaStream_t s) {
+                      uint32_t* status, void* kscratch, cudaStream_t s) {
   // the most any E <= kMaxExperts needs, so one attribute serves every launch
   static const size_t kMaxSmem = [] {
     size_t m = 0;
@@ -369,19 +450,33 @@ cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensor
   }();
   cudaError_t err = set_smem_once<route_tc_kernel<KB>>(kMaxSmem);
   if (err != cudaSuccess) return err;
+  DeviceInfo di;
+  if ((err = device_info(&di)) != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
-  return launch_pdl(route_tc_kernel<KB>, dim3(nch), dim3(kThreads), smem_bytes(c.E, EP), s, mx, mw, bg, c.T, c.d,
-                    c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status,
-                    (int)lists_offset(c.E, EP));
+  const int nks = kscratch != nullptr ? kslices(c, di.sms) : 1;
+  int* karrive = static_cast<int*>(kscratch);
+  float* kpart = nks > 1 ? reinterpret_cast<float*>(static_cast<char*>(kscratch) + karrive_bytes(nch)) : nullptr;
+  if (nks > 1 && (err = cudaMemsetAsync(karrive, 0, sizeof(int) * (size_t)nch, s)) != cudaSuccess) return err;
+  return launch_pdl(route_tc_kernel<KB>, dim3(nch * nks), dim3(kThreads), smem_bytes(c.E, EP), s, mx, mw, bg, c.T,
+                    c.d, c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status,
+                    (int)lists_offset(c.E, EP), kpart, karrive, nks);
 }
 
 }  // namespace
 
 bool route_tc_supported(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.k <= 8; }
 
+size_t route_tc_scratch_bytes(const moe_config& c) {
+  if (!route_tc_supported(c) || c.T <= 0) return 0;
+  const int n = kslices(c, 1LL << 30);   // the most any device could choose
+  if (n == 1) return 0;
+  const int nch = num_chunks(c.T);
+  return karrive_bytes(nch) + (size_t)nch * n * RM * c.E * sizeof(float);
+}
+
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, uint32_t* status, cudaStream_t s) {
+                            int32_t* ntie, uint32_t* status, void* kscratch, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int EP = ((c.E + 15) / 16) * 16;
   CUtensorMap mx, mw;
@@ -389,7 +484,7 @@ cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, 
       !make_map(&mw, wg, (uint64_t)c.E, (uint64_t)c.d, false, (uint32_t)EP))
     return cudaErrorInvalidValue;
 #define MOE_ROUTE_K(K) \
-  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, s)
+  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, kscratch, s)
   switch (c.k) {
     MOE_ROUTE_K(1); MOE_ROUTE_K(2); MOE_ROUTE_K(3); MOE_ROUTE_K(4);
     MOE_ROUTE_K(5); MOE_ROUTE_K(6); MOE_ROUTE_K(7); MOE_ROUTE_K(8);

@@ -69,6 +69,9 @@ MEDIUM = [
     # entries and dependency counters, many experts with no rows
     W("m_E256_k2", T=900, d=64, E=256, F=64, k=2, act=mw.SWIGLU, dtype=mw.BF16, capacity_factor=1.5, lam=1.0,
       zipf_bias=True, seed=32),
+    # gate GEMM cut over the model width (2 chunks x 4 slices of 6 k-blocks)
+    W("m_ksplit", T=200, d=1536, E=32, F=96, k=4, act=mw.SWIGLU, dtype=mw.BF16, capacity_factor=1.25, lam=1.0,
+      seed=35),
 ]
 
 

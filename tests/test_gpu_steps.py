@@ -35,6 +35,14 @@ MEDIUM = {
                           capacity_factor=1.25, seed=19),
     "pair_swiglu_lambda": W("pair_swiglu_lambda", T=1500, d=192, E=3, F=208, k=2, act=mw.SWIGLU, dtype=mw.BF16,
                             lam=1.0, seed=20),
+    # model widths of more than one ring of gate loads on few chunks: the gate
+    # GEMM is cut over the model width (4 slices here, the last one 5 k-blocks
+    # with a zero-filled tail, d = 1072), partials summed by the last CTA;
+    # E = 24 is not a multiple of 16, with normalisation and a gate bias
+    "ksplit_lambda_bias": W("ksplit_lambda_bias", T=300, d=1072, E=24, F=64, k=3, act=mw.SWIGLU, dtype=mw.BF16,
+                            capacity_factor=1.0, lam=1.0, zipf_bias=True, seed=33),
+    # one chunk, the largest expert count and k (4 slices of 2 k-blocks)
+    "ksplit_E256_k8": W("ksplit_E256_k8", T=64, d=512, E=256, F=32, k=8, act=mw.RELU, dtype=mw.BF16, seed=34),
 }
 
 
