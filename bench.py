@@ -420,6 +420,9 @@ def main():
         # row weights; out is zeroed before each call, outside the events.
         fused = fused_combine(w)
         one_launch = fused and w.T * w.k < 512 * w.E
+        # without the fused combine, bf16 layers on 1-SM tiles run the expert
+        # step as one launch writing yp (moe_expert_ffn and the forward alike)
+        plain_launch = (not fused) and w.dtype == mw.BF16 and w.T * w.k < 512 * w.E
         if fused:
             row_w = sv(L.row_w, A, torch.float32)
             out_fc = torch.empty_like(out)
@@ -458,6 +461,8 @@ def main():
             kname, nl = "tc_expert_mlp (steps 4-5 in one launch: both expert layers + the combine)", 1
         elif fused:
             kname, nl = "tc_grouped_gemm(_pair) (layer 1, then layer 2 with the combine fused: 2 launches)", 2
+        elif plain_launch:
+            kname, nl = "tc_expert_mlp (step 4 in one launch: both expert layers, writing yp)", 1
         else:
             kname, nl = "tc_grouped_gemm(_pair) (expert FFN step: 2 launches, layer 1 + layer 2)", 2
         roofline.update({

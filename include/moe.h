@@ -270,8 +270,8 @@ moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_str
  * convention for users that cannot hand out device memory.
  *   Arguments, layout, ownership and results: as moe_permute, minus ws.
  *   Limit: moe_scratch_size(cfg) <= MOE_STATIC_SCRATCH_BYTES, else
- *     MOE_ERR_UNSUPPORTED before any device work (e.g. E = 64 experts allows
- *     T up to about 347k tokens).
+ *     MOE_ERR_UNSUPPORTED before any device work (e.g. E = 64 experts, k = 2
+ *     allows T up to about 344k tokens on the bf16 path, 347k on fp32).
  *   The first call on a device looks up the array's address (that device
  *     must be current) and returns MOE_ERR_CUDA if the lookup fails.
  *   Every scratch word the kernels read is written earlier in the same call;

@@ -44,6 +44,7 @@ Scratch scratch_layout(const moe_config& c) {
   s.psum = off;  off = align256(off + sizeof(float) * (size_t)c.E * nch);
   s.ntie = off;  off = align256(off + sizeof(int32_t) * nch);
   s.status = off; off = align256(off + sizeof(uint32_t));
+  s.mlp = off;    off = align256(off + (c.dtype == MOE_DTYPE_BF16 ? sizeof(int) * expert_mlp_counters(c) : 0));
   s.kslice = off; off = align256(off + route_tc_scratch_bytes(c));
   s.total = off > 0 ? off : 256;
   return s;
@@ -171,6 +172,21 @@ bool one_launch(const moe_config& c) {
          sizeof(int) * expert_mlp_counters(c) <= sizeof(float) * (size_t)c.T * c.k * c.d;
 }
 
+// Without the fused combine, the two expert layers on 1-SM tiles still run as
+// one launch that writes yp (the expert step on its own, and the forward when
+// k > 2); the tile queue's counters live in scratch.
+bool one_launch_plain(const moe_config& c) {
+  return c.dtype == MOE_DTYPE_BF16 && c.T > 0 && !pair_tiles(c);
+}
+moe_status expert_mlp_plain(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
+                            const void* w2, void* h, void* yp, moe_stats* stats, int* counters,
+                            bool counters_zeroed, cudaStream_t s) {
+  if (!counters_zeroed && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, nullptr, static_cast<float*>(yp), counters,
+                                       &stats->status, s));
+}
+
 // Steps 4-5 fused (out zeroed beforehand); counters: the yp region.
 moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* offsets, const int32_t* src_tok,
                            const float* row_w, const void* w1, const void* w2, void* h, float* out, int* counters,
@@ -179,7 +195,7 @@ moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* o
   if (one_launch(c)) {
     if (!counters_zeroed && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
       return MOE_ERR_CUDA;
-    return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, comb, counters, &stats->status, s));
+    return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, &comb, nullptr, counters, &stats->status, s));
   }
   return expert_ffn(c, xp, offsets, w1, w2, h, yp, stats, s, &comb);
 }
@@ -277,7 +293,10 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* 
   const Scratch sc = scratch_layout(c);
   if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
   if ((st = check_device(c.dtype == MOE_DTYPE_BF16)) != MOE_OK) return st;
-  return expert_ffn(c, xp, offsets, W1, W2, h, yp, stats, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (one_launch_plain(c))
+    return expert_mlp_plain(c, xp, offsets, W1, W2, h, yp, stats, at<int>(ws, sc.mlp), false, s);
+  return expert_ffn(c, xp, offsets, W1, W2, h, yp, stats, s);
 }
 
 moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* xp, const int32_t* offsets,
@@ -339,10 +358,14 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   void* yp = at<char>(ws, L.yp);
 
   const bool fuse = fused_combine(c);
-  int* counters = at<int>(ws, L.yp);
+  // the tile queue's counters: the yp region when step 5 is fused (yp is
+  // then never written), else the scratch region
+  const bool plain1 = !fuse && one_launch_plain(c);
+  int* counters = plain1 ? at<int>(scr, sc.mlp) : at<int>(ws, L.yp);
   if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   // the tile-queue counters are zeroed here, ahead of the kernel chain
-  if (one_launch(c) && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
+  if ((one_launch(c) || plain1) &&
+      cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
   // near-tie counts of every chunk in scratch, so step 3 starts from the
@@ -362,7 +385,11 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   if (fuse)   // steps 4-5: the second layer adds the gate-weighted expert outputs into out
     return experts_combine(c, at<char>(ws, L.xp), offsets, at<int32_t>(ws, L.src_tok), row_w, W1, W2,
                            at<char>(ws, L.h), out_f, counters, yp, stats, true, s);
-  st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);
+  if (plain1)
+    st = expert_mlp_plain(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, counters, true,
+                          s);
+  else
+    st = expert_ffn(c, at<char>(ws, L.xp), offsets, W1, W2, at<char>(ws, L.h), yp, stats, s);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));
 }

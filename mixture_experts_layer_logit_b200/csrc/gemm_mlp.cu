@@ -1,5 +1,6 @@
-// Steps 4-5 in one persistent launch: both expert layers and the fused
-// combine, with the tiles of the two layers drawn from one dynamic queue.
+// Step 4, and with k <= 2 step 5, in one persistent launch: both expert
+// layers (and the fused combine) with the tiles of the two layers drawn from
+// one dynamic queue.
 //
 // The experts' two layers are grouped GEMMs over the expert segments
 // (Megatron-Core best-practice page, "Megatron-Core MoE的关键特性":
@@ -10,10 +11,12 @@
 // "1. MoE 设计").
 //
 // Two separate launches leave SMs idle at the end of each layer (the layers'
-// 128 x 256 tiles fill 4.3 and 2.2 waves on the FastMoE layer).  Here one
-// grid of one CTA per SM takes tiles from a global counter: first every
-// layer-1 tile (h = act(xp W1^T)), then every layer-2 tile (out += w * (h W2^T)
-// for the token of each row; at most two additions per output, k <= 2).  A
+// 128 x 256 tiles fill 4.3 and 2.2 waves on the FastMoE layer, 2.8 and 2.05
+// on the top-6 decode layer).  Here one grid of one CTA per SM takes tiles
+// from a global counter: first every layer-1 tile (h = act(xp W1^T)), then
+// every layer-2 tile.  With COMB (k <= 2) a layer-2 tile adds w * (h W2^T)
+// into the token row of out (at most two additions per output); without it,
+// it stores the fp32 rows of yp for the separate combine kernel.  A
 // layer-2 tile needs the h rows of its m-tile from all layer-1 n-tiles: each
 // epilogue warp of a finished layer-1 tile adds 1 to the m-tile's counter
 // (a release after its h stores), and the TMA producer of a
@@ -63,7 +66,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
 struct MlpParams {
   const int32_t* offsets;
   void* h;                  // [rows][F] hidden (16-bit)
-  float* out;               // [T][d] layer output, zeroed beforehand
+  float* out;               // COMB: [T][d] layer output, zeroed beforehand; else [rows][d] yp
   const int32_t* src_tok;   // token of each permuted row
   const float* row_w;       // gate weight of each permuted row
   int E, d, F;
@@ -92,7 +95,7 @@ __device__ __forceinline__ MlpTile mlp_tile(const Tail* tail, int E, int T1, int
   return t;
 }
 
-template <int ACT, bool F16>
+template <int ACT, bool F16, bool COMB>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -292,7 +295,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         if (lane == 0) red_release_gpu_add(p.dep + t.m, 1);
       } else {
         const int nrows = warp_rows(p2, wrow0, t.c.rows - qw * 32, lane);
-        if (nrows > 0) store_tile<kCombine, F16>(p2, tb, wrow0, nrows, t.c.n0, stg, lane, over);
+        if (nrows > 0) store_tile<COMB ? kCombine : kPlain, F16>(p2, tb, wrow0, nrows, t.c.n0, stg, lane, over);
       }
       if (F16 && over) atomicOr(p.status, MOE_DEV_RANGE);
       tc_fence_before();
@@ -314,12 +317,16 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
   }
 }
 
-template <int ACT, bool F16>
+template <int ACT, bool F16, bool COMB>
 cudaError_t launch_t(const CUtensorMap (&maps)[4], const MlpParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_expert_mlp<ACT, F16>>(kSmemBytes);
+  cudaError_t err = set_smem_once<tc_expert_mlp<ACT, F16, COMB>>(kSmemBytes);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_expert_mlp<ACT, F16>, dim3(grid), dim3(kThreads), kSmemBytes, s, maps[0], maps[1], maps[2],
-                    maps[3], p);
+  return launch_pdl(tc_expert_mlp<ACT, F16, COMB>, dim3(grid), dim3(kThreads), kSmemBytes, s, maps[0], maps[1],
+                    maps[2], maps[3], p);
+}
+template <int ACT, bool F16>
+cudaError_t launch_c(const CUtensorMap (&maps)[4], const MlpParams& p, bool comb, int grid, cudaStream_t s) {
+  return comb ? launch_t<ACT, F16, true>(maps, p, grid, s) : launch_t<ACT, F16, false>(maps, p, grid, s);
 }
 
 }  // namespace
@@ -329,9 +336,10 @@ size_t expert_mlp_counters(const moe_config& c) {
 }
 
 cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
-                              const void* w2, void* h, const CombineOut& comb, int* counters, uint32_t* status,
-                              cudaStream_t s) {
+                              const void* w2, void* h, const CombineOut* comb, float* yp, int* counters,
+                              uint32_t* status, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
+  if (comb == nullptr && yp == nullptr) return cudaErrorInvalidValue;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
@@ -344,15 +352,16 @@ cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t
       !make_map(&maps[2], h, rows, (uint64_t)c.F, f16) ||
       !make_map(&maps[3], w2, (uint64_t)c.E * c.d, (uint64_t)c.F, f16))
     return cudaErrorInvalidValue;
-  MlpParams p{offsets, h, comb.out, comb.src_tok, comb.row_w, c.E, c.d, c.F, F1, comb.T, (int)rows,
-              counters, counters + 1, status};
+  MlpParams p{offsets, h, comb ? comb->out : yp, comb ? comb->src_tok : nullptr, comb ? comb->row_w : nullptr,
+              c.E, c.d, c.F, F1, comb ? comb->T : 0, (int)rows, counters, counters + 1, status};
+  const bool cb = comb != nullptr;
   const long long mt_max = (long long)(rows / BM) + c.E;
   const long long nt = (c.act == MOE_ACT_SWIGLU ? (c.F + BN / 2 - 1) / (BN / 2) : (c.F + BN - 1) / BN) +
                        (c.d + BN - 1) / BN;
   const int grid = (int)std::min<long long>(mt_max * nt, di.sms);
   if (c.act == MOE_ACT_SWIGLU)
-    return f16 ? launch_t<kSwiglu, true>(maps, p, grid, s) : launch_t<kSwiglu, false>(maps, p, grid, s);
-  return f16 ? launch_t<kRelu, true>(maps, p, grid, s) : launch_t<kRelu, false>(maps, p, grid, s);
+    return f16 ? launch_c<kSwiglu, true>(maps, p, cb, grid, s) : launch_c<kSwiglu, false>(maps, p, cb, grid, s);
+  return f16 ? launch_c<kRelu, true>(maps, p, cb, grid, s) : launch_c<kRelu, false>(maps, p, cb, grid, s);
 }
 
 }  // namespace moe

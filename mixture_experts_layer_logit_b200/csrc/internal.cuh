@@ -24,6 +24,7 @@ struct Scratch {
   size_t psum;      // float [nchunks][E]   per-chunk sums of softmax probabilities
   size_t ntie;      // int32 [nchunks]      near-tie tokens per chunk
   size_t status;    // uint32               device error bits of a standalone moe_route
+  size_t mlp;       // int32 [expert_mlp_counters] tile queue of the one-launch expert kernel (bf16)
   size_t kslice;    // the route's K-slice arrival counters and partial logits (may be empty); last
   size_t total;
 };
@@ -84,13 +85,14 @@ struct CombineOut {
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
                                  uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
-// Steps 4-5 in one launch for the bf16 path with k <= 2: both expert layers
-// and the fused combine from one dynamic tile queue.  `counters` holds
-// expert_mlp_counters(c) ints, zeroed before the launch.
+// Both expert layers in one launch on the bf16 path, from one dynamic tile
+// queue: with comb (k <= 2) the second layer adds into comb->out (the fused
+// step 5), else it writes fp32 yp.  `counters` holds expert_mlp_counters(c)
+// ints, zeroed before the launch.
 size_t expert_mlp_counters(const moe_config& c);
 cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
-                              const void* w2, void* h, const CombineOut& comb, int* counters, uint32_t* status,
-                              cudaStream_t s);
+                              const void* w2, void* h, const CombineOut* comb, float* yp, int* counters,
+                              uint32_t* status, cudaStream_t s);
 // The same with 2-SM pair tiles (tcgen05.mma.cta_group::2, 256 x 256).
 cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
                                       const void* w1, const void* w2, void* h, void* yp,
