@@ -160,3 +160,46 @@ def test_workspace_layout_is_disjoint_and_aligned(L):
 def test_scratch_grows_with_tokens(L):
     assert moe.moe_scratch_size(cfg(T=64)) < moe.moe_scratch_size(cfg(T=64 * 100))
     assert moe.moe_scratch_size(cfg(T=0)) > 0
+
+
+def _max_tokens(limit, **kw):
+    """Largest T whose scratch fits in `limit` bytes (binary search on the host size function)."""
+    lo, hi = 1, 1 << 22
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if moe.moe_scratch_size(cfg(T=mid, **kw)) <= limit:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
+def test_static_scratch_limit_as_documented(L):
+    # include/moe.h: E = 64, k = 2 fits about 344k tokens on the bf16 path
+    # (its scratch also holds the expert kernel's tile-queue counters) and
+    # 347k on fp32
+    limit = 2 << 20
+    t_bf16 = _max_tokens(limit, d=512, E=64, F=1024, k=2)
+    t_f32 = _max_tokens(limit, d=512, E=64, F=1024, k=2, dtype="f32")
+    assert abs(t_bf16 - 344_000) < 1_000, t_bf16
+    assert abs(t_f32 - 347_000) < 1_000, t_f32
+
+
+def test_route_split_scratch_only_for_wide_layers_on_few_chunks(L):
+    # the gate GEMM is cut over the model width (partial logits in scratch)
+    # only when its reduction needs more than one ring of loads and the batch
+    # has at most 74 chunks of 128 tokens: decode (d = 2048, one chunk) splits
+    # 8 ways, 8 x 128 x 64 fp32 partials; FastMoE (d = 512) and a batch of
+    # 128 chunks do not
+    decode = moe.moe_scratch_size(cfg(T=64, d=2048, E=64, F=1408, k=6, act="swiglu"))
+    assert decode >= 8 * 128 * 64 * 4
+    fastmoe = moe.moe_scratch_size(cfg(T=8192, d=512, E=64, F=1024, k=2))
+    wide_many = moe.moe_scratch_size(cfg(T=16384, d=2048, E=64, F=1408, k=6, act="swiglu"))
+    narrow = moe.moe_scratch_size(cfg(T=64, d=512, E=64, F=1408, k=6, act="swiglu"))
+    assert narrow < 8 * 128 * 64 * 4
+    # no partials: every byte is accounted for by the per-chunk tables and the
+    # tile-queue counters (a few 256-byte alignment pads aside)
+    for s, T, k in ((fastmoe, 8192, 2), (wide_many, 16384, 6)):
+        nch = (T + 127) // 128
+        tables = 4 * (3 * 64 * nch + nch + 1) + 4 * (2 + T * k // 128 + 64)
+        assert s <= tables + 8 * 256, (s, tables)
