@@ -4,7 +4,7 @@
 
 Each csrc/*.cu is compiled to an object under _build/ (parallel), then linked
 into mixture_experts_layer_logit_b200/libmoe.so.  The CUDA runtime is linked
-statically; the driver's tensor-map encoder is reached through the runtime's
+statically; the CUDA driver's tensor-map encoder is reached through the runtime's
 driver entry-point query, so the library needs no libcuda link.  The build is
 skipped when the library is newer than every source and header.
 """
