@@ -136,10 +136,10 @@ moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* 
                              int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                              int32_t* src_tok, void* xp, moe_stats* stats, const Scratch& sc, void* ws,
                              cudaStream_t s, const float* topk_w = nullptr, float* row_w = nullptr,
-                             float* out = nullptr) {
+                             float* out = nullptr, int* zero = nullptr, int nzero = 0) {
   return cuda_status(launch_permute(c, capacity_of(c), x, topk_idx, at<int32_t>(ws, sc.hist),
                                     at<int32_t>(ws, sc.choff), prob_mean, psum, ntie, counts, kept, offsets,
-                                    row_of, src_tok, xp, stats, s, topk_w, row_w, out));
+                                    row_of, src_tok, xp, stats, s, topk_w, row_w, out, zero, nzero));
 }
 
 // Mean assignments per expert from which the expert GEMMs use 2-SM tiles.
@@ -363,8 +363,12 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   const bool plain1 = !fuse && one_launch_plain(c);
   int* counters = plain1 ? at<int>(scr, sc.mlp) : at<int>(ws, L.yp);
   if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  // the tile-queue counters are zeroed here, ahead of the kernel chain
-  if ((one_launch(c) || plain1) &&
+  // the tile-queue counters are zeroed by the scatter's prologue when it runs
+  // scatter_kernel (no memset node between kernels), else here, ahead of the
+  // kernel chain
+  const bool mlp1 = one_launch(c) || plain1;
+  const bool zero_in_scatter = mlp1 && scatter_zeroes(c);
+  if (mlp1 && !zero_in_scatter &&
       cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // steps 1-2: the route kernel also leaves the histogram, probability sums and
@@ -380,7 +384,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
                          c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, at<int32_t>(ws, L.counts),
                          at<int32_t>(ws, L.kept), offsets, row_of, at<int32_t>(ws, L.src_tok),
                          at<char>(ws, L.xp), stats, sc, scr, s, fuse ? w : nullptr, fuse ? row_w : nullptr,
-                         fuse ? out_f : nullptr);
+                         fuse ? out_f : nullptr, zero_in_scatter ? counters : nullptr,
+                         zero_in_scatter ? (int)expert_mlp_counters(c) : 0);
   if (st != MOE_OK) return st;
   if (fuse)   // steps 4-5: the second layer adds the gate-weighted expert outputs into out
     return experts_combine(c, at<char>(ws, L.xp), offsets, at<int32_t>(ws, L.src_tok), row_w, W1, W2,

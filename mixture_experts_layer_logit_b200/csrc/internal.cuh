@@ -67,7 +67,11 @@ cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, con
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
                            const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
                            int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
-                           const float* topk_w = nullptr, float* row_w = nullptr, float* out = nullptr);
+                           const float* topk_w = nullptr, float* row_w = nullptr, float* out = nullptr,
+                           int* zero = nullptr, int nzero = 0);
+// True when the permutation runs scatter_kernel, whose prologue can zero the
+// `zero` ints of launch_permute (T > 0 and k <= 8); otherwise they are ignored.
+inline bool scatter_zeroes(const moe_config& c) { return c.T > 0 && c.k <= 8; }
 // Expert FFN on CUDA cores (fp32 path).
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
                                    const void* w1, const void* w2, void* h, void* yp, uint32_t* status,

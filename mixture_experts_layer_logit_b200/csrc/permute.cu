@@ -267,6 +267,8 @@ struct ScatterArgs {
   const float* topk_w;        // with row_w: the gate weight of each kept row is
   float* row_w;               //   copied to row_w[row] (fused combine)
   float* out;                 // fused combine: the layer output, zeroed here
+  int* zero;                  // or NULL: nzero ints zeroed here (the next kernel's tile-queue counters)
+  int nzero;
   uint32_t* status;           // device error bits (a bounded wait that gave up)
   int T, d, E, k, nch, capacity;
   int slice_vec;              // 16-byte vectors of a row per column slice (gridDim.y slices)
@@ -341,6 +343,10 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
     for (int i = lane; i < ntok; i += 32)
       tc::bulk_load(tc::smem_u32(xs + (size_t)i * W), src + (size_t)i * nvec * 16, (uint32_t)(W * 16), bar);
   }
+  // the expert kernel's counters: nothing reads them before that kernel's
+  // own wait on this grid, and nothing earlier on the stream still runs
+  if (a.zero != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < a.nzero; i += kScatterThreads) a.zero[i] = 0;
   if (a.out != nullptr) {
     constexpr int kOutVec = 16 / (int)sizeof(TX) / 4;   // float4 of out per 16-byte vector of x
     const int wo = W * kOutVec;
@@ -627,7 +633,7 @@ cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, con
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
                            const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
                            int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
-                           const float* topk_w, float* row_w, float* out) {
+                           const float* topk_w, float* row_w, float* out, int* zero, int nzero) {
   ScatterArgs a{};
   a.topk_idx = topk_idx;
   a.hist = hist;
@@ -644,6 +650,8 @@ cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, con
   a.topk_w = topk_w;
   a.row_w = row_w;
   a.out = out;
+  a.zero = zero;
+  a.nzero = nzero;
   a.status = &stats->status;
   a.T = c.T;
   a.d = c.d;
