@@ -61,11 +61,15 @@ class DeviceLayer:
         self.hdt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[self.hidden]
 
     # ---------------------------------------------------------- whole layer
-    def forward(self):
+    def forward(self, poison=None):
+        """poison: a byte value the workspace and out are filled with first."""
         n, L = moe.moe_workspace_size(self.cfg)
         assert n > 0
         ws = dev_bytes(n)
         out = torch.empty((self.T, self.w.d), dtype=torch.float32, device="cuda")
+        if poison is not None:
+            ws.fill_(poison)
+            out.view(torch.uint8).fill_(poison)
         stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
         moe.moe_layer_forward(self.cfg, self.x, self.wg, self.bias, self.w1, self.w2, out, stats, ws)
         torch.cuda.synchronize()

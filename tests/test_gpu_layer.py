@@ -102,6 +102,22 @@ def test_layer_bf16_hidden(name):
     run_and_check(L)
 
 
+@pytest.mark.parametrize("name", ["m_swiglu_lam", "m_relu_cap", "m_ksplit"])
+def test_layer_poisoned_workspace(name):
+    """Every workspace word the forward reads is written earlier in the same
+    call, so a workspace and output filled with 0xFF bytes give the same
+    result.  This covers the expert kernel's tile-queue counters, which the
+    scatter zeroes (in the yp region for k <= 2, in scratch for k > 2), and the
+    route's arrival counters on a model-width split (m_ksplit)."""
+    w = next(m for m in MEDIUM if m.name == name)
+    L = DeviceLayer(w)
+    a = L.forward()
+    b = L.forward(poison=0xFF)
+    assert b["stats"]["status"] == 0
+    assert torch.equal(a["out"], b["out"])
+    assert a["stats"] == b["stats"]
+
+
 def test_layer_deterministic():
     L = DeviceLayer(MEDIUM[1])
     a = L.forward()
