@@ -6,7 +6,10 @@
 A step is one moe_layer_forward (gate GEMM + normalisation/top-k, permutation
 with capacity, both grouped expert GEMMs, combine) over one batch of
 synthetic tokens already resident in HBM; by default it is replayed from a
-CUDA graph.  Between timed steps a 512 MiB memset flushes the 126 MB L2, and
+CUDA graph.  The headline workload is the Mixtral-8x7B-shaped dropless layer
+(T 16384, d 4096, 8 SwiGLU experts of 14336, top-2), the largest that fits
+one GPU; the FastMoE Transformer-XL layer is timed the same way and reported
+under "extra".  Between timed steps a 512 MiB memset flushes the 126 MB L2, and
 each step is bracketed by its own CUDA events (the flush is outside them).
 Under torchrun each rank runs an independent replica on its own token shard
 (weak scaling; no collective on the data path) and the reported time is the
@@ -21,7 +24,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -39,8 +41,15 @@ METRIC = "MoE layer fwd tokens/s at 1 B200; % bf16 tensor peak (GEMM), % HBM BW 
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
-GEMM_PROFILE = os.path.join(ROOT, "profiles", "tc_expert_mlp_fastmoe_txl.md")
-GEMM_SOURCE = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc", "gemm_mlp.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "mixture_experts_layer_logit_b200", "csrc")
+# source files of each expert kernel (the DRAM traffic ncu measured is only
+# reported while they are unchanged)
+KERNEL_SOURCES = {
+    "tc_expert_mlp": ["gemm_mlp.cu", "gemm_common.cuh", "tc_ptx.cuh"],
+    "tc_grouped_gemm_pair": ["gemm_tc2.cu", "gemm_common.cuh", "tc_ptx.cuh"],
+    "tc_grouped_gemm": ["gemm_tc.cu", "gemm_common.cuh", "tc_ptx.cuh"],
+}
 
 
 def parse_args():
@@ -49,6 +58,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=mw.BENCH_WORKLOAD, choices=sorted(mw.WORKLOADS))
+    ap.add_argument("--extra", default=",".join(mw.BENCH_EXTRA_WORKLOADS),
+                    help="comma-separated workloads also timed on the device (1 GPU only); '' for none")
+    ap.add_argument("--hidden", default="f16", choices=["f16", "bf16"],
+                    help="element type of the expert hidden activation and W2 on the bf16 path")
     ap.add_argument("--impl", default="moe", choices=["moe", "reference"])
     ap.add_argument("--no-graph", action="store_true", help="launch the C ABI call directly instead of a graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -82,12 +95,14 @@ def graph_kernel_nodes(graph) -> int:
     return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
 
 
-def workload_config(w: mw.Workload, n_gpus: int, graph: bool):
+def workload_config(w: mw.Workload, n_gpus: int, graph: bool, hidden: str = "f16"):
     return {"workload": w.name, "tokens_per_gpu": w.T, "global_batch": w.T * n_gpus, "d_model": w.d,
             "experts": w.E, "ffn_hidden": w.F, "top_k": w.k, "activation": w.act,
             "capacity_factor": w.capacity_factor if w.capacity_factor > 0 else "dropless",
             "lambda": w.lam, "gate_bias": "zipf1.2" if w.zipf_bias else None,
-            "hidden_dtype": "f16" if w.dtype == mw.BF16 else "f32", "out_dtype": "f32",
+            "hidden_dtype": hidden if w.dtype == mw.BF16 else "f32",
+            "precision": ("x, W_gate, W1 bf16; h and W2 " + hidden + "; fp32 accumulation; out fp32")
+            if w.dtype == mw.BF16 else "fp32 throughout", "out_dtype": "f32",
             "parallelism": "replicas" if n_gpus == 1 else f"dp{n_gpus} replicas",
             "l2": "flushed between steps (512 MiB memset outside the timed events)",
             "cuda_graph": graph}
@@ -155,7 +170,7 @@ def run_reference(a):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, 1, False),
+            "config": workload_config(w, 1, False, a.hidden),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"each step: float64 oracle forward of the first {Ts} of {w.T} tokens"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -242,16 +257,24 @@ def fused_combine(w: mw.Workload) -> bool:
     return w.dtype == mw.BF16 and w.k <= 2
 
 
-def committed_traffic():
-    """DRAM bytes per grouped-GEMM launch from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
+def source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summaries (profiles/traffic.json), if they were taken on the current
+    kernel sources (else None)."""
     try:
-        src = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()[:16]
-        txt = open(GEMM_PROFILE).read()
-        m_hash = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
-        m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-        if m_hash and m_tr and m_hash.group(1) == src:
-            return float(m_tr.group(1))
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d[f"{kernel}@{workload}"]
+        if e["source_sha256_16"] == source_hash(kernel):
+            return float(e["traffic_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -282,6 +305,245 @@ def job_tokens_per_second(world: int, tokens_per_rank: int, ms_per_step: float) 
 
 
 # ------------------------------------------------------------------ main
+class Layer:
+    """One workload's inputs, weights and buffers on the device."""
+
+    def __init__(self, moe, w: mw.Workload, rank: int, dev, hidden: str):
+        import torch
+        self.w = w
+        self.inp = replica_inputs(w, rank)
+        self.cfg = moe.make_config(w.T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam,
+                                   hidden if w.dtype == mw.BF16 else None)
+        self.tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
+        self.x = mw.to_device(self.inp.x, dev)
+        self.wg, self.bias = mw.to_device(self.inp.wg, dev), mw.to_device(self.inp.bias, dev)
+        self.w1 = mw.to_device(self.inp.w1, dev)
+        # weight preparation at load time (not part of a step): W2 in the hidden type
+        self.w2 = moe.prepare_w2(self.cfg, mw.to_device(self.inp.w2, dev))
+        nbytes, self.lay = moe.moe_workspace_size(self.cfg)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.out = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
+        self.stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
+        self.moe = moe
+
+    def fwd(self, x=None, out=None, stats=None):
+        self.moe.moe_layer_forward(self.cfg, self.x if x is None else x, self.wg, self.bias, self.w1, self.w2,
+                                   self.out if out is None else out, self.stats if stats is None else stats,
+                                   self.ws)
+
+
+def timed(fn, steps, flush):
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in evs:
+        if flush is not None:
+            flush.zero_()
+        e0.record()
+        fn()
+        e1.record()
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in evs]
+
+
+def capture(L: Layer, no_graph: bool):
+    """(run, launches per step, graph): one forward captured as a CUDA graph;
+    its kernel nodes are the launches of a step."""
+    import torch
+    L.fwd()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(graph):
+        L.fwd()
+    launches = graph_kernel_nodes(graph)
+    if no_graph:
+        graph.reset()
+        return L.fwd, launches, None
+    return graph.replay, launches, graph
+
+
+def expert_kernel(w: mw.Workload):
+    """(kernel name, launches per step, description) of the expert step the forward runs."""
+    fused = fused_combine(w)
+    pair = w.dtype == mw.BF16 and w.T * w.k >= 512 * w.E
+    if w.dtype != mw.BF16:
+        return "simt_grouped_gemm", 2, "simt_grouped_gemm (fp32 expert FFN, 2 launches)"
+    if not pair:
+        if fused:
+            return "tc_expert_mlp", 1, "tc_expert_mlp (steps 4-5 in one launch: both expert layers + the combine)"
+        return "tc_expert_mlp", 1, "tc_expert_mlp (step 4 in one launch: both expert layers, writing yp)"
+    if fused:
+        return ("tc_grouped_gemm_pair", 2, "tc_grouped_gemm_pair (2-SM pair tiles; layer 1 with the activation, "
+                "then layer 2 with the combine fused: 2 launches)")
+    return "tc_grouped_gemm_pair", 2, "tc_grouped_gemm_pair (2-SM pair tiles; layer 1 + layer 2: 2 launches)"
+
+
+def breakdown_roofline(L: Layer, a, flush, pk, pk_src, dev):
+    """Per-step times through the step entry points, and the roofline of the
+    dominant kernel (the expert step the forward runs), from CUDA events."""
+    import torch
+    moe, w, lay, ws = L.moe, L.w, L.lay, L.ws
+    A = w.T * w.k
+    sv = lambda off, n, dt: ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)  # noqa: E731
+    idx, tw, gap = sv(lay.topk_idx, A, torch.int32), sv(lay.topk_w, A, torch.float32), sv(lay.gap, w.T, torch.float32)
+    counts, kept = sv(lay.counts, w.E, torch.int32), sv(lay.kept, w.E, torch.int32)
+    offs = sv(lay.offsets, w.E + 1, torch.int32)
+    row_of, src_tok = sv(lay.row_of, A, torch.int32), sv(lay.src_tok, A, torch.int32)
+    hdt = {moe.MOE_DTYPE_F16: torch.float16, moe.MOE_DTYPE_BF16: torch.bfloat16}.get(L.cfg.hidden_dtype,
+                                                                                      torch.float32)
+    xp, h, yp = sv(lay.xp, A * w.d, L.tdt), sv(lay.h, A * w.F, hdt), sv(lay.yp, A * w.d, torch.float32)
+    scr = ws[lay.scratch:]
+    pm = torch.empty(w.E, dtype=torch.float32, device=dev)
+    names = ["route", "permute", "expert_ffn", "combine"]
+    acc = {n: 0.0 for n in names}
+    for i in range(a.warmup + a.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record()
+        moe.moe_route(L.cfg, L.x, L.wg, L.bias, idx, tw, gap, pm, scr)
+        ev[1].record()
+        moe.moe_permute(L.cfg, L.x, idx, gap, pm, counts, kept, offs, row_of, src_tok, xp, L.stats, scr)
+        ev[2].record()
+        moe.moe_expert_ffn(L.cfg, xp, offs, L.w1, L.w2, h, yp, L.stats, scr)
+        ev[3].record()
+        moe.moe_combine(L.cfg, yp, row_of, tw, L.out)
+        ev[4].record()
+        torch.cuda.synchronize()
+        if i >= a.warmup:
+            for j, n in enumerate(names):
+                acc[n] += ev[j].elapsed_time(ev[j + 1])
+    breakdown = {n: acc[n] / a.steps for n in names}
+    offsets = offs.cpu().numpy()
+    sb = step_bytes(w, offsets)
+    # The forward's own steps 4-5 on bf16 layers with k <= 2: the expert kernel
+    # with the combine fused in, fed the forward's permuted rows and row
+    # weights; out is zeroed before each call, outside the events.
+    fused = fused_combine(w)
+    if fused:
+        row_w = sv(lay.row_w, A, torch.float32)
+        out_fc = torch.empty_like(L.out)
+        t_fc = 0.0
+        for i in range(a.warmup + a.steps):
+            flush.zero_()
+            out_fc.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            moe.moe_expert_ffn_combine(L.cfg, xp, offs, src_tok, row_w, L.w1, L.w2, h, out_fc, L.stats, ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= a.warmup:
+                t_fc += e0.elapsed_time(e1)
+        breakdown["experts_combine"] = t_fc / a.steps
+        del out_fc
+    rl = {}
+    for n in ["route", "permute", "combine"]:
+        gbs = sb[n] / (breakdown[n] * 1e-3) / 1e9
+        rl[n] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                 "frac": gbs / pk["hbm_gbs"], "bytes": sb[n]}
+    step = "experts_combine" if fused else "expert_ffn"
+    t_ffn = breakdown[step] * 1e-3
+    tflops = sb["expert_flops"] / t_ffn / 1e12
+    gbs = sb[step] / t_ffn / 1e9
+    t_hbm = sb[step] / (pk["hbm_gbs"] * 1e9)
+    t_tc = sb["expert_flops"] / (pk["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    kname, nl, kdesc = expert_kernel(w)
+    traffic = committed_traffic(kname, w.name) if kname in KERNEL_SOURCES else None
+    if bound == "hbm":
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm_gbs"], "traffic": traffic}
+    else:
+        roofline = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": tflops / pk["bf16_tflops"], "traffic": traffic}
+    roofline.update({
+        "kernel": kdesc, "peak_kind": "burst (the expert step is timed on its own)",
+        "launches_per_step": nl, "algorithmic_bytes_per_launch": sb[step] / nl,
+        "algorithmic_flops_per_launch": sb["expert_flops"] / nl, "launch_ms": breakdown[step] / nl,
+        "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"],
+        "tensor_frac_of_sustained": tflops / pk["bf16_tflops_sustained"], "hbm_gbs": gbs,
+        "hbm_frac": gbs / pk["hbm_gbs"], "weight_bytes": sb["weight_bytes"],
+        "peak_source": "measured (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback (recipe)",
+        "other_steps": rl})
+    return breakdown, roofline
+
+
+def e2e_measure(L: Layer, a, flush, graph_ok: bool, barrier, max_over_ranks, world: int, dev):
+    """Every step copies its tokens from pinned host memory to the device, runs
+    the layer through the C ABI and reads the output and statistics back.  Two
+    buffer slots and three streams (host-to-device, compute, device-to-host)
+    let the copies of one step overlap the compute of the next; each step
+    still starts from a flushed L2."""
+    import torch
+    moe, w, x, out, stats = L.moe, L.w, L.x, L.out, L.stats
+    x_host = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for _ in range(2)]
+    for xh in x_host:
+        xh.copy_(x.cpu())
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    st_host = [torch.empty(stats.shape, dtype=stats.dtype).pin_memory() for _ in range(2)]
+    xs = [x, torch.empty_like(x)]
+    outs = [out, torch.empty_like(out)]
+    sts = [stats, torch.zeros_like(stats)]
+    s_h2d, s_comp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    slot_runs = []
+    for i in range(2):
+        def slot_fwd(i=i):
+            L.fwd(xs[i], outs[i], sts[i])
+        if not graph_ok:
+            slot_runs.append(slot_fwd)
+        else:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_comp):
+                slot_fwd()
+            slot_runs.append(g)
+    ev_h2d = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_d2h = [torch.cuda.Event() for _ in range(2)]
+
+    def pipelined(steps):
+        for i in range(steps):
+            k = i % 2
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(ev_comp[k])        # the layer of step i-2 has read xs[k]
+                xs[k].copy_(x_host[k], non_blocking=True)
+                ev_h2d[k].record(s_h2d)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_h2d[k])
+                if i >= 2:
+                    s_comp.wait_event(ev_d2h[k])        # step i-2's output has been read back
+                flush.zero_()
+                r = slot_runs[k]
+                r.replay() if hasattr(r, "replay") else r()
+                ev_comp[k].record(s_comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_comp[k])
+                out_host[k].copy_(outs[k], non_blocking=True)
+                st_host[k].copy_(sts[k], non_blocking=True)
+                ev_d2h[k].record(s_d2h)
+
+    pipelined(a.warmup)
+    torch.cuda.synchronize()
+    barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(s_h2d)
+    s_comp.wait_event(e_start)
+    s_d2h.wait_event(e_start)
+    pipelined(a.steps)
+    s_h2d.wait_stream(s_d2h)
+    s_h2d.wait_stream(s_comp)
+    e_end.record(s_h2d)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / a.steps
+    assert int(st_host[(a.steps - 1) % 2].view(torch.int32)[6]) == 0, "device status after the e2e steps"
+    res = {"value": world * w.T / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+           "h2d_bytes_per_step": x.numel() * x.element_size(),
+           "d2h_bytes_per_step": out.numel() * out.element_size() + stats.numel(),
+           "pipeline": "2 buffer slots; host-to-device, compute and device-to-host streams overlap across steps"}
+    del slot_runs
+    return res
+
+
 def main():
     a = parse_args()
     if a.impl == "reference":
@@ -308,49 +570,6 @@ def main():
         dist.barrier()
     moe.lib()
 
-    w = mw.WORKLOADS[a.workload]
-    inp = replica_inputs(w, rank)
-    cfg = moe.make_config(w.T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam)
-    tdt = torch.bfloat16 if w.dtype == mw.BF16 else torch.float32
-    x = mw.to_device(inp.x, dev)
-    wg, bias = mw.to_device(inp.wg, dev), mw.to_device(inp.bias, dev)
-    w1 = mw.to_device(inp.w1, dev)
-    # weight preparation at load time (not part of a step): W2 in the hidden type
-    w2 = moe.prepare_w2(cfg, mw.to_device(inp.w2, dev))
-    nbytes, lay = moe.moe_workspace_size(cfg)
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    out = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
-    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def fwd():
-        moe.moe_layer_forward(cfg, x, wg, bias, w1, w2, out, stats, ws)
-
-    fwd()
-    torch.cuda.synchronize()
-    # one step captured as a CUDA graph; its kernel nodes are the launches of a step
-    graph = torch.cuda.CUDAGraph(keep_graph=True)
-    with torch.cuda.graph(graph):
-        fwd()
-    launches_per_step = graph_kernel_nodes(graph)
-    run = fwd
-    if a.no_graph:
-        graph.reset()
-        graph = None
-    else:
-        run = graph.replay
-
-    def timed(fn, steps, flush_between=True):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-        for e0, e1 in evs:
-            if flush_between:
-                flush.zero_()
-            e0.record()
-            fn()
-            e1.record()
-        torch.cuda.synchronize()
-        return [e0.elapsed_time(e1) for e0, e1 in evs]
-
     def barrier():
         torch.cuda.synchronize()
         if world > 1:
@@ -360,8 +579,14 @@ def main():
     def max_over_ranks(v: float) -> float:
         return reduce_max_over_ranks(v, world, dev)
 
+    pk, pk_src = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
     # ---------------------------------------------------------- headline
-    timed(run, a.warmup)
+    w = mw.WORKLOADS[a.workload]
+    L = Layer(moe, w, rank, dev, a.hidden)
+    run, launches_per_step, graph = capture(L, a.no_graph)
+    timed(run, a.warmup, flush)
     barrier()
     gpu_id = str(local)
     try:
@@ -371,201 +596,63 @@ def main():
     sampler = ClockSampler(gpu_id)
     sampler.start()
     barrier()
-    times = timed(run, a.steps)
+    times = timed(run, a.steps, flush)
     barrier()
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(times))
     ms = total_ms / a.steps
     value = job_tokens_per_second(world, w.T, ms)
-    st = moe.read_stats(stats)
-    offsets = ws[lay.offsets:lay.offsets + 4 * (w.E + 1)].view(torch.int32).cpu().numpy()
+    st = moe.read_stats(L.stats)
     assert st["status"] == 0, f"device status {st['status']}"
 
-    # ------------------------------------------- per-step breakdown (rank-local)
-    pk, pk_src = peaks()
-    sb = step_bytes(w, offsets)
-    breakdown = None
-    roofline = None
+    breakdown = roofline = None
     if not a.no_breakdown:
-        A = w.T * w.k
-        L = lay
-        sv = lambda off, n, dt: ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)  # noqa: E731
-        idx, tw, gap = sv(L.topk_idx, A, torch.int32), sv(L.topk_w, A, torch.float32), sv(L.gap, w.T, torch.float32)
-        counts, kept, offs = sv(L.counts, w.E, torch.int32), sv(L.kept, w.E, torch.int32), sv(L.offsets, w.E + 1, torch.int32)
-        row_of, src_tok = sv(L.row_of, A, torch.int32), sv(L.src_tok, A, torch.int32)
-        xp, h, yp = sv(L.xp, A * w.d, tdt), sv(L.h, A * w.F, tdt), sv(L.yp, A * w.d, torch.float32)
-        scr = ws[L.scratch:]
-        pm = torch.empty(w.E, dtype=torch.float32, device=dev)
-        names = ["route", "permute", "expert_ffn", "combine"]
-        acc = {n: 0.0 for n in names}
-        for i in range(a.warmup + a.steps):
-            flush.zero_()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-            ev[0].record()
-            moe.moe_route(cfg, x, wg, bias, idx, tw, gap, pm, scr)
-            ev[1].record()
-            moe.moe_permute(cfg, x, idx, gap, pm, counts, kept, offs, row_of, src_tok, xp, stats, scr)
-            ev[2].record()
-            moe.moe_expert_ffn(cfg, xp, offs, w1, w2, h, yp, stats, scr)
-            ev[3].record()
-            moe.moe_combine(cfg, yp, row_of, tw, out)
-            ev[4].record()
-            torch.cuda.synchronize()
-            if i >= a.warmup:
-                for j, n in enumerate(names):
-                    acc[n] += ev[j].elapsed_time(ev[j + 1])
-        breakdown = {n: acc[n] / a.steps for n in names}
-        # The forward's own steps 4-5 on bf16 layers with k <= 2: the expert
-        # kernel with the combine fused in, fed the forward's permuted rows and
-        # row weights; out is zeroed before each call, outside the events.
-        fused = fused_combine(w)
-        one_launch = fused and w.T * w.k < 512 * w.E
-        # without the fused combine, bf16 layers on 1-SM tiles run the expert
-        # step as one launch writing yp (moe_expert_ffn and the forward alike)
-        plain_launch = (not fused) and w.dtype == mw.BF16 and w.T * w.k < 512 * w.E
-        if fused:
-            row_w = sv(L.row_w, A, torch.float32)
-            out_fc = torch.empty_like(out)
-            t_fc = 0.0
-            for i in range(a.warmup + a.steps):
-                flush.zero_()
-                out_fc.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                moe.moe_expert_ffn_combine(cfg, xp, offs, src_tok, row_w, w1, w2, h, out_fc, stats, ws)
-                e1.record()
-                torch.cuda.synchronize()
-                if i >= a.warmup:
-                    t_fc += e0.elapsed_time(e1)
-            breakdown["experts_combine"] = t_fc / a.steps
-        rl = {}
-        for n in ["route", "permute", "combine"]:
-            gbs = sb[n] / (breakdown[n] * 1e-3) / 1e9
-            rl[n] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / pk["hbm_gbs"], "bytes": sb[n]}
-        step = "experts_combine" if fused else "expert_ffn"
-        t_ffn = breakdown[step] * 1e-3
-        tflops = sb["expert_flops"] / t_ffn / 1e12
-        gbs = sb[step] / t_ffn / 1e9
-        t_hbm = sb[step] / (pk["hbm_gbs"] * 1e9)
-        t_tc = sb["expert_flops"] / (pk["bf16_tflops"] * 1e12)
-        bound = "hbm" if t_hbm >= t_tc else "tensor"
-        traffic = committed_traffic() if (a.workload == mw.BENCH_WORKLOAD and one_launch) else None
-        if bound == "hbm":
-            roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": gbs / pk["hbm_gbs"], "traffic": traffic}
-        else:
-            roofline = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": tflops / pk["bf16_tflops"], "traffic": traffic}
-        if one_launch:
-            kname, nl = "tc_expert_mlp (steps 4-5 in one launch: both expert layers + the combine)", 1
-        elif fused:
-            kname, nl = "tc_grouped_gemm(_pair) (layer 1, then layer 2 with the combine fused: 2 launches)", 2
-        elif plain_launch:
-            kname, nl = "tc_expert_mlp (step 4 in one launch: both expert layers, writing yp)", 1
-        else:
-            kname, nl = "tc_grouped_gemm(_pair) (expert FFN step: 2 launches, layer 1 + layer 2)", 2
-        roofline.update({
-            "kernel": kname,
-            "launches_per_step": nl, "algorithmic_bytes_per_launch": sb[step] / nl,
-            "algorithmic_flops_per_launch": sb["expert_flops"] / nl, "launch_ms": breakdown[step] / nl,
-            "tensor_tflops": tflops, "tensor_frac": tflops / pk["bf16_tflops"], "hbm_gbs": gbs,
-            "hbm_frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured"
-            else "fallback (recipe)", "other_steps": rl})
-
-    # ------------------------------------------------------------------ e2e
-    # Every step copies its tokens from pinned host memory to the device, runs
-    # the layer through the C ABI and reads the output and statistics back.
-    # Two buffer slots and three streams (host-to-device, compute,
-    # device-to-host) let the copies of one step overlap the compute of the
-    # next; each step still starts from a flushed L2.
+        breakdown, roofline = breakdown_roofline(L, a, flush, pk, pk_src, dev)
     e2e = None
     if not a.no_e2e:
-        x_host = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for _ in range(2)]
-        for xh in x_host:
-            xh.copy_(x.cpu())
-        out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-        st_host = [torch.empty(stats.shape, dtype=stats.dtype).pin_memory() for _ in range(2)]
-        xs = [x, torch.empty_like(x)]
-        outs = [out, torch.empty_like(out)]
-        sts = [stats, torch.zeros_like(stats)]
-        s_h2d, s_comp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        slot_runs = []
-        for i in range(2):
-            def slot_fwd(i=i):
-                moe.moe_layer_forward(cfg, xs[i], wg, bias, w1, w2, outs[i], sts[i], ws)
-            if a.no_graph:
-                slot_runs.append(slot_fwd)
-            else:
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=s_comp):
-                    slot_fwd()
-                slot_runs.append(g)
-        ev_h2d = [torch.cuda.Event() for _ in range(2)]
-        ev_comp = [torch.cuda.Event() for _ in range(2)]
-        ev_d2h = [torch.cuda.Event() for _ in range(2)]
-
-        def pipelined(steps):
-            for i in range(steps):
-                k = i % 2
-                with torch.cuda.stream(s_h2d):
-                    if i >= 2:
-                        s_h2d.wait_event(ev_comp[k])        # the layer of step i-2 has read xs[k]
-                    xs[k].copy_(x_host[k], non_blocking=True)
-                    ev_h2d[k].record(s_h2d)
-                with torch.cuda.stream(s_comp):
-                    s_comp.wait_event(ev_h2d[k])
-                    if i >= 2:
-                        s_comp.wait_event(ev_d2h[k])        # step i-2's output has been read back
-                    flush.zero_()
-                    r = slot_runs[k]
-                    r.replay() if hasattr(r, "replay") else r()
-                    ev_comp[k].record(s_comp)
-                with torch.cuda.stream(s_d2h):
-                    s_d2h.wait_event(ev_comp[k])
-                    out_host[k].copy_(outs[k], non_blocking=True)
-                    st_host[k].copy_(sts[k], non_blocking=True)
-                    ev_d2h[k].record(s_d2h)
-
-        pipelined(a.warmup)
-        torch.cuda.synchronize()
-        barrier()
-        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e_start.record(s_h2d)
-        s_comp.wait_event(e_start)
-        s_d2h.wait_event(e_start)
-        pipelined(a.steps)
-        s_h2d.wait_stream(s_d2h)
-        s_h2d.wait_stream(s_comp)
-        e_end.record(s_h2d)
-        torch.cuda.synchronize()
-        barrier()
-        e_ms = max_over_ranks(e_start.elapsed_time(e_end)) / a.steps
-        assert int(st_host[(a.steps - 1) % 2].view(torch.int32)[6]) == 0, "device status after the e2e steps"
-        e2e = {"value": world * w.T / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
-               "h2d_bytes_per_step": x.numel() * x.element_size(),
-               "d2h_bytes_per_step": out.numel() * out.element_size() + stats.numel(),
-               "pipeline": "2 buffer slots; host-to-device, compute and device-to-host streams overlap across steps"}
-        del slot_runs
-
+        e2e = e2e_measure(L, a, flush, graph is not None, barrier, max_over_ranks, world, dev)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, a.cpu_seconds)
+        cpu = cpu_baseline(w, L.inp, a.cpu_seconds)
+    if graph is not None:
+        del graph
+    del run, L
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------ further workloads (1 GPU only)
+    extra = {}
+    names = [n for n in a.extra.split(",") if n and n != a.workload] if world == 1 else []
+    for name in names:
+        we = mw.WORKLOADS[name]
+        Le = Layer(moe, we, rank, dev, a.hidden)
+        run_e, nl_e, g_e = capture(Le, a.no_graph)
+        timed(run_e, a.warmup, flush)
+        t_e = timed(run_e, a.steps, flush)
+        ms_e = sum(t_e) / a.steps
+        st_e = moe.read_stats(Le.stats)
+        assert st_e["status"] == 0, f"device status {st_e['status']} on {name}"
+        ent = {"value": we.T / (ms_e / 1e3), "unit": UNIT, "ms_per_step": ms_e,
+               "config": workload_config(we, 1, g_e is not None, a.hidden), "gpu_launches_per_step": nl_e}
+        if not a.no_breakdown:
+            ent["breakdown_ms"], ent["roofline"] = breakdown_roofline(Le, a, flush, pk, pk_src, dev)
+        extra[name] = ent
+        if g_e is not None:
+            del g_e
+        del run_e, Le
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16" if w.dtype == mw.BF16 else "f32", "data": "synthetic",
-                "config": workload_config(w, world, graph is not None),
+                "config": workload_config(w, world, not a.no_graph, a.hidden),
                 "gpu_launches": launches_per_step * a.steps,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "breakdown_ms": breakdown,
                 "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "rows_kept": st["rows_kept"],
-                          "capacity": st["capacity"], "near_tie_count": st["near_tie_count"]}}
+                          "capacity": st["capacity"], "near_tie_count": st["near_tie_count"]},
+                "extra": extra}
         print(json.dumps(line), flush=True)
-    if graph is not None:
-        del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
