@@ -7,5 +7,5 @@ from .moe_oracle import (  # noqa: F401
     LayerConfig, Routing, Dispatch, Forward, RELU, SWIGLU,
     gate_logits, normalise_logits, softmax, top_k, route, capacity, dispatch,
     expert_hidden, expert_ffn, expert_segments, combine, forward, forward_tokens,
-    brute_force,
+    brute_force, log_partition, z_loss, adaptive_aux_coef,
 )

@@ -30,6 +30,15 @@ upcast exactly), written to be checked against the pages by eye:
   Skywork slides' slide 7 formula is blank): Switch form
   aux = E * sum_e f_e * P_e with f_e the fraction of pre-drop assignments to
   expert e and P_e the mean full-softmax probability of expert e.
+* Router z-loss (Megatron-Core page, "Megatron-Core MoE的关键特性", which
+  names Z-Loss among the load-balancing methods without a formula).  Reading:
+  the mean over tokens of the squared log-partition function of the scores the
+  softmax takes (z_hat when lambda > 0, else z).
+* Adaptive aux-loss coefficient (Skywork-MoE release, "2.自适应的Aux Loss";
+  slides, slide 7: layer-wise coefficients, raised when the token drop rate
+  rises and lowered when it falls; the formula itself is not on the pages).
+  Reading: per layer, alpha <- beta * alpha + (1 - beta) * xi * drop_rate, an
+  exponential moving average of a target proportional to the drop rate.
 * Experts: two-layer MLP with ReLU (FastMoE announcement, Transformer-XL
   experiment: 512->1024->512) or the gated SwiGLU pair whose gate and up
   projections are stored concatenated, gate first (Megatron-Core page,
@@ -140,6 +149,7 @@ class Routing:
     w: np.ndarray        # renormalised gate weights of the selected experts    [T, k]
     gap: np.ndarray      # k-th minus (k+1)-th score                            [T]
     prob_mean: np.ndarray  # P_e = mean_t p[t, e]                               [E]
+    z_loss: float = float("nan")  # mean_t (log sum_e exp s[t, e])^2 (NaN when T == 0)
 
 
 def route(x, wg, bias, cfg: LayerConfig, forced_mask: Optional[np.ndarray] = None,
@@ -162,7 +172,31 @@ def route(x, wg, bias, cfg: LayerConfig, forced_mask: Optional[np.ndarray] = Non
         idx[forced_mask] = np.asarray(forced_idx)[forced_mask]
     psel = np.take_along_axis(p, idx, axis=1)
     w = psel / psel.sum(axis=1, keepdims=True)
-    return Routing(s=s, p=p, idx=idx, w=w, gap=gap, prob_mean=p.mean(axis=0))
+    return Routing(s=s, p=p, idx=idx, w=w, gap=gap, prob_mean=p.mean(axis=0), z_loss=z_loss(s))
+
+
+def log_partition(s: np.ndarray) -> np.ndarray:
+    """lse[t] = log sum_e exp(s[t, e]), the row maximum taken out first."""
+    m = s.max(axis=1)
+    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+
+
+def z_loss(s: np.ndarray) -> float:
+    """Router z-loss: (1/T) sum_t (log sum_e exp s[t, e])^2 over the scores the
+    softmax takes (Megatron-Core page, "Megatron-Core MoE的关键特性": Z-Loss; the
+    formula is this reading).  NaN for an empty batch."""
+    if s.shape[0] == 0:
+        return float("nan")
+    return float(np.mean(log_partition(s) ** 2))
+
+
+def adaptive_aux_coef(alpha: float, drop_rate: float, beta: float, xi: float) -> float:
+    """One step of the layer-wise adaptive aux-loss coefficient (Skywork-MoE
+    release, "2.自适应的Aux Loss"; slides, slide 7: raise the coefficient when
+    the drop rate rises, lower it when it falls).  Reading: the coefficient is
+    an exponential moving average, with smoothing beta, of xi times the drop
+    rate of the step just taken."""
+    return beta * alpha + (1.0 - beta) * xi * drop_rate
 
 
 # ---------------------------------------------------- step 3: capacity/permute

@@ -94,6 +94,37 @@ def check_closed_forms():
     return bad
 
 
+def check_losses():
+    """Closed forms of the router z-loss and of the adaptive aux coefficient."""
+    bad = []
+    c = _cases()
+    for name in ["z_loss_constant_scores", "z_loss_two_tokens"]:
+        cs = c[name]
+        got = om.z_loss(np.array(cs["scores"], dtype=np.float64))
+        if not abs(got - cs["expected_z_loss"]) <= 1e-12 * max(1.0, abs(cs["expected_z_loss"])):
+            bad.append(f"{name}: {got}")
+    cs = c["z_loss_after_normalisation"]
+    x = np.array(cs["x"]); wg = np.array(cs["wg"])
+    cfg = oracle.LayerConfig(T=1, d=2, E=2, F=1, k=cs["k"], lam=cs["lam"])
+    got = om.route(x, wg, None, cfg).z_loss
+    if not abs(got - cs["expected_z_loss"]) <= 1e-13:
+        bad.append(f"z_loss_after_normalisation: {got}")
+    if not math.isnan(om.z_loss(np.zeros((0, 3)))):
+        bad.append("z_loss of an empty batch")
+    cs = c["adaptive_aux_coef_constant_drop_rate"]
+    a = cs["alpha0"]
+    for _ in range(cs["steps"]):
+        a = om.adaptive_aux_coef(a, cs["drop_rate"], cs["beta"], cs["xi"])
+    if not abs(a - cs["expected_alpha"]) <= 1e-15:
+        bad.append(f"adaptive_aux_coef: {a}")
+    # the coefficient rises with the drop rate and falls with it
+    up = om.adaptive_aux_coef(0.05, 0.3, 0.8, 1.0)
+    down = om.adaptive_aux_coef(0.05, 0.01, 0.8, 1.0)
+    if not (down < 0.05 < up):
+        bad.append(f"adaptive_aux_coef direction: {down} {up}")
+    return bad
+
+
 def dataclass_replace(cfg, **kw):
     import dataclasses
     return dataclasses.replace(cfg, **kw)
@@ -250,6 +281,10 @@ def test_special_cases():
     assert check_special_cases() == []
 
 
+def test_losses_closed_forms():
+    assert check_losses() == []
+
+
 def test_capacity_formula_values():
     # the capacities of the workloads: ceil(cf * T * k / E)
     cases = [((8192, 2, 64, 1.25), 320), ((4096, 2, 16, 1.0), 512), ((64, 6, 64, 1.0), 6),
@@ -300,7 +335,8 @@ def test_workload_generator_is_seeded_and_bf16_exact():
 
 # -------------------------------------------------- planted mistakes (CPU)
 def _all_pins():
-    return check_closed_forms() + check_brute_force() + check_invariants() + check_special_cases()
+    return (check_closed_forms() + check_brute_force() + check_invariants() + check_special_cases() +
+            check_losses())
 
 
 def _mut_sample_std(z, lam):
@@ -385,6 +421,26 @@ def _mut_gate_transposed_bias_sign(x, wg, bias=None):
     return z
 
 
+def _mut_z_loss_not_squared(s):
+    if s.shape[0] == 0:
+        return float("nan")
+    return float(np.mean(om.log_partition(s)))
+
+
+def _mut_z_loss_summed(s):
+    if s.shape[0] == 0:
+        return float("nan")
+    return float(np.sum(om.log_partition(s) ** 2))
+
+
+def _mut_log_partition_is_max(s):
+    return s.max(axis=1)
+
+
+def _mut_coef_beta_swapped(alpha, drop_rate, beta, xi):
+    return (1.0 - beta) * alpha + beta * xi * drop_rate
+
+
 MUTATIONS = {
     "sample_std": ("normalise_logits", _mut_sample_std),
     "lambda_ignored": ("normalise_logits", _mut_no_scale),
@@ -396,6 +452,10 @@ MUTATIONS = {
     "capacity_floor": ("capacity", _mut_capacity_floor),
     "aux_uses_kept_counts": ("dispatch", _mut_aux_postdrop),
     "bias_sign_flipped": ("gate_logits", _mut_gate_transposed_bias_sign),
+    "z_loss_not_squared": ("z_loss", _mut_z_loss_not_squared),
+    "z_loss_summed_over_tokens": ("z_loss", _mut_z_loss_summed),
+    "log_partition_is_the_max": ("log_partition", _mut_log_partition_is_max),
+    "coef_smoothing_swapped": ("adaptive_aux_coef", _mut_coef_beta_swapped),
 }
 
 
