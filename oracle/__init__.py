@@ -1,4 +1,4 @@
-"""Float64 CPU oracle of the MoE layer forward pass (test infrastructure only).
+"""Float64 CPU oracle of the MoE layer, forward and backward (test infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
 reference legs may import this package; the CUDA product path never does.
@@ -8,4 +8,8 @@ from .moe_oracle import (  # noqa: F401
     gate_logits, normalise_logits, softmax, top_k, route, capacity, dispatch,
     expert_hidden, expert_ffn, expert_segments, combine, forward, forward_tokens,
     brute_force, log_partition, z_loss, adaptive_aux_coef,
+)
+from .moe_backward import (  # noqa: F401
+    Grads, loss, backward, expert_backward, normalise_backward, silu_grad, gate_weight_backward,
+    aux_prob_grad, softmax_backward, z_loss_score_grad,
 )
