@@ -393,13 +393,14 @@ def breakdown_roofline(L: Layer, a, flush, pk, pk_src, dev):
     xp, h, yp = sv(lay.xp, A * w.d, L.tdt), sv(lay.h, A * w.F, hdt), sv(lay.yp, A * w.d, torch.float32)
     scr = ws[lay.scratch:]
     pm = torch.empty(w.E, dtype=torch.float32, device=dev)
+    zl = torch.empty(1, dtype=torch.float32, device=dev)
     names = ["route", "permute", "expert_ffn", "combine"]
     acc = {n: 0.0 for n in names}
     for i in range(a.warmup + a.steps):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         ev[0].record()
-        moe.moe_route(L.cfg, L.x, L.wg, L.bias, idx, tw, gap, pm, scr)
+        moe.moe_route(L.cfg, L.x, L.wg, L.bias, idx, tw, gap, pm, scr, z_loss=zl)
         ev[1].record()
         moe.moe_permute(L.cfg, L.x, idx, gap, pm, counts, kept, offs, row_of, src_tok, xp, L.stats, scr)
         ev[2].record()
@@ -649,7 +650,8 @@ def main():
                 "gpu_launches": launches_per_step * a.steps,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "breakdown_ms": breakdown,
-                "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "rows_kept": st["rows_kept"],
+                "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "z_loss": st["z_loss"],
+                          "rows_kept": st["rows_kept"],
                           "capacity": st["capacity"], "near_tie_count": st["near_tie_count"]},
                 "extra": extra}
         print(json.dumps(line), flush=True)

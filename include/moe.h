@@ -108,7 +108,10 @@ typedef struct moe_config {
 /* Per-forward statistics, in DEVICE memory, written by moe_permute (and by
  * moe_layer_forward).  Drop-token rate and load balance are the quantities the
  * Skywork-MoE adaptive aux-loss controller monitors (Skywork-MoE release,
- * section "2.自适应的Aux Loss"). */
+ * section "2.自适应的Aux Loss"; see moe_aux_coef_update).  The router z-loss
+ * is the Z-Loss the Megatron-Core best-practice page names among its
+ * load-balancing methods (section "Megatron-Core MoE的关键特性"); the pages
+ * give no formula, and the one above is the reading this library takes. */
 typedef struct moe_stats {
   int32_t drop_count;        /* assignments dropped by the capacity */
   int32_t rows_kept;         /* offsets[E] = T*k - drop_count */
@@ -117,7 +120,9 @@ typedef struct moe_stats {
   float drop_rate;           /* drop_count / (T*k); 0 when T == 0 */
   float aux_loss;            /* E * sum_e (counts_e/(T*k)) * P_e (pre-drop counts); NaN if P not given or T == 0 */
   uint32_t status;           /* MOE_DEV_* bits; cleared by moe_permute, OR-ed by later steps */
-  int32_t reserved;
+  float z_loss;              /* router z-loss (1/T) sum_t (log sum_e exp s[t, e])^2 over the scores the
+                                softmax takes (z_hat when lambda > 0, else z); written by
+                                moe_layer_forward, NaN from a standalone moe_permute or when T == 0 */
 } moe_stats;
 
 /* Byte offsets of the intermediates inside a moe_layer_forward workspace
@@ -153,10 +158,11 @@ size_t moe_workspace_size(const moe_config* cfg, moe_ws_layout* layout);
  *   gap[T] fp32: k-th minus (k+1)-th largest score (z_hat or z), +inf if k == E.
  *   prob_mean[E] fp32 or NULL: P_e = mean over tokens of the full softmax
  *     probability of expert e (input of the aux loss).
+ *   z_loss fp32 scalar or NULL: the router z-loss of the batch (moe_stats.z_loss).
  *   ws: at least moe_scratch_size(cfg) bytes.
  */
 moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
-                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean,
+                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean, float* z_loss,
                      void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
@@ -226,6 +232,30 @@ moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* xp, const i
                                   moe_stream_t stream);
 
 /*
+ * Step 4 over caller-given row segments that share the weights of E experts:
+ * the expert-parallel form of the step.  With the experts partitioned over G
+ * GPUs (FastMoE announcement, "特色四", Figure 6: each worker holds its own
+ * experts and the inputs of an expert are sent to its worker), a GPU receives
+ * from each of the G source ranks that rank's rows for its E local experts,
+ * expert by expert; the G blocks of E segments are run as they arrived.
+ * Segment i holds rows [seg_offsets[i], seg_offsets[i+1]) of xp and runs
+ * through local expert i % E:
+ *   cfg: d, F, act, dtype, hidden_dtype as for the layer; E = the experts
+ *     whose weights W1[E, F1, d] and W2[E, d, F] are given; T, k,
+ *     capacity_factor and lambda are ignored.
+ *   nseg (1..256) segments over a buffer of `rows` rows: seg_offsets[nseg+1]
+ *     device int32, non-decreasing inside [0, rows] (else MOE_DEV_BOUNDS and
+ *     nothing is computed); xp[rows, d], h[rows, F] (hidden_dtype) and
+ *     yp[rows, d] fp32 as in moe_expert_ffn, written for rows
+ *     [0, seg_offsets[nseg]).
+ *   ws: at least moe_segments_scratch_size(cfg, nseg, rows) bytes.
+ */
+size_t moe_segments_scratch_size(const moe_config* cfg, int32_t nseg, int32_t rows);
+moe_status moe_expert_ffn_segments(const moe_config* cfg, int32_t nseg, int32_t rows, const int32_t* seg_offsets,
+                                   const void* xp, const void* W1, const void* W2, void* h, void* yp,
+                                   moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Step 5: un-permute and combine.  out[t] = sum over j = 0..k-1 with
  * row_of[t, j] >= 0 of topk_w[t, j] * yp[row_of[t, j]], accumulated in fp32 in
  * slot order; 0 for a token whose slots were all dropped (the residual path
@@ -248,6 +278,38 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * The backward of the layer: the gradients of
+ *     L = sum_{t,i} dout[t, i] out[t, i] + aux_coef * aux_loss + z_coef * z_loss
+ * with respect to x, W_gate, the gate bias, W1 and W2, for a forward already
+ * run by moe_layer_forward on the same inputs.  The layer's figures on the
+ * pages are training figures (FastMoE announcement, "特色三"; Skywork-MoE
+ * release, "训练Infra"), and the aux loss (Switch form, pre-drop counts) and
+ * its coefficient and the z-loss are those of moe_stats and moe_aux_coef_update.
+ * The forward's discrete choices (selected experts, capacity drops, counts)
+ * carry no gradient and are read from its workspace `fws`.
+ *   x, Wg, bg (or NULL), W1 as for the forward; W2[E, d, F] in the element
+ *     type of x (bf16 on the bf16 path, not the fp16 copy an fp16 hidden
+ *     activation uses; fp32 on the fp32 path).
+ *   dout[T, d] fp32: the gradient of L with respect to out.
+ *   fws: the workspace of that forward (moe_workspace_size bytes), unchanged
+ *     since.
+ *   Outputs, all fp32 and fully written: dx[T, d], dWg[E, d], dbg[E] (or
+ *     NULL), dW1[E, F1, d], dW2[E, d, F]; dw[T, k] (or NULL): the gradient of
+ *     the gate weights topk_w (0 for a dropped slot).
+ *   ws: at least moe_backward_workspace_size(cfg) bytes (256-byte aligned).
+ *   stats: device moe_stats; device-detected errors are OR-ed into status
+ *     (clear it before the call for a clean record).
+ * The expert GEMMs run on the tensor cores (bf16 operands, fp32 accumulation:
+ * dout is rounded to bf16 for them) on the bf16 path and in fp32 FFMA on the
+ * fp32 path.  Gradients are written, never accumulated into.
+ */
+size_t moe_backward_workspace_size(const moe_config* cfg);
+moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* Wg, const float* bg, const void* W1,
+                              const void* W2, const float* dout, float aux_coef, float z_coef, const void* fws,
+                              size_t fws_bytes, float* dx, float* dWg, float* dbg, float* dW1, float* dW2,
+                              float* dw, moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Weight preparation (run once when the weights are loaded, not per forward):
  * dst[i] = fp16(src[i]) for n bf16 values, round to nearest even; values
  * beyond the fp16 range saturate to +-65504.  Every bf16 value of magnitude in
@@ -257,6 +319,44 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
  * the pages: it prepares the storage format of the second expert layer.
  */
 moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_stream_t stream);
+
+/*
+ * Layer-wise adaptive aux-loss coefficient (Skywork-MoE release, section
+ * "2.自适应的Aux Loss"; slides, slide 7: each layer's coefficient is raised
+ * when its token drop rate rises and lowered when it falls, to keep the drop
+ * rate in a suitable band).  The pages give no formula; the reading taken is
+ * an exponential moving average of a target proportional to the drop rate:
+ *     coef <- beta * coef + (1 - beta) * xi * drop_rate
+ * with smoothing 0 <= beta <= 1 and sensitivity xi >= 0 (both finite).
+ *
+ * moe_aux_coef_update: on the device, after a forward: reads stats->drop_rate
+ *   (device moe_stats of that layer) and updates *coef (device fp32) in place,
+ *   one thread on `stream`, no host synchronisation.  MOE_ERR_ARG for a NULL
+ *   or misaligned pointer or beta / xi out of range.
+ * moe_aux_coef_next: the same step on the host: *next = the updated value of
+ *   coef given drop_rate (0 <= drop_rate <= 1).  MOE_ERR_ARG on a bad value.
+ */
+moe_status moe_aux_coef_update(const moe_stats* stats, float* coef, float beta, float xi, moe_stream_t stream);
+moe_status moe_aux_coef_next(float coef, float drop_rate, float beta, float xi, float* next);
+
+/*
+ * Test hook for the failure path of the bounded waits.  No counterpart on the
+ * pages.  Every wait inside the kernels gives up after a limit (2 s by
+ * default), sets MOE_DEV_TIMEOUT in moe_stats.status, stops the kernel's other
+ * roles, waits for its own copies and MMAs in flight, frees its tensor memory
+ * and returns, so that the context stays usable.  This call lets a test reach
+ * that path without a GPU fault, in the one-launch expert kernel (bf16 path,
+ * 1-SM tiles, the kernel moe_layer_forward and moe_expert_ffn run on layers
+ * with T*k < 512*E):
+ *   wait_ns: limit of that kernel's waits in ns (0 = the default 2 s; at most
+ *     60 s);
+ *   extra_dependency: added to the number of layer-1 releases a layer-2 tile
+ *     waits for (0 = none; > 0 makes that wait unreachable, so it runs out).
+ * The setting is process-wide and applies to launches made after the call;
+ * MOE_ERR_ARG for wait_ns > 60 s or extra_dependency < 0.  Not for use
+ * outside tests.
+ */
+moe_status moe_testing_set_expert_wait(uint64_t wait_ns, int32_t extra_dependency);
 
 /* Size of the library's fixed device scratch array used by moe_permute_static. */
 #define MOE_STATIC_SCRATCH_BYTES (2u << 20)
@@ -271,9 +371,13 @@ moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_str
  *   Arguments, layout, ownership and results: as moe_permute, minus ws.
  *   Limit: moe_scratch_size(cfg) <= MOE_STATIC_SCRATCH_BYTES, else
  *     MOE_ERR_UNSUPPORTED before any device work (e.g. E = 64 experts, k = 2
- *     allows T up to about 344k tokens on the bf16 path, 347k on fp32).
+ *     allows T up to about 342k tokens on the bf16 path, 345k on fp32).
  *   The first call on a device looks up the array's address (that device
- *     must be current) and returns MOE_ERR_CUDA if the lookup fails.
+ *     must be current; make this first call before any stream capture) and
+ *     returns MOE_ERR_CUDA if the lookup fails; a failed lookup is retried by
+ *     the next call, a successful one is kept for the life of the process.
+ *     cudaDeviceReset destroys the array, and the kept address with it: do
+ *     not call this entry point on a device after resetting it.
  *   Every scratch word the kernels read is written earlier in the same call;
  *     the one value that must start at zero, stats->status, is cleared by the
  *     call on `stream`.

@@ -20,7 +20,9 @@ __all__ = [
     "LIB_PATH", "MoeError", "moe_config", "moe_stats", "moe_ws_layout", "lib", "make_config",
     "moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "moe_permute_static",
-    "moe_expert_ffn_combine", "MOE_STATIC_SCRATCH_BYTES", "prepare_w2",
+    "moe_expert_ffn_combine", "MOE_STATIC_SCRATCH_BYTES", "prepare_w2", "moe_aux_coef_update",
+    "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_segments_scratch_size", "moe_expert_ffn_segments",
+    "moe_backward_workspace_size", "moe_layer_backward",
     "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
     "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
@@ -34,7 +36,10 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE
 
 EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size", "moe_route",
                     "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-                    "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine"]
+                    "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine",
+                    "moe_aux_coef_update", "moe_aux_coef_next", "moe_testing_set_expert_wait",
+                    "moe_segments_scratch_size", "moe_expert_ffn_segments", "moe_backward_workspace_size",
+                    "moe_layer_backward"]
 MOE_STATIC_SCRATCH_BYTES = 2 << 20
 
 
@@ -48,7 +53,7 @@ class moe_config(ctypes.Structure):
 class moe_stats(ctypes.Structure):
     _fields_ = [("drop_count", ctypes.c_int32), ("rows_kept", ctypes.c_int32), ("capacity", ctypes.c_int32),
                 ("near_tie_count", ctypes.c_int32), ("drop_rate", ctypes.c_float), ("aux_loss", ctypes.c_float),
-                ("status", ctypes.c_uint32), ("reserved", ctypes.c_int32)]
+                ("status", ctypes.c_uint32), ("z_loss", ctypes.c_float)]
 
 
 class moe_ws_layout(ctypes.Structure):
@@ -83,7 +88,7 @@ def lib() -> ctypes.CDLL:
     L.moe_scratch_size.restype = ctypes.c_size_t
     L.moe_workspace_size.argtypes = [cfgp, ctypes.POINTER(moe_ws_layout)]
     L.moe_workspace_size.restype = ctypes.c_size_t
-    L.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_permute.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_combine.argtypes = [cfgp, P, P, P, P, P]
@@ -91,8 +96,21 @@ def lib() -> ctypes.CDLL:
     L.moe_convert_bf16_to_f16.argtypes = [P, P, ctypes.c_size_t, P]
     L.moe_permute_static.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P]
     L.moe_expert_ffn_combine.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    f32 = ctypes.c_float
+    L.moe_aux_coef_update.argtypes = [P, P, f32, f32, P]
+    L.moe_aux_coef_next.argtypes = [f32, f32, f32, f32, ctypes.POINTER(f32)]
+    L.moe_testing_set_expert_wait.argtypes = [ctypes.c_uint64, ctypes.c_int32]
+    i32 = ctypes.c_int32
+    L.moe_segments_scratch_size.argtypes = [cfgp, i32, i32]
+    L.moe_segments_scratch_size.restype = ctypes.c_size_t
+    L.moe_expert_ffn_segments.argtypes = [cfgp, i32, i32, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_backward_workspace_size.argtypes = [cfgp]
+    L.moe_backward_workspace_size.restype = ctypes.c_size_t
+    L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, f32, f32, P, ctypes.c_size_t, P, P, P, P, P, P, P, P,
+                                     ctypes.c_size_t, P]
     for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-              "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine"]:
+              "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine", "moe_aux_coef_update",
+              "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_expert_ffn_segments", "moe_layer_backward"]:
         getattr(L, n).restype = st
     _lib = L
     return L
@@ -153,10 +171,11 @@ def moe_workspace_size(cfg: moe_config):
     return n, L
 
 
-def moe_route(cfg, x, Wg, bg, topk_idx, topk_w, gap, prob_mean, ws, stream=None):
+def moe_route(cfg, x, Wg, bg, topk_idx, topk_w, gap, prob_mean, ws, stream=None, z_loss=None):
+    """z_loss: optional device fp32 scalar that receives the router z-loss."""
     _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg), _ptr(topk_idx),
-                                        _ptr(topk_w), _ptr(gap), _ptr(prob_mean), _ptr(ws), _nbytes(ws),
-                                        _stream(stream)))
+                                        _ptr(topk_w), _ptr(gap), _ptr(prob_mean), _ptr(z_loss), _ptr(ws),
+                                        _nbytes(ws), _stream(stream)))
 
 
 def moe_permute(cfg, x, topk_idx, gap, prob_mean, counts, kept, offsets, row_of, src_tok, xp, stats, ws,
@@ -192,6 +211,19 @@ def moe_expert_ffn_combine(cfg, xp, offsets, src_tok, row_w, W1, W2, h, out, sta
                                         _stream(stream)))
 
 
+def moe_segments_scratch_size(cfg: moe_config, nseg: int, rows: int) -> int:
+    return lib().moe_segments_scratch_size(ctypes.byref(cfg), nseg, rows)
+
+
+def moe_expert_ffn_segments(cfg, nseg, rows, seg_offsets, xp, W1, W2, h, yp, stats, ws, stream=None):
+    """Step 4 over nseg caller-given segments of a rows-row buffer; segment i
+    runs through local expert i % cfg.E (the expert-parallel form)."""
+    _check("moe_expert_ffn_segments",
+           lib().moe_expert_ffn_segments(ctypes.byref(cfg), nseg, rows, _ptr(seg_offsets), _ptr(xp), _ptr(W1),
+                                         _ptr(W2), _ptr(h), _ptr(yp), _ptr(stats), _ptr(ws), _nbytes(ws),
+                                         _stream(stream)))
+
+
 def moe_combine(cfg, yp, row_of, topk_w, out, stream=None):
     _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(yp), _ptr(row_of), _ptr(topk_w),
                                             _ptr(out), _stream(stream)))
@@ -201,6 +233,40 @@ def moe_layer_forward(cfg, x, Wg, bg, W1, W2, out, stats, ws, stream=None):
     _check("moe_layer_forward", lib().moe_layer_forward(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg),
                                                         _ptr(W1), _ptr(W2), _ptr(out), _ptr(stats), _ptr(ws),
                                                         _nbytes(ws), _stream(stream)))
+
+
+def moe_aux_coef_update(stats, coef, beta: float, xi: float, stream=None):
+    """On the device: coef <- beta * coef + (1 - beta) * xi * stats.drop_rate
+    (stats: device moe_stats bytes, coef: device fp32 scalar)."""
+    _check("moe_aux_coef_update", lib().moe_aux_coef_update(_ptr(stats), _ptr(coef), beta, xi, _stream(stream)))
+
+
+def moe_aux_coef_next(coef: float, drop_rate: float, beta: float, xi: float) -> float:
+    """The same update on the host (no device involved)."""
+    out = ctypes.c_float()
+    _check("moe_aux_coef_next", lib().moe_aux_coef_next(coef, drop_rate, beta, xi, ctypes.byref(out)))
+    return out.value
+
+
+def moe_testing_set_expert_wait(wait_ns: int, extra_dependency: int):
+    """Test hook: limit of the one-launch expert kernel's waits (0 = default)
+    and an amount added to its layer-2 dependency target (> 0: unreachable)."""
+    _check("moe_testing_set_expert_wait", lib().moe_testing_set_expert_wait(wait_ns, extra_dependency))
+
+
+def moe_backward_workspace_size(cfg: moe_config) -> int:
+    return lib().moe_backward_workspace_size(ctypes.byref(cfg))
+
+
+def moe_layer_backward(cfg, x, Wg, bg, W1, W2, dout, aux_coef, z_coef, fws, dx, dWg, dbg, dW1, dW2, dw, stats, ws,
+                       stream=None):
+    """Gradients of <dout, out> + aux_coef * aux + z_coef * z_loss for the forward
+    whose workspace is fws (see include/moe.h)."""
+    _check("moe_layer_backward",
+           lib().moe_layer_backward(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg), _ptr(W1), _ptr(W2), _ptr(dout),
+                                    aux_coef, z_coef, _ptr(fws), _nbytes(fws), _ptr(dx), _ptr(dWg), _ptr(dbg),
+                                    _ptr(dW1), _ptr(dW2), _ptr(dw), _ptr(stats), _ptr(ws), _nbytes(ws),
+                                    _stream(stream)))
 
 
 def moe_convert_bf16_to_f16(src, dst, n: Optional[int] = None, stream=None):

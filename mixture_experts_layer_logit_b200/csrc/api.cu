@@ -3,6 +3,8 @@
 #include "internal.cuh"
 
 #include <math.h>
+
+#include <algorithm>
 #include <mutex>
 
 namespace moe {
@@ -43,6 +45,7 @@ Scratch scratch_layout(const moe_config& c) {
   s.choff = off; off = align256(off + sizeof(int32_t) * (size_t)c.E * nch);
   s.psum = off;  off = align256(off + sizeof(float) * (size_t)c.E * nch);
   s.ntie = off;  off = align256(off + sizeof(int32_t) * nch);
+  s.zsum = off;  off = align256(off + sizeof(float) * nch);
   s.status = off; off = align256(off + sizeof(uint32_t));
   s.mlp = off;    off = align256(off + (c.dtype == MOE_DTYPE_BF16 ? sizeof(int) * expert_mlp_counters(c) : 0));
   s.kslice = off; off = align256(off + route_tc_scratch_bytes(c));
@@ -132,14 +135,14 @@ T* at(void* base, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(b
 
 // step 3 given the histogram already in scratch
 moe_status permute_from_hist(const moe_config& c, const void* x, const int32_t* topk_idx,
-                             const float* prob_mean, const float* psum, const int32_t* ntie,
+                             const float* prob_mean, const float* psum, const int32_t* ntie, const float* zsum,
                              int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                              int32_t* src_tok, void* xp, moe_stats* stats, const Scratch& sc, void* ws,
                              cudaStream_t s, const float* topk_w = nullptr, float* row_w = nullptr,
                              float* out = nullptr, int* zero = nullptr, int nzero = 0) {
   return cuda_status(launch_permute(c, capacity_of(c), x, topk_idx, at<int32_t>(ws, sc.hist),
-                                    at<int32_t>(ws, sc.choff), prob_mean, psum, ntie, counts, kept, offsets,
-                                    row_of, src_tok, xp, stats, s, topk_w, row_w, out, zero, nzero));
+                                    at<int32_t>(ws, sc.choff), prob_mean, psum, ntie, zsum, counts, kept,
+                                    offsets, row_of, src_tok, xp, stats, s, topk_w, row_w, out, zero, nzero));
 }
 
 // Mean assignments per expert from which the expert GEMMs use 2-SM tiles.
@@ -148,15 +151,16 @@ bool pair_tiles(const moe_config& c) { return (long long)c.T * c.k >= kPairRowsP
 
 moe_status expert_ffn(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                       const void* w2, void* h, void* yp, moe_stats* stats, cudaStream_t s,
-                      const CombineOut* comb = nullptr) {
+                      const CombineOut* comb = nullptr, int e_mod = 0) {
   if (c.dtype == MOE_DTYPE_BF16) {
     // 2-SM pair tiles (256 rows) pay off once the expert segments hold a few
     // hundred rows on average; short segments waste half a pair tile.
     if (pair_tiles(c))
-      return cuda_status(launch_expert_ffn_tc_pair(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
-    return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb));
+      return cuda_status(
+          launch_expert_ffn_tc_pair(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb, e_mod));
+    return cuda_status(launch_expert_ffn_tc(c, xp, offsets, w1, w2, h, yp, &stats->status, s, comb, e_mod));
   }
-  return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, &stats->status, s));
+  return cuda_status(launch_expert_ffn_simt(c, xp, offsets, w1, w2, h, yp, &stats->status, s, e_mod));
 }
 
 // The forward fuses step 5 into the second expert GEMM when a token has at
@@ -180,11 +184,23 @@ bool one_launch_plain(const moe_config& c) {
 }
 moe_status expert_mlp_plain(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                             const void* w2, void* h, void* yp, moe_stats* stats, int* counters,
-                            bool counters_zeroed, cudaStream_t s) {
+                            bool counters_zeroed, cudaStream_t s, int e_mod = 0) {
   if (!counters_zeroed && cudaMemsetAsync(counters, 0, sizeof(int) * expert_mlp_counters(c), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, nullptr, static_cast<float*>(yp), counters,
-                                       &stats->status, s));
+                                       &stats->status, s, e_mod));
+}
+
+// The configuration step 4 runs with over `nseg` caller-given segments of a
+// `rows`-row buffer: one "assignment" per row, one tile-table entry per segment.
+moe_config segments_config(const moe_config& c, int nseg, int rows) {
+  moe_config cc = c;
+  cc.T = rows;
+  cc.k = 1;
+  cc.E = nseg;
+  cc.capacity_factor = 0.f;
+  cc.lambda = 0.f;
+  return cc;
 }
 
 // Steps 4-5 fused (out zeroed beforehand); counters: the yp region.
@@ -198,6 +214,41 @@ moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* o
     return cuda_status(launch_expert_mlp(c, xp, offsets, w1, w2, h, &comb, nullptr, counters, &stats->status, s));
   }
   return expert_ffn(c, xp, offsets, w1, w2, h, yp, stats, s, &comb);
+}
+
+// Layout of the backward workspace (each region 256-byte aligned).
+struct BwdLayout {
+  int rows;
+  int nsplit, tok_per_split, col_tiles;
+  size_t pad_offsets, xp, dout_perm, wrow, u, du, hw, dwpart, dxp, z, dz, dwg_part, total;
+};
+
+BwdLayout bwd_layout(const moe_config& c) {
+  BwdLayout L{};
+  const size_t es = elem_size(c);
+  const int F1 = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  const long long rows = (long long)c.T * c.k + (long long)(bwd_pad_rows() - 1) * c.E;
+  L.rows = (int)((rows + 127) / 128 * 128);
+  const int col = c.dtype == MOE_DTYPE_BF16 ? bwd_tc_col_tile() : bwd_simt_col_tile();
+  L.col_tiles = (c.F + col - 1) / col;
+  L.tok_per_split = std::max(256, (((c.T + 63) / 64) + 63) / 64 * 64);
+  L.nsplit = std::max(1, (c.T + L.tok_per_split - 1) / L.tok_per_split);
+  const size_t R = (size_t)L.rows, T = (size_t)c.T, E = (size_t)c.E, d = (size_t)c.d;
+  size_t off = 0;
+  L.pad_offsets = off; off = align256(off + 4 * (E + 1));
+  L.xp = off;          off = align256(off + es * R * d);
+  L.dout_perm = off;   off = align256(off + es * R * d);
+  L.wrow = off;        off = align256(off + 4 * R);
+  L.u = off;           off = align256(off + 4 * R * (size_t)F1);
+  L.du = off;          off = align256(off + es * R * (size_t)F1);
+  L.hw = off;          off = align256(off + es * R * (size_t)c.F);
+  L.dwpart = off;      off = align256(off + 4 * R * (size_t)L.col_tiles);
+  L.dxp = off;         off = align256(off + 4 * R * d);
+  L.z = off;           off = align256(off + 4 * T * E);
+  L.dz = off;          off = align256(off + 4 * T * E);
+  L.dwg_part = off;    off = align256(off + 4 * (size_t)L.nsplit * E * (d + 1));
+  L.total = off;
+  return L;
 }
 
 }  // namespace
@@ -228,7 +279,7 @@ size_t moe_workspace_size(const moe_config* cfg, moe_ws_layout* layout) {
 }
 
 moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
-                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean,
+                     int32_t* topk_idx, float* topk_w, float* gap, float* prob_mean, float* z_loss,
                      void* ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
@@ -236,17 +287,25 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const
   if (c.T > 0 && (x == nullptr || Wg == nullptr || topk_idx == nullptr || topk_w == nullptr || gap == nullptr))
     return MOE_ERR_ARG;
   if (!aligned16(x) || !aligned16(Wg) || !aligned4(bg) || !aligned4(topk_idx) || !aligned4(topk_w) ||
-      !aligned4(gap) || !aligned4(prob_mean))
+      !aligned4(gap) || !aligned4(prob_mean) || !aligned4(z_loss))
     return MOE_ERR_ARG;
   const Scratch sc = scratch_layout(c);
   if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
   if ((st = check_device(false)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(c, x, Wg, bg, topk_idx, topk_w, gap, at<int32_t>(ws, sc.hist),
-                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<uint32_t>(ws, sc.status),
-                               at<char>(ws, sc.kslice), s);
+                               at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<float>(ws, sc.zsum),
+                               at<uint32_t>(ws, sc.status), at<char>(ws, sc.kslice), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  if (prob_mean != nullptr) e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s);
+  if (c.T == 0) {   // empty batch: P_e and the z-loss are not defined
+    if (prob_mean != nullptr && cudaMemsetAsync(prob_mean, 0xff, sizeof(float) * (size_t)c.E, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (z_loss != nullptr && cudaMemsetAsync(z_loss, 0xff, sizeof(float), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (prob_mean != nullptr && (e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (z_loss != nullptr) e = launch_z_loss(c, at<float>(ws, sc.zsum), z_loss, s);
   return cuda_status(e);
 }
 
@@ -274,7 +333,7 @@ moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk
                               &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return permute_from_hist(c, x, topk_idx, prob_mean, nullptr,
-                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, counts, kept,
+                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, nullptr, counts, kept,
                            offsets, row_of, src_tok, xp, stats, sc, ws, s);
 }
 
@@ -375,13 +434,14 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   // near-tie counts of every chunk in scratch, so step 3 starts from the
   // histograms (the scatter scans them itself)
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
-                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), &stats->status,
-                               at<char>(scr, sc.kslice), s);
+                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), at<float>(scr, sc.zsum),
+                               &stats->status, at<char>(scr, sc.kslice), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   float* row_w = at<float>(ws, L.row_w);
   float* out_f = static_cast<float*>(out);
   st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
-                         c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, at<int32_t>(ws, L.counts),
+                         c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, c.T > 0 ? at<float>(scr, sc.zsum) : nullptr,
+                         at<int32_t>(ws, L.counts),
                          at<int32_t>(ws, L.kept), offsets, row_of, at<int32_t>(ws, L.src_tok),
                          at<char>(ws, L.xp), stats, sc, scr, s, fuse ? w : nullptr, fuse ? row_w : nullptr,
                          fuse ? out_f : nullptr, zero_in_scatter ? counters : nullptr,
@@ -426,8 +486,137 @@ moe_status moe_permute_static(const moe_config* cfg, const void* x, const int32_
                               &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return permute_from_hist(c, x, topk_idx, prob_mean, nullptr,
-                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, counts, kept,
+                           (gap != nullptr && c.T > 0) ? at<int32_t>(ws, sc.ntie) : nullptr, nullptr, counts, kept,
                            offsets, row_of, src_tok, xp, stats, sc, ws, s);
+}
+
+moe_status moe_aux_coef_update(const moe_stats* stats, float* coef, float beta, float xi, moe_stream_t stream) {
+  if (stats == nullptr || coef == nullptr || !aligned4(stats) || !aligned4(coef)) return MOE_ERR_ARG;
+  if (!(beta >= 0.f && beta <= 1.f) || !(xi >= 0.f) || !isfinite(xi)) return MOE_ERR_ARG;
+  moe_status st = check_device(false);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_aux_coef_update(stats, coef, beta, xi, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_aux_coef_next(float coef, float drop_rate, float beta, float xi, float* next) {
+  if (next == nullptr || !isfinite(coef) || !(drop_rate >= 0.f && drop_rate <= 1.f)) return MOE_ERR_ARG;
+  if (!(beta >= 0.f && beta <= 1.f) || !(xi >= 0.f) || !isfinite(xi)) return MOE_ERR_ARG;
+  *next = aux_coef_step(coef, drop_rate, beta, xi);
+  return MOE_OK;
+}
+
+size_t moe_segments_scratch_size(const moe_config* cfg, int32_t nseg, int32_t rows) {
+  if (check_config(cfg) != MOE_OK || nseg < 1 || nseg > kMaxExperts || rows < 0) return 0;
+  const moe_config cc = segments_config(*cfg, nseg, rows);
+  if (check_config(&cc) != MOE_OK) return 0;
+  return scratch_layout(cc).total;
+}
+
+moe_status moe_expert_ffn_segments(const moe_config* cfg, int32_t nseg, int32_t rows, const int32_t* seg_offsets,
+                                   const void* xp, const void* W1, const void* W2, void* h, void* yp,
+                                   moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (nseg < 1 || rows < 0) return MOE_ERR_ARG;
+  if (nseg > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  const moe_config cc = segments_config(*cfg, nseg, rows);
+  if ((st = check_config(&cc)) != MOE_OK) return st;
+  if (seg_offsets == nullptr || stats == nullptr) return MOE_ERR_ARG;
+  if (rows > 0 && (xp == nullptr || W1 == nullptr || W2 == nullptr || h == nullptr || yp == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(xp) || !aligned16(W1) || !aligned16(W2) || !aligned16(h) || !aligned16(yp) ||
+      !aligned4(seg_offsets) || !aligned4(stats))
+    return MOE_ERR_ARG;
+  const Scratch sc = scratch_layout(cc);
+  if ((st = check_ws(ws, ws_bytes, sc.total)) != MOE_OK) return st;
+  if ((st = check_device(cc.dtype == MOE_DTYPE_BF16)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return MOE_OK;
+  if (one_launch_plain(cc))
+    return expert_mlp_plain(cc, xp, seg_offsets, W1, W2, h, yp, stats, at<int>(ws, sc.mlp), false, s, cfg->E);
+  return expert_ffn(cc, xp, seg_offsets, W1, W2, h, yp, stats, s, nullptr, cfg->E);
+}
+
+size_t moe_backward_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return bwd_layout(*cfg).total;
+}
+
+moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* Wg, const float* bg, const void* W1,
+                              const void* W2, const float* dout, float aux_coef, float z_coef, const void* fws,
+                              size_t fws_bytes, float* dx, float* dWg, float* dbg, float* dW1, float* dW2,
+                              float* dw, moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (stats == nullptr || Wg == nullptr || W1 == nullptr || W2 == nullptr || dWg == nullptr || dW1 == nullptr ||
+      dW2 == nullptr)
+    return MOE_ERR_ARG;
+  if (c.T > 0 && (x == nullptr || dout == nullptr || dx == nullptr)) return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned4(bg) || !aligned16(W1) || !aligned16(W2) || !aligned16(dout) ||
+      !aligned16(dx) || !aligned16(dWg) || !aligned4(dbg) || !aligned16(dW1) || !aligned16(dW2) || !aligned4(dw) ||
+      !aligned4(stats))
+    return MOE_ERR_ARG;
+  if (!isfinite(aux_coef) || !isfinite(z_coef)) return MOE_ERR_ARG;
+  const moe_ws_layout FL = layout_of(c);
+  if ((st = check_ws(const_cast<void*>(fws), fws_bytes, FL.total)) != MOE_OK) return st;
+  const BwdLayout BL = bwd_layout(c);
+  if ((st = check_ws(ws, ws_bytes, BL.total)) != MOE_OK) return st;
+  if ((st = check_device(c.dtype == MOE_DTYPE_BF16)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int F1 = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  if (c.T == 0) {   // no token: every weight gradient is zero
+    if (cudaMemsetAsync(dW1, 0, sizeof(float) * (size_t)c.E * F1 * c.d, s) != cudaSuccess ||
+        cudaMemsetAsync(dW2, 0, sizeof(float) * (size_t)c.E * c.d * c.F, s) != cudaSuccess ||
+        cudaMemsetAsync(dWg, 0, sizeof(float) * (size_t)c.E * c.d, s) != cudaSuccess ||
+        (dbg != nullptr && cudaMemsetAsync(dbg, 0, sizeof(float) * (size_t)c.E, s) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  void* f = const_cast<void*>(fws);
+  BwdState b{};
+  b.topk_idx = at<int32_t>(f, FL.topk_idx);
+  b.topk_w = at<float>(f, FL.topk_w);
+  b.counts = at<int32_t>(f, FL.counts);
+  b.offsets = at<int32_t>(f, FL.offsets);
+  b.row_of = at<int32_t>(f, FL.row_of);
+  b.src_tok = at<int32_t>(f, FL.src_tok);
+  b.pad_offsets = at<int32_t>(ws, BL.pad_offsets);
+  b.rows_alloc = BL.rows;
+  b.xp = at<char>(ws, BL.xp);
+  b.dout_perm = at<char>(ws, BL.dout_perm);
+  b.wrow = at<float>(ws, BL.wrow);
+  b.u = at<float>(ws, BL.u);
+  b.du = at<char>(ws, BL.du);
+  b.hw = at<char>(ws, BL.hw);
+  b.dwpart = at<float>(ws, BL.dwpart);
+  b.dxp = at<float>(ws, BL.dxp);
+  b.z = at<float>(ws, BL.z);
+  b.dz = at<float>(ws, BL.dz);
+  b.dwg_part = at<float>(ws, BL.dwg_part);
+  b.nsplit = BL.nsplit;
+  b.tok_per_split = BL.tok_per_split;
+  b.status = &stats->status;
+  // padded rows: x, dout and the gate weight of every kept assignment
+  if (launch_bwd_front(c, x, dout, b, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // the first layer's pre-activation u = xp W1[e]^T, then the expert layers' gradients
+  cudaError_t e;
+  if (c.dtype == MOE_DTYPE_BF16) {
+    e = launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);
+    if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, W1, W2, dW1, dW2, s);
+  } else {
+    e = launch_grouped_plain_simt(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);
+    if (e == cudaSuccess) e = launch_expert_backward_simt(c, b, W1, W2, dW1, dW2, s);
+  }
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // the gate: scores, logits, dx and dW_gate
+  return cuda_status(launch_bwd_gate(c, x, Wg, bg, b, aux_coef, z_coef, dx, dWg, dbg, dw, s));
+}
+
+moe_status moe_testing_set_expert_wait(uint64_t wait_ns, int32_t extra_dependency) {
+  if (wait_ns > 60000000000ull || extra_dependency < 0) return MOE_ERR_ARG;
+  set_expert_mlp_test_hooks(wait_ns, extra_dependency);
+  return MOE_OK;
 }
 
 }  // extern "C"

@@ -35,7 +35,13 @@ struct Params {
   const int32_t* src_tok;   // kCombine: token of each permuted row
   const float* row_w;       // kCombine: gate weight of each permuted row
   int out_rows;             // kCombine: token rows of the output
+  int e_mod;                // weight blocks: segment e uses block e % e_mod (0: e itself)
 };
+
+// Weight block of segment e: segments may outnumber the experts whose
+// weights are given (the segments of several source ranks, each holding the
+// same local experts in turn).
+__device__ __forceinline__ int weight_block(const Params& p, int e) { return p.e_mod > 0 ? e % p.e_mod : e; }
 
 // Two fp32 values -> one 32-bit pair of the hidden type (round to nearest
 // even).  fp16 saturates at +-65504 (NaN passes through) and notes it in `over`.

@@ -33,6 +33,7 @@
 #include "gemm_common.cuh"
 
 #include <algorithm>
+#include <atomic>
 
 namespace moe {
 namespace {
@@ -76,6 +77,9 @@ struct MlpParams {
   int* sched;               // [0]: next tile to claim; zeroed beforehand
   int* dep;                 // per global m-tile: layer-1 n-tiles finished; zeroed beforehand
   uint32_t* status;
+  unsigned long long wait_ns;   // limit of every bounded wait (kWaitNs unless a test shortens it)
+  int dep_extra;                // added to the layer-2 dependency target (0 unless a test sets it)
+  int e_mod;                    // weight blocks: segment e uses block e % e_mod
 };
 
 // the tile's layer, coordinates and global m-tile index
@@ -174,7 +178,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       for (int n = 0; ok; ++n) {
         const int q = n % kQueue;
         const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
-        if (!mbar_wait(qempty0 + 8 * q, qph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+        if (!mbar_wait(qempty0 + 8 * q, qph ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         int L = atomicAdd(p.sched, 1);
         if (L >= total) L = -1;
         tail->queue[q] = L;
@@ -185,21 +189,21 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         const CUtensorMap* mB = t.l2 ? &tmB2 : &tmB1;
         int b0, b1;
         if (!t.l2) {
-          b0 = t.c.e * p.F1 + t.c.n0;
+          b0 = (t.c.e % p.e_mod) * p.F1 + t.c.n0;
           b1 = (ACT == kSwiglu) ? b0 + p.F : b0 + BN / 2;
         } else {
-          b0 = t.c.e * p.d + t.c.n0;
+          b0 = (t.c.e % p.e_mod) * p.d + t.c.n0;
           b1 = b0 + BN / 2;
         }
         if (t.l2) {   // the h rows of this m-tile: every layer-1 n-tile, 4 epilogue warps each
-          if (!wait_flag_geq(p.dep + t.m, 4 * nt1, abort_flag, kWaitNs)) { ok = false; break; }
+          if (!wait_flag_geq(p.dep + t.m, 4 * nt1 + p.dep_extra, abort_flag, p.wait_ns)) { ok = false; break; }
           fence_proxy_async_global();
         }
         const int nkb = t.l2 ? nkb2 : nkb1;
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           const uint32_t sa = base + (uint32_t)(s * STAGE_BYTES);
           mbar_expect_tx(full0 + 8 * s, STAGE_BYTES);
           tma_load_2d(sa, mA, full0 + 8 * s, kb * BK, t.c.row0);
@@ -223,7 +227,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       for (int n = 0; ok; ++n) {
         const int q = n % kQueue;
         const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
-        if (!mbar_wait(qfull0 + 8 * q, qph, abort_flag, kWaitNs)) { ok = false; break; }
+        if (!mbar_wait(qfull0 + 8 * q, qph, abort_flag, p.wait_ns)) { ok = false; break; }
         const int L = tail->queue[q];
         mbar_arrive(qempty0 + 8 * q);
         if (L < 0) break;
@@ -232,13 +236,13 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         const uint32_t idesc = l2 ? kIdesc2 : kIdesc1;
         const int acc = tl & 1;
         const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
-        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kWaitNs)) { ok = false; break; }
+          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + (uint32_t)(s * STAGE_BYTES);
           const uint64_t ad = sdesc(sa), bd = sdesc(sa + A_BYTES);
@@ -268,7 +272,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
     for (int n = 0;; ++n) {
       const int q = n % kQueue;
       const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
-      ok = mbar_wait(qfull0 + 8 * q, qph, abort_flag, kWaitNs);
+      ok = mbar_wait(qfull0 + 8 * q, qph, abort_flag, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const int L = tail->queue[q];
@@ -278,7 +282,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       const MlpTile t = mlp_tile<ACT>(tail, p.E, T1, L);
       const int acc = tl & 1;
       const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
-      ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kWaitNs);
+      ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -329,7 +333,15 @@ cudaError_t launch_c(const CUtensorMap (&maps)[4], const MlpParams& p, bool comb
   return comb ? launch_t<ACT, F16, true>(maps, p, grid, s) : launch_t<ACT, F16, false>(maps, p, grid, s);
 }
 
+std::atomic<unsigned long long> g_wait_ns{kWaitNs};
+std::atomic<int> g_dep_extra{0};
+
 }  // namespace
+
+void set_expert_mlp_test_hooks(unsigned long long wait_ns, int dep_extra) {
+  g_wait_ns.store(wait_ns != 0 ? wait_ns : kWaitNs);
+  g_dep_extra.store(dep_extra);
+}
 
 size_t expert_mlp_counters(const moe_config& c) {
   return 1 + (size_t)c.T * c.k / BM + (size_t)c.E + 1;
@@ -337,7 +349,7 @@ size_t expert_mlp_counters(const moe_config& c) {
 
 cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                               const void* w2, void* h, const CombineOut* comb, float* yp, int* counters,
-                              uint32_t* status, cudaStream_t s) {
+                              uint32_t* status, cudaStream_t s, int e_mod) {
   if (c.T == 0) return cudaSuccess;
   if (comb == nullptr && yp == nullptr) return cudaErrorInvalidValue;
   DeviceInfo di;
@@ -346,14 +358,16 @@ cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t
   const bool f16 = c.hidden_dtype == MOE_DTYPE_F16;
   const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
+  const int EW = e_mod > 0 ? e_mod : c.E;   // experts whose weights are given
   CUtensorMap maps[4];
   if (!make_map(&maps[0], xp, rows, (uint64_t)c.d, false) ||
-      !make_map(&maps[1], w1, (uint64_t)c.E * F1, (uint64_t)c.d, false) ||
+      !make_map(&maps[1], w1, (uint64_t)EW * F1, (uint64_t)c.d, false) ||
       !make_map(&maps[2], h, rows, (uint64_t)c.F, f16) ||
-      !make_map(&maps[3], w2, (uint64_t)c.E * c.d, (uint64_t)c.F, f16))
+      !make_map(&maps[3], w2, (uint64_t)EW * c.d, (uint64_t)c.F, f16))
     return cudaErrorInvalidValue;
   MlpParams p{offsets, h, comb ? comb->out : yp, comb ? comb->src_tok : nullptr, comb ? comb->row_w : nullptr,
-              c.E, c.d, c.F, F1, comb ? comb->T : 0, (int)rows, counters, counters + 1, status};
+              c.E, c.d, c.F, F1, comb ? comb->T : 0, (int)rows, counters, counters + 1, status,
+              g_wait_ns.load(), g_dep_extra.load(), EW};
   const bool cb = comb != nullptr;
   const long long mt_max = (long long)(rows / BM) + c.E;
   const long long nt = (c.act == MOE_ACT_SWIGLU ? (c.F + BN / 2 - 1) / (BN / 2) : (c.F + BN - 1) / BN) +

@@ -21,7 +21,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads)
 simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, float* __restrict__ C,
                   const int32_t* __restrict__ offsets, int E, int K, int Nout, int NB, int F, int rows_alloc,
-                  uint32_t* __restrict__ status) {
+                  int EW, uint32_t* __restrict__ status) {
   __shared__ int tstart[kMaxExperts + 1];
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Bs[kBK][kBN + 4];
@@ -38,6 +38,7 @@ simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, floa
 
   for (int L = blockIdx.x; L < total; L += gridDim.x) {
     const int e = tile_expert(tstart, E, L);
+    const int we = e % EW;   // weight block of segment e
     const int seg0 = offsets[e], M = offsets[e + 1] - seg0;
     const int mt = (M + kBM - 1) / kBM;
     const int local = L - tstart[e];
@@ -59,8 +60,8 @@ simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, floa
       for (int i = tid; i < kBN * kBK; i += kThreads) {
         const int n = i / kBK, kk = i % kBK;
         const bool ok = (n0 + n < Nout) && (k0 + kk < K);
-        Bs[kk][n] = ok ? B[((size_t)e * NB + n0 + n) * K + k0 + kk] : 0.f;
-        if (MODE == kSwiglu) Bu[kk][n] = ok ? B[((size_t)e * NB + F + n0 + n) * K + k0 + kk] : 0.f;
+        Bs[kk][n] = ok ? B[((size_t)we * NB + n0 + n) * K + k0 + kk] : 0.f;
+        if (MODE == kSwiglu) Bu[kk][n] = ok ? B[((size_t)we * NB + F + n0 + n) * K + k0 + kk] : 0.f;
       }
       __syncthreads();
 #pragma unroll
@@ -99,9 +100,22 @@ simt_grouped_gemm(const float* __restrict__ A, const float* __restrict__ B, floa
 
 }  // namespace
 
+cudaError_t launch_grouped_plain_simt(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                      const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s) {
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const long long tiles = ((long long)rows_alloc / kBM + c.E) * ((Nout + kBN - 1) / kBN);
+  simt_grouped_gemm<kPlain><<<(int)std::min<long long>(tiles, 8LL * di.sms), kThreads, 0, s>>>(
+      static_cast<const float*>(A), static_cast<const float*>(B), out, offsets, c.E, K, Nout, Nout, 0, rows_alloc,
+      c.E, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
                                    const void* w1, const void* w2, void* h, void* yp, uint32_t* status,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, int e_mod) {
+  const int EW = e_mod > 0 ? e_mod : c.E;
   if (c.T == 0) return cudaSuccess;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
@@ -117,15 +131,15 @@ cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const in
   if (c.act == MOE_ACT_SWIGLU)
     simt_grouped_gemm<kSwiglu><<<grid_for(c.F), kThreads, 0, s>>>(X, static_cast<const float*>(w1), H,
                                                                    offsets, c.E, c.d, c.F, 2 * c.F, c.F, (int)A,
-                                                                   status);
+                                                                   EW, status);
   else
     simt_grouped_gemm<kRelu><<<grid_for(c.F), kThreads, 0, s>>>(X, static_cast<const float*>(w1), H,
-                                                                 offsets, c.E, c.d, c.F, c.F, 0, (int)A, status);
+                                                                 offsets, c.E, c.d, c.F, c.F, 0, (int)A, EW, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   simt_grouped_gemm<kPlain><<<grid_for(c.d), kThreads, 0, s>>>(H, static_cast<const float*>(w2),
                                                                 static_cast<float*>(yp), offsets, c.E,
-                                                                c.F, c.d, c.d, 0, (int)A, status);
+                                                                c.F, c.d, c.d, 0, (int)A, EW, status);
   return cudaGetLastError();
 }
 

@@ -119,7 +119,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       bool ok = true;
       for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
         const TileCoord c = decode_tile<MODE, BM>(tail->tstart, tail->seg, p.E, L);
-        const int b0 = c.e * p.b_rows + c.n0;
+        const int b0 = weight_block(p, c.e) * p.b_rows + c.n0;
         const int b1 = (MODE == kSwiglu) ? b0 + p.up_off : b0 + BN / 2;
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % STAGES;
@@ -224,7 +224,8 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const Param
 template <bool F16>
 cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                           const void* w2, void* h, void* yp, uint32_t* status, int sms, cudaStream_t s,
-                          const CombineOut* comb) {
+                          const CombineOut* comb, int e_mod) {
+  const int EW = e_mod > 0 ? e_mod : c.E;   // experts whose weights are given
   const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
   const long long mt_max = (long long)(rows / BM) + c.E;
@@ -232,9 +233,10 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
   cudaError_t err;
 
   // layer 1: h = act(xp W1[e]^T)
-  if (!make_map(&ma, xp, rows, (uint64_t)c.d, false) || !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false))
+  if (!make_map(&ma, xp, rows, (uint64_t)c.d, false) || !make_map(&mb, w1, (uint64_t)EW * F1, (uint64_t)c.d, false))
     return cudaErrorInvalidValue;
   Params p1{offsets, h, c.E, c.d, c.F, F1, c.F, (int)rows, status};
+  p1.e_mod = e_mod;
   if (c.act == MOE_ACT_SWIGLU) {
     const long long nt = (c.F + BN / 2 - 1) / (BN / 2);
     err = launch_one<kSwiglu, F16>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, sms), s);
@@ -246,9 +248,10 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
 
   // layer 2: yp = h W2[e]^T, kept in fp32 so that the combine adds unrounded
   // expert outputs
-  if (!make_map(&ma, h, rows, (uint64_t)c.F, F16) || !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F, F16))
+  if (!make_map(&ma, h, rows, (uint64_t)c.F, F16) || !make_map(&mb, w2, (uint64_t)EW * c.d, (uint64_t)c.F, F16))
     return cudaErrorInvalidValue;
   Params p2{offsets, yp, c.E, c.F, c.d, c.d, 0, (int)rows, status};
+  p2.e_mod = e_mod;
   const long long nt2 = (c.d + BN - 1) / BN;
   const int g2 = (int)std::min<long long>(mt_max * nt2, sms);
   if (comb != nullptr) {   // step 5 fused: gate-weighted sums into the token rows of out
@@ -263,16 +266,30 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
 
 }  // namespace
 
+cudaError_t launch_grouped_plain_tc(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                    const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s) {
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, (uint64_t)rows_alloc, (uint64_t)K, false) ||
+      !make_map(&mb, B, (uint64_t)c.E * Nout, (uint64_t)K, false))
+    return cudaErrorInvalidValue;
+  Params p{offsets, out, c.E, K, Nout, Nout, 0, rows_alloc, status};
+  const long long tiles = ((long long)rows_alloc / BM + c.E) * ((Nout + BN - 1) / BN);
+  return launch_one<kPlain, false>(ma, mb, p, (int)std::min<long long>(tiles, di.sms), s);
+}
+
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
-                                 uint32_t* status, cudaStream_t s, const CombineOut* comb) {
+                                 uint32_t* status, cudaStream_t s, const CombineOut* comb, int e_mod) {
   if (c.T == 0) return cudaSuccess;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
   if (c.hidden_dtype == MOE_DTYPE_F16)
-    return launch_layers<true>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb);
-  return launch_layers<false>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb);
+    return launch_layers<true>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb, e_mod);
+  return launch_layers<false>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb, e_mod);
 }
 
 }  // namespace moe

@@ -125,7 +125,8 @@ tc_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_const
       for (int L = pair; L < total && ok; L += npairs) {
         const TileCoord c = decode_tile<MODE, PM>(tail->tstart, tail->seg, p.E, L);
         const int arow = c.row0 + HM * (int)rank;
-        const int brow = c.e * p.b_rows + c.n0 + (rank == 0 ? 0 : (MODE == kSwiglu ? p.up_off : HN));
+        const int brow =
+            weight_block(p, c.e) * p.b_rows + c.n0 + (rank == 0 ? 0 : (MODE == kSwiglu ? p.up_off : HN));
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -227,7 +228,8 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const Param
 template <bool F16>
 cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                           const void* w2, void* h, void* yp, uint32_t* status, int sms, cudaStream_t s,
-                          const CombineOut* comb) {
+                          const CombineOut* comb, int e_mod) {
+  const int EW = e_mod > 0 ? e_mod : c.E;   // experts whose weights are given
   const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
   const long long mt_max = (long long)(rows / PM) + c.E;
@@ -236,9 +238,10 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
   cudaError_t err;
 
   // layer 1: h = act(xp W1[e]^T)
-  if (!make_map(&ma, xp, rows, (uint64_t)c.d, false) || !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false))
+  if (!make_map(&ma, xp, rows, (uint64_t)c.d, false) || !make_map(&mb, w1, (uint64_t)EW * F1, (uint64_t)c.d, false))
     return cudaErrorInvalidValue;
   Params p1{offsets, h, c.E, c.d, c.F, F1, c.F, (int)rows, status};
+  p1.e_mod = e_mod;
   if (c.act == MOE_ACT_SWIGLU) {
     const long long nt = (c.F + BN / 2 - 1) / (BN / 2);
     err = launch_one<kSwiglu, F16>(ma, mb, p1, (int)std::min<long long>(mt_max * nt, max_pairs), s);
@@ -249,9 +252,10 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
   if (err != cudaSuccess) return err;
 
   // layer 2: yp = h W2[e]^T in fp32
-  if (!make_map(&ma, h, rows, (uint64_t)c.F, F16) || !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F, F16))
+  if (!make_map(&ma, h, rows, (uint64_t)c.F, F16) || !make_map(&mb, w2, (uint64_t)EW * c.d, (uint64_t)c.F, F16))
     return cudaErrorInvalidValue;
   Params p2{offsets, yp, c.E, c.F, c.d, c.d, 0, (int)rows, status};
+  p2.e_mod = e_mod;
   const long long nt2 = (c.d + BN - 1) / BN;
   const int g2 = (int)std::min<long long>(mt_max * nt2, max_pairs);
   if (comb != nullptr) {   // step 5 fused: gate-weighted sums into the token rows of out
@@ -268,14 +272,14 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
 
 cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
                                       const void* w1, const void* w2, void* h, void* yp,
-                                      uint32_t* status, cudaStream_t s, const CombineOut* comb) {
+                                      uint32_t* status, cudaStream_t s, const CombineOut* comb, int e_mod) {
   if (c.T == 0) return cudaSuccess;
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
   if (c.hidden_dtype == MOE_DTYPE_F16)
-    return launch_layers<true>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb);
-  return launch_layers<false>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb);
+    return launch_layers<true>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb, e_mod);
+  return launch_layers<false>(c, xp, offsets, w1, w2, h, yp, status, di.sms, s, comb, e_mod);
 }
 
 }  // namespace moe

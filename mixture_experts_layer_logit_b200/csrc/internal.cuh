@@ -23,6 +23,7 @@ struct Scratch {
   size_t choff;     // int32 [E][nchunks]   exclusive prefix over chunks
   size_t psum;      // float [nchunks][E]   per-chunk sums of softmax probabilities
   size_t ntie;      // int32 [nchunks]      near-tie tokens per chunk
+  size_t zsum;      // float [nchunks]      per-chunk sums of squared log-partitions (router z-loss)
   size_t status;    // uint32               device error bits of a standalone moe_route
   size_t mlp;       // int32 [expert_mlp_counters] tile queue of the one-launch expert kernel (bf16)
   size_t kslice;    // the route's K-slice arrival counters and partial logits (may be empty); last
@@ -38,12 +39,12 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Every launcher enqueues on `s` and returns cudaGetLastError().
 
 // Route: logits, normalisation, softmax, top-k; per-chunk histogram, probability
-// sums and near-tie counts into scratch.  TX = float or __nv_bfloat16.
+// sums, near-tie counts and z-loss sums into scratch.  TX = float or __nv_bfloat16.
 // kscratch: route_tc_scratch_bytes(c) bytes (or NULL: no K-slice split).
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
-                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, void* kscratch,
-                         cudaStream_t s);
+                         int32_t* hist, float* psum, int32_t* ntie, float* zsum, uint32_t* status,
+                         void* kscratch, cudaStream_t s);
 // The same on tcgen05 tensor cores (bf16, k <= 8).
 bool route_tc_supported(const moe_config& c);
 // Scratch bytes of the tensor-core route's model-width split (0 when it never
@@ -51,31 +52,37 @@ bool route_tc_supported(const moe_config& c);
 size_t route_tc_scratch_bytes(const moe_config& c);
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, uint32_t* status, void* kscratch, cudaStream_t s);
+                            int32_t* ntie, float* zsum, uint32_t* status, void* kscratch, cudaStream_t s);
 // prob_mean[e] = sum over chunks of psum / T (fixed order).
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
+// *z_loss = sum over chunks of zsum / T (fixed order).
+cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s);
+// *coef = beta * *coef + (1 - beta) * xi * stats->drop_rate (one thread).
+cudaError_t launch_aux_coef_update(const moe_stats* stats, float* coef, float beta, float xi, cudaStream_t s);
 // Histogram of topk_idx per chunk (+ near ties from gap when given).
 cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const float* gap,
                         int32_t* hist, int32_t* ntie, uint32_t* status, cudaStream_t s);
 // Step 3 after the histograms: counts, kept, offsets, statistics, stable
 // ranks, the capacity test, row_of/src_tok and the gather xp[row] = x[t].
 // Either prob_mean (standalone) or psum (fused forward) or neither supplies
-// P_e for the aux loss; choff is scratch for the chunk offsets when the scan
+// P_e for the aux loss; zsum (fused forward) or NULL (z_loss = NaN) the z-loss; choff is scratch for the chunk offsets when the scan
 // runs as its own kernel.  With row_w and out (fused combine, k <= 8 path):
 // row_w[row] = topk_w of each kept assignment and out is zeroed.
 cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
-                           const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
-                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
-                           const float* topk_w = nullptr, float* row_w = nullptr, float* out = nullptr,
-                           int* zero = nullptr, int nzero = 0);
+                           const int32_t* ntie, const float* zsum, int32_t* counts, int32_t* kept,
+                           int32_t* offsets, int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                           cudaStream_t s, const float* topk_w = nullptr, float* row_w = nullptr,
+                           float* out = nullptr, int* zero = nullptr, int nzero = 0);
 // True when the permutation runs scatter_kernel, whose prologue can zero the
 // `zero` ints of launch_permute (T > 0 and k <= 8); otherwise they are ignored.
 inline bool scatter_zeroes(const moe_config& c) { return c.T > 0 && c.k <= 8; }
 // Expert FFN on CUDA cores (fp32 path).
+// e_mod > 0: c.E counts row segments, and segment e uses the weights of
+// expert e % e_mod (of e_mod given); 0: segment e is expert e.
 cudaError_t launch_expert_ffn_simt(const moe_config& c, const void* xp, const int32_t* offsets,
                                    const void* w1, const void* w2, void* h, void* yp, uint32_t* status,
-                                   cudaStream_t s);
+                                   cudaStream_t s, int e_mod = 0);
 // Fused step 5 for the bf16 path with k <= 2: layer 2 adds row_w[row] * y of
 // every permuted row into out[src_tok[row]] (out zeroed beforehand) instead
 // of writing yp.
@@ -88,7 +95,8 @@ struct CombineOut {
 // Expert FFN on tcgen05 tensor cores (bf16 path).
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,
                                  const void* w1, const void* w2, void* h, void* yp,
-                                 uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
+                                 uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr,
+                                 int e_mod = 0);
 // Both expert layers in one launch on the bf16 path, from one dynamic tile
 // queue: with comb (k <= 2) the second layer adds into comb->out (the fused
 // step 5), else it writes fp32 yp.  `counters` holds expert_mlp_counters(c)
@@ -96,14 +104,75 @@ cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int3
 size_t expert_mlp_counters(const moe_config& c);
 cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
                               const void* w2, void* h, const CombineOut* comb, float* yp, int* counters,
-                              uint32_t* status, cudaStream_t s);
+                              uint32_t* status, cudaStream_t s, int e_mod = 0);
+// Test hooks of the one-launch expert kernel (see moe_testing_set_expert_wait):
+// the limit of its bounded waits (0 = the default 2 s) and an amount added to
+// the layer-2 dependency target (0 = none; > 0 makes that wait unreachable).
+void set_expert_mlp_test_hooks(unsigned long long wait_ns, int dep_extra);
 // The same with 2-SM pair tiles (tcgen05.mma.cta_group::2, 256 x 256).
 cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
                                       const void* w1, const void* w2, void* h, void* yp,
-                                      uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr);
+                                      uint32_t* status, cudaStream_t s, const CombineOut* comb = nullptr,
+                                      int e_mod = 0);
+// ------------------------------------------------------------- backward
+// Buffers of the layer's backward: the forward's discrete choices (read from
+// its workspace) and the backward workspace.  Padded rows: every expert's
+// kept rows, its segment padded with zero rows to a multiple of
+// bwd_pad_rows(); rows_alloc bounds them.
+struct BwdState {
+  const int32_t* topk_idx;   // [T][k]   forward: selected experts
+  const float* topk_w;       // [T][k]   forward: gate weights
+  const int32_t* counts;     // [E]      forward: pre-drop counts
+  const int32_t* offsets;    // [E+1]    forward: permuted row offsets
+  const int32_t* row_of;     // [T][k]   forward: permuted row of a slot (-1 dropped)
+  const int32_t* src_tok;    // [A]      forward: token of a permuted row
+  int32_t* pad_offsets;      // [E+1]
+  int rows_alloc;
+  void* xp;                  // [rows][d]   x of each padded row (element type of the path)
+  void* dout_perm;           // [rows][d]   dout of each padded row (element type of the path)
+  float* wrow;               // [rows]      gate weight of each padded row
+  float* u;                  // [rows][F1]  first-layer pre-activation
+  void* du;                  // [rows][F1]  (element type of the path)
+  void* hw;                  // [rows][F]   w * h (element type of the path)
+  float* dwpart;             // [column tiles of F][rows]
+  float* dxp;                // [rows][d]
+  float* z;                  // [T][E] logits
+  float* dz;                 // [T][E]
+  float* dwg_part;           // [nsplit][E][d + 1]
+  int nsplit, tok_per_split;
+  uint32_t* status;
+};
+int bwd_pad_rows();
+int bwd_tc_col_tile();     // columns of a tensor-core backward tile (the dw partials per row)
+int bwd_simt_col_tile();
+// prep (padded offsets) and gather (x, dout, gate weight of every padded row)
+cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
+                             cudaStream_t s);
+// the expert layers' gradients: dh with the activation backward, dxp, dW2, dW1
+cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
+                                      float* dw1, float* dw2, cudaStream_t s);
+cudaError_t launch_expert_backward_simt(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
+                                        float* dw1, float* dw2, cudaStream_t s);
+// out[rows][Nout] = A[rows][K] B_e[Nout][K]^T over the segments of offsets (E of them), fp32 out
+cudaError_t launch_grouped_plain_tc(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                    const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s);
+cudaError_t launch_grouped_plain_simt(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                      const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s);
+// the gate's gradient (logits recomputed), dx and dW_gate / db
+cudaError_t launch_bwd_gate(const moe_config& c, const void* x, const void* wg, const float* bg, const BwdState& st,
+                            float aux_coef, float z_coef, float* dx, float* dwg, float* dbg, float* dw_out,
+                            cudaStream_t s);
+
 // Combine.
 cudaError_t launch_combine(const moe_config& c, const void* yp, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s);
+
+// One step of the layer-wise adaptive aux-loss coefficient (Skywork-MoE
+// release, "2.自适应的Aux Loss"): an exponential moving average, smoothing
+// beta, of xi times the drop rate.  The same expression on host and device.
+__host__ __device__ inline float aux_coef_step(float coef, float drop_rate, float beta, float xi) {
+  return beta * coef + (1.f - beta) * (xi * drop_rate);
+}
 
 // Device properties cached per device (SM count, compute capability).
 struct DeviceInfo {

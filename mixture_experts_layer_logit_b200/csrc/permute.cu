@@ -89,6 +89,18 @@ __device__ __forceinline__ void expert_totals(const int32_t* __restrict__ hist, 
   *prefix = warp_sum(pre);
 }
 
+// Sum of the per-chunk sums of squared log-partitions (the router z-loss
+// numerator) in a fixed order: lanes stride over the chunks in double, then a
+// butterfly.  NaN when the route left none.
+__device__ __forceinline__ double chunk_zsum(const float* __restrict__ zsum, int nch, int lane) {
+  if (zsum == nullptr) return (double)NAN;
+  double s = 0.0;
+  for (int c = lane; c < nch; c += 32) s += (double)zsum[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
+  return s;
+}
+
 __device__ __forceinline__ int chunk_ties(const int32_t* __restrict__ ntie, int nch, int lane) {
   int s = 0;
   if (ntie != nullptr)
@@ -149,9 +161,10 @@ __device__ __forceinline__ void block_expert_totals(const int32_t* __restrict__ 
 // Switch aux loss E * sum_e (count_e / (T k)) * P_e in double (the sum of
 // count_e * P_e is divided by T k once: double divisions are slow).  Writes the
 // offsets to s_off when given and the global results when `out` is set.
-__device__ __forceinline__ void expert_offsets(const int* s_counts, const float* s_p, int s_ntie, int E, int T,
-                                               int k, int capacity, int* s_off, bool out, int32_t* counts,
-                                               int32_t* kept, int32_t* offsets, moe_stats* stats, int lane) {
+__device__ __forceinline__ void expert_offsets(const int* s_counts, const float* s_p, int s_ntie, double s_z,
+                                               int E, int T, int k, int capacity, int* s_off, bool out,
+                                               int32_t* counts, int32_t* kept, int32_t* offsets, moe_stats* stats,
+                                               int lane) {
   constexpr int PER = kMaxExperts / 32;
   int kv[PER];
   int local = 0, drop = 0;
@@ -205,6 +218,7 @@ __device__ __forceinline__ void expert_offsets(const int* s_counts, const float*
     stats->near_tie_count = s_ntie;
     stats->drop_rate = (T > 0) ? (float)((double)drop / A) : 0.f;
     stats->aux_loss = (T > 0) ? (float)((double)E * aux / A) : NAN;
+    stats->z_loss = (T > 0) ? (float)(s_z / (double)T) : NAN;
   }
 }
 
@@ -212,11 +226,12 @@ __device__ __forceinline__ void expert_offsets(const int* s_counts, const float*
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int nch, int T, int E, int k,
             int capacity, const float* __restrict__ prob_mean, const float* __restrict__ psum,
-            const int32_t* __restrict__ ntie, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
-            int32_t* __restrict__ offsets, moe_stats* __restrict__ stats) {
+            const int32_t* __restrict__ ntie, const float* __restrict__ zsum, int32_t* __restrict__ counts,
+            int32_t* __restrict__ kept, int32_t* __restrict__ offsets, moe_stats* __restrict__ stats) {
   __shared__ int s_counts[kMaxExperts];
   __shared__ float s_p[kMaxExperts];
   __shared__ int s_ntie;
+  __shared__ double s_z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = kScanThreads / 32;
   pdl_wait();
@@ -228,10 +243,15 @@ scan_kernel(const int32_t* __restrict__ hist, int32_t* __restrict__ choff, int n
   block_expert_totals<kScanThreads>(hist, psum, prob_mean, E, nch, 0, T, true, s_counts, nullptr, s_p);
   if (warp == nwarps - 1) {
     const int nt = chunk_ties(ntie, nch, lane);
-    if (lane == 0) s_ntie = nt;
+    const double z = chunk_zsum(zsum, nch, lane);
+    if (lane == 0) {
+      s_ntie = nt;
+      s_z = z;
+    }
   }
   __syncthreads();
-  if (warp == 0) expert_offsets(s_counts, s_p, s_ntie, E, T, k, capacity, nullptr, true, counts, kept, offsets, stats, lane);
+  if (warp == 0)
+    expert_offsets(s_counts, s_p, s_ntie, s_z, E, T, k, capacity, nullptr, true, counts, kept, offsets, stats, lane);
 }
 
 // ------------------------------------------------------------------ scatter
@@ -258,6 +278,7 @@ struct ScatterArgs {
   const float* prob_mean;     // FUSED, statistics block: P_e given, or
   const float* psum;          //   summed from the per-chunk probability sums
   const int32_t* ntie;
+  const float* zsum;          // per-chunk sums of squared log-partitions (z-loss), or NULL
   int32_t* counts;
   int32_t* kept;
   int32_t* offsets;           // read (separate scan) or written by the statistics block (FUSED)
@@ -299,6 +320,7 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
   __shared__ int s_pre[kMaxExperts], s_off[kMaxExperts], s_counts[kMaxExperts];
   __shared__ float s_p[kMaxExperts];
   __shared__ int s_ntie;
+  __shared__ double s_z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
   const int E = a.E, k = a.k, T = a.T;
@@ -312,11 +334,15 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
                                          s_p);
     if (warp == kWarps - 1) {
       const int nt = chunk_ties(a.ntie, a.nch, lane);
-      if (lane == 0) s_ntie = nt;
+      const double z = chunk_zsum(a.zsum, a.nch, lane);
+      if (lane == 0) {
+        s_ntie = nt;
+        s_z = z;
+      }
     }
     __syncthreads();
     if (warp == 0)
-      expert_offsets(s_counts, s_p, s_ntie, E, T, k, a.capacity, nullptr, true, a.counts, a.kept, a.offsets,
+      expert_offsets(s_counts, s_p, s_ntie, s_z, E, T, k, a.capacity, nullptr, true, a.counts, a.kept, a.offsets,
                      a.stats, lane);
     return;
   }
@@ -382,7 +408,7 @@ scatter_kernel(const TX* __restrict__ x, TX* __restrict__ xp, const ScatterArgs 
                                          nullptr);
     __syncthreads();
     if (warp == 0)
-      expert_offsets(s_counts, nullptr, 0, E, T, k, a.capacity, s_off, false, nullptr, nullptr, nullptr, nullptr,
+      expert_offsets(s_counts, nullptr, 0, 0.0, E, T, k, a.capacity, s_off, false, nullptr, nullptr, nullptr, nullptr,
                      lane);
   } else {
     for (int e = threadIdx.x; e < E; e += kScatterThreads) {
@@ -613,8 +639,8 @@ cudaError_t launch_permute_t(const moe_config& c, const void* x, void* xp, Scatt
   if (c.T > 0 && c.k <= 8 && (long long)c.E * a.nch <= kFusedHistMax)
     return launch_scatter_t<TX, true>(c, xx, pp, a, s);
   cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, a.hist, a.choff,
-                             a.nch, c.T, c.E, c.k, a.capacity, a.prob_mean, a.psum, a.ntie, a.counts, a.kept,
-                             a.offsets, a.stats);
+                             a.nch, c.T, c.E, c.k, a.capacity, a.prob_mean, a.psum, a.ntie, a.zsum, a.counts,
+                             a.kept, a.offsets, a.stats);
   if (e != cudaSuccess || c.T == 0) return e;
   if (c.k <= 8) return launch_scatter_t<TX, false>(c, xx, pp, a, s);
   return launch_generic_t<TX>(c, xx, pp, a, s);
@@ -631,9 +657,9 @@ cudaError_t launch_hist(const moe_config& c, const int32_t* topk_idx, const floa
 
 cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, const int32_t* topk_idx,
                            const int32_t* hist, int32_t* choff, const float* prob_mean, const float* psum,
-                           const int32_t* ntie, int32_t* counts, int32_t* kept, int32_t* offsets,
-                           int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats, cudaStream_t s,
-                           const float* topk_w, float* row_w, float* out, int* zero, int nzero) {
+                           const int32_t* ntie, const float* zsum, int32_t* counts, int32_t* kept,
+                           int32_t* offsets, int32_t* row_of, int32_t* src_tok, void* xp, moe_stats* stats,
+                           cudaStream_t s, const float* topk_w, float* row_w, float* out, int* zero, int nzero) {
   ScatterArgs a{};
   a.topk_idx = topk_idx;
   a.hist = hist;
@@ -641,6 +667,7 @@ cudaError_t launch_permute(const moe_config& c, int capacity, const void* x, con
   a.prob_mean = prob_mean;
   a.psum = psum;
   a.ntie = ntie;
+  a.zsum = zsum;
   a.counts = counts;
   a.kept = kept;
   a.offsets = offsets;

@@ -10,8 +10,10 @@
 // probabilities renormalised to sum to 1.
 //
 // The CTA also leaves, for the permutation step, its per-expert histogram, its
-// per-expert sum of softmax probabilities (for the Switch aux loss) and its
-// near-tie count in the scratch workspace.
+// per-expert sum of softmax probabilities (for the Switch aux loss), its
+// near-tie count and its sum of squared log-partitions (the router z-loss;
+// Megatron-Core best-practice page, "Megatron-Core MoE的关键特性") in the
+// scratch workspace.
 #include "internal.cuh"
 
 #include <math.h>
@@ -55,7 +57,8 @@ struct RouteSmem {
   static constexpr size_t pbuf = seli + sizeof(int) * 8 * EP;              // float [8][EP]
   static constexpr size_t hist = pbuf + sizeof(float) * 8 * EP;            // int   [EP]
   static constexpr size_t misc = hist + sizeof(int) * EP;                  // int   [4]
-  static constexpr size_t total = misc + 16;
+  static constexpr size_t zpart = misc + 16;                               // float [8] per-warp z-loss sums
+  static constexpr size_t total = zpart + sizeof(float) * (kThreads / 32);
 };
 
 template <int NJ, typename TX>
@@ -64,7 +67,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
              int T, int d, int E, int k, float lam,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
              int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-             int nch) {
+             float* __restrict__ zsum_out, int nch) {
   using L = RouteSmem<NJ>;
   constexpr int EP = L::EP;
   constexpr int V = VecLoad<TX>::N;
@@ -78,6 +81,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
   float (*pbuf)[EP] = reinterpret_cast<float (*)[EP]>(smem + L::pbuf);
   int* shist = reinterpret_cast<int*>(smem + L::hist);
   int* misc = reinterpret_cast<int*>(smem + L::misc);
+  float* zpart = reinterpret_cast<float*>(smem + L::zpart);
 
   const int tid = threadIdx.x;
   const int chunk = blockIdx.x;
@@ -152,6 +156,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
   float pacc[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) pacc[i] = 0.f;
+  float zacc = 0.f;   // this warp's rows: sum of squared log-partitions (router z-loss)
 
   for (int r = warp; r < rows; r += kThreads / 32) {
     const int t = t0 + r;
@@ -188,7 +193,10 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
       p[i] = ok[i] ? expf(v[i] - m) : 0.f;
       ps += p[i];
     }
-    const float inv = 1.f / warp_sum(ps);
+    const float psum_row = warp_sum(ps);
+    const float inv = 1.f / psum_row;
+    const float lse = m + logf(psum_row);
+    zacc += lse * lse;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       p[i] *= inv;
@@ -251,6 +259,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
     const int e = lane + 32 * i;
     if (e < EP) pbuf[warp][e] = pacc[i];
   }
+  if (lane == 0) zpart[warp] = zacc;
   __syncthreads();
   for (int e = tid; e < E; e += kThreads) {
     float s = 0.f;
@@ -259,7 +268,23 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
     psum_out[(size_t)chunk * E + e] = s;
     hist_out[(size_t)e * nch + chunk] = shist[e];
   }
-  if (tid == 0) ntie_out[chunk] = misc[0];
+  if (tid == 0) {
+    ntie_out[chunk] = misc[0];
+    float z = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) z += zpart[w];   // fixed warp order
+    zsum_out[chunk] = z;
+  }
+}
+
+// Router z-loss of a standalone route: sum of the per-chunk sums / T.
+__global__ void z_loss_kernel(const float* __restrict__ zsum, int nch, int T, float* __restrict__ z_loss) {
+  const int lane = threadIdx.x;
+  double s = 0.0;
+  for (int c = lane; c < nch; c += 32) s += (double)zsum[c];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) *z_loss = (float)(s / (double)T);
 }
 
 // One warp per expert: lanes stride over the chunks, then a fixed-order
@@ -278,40 +303,45 @@ __global__ void prob_mean_kernel(const float* __restrict__ psum, int nch, int E,
 template <int NJ, typename TX>
 cudaError_t launch_route_nj(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* idx, float* w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, cudaStream_t s) {
+                            int32_t* ntie, float* zsum, cudaStream_t s) {
   const size_t smem = RouteSmem<NJ>::total;
   auto kern = route_kernel<NJ, TX>;
   cudaError_t err = set_smem_once<route_kernel<NJ, TX>>(smem);
   if (err != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
   kern<<<nch, kThreads, smem, s>>>(static_cast<const TX*>(x), static_cast<const TX*>(wg), bg,
-                                   c.T, c.d, c.E, c.k, c.lambda, idx, w, gap, hist, psum, ntie, nch);
+                                   c.T, c.d, c.E, c.k, c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch);
   return cudaGetLastError();
 }
 
 template <typename TX>
 cudaError_t launch_route_t(const moe_config& c, const void* x, const void* wg, const float* bg,
                            int32_t* idx, float* w, float* gap, int32_t* hist, float* psum,
-                           int32_t* ntie, cudaStream_t s) {
-  if (c.E <= 16) return launch_route_nj<1, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, s);
-  if (c.E <= 32) return launch_route_nj<2, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, s);
-  if (c.E <= 64) return launch_route_nj<4, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, s);
-  if (c.E <= 128) return launch_route_nj<8, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, s);
-  return launch_route_nj<16, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, s);
+                           int32_t* ntie, float* zsum, cudaStream_t s) {
+  if (c.E <= 16) return launch_route_nj<1, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
+  if (c.E <= 32) return launch_route_nj<2, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
+  if (c.E <= 64) return launch_route_nj<4, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
+  if (c.E <= 128) return launch_route_nj<8, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
+  return launch_route_nj<16, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
-                         int32_t* hist, float* psum, int32_t* ntie, uint32_t* status, void* kscratch,
-                         cudaStream_t s) {
+                         int32_t* hist, float* psum, int32_t* ntie, float* zsum, uint32_t* status,
+                         void* kscratch, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   if (route_tc_supported(c))
-    return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, kscratch, s);
+    return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, kscratch, s);
   if (c.dtype == MOE_DTYPE_BF16)
-    return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, s);
-  return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, s);
+    return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);
+  return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);
+}
+
+cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s) {
+  z_loss_kernel<<<1, 32, 0, s>>>(zsum, num_chunks(c.T), c.T, z_loss);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s) {

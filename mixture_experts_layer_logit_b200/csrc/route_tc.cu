@@ -19,7 +19,9 @@
 // of the experts: partial sums, maxima and top-(k+1) lists are merged through
 // shared memory in quarter order.  Each CTA is one routing chunk of 128 tokens: it also writes the
 // chunk's per-expert histogram, per-expert sum of softmax probabilities
-// (summed in a fixed order) and near-tie count for the permutation step.
+// (summed in a fixed order), near-tie count and sum of squared
+// log-partitions (the router z-loss, Megatron-Core best-practice page,
+// "Megatron-Core MoE的关键特性") for the permutation step.
 //
 // A small batch with a wide model (decode: one chunk, d = 2048) would leave
 // the reduction to one SM, one ring of loads after another.  There the model
@@ -58,6 +60,7 @@ struct RTail {
   int hist[kMaxExperts];
   float bias[kMaxExperts];
   float part[kSplit][4][RM];       // per quarter: sum, squares, max, exp-sum of each row
+  float zrow[RM];                  // squared log-partition of each row (router z-loss)
 };
 
 // The top lists of quarters 1..3 of each row: (score, expert) pairs.  They
@@ -146,7 +149,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
                 int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-                int nch, uint32_t* __restrict__ status, int lists_off, float* __restrict__ kpart,
+                float* __restrict__ zsum_out, int nch, uint32_t* __restrict__ status, int lists_off,
+                float* __restrict__ kpart,
                 int* __restrict__ karrive, int nks) {
   constexpr int k = KB;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -363,6 +367,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     const float S = ((part[0][3][row] + part[1][3][row]) + part[2][3][row]) + part[3][3][row];
     const float invS = 1.f / S;
     if (qtr == 0) {
+      const float lse = m + logf(S);   // log sum_e exp(score): the router z-loss term of this row
+      tail->zrow[row] = valid ? lse * lse : 0.f;
       // the other quarters' lists, in quarter order: their experts all have
       // higher indices, so inserting them keeps lowest-index-wins order
 #pragma unroll
@@ -415,6 +421,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       hist_out[(size_t)e * nch + chunk] = tail->hist[e];
     }
     if (tid == 0) ntie_out[chunk] = tail->ntie;
+    if (warp == 0) {   // the chunk's z-loss sum, in a fixed order
+      float z = ((tail->zrow[lane] + tail->zrow[lane + 32]) + tail->zrow[lane + 64]) + tail->zrow[lane + 96];
+      z = warp_sum(z);
+      if (lane == 0) zsum_out[chunk] = z;
+    }
   }   // lead
   if (warp == 1) {
     tc_fence_after();
@@ -441,7 +452,7 @@ size_t karrive_bytes(int nch) { return ((size_t)nch * sizeof(int) + 255) & ~(siz
 template <int KB>
 cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
                       int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
-                      uint32_t* status, void* kscratch, cudaStream_t s) {
+                      float* zsum, uint32_t* status, void* kscratch, cudaStream_t s) {
   // the most any E <= kMaxExperts needs, so one attribute serves every launch
   static const size_t kMaxSmem = [] {
     size_t m = 0;
@@ -458,7 +469,7 @@ cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensor
   float* kpart = nks > 1 ? reinterpret_cast<float*>(static_cast<char*>(kscratch) + karrive_bytes(nch)) : nullptr;
   if (nks > 1 && (err = cudaMemsetAsync(karrive, 0, sizeof(int) * (size_t)nch, s)) != cudaSuccess) return err;
   return launch_pdl(route_tc_kernel<KB>, dim3(nch * nks), dim3(kThreads), smem_bytes(c.E, EP), s, mx, mw, bg, c.T,
-                    c.d, c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, nch, status,
+                    c.d, c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch, status,
                     (int)lists_offset(c.E, EP), kpart, karrive, nks);
 }
 
@@ -476,7 +487,7 @@ size_t route_tc_scratch_bytes(const moe_config& c) {
 
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, uint32_t* status, void* kscratch, cudaStream_t s) {
+                            int32_t* ntie, float* zsum, uint32_t* status, void* kscratch, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int EP = ((c.E + 15) / 16) * 16;
   CUtensorMap mx, mw;
@@ -484,7 +495,7 @@ cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, 
       !make_map(&mw, wg, (uint64_t)c.E, (uint64_t)c.d, false, (uint32_t)EP))
     return cudaErrorInvalidValue;
 #define MOE_ROUTE_K(K) \
-  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, status, kscratch, s)
+  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, kscratch, s)
   switch (c.k) {
     MOE_ROUTE_K(1); MOE_ROUTE_K(2); MOE_ROUTE_K(3); MOE_ROUTE_K(4);
     MOE_ROUTE_K(5); MOE_ROUTE_K(6); MOE_ROUTE_K(7); MOE_ROUTE_K(8);

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "internal.cuh"
+#include "bounded_wait.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -54,15 +55,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // ns or, when `abort_flag` is given, once another role has given up.
 static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
                                        unsigned long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = now_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (now_ns() - t0 > limit) return false;
-    }
-  }
+  return bounded_poll([&] { return mbar_try_wait(bar, parity); }, [] { return now_ns(); }, [] {}, abort_flag,
+                      limit, 32u);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
   asm volatile(
@@ -127,16 +121,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // once `abort_flag` is raised.
 static __device__ __noinline__ bool wait_flag_geq(const int* p, int target, const volatile int* abort_flag,
                                                   unsigned long long limit) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const unsigned long long t0 = now_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(p) >= target) return true;
-    if ((i & 15u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (now_ns() - t0 > limit) return false;
-    }
-  }
+  return bounded_poll([&] { return ld_acquire_gpu(p) >= target; }, [] { return now_ns(); },
+                      [] { __nanosleep(64); }, abort_flag, limit, 16u);
 }
 
 // ---- CTA pairs (a cluster of two CTAs sharing one tcgen05 MMA, cta_group::2)
@@ -233,6 +219,21 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   d |= (uint64_t)2 << 61;               // SWIZZLE_128B
   return d;
 }
+
+// Shared-memory matrix descriptor of an MN-major operand: 128-byte swizzle,
+// rows of 64 16-bit MN elements (128 bytes) along K, 8-row groups 1024 bytes
+// apart (SBO), successive 64-element MN blocks `lbo` bytes apart (LBO).  One
+// K = 16 step of the MMA advances the start address by 16 rows (2048 bytes).
+__device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;   // leading byte offset: the next 64-element MN block
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: the next 8 K rows
+  d |= (uint64_t)1 << 46;                        // version
+  d |= (uint64_t)2 << 61;                        // SWIZZLE_128B
+  return d;
+}
+// instruction descriptor bits that mark A (bit 15) or B (bit 16) as MN-major
+constexpr uint32_t kIdescAMN = 1u << 15, kIdescBMN = 1u << 16;
 
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

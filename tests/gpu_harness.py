@@ -90,13 +90,16 @@ class DeviceLayer:
     def scratch(self):
         return dev_bytes(moe.moe_scratch_size(self.cfg))
 
-    def route(self, want_prob_mean=True):
+    def route(self, want_prob_mean=True, want_z_loss=False):
         T, k, E = self.T, self.w.k, self.w.E
         idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
         wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
         gap = torch.empty((T,), dtype=torch.float32, device="cuda")
         pm = torch.empty((E,), dtype=torch.float32, device="cuda") if want_prob_mean else None
-        moe.moe_route(self.cfg, self.x, self.wg, self.bias, idx, wt, gap, pm, self.scratch())
+        zl = torch.empty((1,), dtype=torch.float32, device="cuda") if want_z_loss else None
+        moe.moe_route(self.cfg, self.x, self.wg, self.bias, idx, wt, gap, pm, self.scratch(), z_loss=zl)
+        if want_z_loss:
+            return idx, wt, gap, pm, zl
         return idx, wt, gap, pm
 
     def permute(self, idx, gap=None, prob_mean=None):

@@ -39,6 +39,10 @@ def run_and_check(L: DeviceLayer, sample: int = 0, seed: int = 0):
     if L.T > 0:
         assert abs(st["aux_loss"] - d.aux) <= 1e-4 * max(1.0, abs(d.aux))
         assert abs(st["drop_rate"] - d.drop_rate) <= 1e-6
+        # router z-loss over every token (it does not depend on the selection)
+        assert abs(st["z_loss"] - r0.z_loss) <= 1e-4 * abs(r0.z_loss), (st["z_loss"], r0.z_loss)
+    else:
+        assert np.isnan(st["z_loss"]) and np.isnan(st["aux_loss"])
     out = res["out"]
     if sample and sample < L.T:
         toks = np.sort(np.random.default_rng(seed).choice(L.T, size=sample, replace=False))
@@ -88,6 +92,7 @@ def test_layer_empty_tokens():
     assert res["stats"]["rows_kept"] == 0 and res["stats"]["drop_count"] == 0
     assert np.all(res["offsets"] == 0) and np.all(res["counts"] == 0)
     assert res["stats"]["drop_rate"] == 0.0 and np.isnan(res["stats"]["aux_loss"])
+    assert np.isnan(res["stats"]["z_loss"])
 
 
 @pytest.mark.parametrize("name", ["fastmoe_txl", "m_relu_cap", "m_multi_tile"])

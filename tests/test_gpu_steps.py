@@ -59,7 +59,7 @@ def oracle_inputs(L: DeviceLayer):
 
 def test_route(layer):
     L = layer
-    idx, wt, gap, pm = L.route()
+    idx, wt, gap, pm, zl = L.route(want_z_loss=True)
     torch.cuda.synchronize()
     x, wg, b, _, _ = oracle_inputs(L)
     r = om.route(x, wg, b, lcfg_of(L.w, L.T))
@@ -77,6 +77,8 @@ def test_route(layer):
     assert np.array_equal(np.isfinite(dg), fin)
     assert np.max(np.abs(dg[fin] - r.gap[fin]), initial=0.0) < 1e-4
     assert np.allclose(pm.cpu().numpy(), r.prob_mean, rtol=1e-5, atol=1e-7)
+    # router z-loss: mean over tokens of the squared log-partition of the scores
+    assert abs(float(zl.item()) - r.z_loss) <= 1e-4 * abs(r.z_loss), (float(zl.item()), r.z_loss)
 
 
 def test_permute_exact(layer):
@@ -329,3 +331,25 @@ def test_expert_ffn_short_layer_any_segment(offsets):
     xp64 = xp.float().cpu().numpy().astype(np.float64)
     _, yp_ref = om.expert_segments(xp64[:n], np.array(offsets), w1, w2, cfg)
     check_out(to_np64(yp[:n]), yp_ref, w.dtype)
+
+
+def test_adaptive_aux_coef_on_the_device_follows_the_oracle():
+    """moe_aux_coef_update, chained on the stream over scripted drop rates
+    written into a device moe_stats, against the oracle's coefficient step."""
+    import ctypes
+    from oracle import moe_oracle as om
+    beta, xi = 0.8, 0.25
+    rates = [0.4, 0.4, 0.3, 0.1, 0.0, 0.0, 0.05, 0.5]
+    coef = torch.full((1,), 0.02, dtype=torch.float32, device="cuda")
+    ref = 0.02
+    got = []
+    for d in rates:
+        st = moe.moe_stats()
+        st.drop_rate = d
+        stats = torch.frombuffer(bytearray(bytes(st)), dtype=torch.uint8).cuda()
+        moe.moe_aux_coef_update(stats, coef, beta, xi)
+        ref = om.adaptive_aux_coef(ref, d, beta, xi)
+        got.append((float(coef.item()), ref))
+    for g, r in got:
+        assert abs(g - r) <= 1e-6 * max(1.0, abs(r)), got
+    assert ctypes.sizeof(moe.moe_stats) == moe.STATS_BYTES

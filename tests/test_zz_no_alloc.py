@@ -99,9 +99,9 @@ def test_two_static_calls_match_moe_permute():
         torch.cuda.synchronize()
         for name in ("counts", "kept", "offsets", "row_of"):
             assert torch.equal(got[name], ref[name]), (w.name, name)
-        # every moe_stats field but the trailing `reserved` word, which no entry point writes
-        n = moe.STATS_BYTES - 4
-        assert torch.equal(got["stats"][:n], ref["stats"][:n]), w.name
+        # every moe_stats field, bit for bit (z_loss is NaN from both: a
+        # standalone permutation has no router scores)
+        assert torch.equal(got["stats"], ref["stats"]), w.name
         rows = int(ref["offsets"][E].item())
         assert rows > 0
         assert torch.equal(got["src_tok"][:rows], ref["src_tok"][:rows]), w.name
