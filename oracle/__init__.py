@@ -13,3 +13,4 @@ from .moe_backward import (  # noqa: F401
     Grads, loss, backward, expert_backward, normalise_backward, silu_grad, gate_weight_backward,
     aux_prob_grad, softmax_backward, z_loss_score_grad,
 )
+from . import moe_fp8  # noqa: F401  (MX FP8 expert weights: forward oracle)

@@ -58,6 +58,8 @@ class Grads:
     dw: np.ndarray      # [T, k]  gradient of the gate weights (0 for dropped slots)
     ds: np.ndarray      # [T, E]  gradient of the scores the softmax takes
     dz: np.ndarray      # [T, E]  gradient of the logits
+    abs_dw1: Optional[np.ndarray] = None   # [E, F1, d]  expert_abs_contractions, when asked for
+    abs_dw2: Optional[np.ndarray] = None   # [E, d, F]
 
 
 def loss(fw: om.Forward, dout: np.ndarray, aux_coef: float = 0.0, z_coef: float = 0.0) -> float:
@@ -100,6 +102,37 @@ def expert_backward(xe, w1e, w2e, dye, act: str, F: int):
     dw1e = du.T @ xe
     dxe = du @ w1e
     return dxe, dw1e, dw2e
+
+
+def expert_abs_contractions(xe, w1e, w2e, dye, act: str, F: int):
+    """The weight-gradient contractions of one expert taken over absolute
+    values: A2 = |dy|^T |h| and A1 = |du|_abs^T |x| with |du|_abs =
+    (|dy| |W2[e]|) * |act'(u)| (SwiGLU: |v silu'(g)| for the gate columns,
+    |silu(g)| for the up columns).  A rounding of relative size eps in every
+    product of a contraction moves its result by at most eps times the same
+    contraction over absolute values; these are the scales the bf16-path
+    weight gradients are compared against."""
+    xe = np.asarray(xe, np.float64)
+    w1e = np.asarray(w1e, np.float64)
+    w2e = np.asarray(w2e, np.float64)
+    u = xe @ w1e.T
+    if act == om.RELU:
+        h = np.maximum(u, 0.0)
+        dact = (u > 0.0).astype(np.float64)
+    else:
+        g, v = u[:, :F], u[:, F:2 * F]
+        with np.errstate(over="ignore"):
+            sg = 1.0 / (1.0 + np.exp(-g))
+        h = g * sg * v
+    ady = np.abs(dye)
+    A2 = ady.T @ np.abs(h)
+    adh = ady @ np.abs(w2e)
+    if act == om.RELU:
+        adu = adh * dact
+    else:
+        adu = np.concatenate([adh * np.abs(v * silu_grad(g)), adh * np.abs(g * sg)], axis=1)
+    A1 = adu.T @ np.abs(xe)
+    return A1, A2
 
 
 def normalise_backward(z: np.ndarray, ds: np.ndarray, lam: float) -> np.ndarray:
@@ -153,7 +186,7 @@ def z_loss_score_grad(s: np.ndarray, p: np.ndarray, z_coef: float) -> np.ndarray
 
 
 def backward(x, wg, bias, w1, w2, cfg: om.LayerConfig, dout, aux_coef: float = 0.0, z_coef: float = 0.0,
-             fw: Optional[om.Forward] = None) -> Grads:
+             fw: Optional[om.Forward] = None, want_abs: bool = False) -> Grads:
     """All gradients of L (module text) for one layer.  fw: the forward of the
     same inputs (computed here when not given; a forced routing in it is kept)."""
     x = np.asarray(x, np.float64)
@@ -170,6 +203,8 @@ def backward(x, wg, bias, w1, w2, cfg: om.LayerConfig, dout, aux_coef: float = 0
     dw = np.zeros((T, k))
     dw1 = np.zeros((E, F1, d))
     dw2 = np.zeros((E, d, F))
+    abs1 = np.zeros((E, F1, d)) if want_abs else None
+    abs2 = np.zeros((E, d, F)) if want_abs else None
     rows_t = dsp.src_tok
     for e in range(E):
         a, b = int(dsp.offsets[e]), int(dsp.offsets[e + 1])
@@ -184,6 +219,8 @@ def backward(x, wg, bias, w1, w2, cfg: om.LayerConfig, dout, aux_coef: float = 0
         dye = r.w[toks, slot][:, None] * dout[toks]
         dxe, dw1[e], dw2[e] = expert_backward(x[toks], w1[e], w2[e], dye, cfg.act, F)
         np.add.at(dx, toks, dxe)
+        if want_abs:
+            abs1[e], abs2[e] = expert_abs_contractions(x[toks], w1[e], w2[e], dye, cfg.act, F)
 
     # ---- gate weights, aux, softmax, z-loss
     dp = gate_weight_backward(r.p, r.idx, r.w, dw) + aux_prob_grad(dsp.counts, T, k, aux_coef)[None, :]
@@ -195,4 +232,4 @@ def backward(x, wg, bias, w1, w2, cfg: om.LayerConfig, dout, aux_coef: float = 0
     dwg = dz.T @ x
     dbias = dz.sum(axis=0)
     dx += dz @ wg
-    return Grads(dx=dx, dwg=dwg, dbias=dbias, dw1=dw1, dw2=dw2, dw=dw, ds=ds, dz=dz)
+    return Grads(dx=dx, dwg=dwg, dbias=dbias, dw1=dw1, dw2=dw2, dw=dw, ds=ds, dz=dz, abs_dw1=abs1, abs_dw2=abs2)

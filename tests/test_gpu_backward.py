@@ -1,0 +1,121 @@
+"""Parity of the layer's backward (moe_layer_backward, through the C ABI)
+against the float64 backward oracle, which is itself pinned by finite
+differences of the forward oracle.
+
+For each layer: the forward runs (moe_layer_forward), then the backward of
+L = <dout, out> + aux_coef * aux + z_coef * z_loss on the forward's workspace.
+Every gradient (dx, dW_gate, db, dW1, dW2 and the gate-weight gradient dw) is
+compared element by element: bf16 path max|err| <= 2e-2 * RMS(ref), fp32 path
+max|err| <= 1e-4 * max|ref|.  Near-tie tokens take the device's selection in
+the oracle (both selections are correct there)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as mw
+import mixture_experts_layer_logit_b200 as moe
+import oracle
+from oracle import moe_oracle as om
+from oracle import moe_backward as ob
+from tests.gpu_harness import DeviceLayer, to_np64
+
+pytestmark = pytest.mark.gpu
+
+W = mw.Workload
+LAYERS = [
+    W("b_relu_cap", T=777, d=256, E=12, F=320, k=3, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.1, seed=71),
+    W("b_swiglu_lam_bias", T=1000, d=192, E=8, F=208, k=2, act=mw.SWIGLU, dtype=mw.BF16, capacity_factor=0.9,
+      lam=1.0, zipf_bias=True, seed=72),
+    W("b_fine_top6", T=500, d=128, E=64, F=176, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True, seed=73),
+    W("b_wide", T=600, d=512, E=4, F=544, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=74),
+    W("b_E1", T=130, d=64, E=1, F=64, k=1, act=mw.RELU, dtype=mw.BF16, seed=75),
+    W("b_fp32_relu", T=300, d=64, E=5, F=96, k=2, act=mw.RELU, dtype=mw.F32, capacity_factor=1.0, seed=76),
+    W("b_fp32_swiglu", T=257, d=32, E=6, F=40, k=3, act=mw.SWIGLU, dtype=mw.F32, lam=0.5, seed=77),
+]
+AUX, ZC = 0.05, 0.01
+
+
+def _close(got, ref, dtype, name):
+    if ref.size == 0:
+        return 0.0
+    err = float(np.max(np.abs(got - ref)))
+    if dtype == mw.BF16:
+        rms = float(np.sqrt(np.mean(ref ** 2)))
+        assert err <= 2e-2 * rms, f"{name}: max|err| {err:.3e} > 2e-2 * RMS {rms:.3e}"
+        return err / rms
+    scale = float(np.max(np.abs(ref)))
+    assert err <= 1e-4 * scale, f"{name}: max|err| {err:.3e} > 1e-4 * max|ref| {scale:.3e}"
+    return err / scale
+
+
+def run_backward(L: DeviceLayer, seed: int):
+    w, cfg = L.w, L.cfg
+    res = L.forward()
+    T, d, E, F, k = L.T, w.d, w.E, w.F, w.k
+    F1 = F if w.act == mw.RELU else 2 * F
+    rng = np.random.default_rng(seed)
+    dout = rng.standard_normal((T, d)).astype(np.float32)
+    w2_bwd = mw.to_device(L.inp.w2)       # W2 in the element type of x (not the fp16 copy)
+    dev = "cuda"
+    dx = torch.empty((max(T, 1), d), dtype=torch.float32, device=dev)
+    dwg = torch.empty((E, d), dtype=torch.float32, device=dev)
+    dbg = torch.empty((E,), dtype=torch.float32, device=dev)
+    dw1 = torch.full((E, F1, d), float("nan"), dtype=torch.float32, device=dev)
+    dw2 = torch.full((E, d, F), float("nan"), dtype=torch.float32, device=dev)
+    dw = torch.empty((max(T, 1), k), dtype=torch.float32, device=dev)
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
+    ws = torch.empty(moe.moe_backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    ws.fill_(0xA5)   # stale contents must not leak into any gradient
+    moe.moe_layer_backward(cfg, L.x, L.wg, L.bias, L.w1, w2_bwd, torch.from_numpy(dout).cuda(), AUX, ZC, res["ws"],
+                           dx, dwg, dbg, dw1, dw2, dw, stats, ws)
+    torch.cuda.synchronize()
+    st = moe.read_stats(stats)
+    assert st["status"] == 0, st
+    # the oracle, with the device's selection on near-tie tokens
+    lc = oracle.LayerConfig.from_workload(w, T)
+    x, wg = mw.to_f64(L.inp.x), mw.to_f64(L.inp.wg)
+    w1, w2 = mw.F64Experts(L.inp.w1), mw.F64Experts(L.inp.w2)
+    r0 = om.route(x, wg, L.inp.bias, lc)
+    forced = r0.gap < 1e-4
+    fw = om.forward(x, wg, L.inp.bias, w1, w2, lc, forced if forced.any() else None,
+                    res["topk_idx"] if forced.any() else None)
+    g = ob.backward(x, wg, L.inp.bias, w1, w2, lc, dout.astype(np.float64), AUX, ZC, fw=fw)
+    out = {}
+    out["dw"] = _close(dw.cpu().numpy().astype(np.float64)[:T], g.dw, w.dtype, "dw")
+    out["dW2"] = _close(to_np64(dw2), g.dw2, w.dtype, "dW2")
+    out["dW1"] = _close(to_np64(dw1), g.dw1, w.dtype, "dW1")
+    out["dx"] = _close(to_np64(dx[:T]), g.dx, w.dtype, "dx")
+    out["dWg"] = _close(to_np64(dwg), g.dwg, w.dtype, "dWg")
+    if L.inp.bias is not None:
+        out["db"] = _close(to_np64(dbg), g.dbias, w.dtype, "db")
+    return out
+
+
+@pytest.mark.parametrize("w", LAYERS, ids=[w.name for w in LAYERS])
+def test_backward_matches_oracle(w):
+    rel = run_backward(DeviceLayer(w), w.seed + 1000)
+    print(w.name, {k: f"{v:.2e}" for k, v in rel.items()})
+
+
+def test_backward_bf16_hidden_config():
+    """A bf16 hidden activation in the forward changes nothing in the backward
+    (it recomputes u in fp32)."""
+    w = LAYERS[1]
+    run_backward(DeviceLayer(w, hidden="bf16"), 5)
+
+
+def test_backward_no_tokens():
+    w = W("b_empty", T=0, d=64, E=4, F=64, k=2, act=mw.RELU, dtype=mw.BF16)
+    L = DeviceLayer(w)
+    res = L.forward()
+    cfg = L.cfg
+    dwg = torch.full((4, 64), 7.0, device="cuda")
+    dw1 = torch.full((4, 64, 64), 7.0, device="cuda")
+    dw2 = torch.full((4, 64, 64), 7.0, device="cuda")
+    dbg = torch.full((4,), 7.0, device="cuda")
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(moe.moe_backward_workspace_size(cfg), 256), dtype=torch.uint8, device="cuda")
+    moe.moe_layer_backward(cfg, None, L.wg, None, L.w1, mw.to_device(L.inp.w2), None, 0.0, 0.0, res["ws"], None,
+                           dwg, dbg, dw1, dw2, None, stats, ws)
+    torch.cuda.synchronize()
+    assert torch.all(dwg == 0) and torch.all(dw1 == 0) and torch.all(dw2 == 0) and torch.all(dbg == 0)

@@ -110,6 +110,20 @@ def test_closed_forms():
     assert check_closed_forms() == []
 
 
+def test_abs_contractions_bound_the_weight_gradients():
+    """expert_abs_contractions: on positive inputs (and a ReLU that passes them
+    all) they equal the weight gradients; in general they bound them."""
+    rng = np.random.default_rng(3)
+    x, w1, w2, dy = (np.abs(rng.standard_normal(s)) for s in [(6, 4), (5, 4), (4, 5), (6, 4)])
+    A1, A2 = ob.expert_abs_contractions(x, w1, w2, dy, om.RELU, 5)
+    _, dw1, dw2 = ob.expert_backward(x, w1, w2, dy, om.RELU, 5)
+    assert np.allclose(A1, dw1, rtol=1e-14) and np.allclose(A2, dw2, rtol=1e-14)
+    x, w1, w2, dy = (rng.standard_normal(s) for s in [(6, 4), (10, 4), (4, 5), (6, 4)])
+    A1, A2 = ob.expert_abs_contractions(x, w1, w2, dy, om.SWIGLU, 5)
+    _, dw1, dw2 = ob.expert_backward(x, w1, w2, dy, om.SWIGLU, 5)
+    assert np.all(np.abs(dw1) <= A1 * (1 + 1e-12)) and np.all(np.abs(dw2) <= A2 * (1 + 1e-12))
+
+
 def test_dropped_slots_carry_no_gradient():
     cfg, x, wg, b, w1, w2, dout = _layer(7, 20, 4, 2, 3, 1, om.RELU, 0.3, 0.0, False)
     fw = om.forward(x, wg, b, w1, w2, cfg)
