@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the layer's backward")
+    ap.add_argument("--no-fp8", action="store_true", help="skip timing the FP8-weight decode layer")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget for cpu_baseline")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
@@ -319,7 +321,9 @@ class Layer:
         self.wg, self.bias = mw.to_device(self.inp.wg, dev), mw.to_device(self.inp.bias, dev)
         self.w1 = mw.to_device(self.inp.w1, dev)
         # weight preparation at load time (not part of a step): W2 in the hidden type
-        self.w2 = moe.prepare_w2(self.cfg, mw.to_device(self.inp.w2, dev))
+        # (the bf16 original is kept for the FP8 weight preparation)
+        self.w2_src = mw.to_device(self.inp.w2, dev)
+        self.w2 = moe.prepare_w2(self.cfg, self.w2_src)
         nbytes, self.lay = moe.moe_workspace_size(self.cfg)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         self.out = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
@@ -467,6 +471,81 @@ def breakdown_roofline(L: Layer, a, flush, pk, pk_src, dev):
     return breakdown, roofline
 
 
+def backward_measure(L: Layer, a, flush, pk, dev):
+    """The layer's backward (moe_layer_backward: all five expert GEMMs, the
+    gate's gradient, dx and dW_gate) after a forward of the same inputs,
+    timed with CUDA events, L2 flushed before each call."""
+    import torch
+    moe, w = L.moe, L.w
+    F1 = w.F if w.act == mw.RELU else 2 * w.F
+    dout = torch.randn((w.T, w.d), dtype=torch.float32, device=dev, generator=torch.Generator(dev).manual_seed(0))
+    dx = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
+    dwg = torch.empty((w.E, w.d), dtype=torch.float32, device=dev)
+    dbg = torch.empty((w.E,), dtype=torch.float32, device=dev)
+    dw1 = torch.empty((w.E, F1, w.d), dtype=torch.float32, device=dev)
+    dw2 = torch.empty((w.E, w.d, w.F), dtype=torch.float32, device=dev)
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device=dev)
+    bws = torch.empty(moe.moe_backward_workspace_size(L.cfg), dtype=torch.uint8, device=dev)
+    L.fwd()
+
+    def bwd():
+        moe.moe_layer_backward(L.cfg, L.x, L.wg, L.bias, L.w1, L.w2, dout, 0.01, 0.001, L.ws, dx, dwg, dbg,
+                               dw1, dw2, None, stats, bws)
+
+    timed(bwd, a.warmup, flush)
+    t = timed(bwd, a.steps, flush)
+    ms = sum(t) / len(t)
+    st = moe.read_stats(stats)
+    assert st["status"] == 0, f"device status {st['status']} in the backward"
+    kept = int(moe.read_stats(L.stats)["rows_kept"])
+    flops = 2.0 * kept * w.d * (3 * F1 + 2 * w.F)
+    tf = flops / (ms * 1e-3) / 1e12
+    res = {"ms_per_step": ms, "tokens_per_s": w.T / (ms * 1e-3), "expert_gemm_flops": flops, "tflops": tf,
+           "tensor_frac": tf / pk["bf16_tflops"], "tensor_frac_of_sustained": tf / pk["bf16_tflops_sustained"],
+           "what": "moe_layer_backward after a forward: u recomputed, dh with the activation backward, dxp, dW2, "
+                   "dW1 (tcgen05), gate gradient, dx, dW_gate; L2 flushed before each call"}
+    del dw1, dw2, bws
+    return res
+
+
+def mxfp8_measure(moe, name: str, a, flush, pk, dev):
+    """The layer with MX FP8 expert weights (moe_layer_forward_mxfp8) on one
+    workload, replayed from a CUDA graph with the L2 flushed between steps,
+    and its expert step (the padded quantised rows, both FP8 GEMMs) against
+    the HBM bytes of the touched experts' FP8 weights."""
+    import torch
+    w = mw.WORKLOADS[name]
+    L = Layer(moe, w, 0, dev, "f16")
+    w1q, w1s, w2q, w2s = moe.prepare_mxfp8(L.cfg, L.w1, L.w2_src)
+    ws = torch.empty(moe.moe_workspace_size_mxfp8(L.cfg), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        moe.moe_layer_forward_mxfp8(L.cfg, L.x, L.wg, L.bias, w1q, w1s, w2q, w2s, L.out, L.stats, ws)
+
+    fwd()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    timed(g.replay, a.warmup, flush)
+    t = timed(g.replay, a.steps, flush)
+    ms = sum(t) / len(t)
+    st = moe.read_stats(L.stats)
+    assert st["status"] == 0, f"device status {st['status']} on the FP8 layer"
+    n, lay = moe.moe_workspace_size(L.cfg)
+    offs = ws[lay.offsets:lay.offsets + 4 * (w.E + 1)].view(torch.int32).cpu().numpy()
+    touched = int(np.sum(np.diff(offs) > 0))
+    F1 = w.F1
+    wbytes = touched * (F1 * w.d + w.d * w.F) * (1 + 1 / 32)   # E4M3 elements + one scale byte per 32
+    res = {"value": w.T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "workload": name,
+           "weights": "MX FP8 (E4M3, UE8M0 scale per 32 along K), both expert layers",
+           "touched_expert_weight_bytes": wbytes,
+           "weight_stream_gbs_over_whole_forward": wbytes / (ms * 1e-3) / 1e9}
+    del g, L, ws, w1q, w1s, w2q, w2s
+    torch.cuda.empty_cache()
+    return res
+
+
 def e2e_measure(L: Layer, a, flush, graph_ok: bool, barrier, max_over_ranks, world: int, dev):
     """Every step copies its tokens from pinned host memory to the device, runs
     the layer through the C ABI and reads the output and statistics back.  Two
@@ -612,6 +691,9 @@ def main():
     e2e = None
     if not a.no_e2e:
         e2e = e2e_measure(L, a, flush, graph is not None, barrier, max_over_ranks, world, dev)
+    backward = None
+    if world == 1 and not a.no_backward and w.dtype == mw.BF16:
+        backward = backward_measure(L, a, flush, pk, dev)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(w, L.inp, a.cpu_seconds)
@@ -642,6 +724,9 @@ def main():
         del run_e, Le
         torch.cuda.empty_cache()
 
+    if world == 1 and not a.no_fp8:
+        extra["fine_decode_dropless_mxfp8"] = mxfp8_measure(moe, "fine_decode_dropless", a, flush, pk, dev)
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
                 "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -653,7 +738,7 @@ def main():
                 "stats": {"drop_rate": st["drop_rate"], "aux_loss": st["aux_loss"], "z_loss": st["z_loss"],
                           "rows_kept": st["rows_kept"],
                           "capacity": st["capacity"], "near_tie_count": st["near_tie_count"]},
-                "extra": extra}
+                "backward": backward, "extra": extra}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

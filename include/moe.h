@@ -287,9 +287,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
  * its coefficient and the z-loss are those of moe_stats and moe_aux_coef_update.
  * The forward's discrete choices (selected experts, capacity drops, counts)
  * carry no gradient and are read from its workspace `fws`.
- *   x, Wg, bg (or NULL), W1 as for the forward; W2[E, d, F] in the element
- *     type of x (bf16 on the bf16 path, not the fp16 copy an fp16 hidden
- *     activation uses; fp32 on the fp32 path).
+ *   x, Wg, bg (or NULL), W1, W2: as for the forward (W2 in hidden_dtype).
  *   dout[T, d] fp32: the gradient of L with respect to out.
  *   fws: the workspace of that forward (moe_workspace_size bytes), unchanged
  *     since.
@@ -299,15 +297,53 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
  *   ws: at least moe_backward_workspace_size(cfg) bytes (256-byte aligned).
  *   stats: device moe_stats; device-detected errors are OR-ed into status
  *     (clear it before the call for a clean record).
- * The expert GEMMs run on the tensor cores (bf16 operands, fp32 accumulation:
- * dout is rounded to bf16 for them) on the bf16 path and in fp32 FFMA on the
- * fp32 path.  Gradients are written, never accumulated into.
+ * The expert GEMMs run on the tensor cores on the bf16 path, with fp32
+ * accumulation and operands of the hidden type: with fp16 (the default),
+ * dout is scaled by a power of two s so that max|s dout| lies in [512, 1024),
+ * x, W1, s dout, s du and w h are rounded to fp16 (saturating at +-65504, which
+ * sets MOE_DEV_RANGE) and every result is scaled back by 1/s; with bf16 they
+ * are bf16.  The fp32 path runs in fp32 FFMA.  The gate's gradient, dx and
+ * dW_gate are fp32.  Gradients are written, never accumulated into.
  */
 size_t moe_backward_workspace_size(const moe_config* cfg);
 moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* Wg, const float* bg, const void* W1,
                               const void* W2, const float* dout, float aux_coef, float z_coef, const void* fws,
                               size_t fws_bytes, float* dx, float* dWg, float* dbg, float* dW1, float* dW2,
                               float* dw, moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The layer with FP8 expert weights.  The Skywork-MoE release serves its model
+ * with FP8 weights (inference section: 146 GB on an 8 x 4090 server); the
+ * pages fix no FP8 format.  This library takes the microscaled (MX) form the
+ * B200 tensor cores run natively (tcgen05.mma kind::mxf8f6f4): E4M3 elements
+ * and one power-of-two scale (UE8M0) per 32 consecutive elements along the
+ * reduction.  A block's scale 2^X is the least that brings every |v| / 2^X
+ * within 448, and elements round to the nearest E4M3 value, ties to even.
+ * Both expert layers run on it: the weights are quantised once by
+ * moe_prepare_mxfp8_weights, the layer-1 input rows and the hidden activation
+ * on every call.  Routing, permutation and combine are the bf16 layer's.
+ *   Shapes: the bf16 path with d and F multiples of 128 (else
+ *     MOE_ERR_UNSUPPORTED); cfg.hidden_dtype is not used.
+ *   moe_mxfp8_weight_bytes: bytes of the four prepared arrays (returned
+ *     through the pointers that are not NULL) and their sum; 0 for an
+ *     unsupported cfg.
+ *   moe_prepare_mxfp8_weights: W1[E, F1, d] and W2[E, d, F] bf16 (device) ->
+ *     W1q, W1s, W2q, W2s (device, 16-byte aligned, sizes from
+ *     moe_mxfp8_weight_bytes).  Their layout is the kernels' own (scales in
+ *     512-byte atoms of 128 rows x 4 blocks; a SwiGLU expert's W1 rows
+ *     interleaved gate/up by 64) and is read only by this library.
+ *   moe_layer_forward_mxfp8: as moe_layer_forward with the prepared weights;
+ *     ws: at least moe_workspace_size_mxfp8(cfg) bytes, whose first
+ *     moe_workspace_size(cfg) bytes have the moe_ws_layout of the bf16 forward
+ *     (yp holds the fp32 expert outputs; the fused combine is not used).
+ */
+size_t moe_mxfp8_weight_bytes(const moe_config* cfg, size_t* w1q, size_t* w1s, size_t* w2q, size_t* w2s);
+moe_status moe_prepare_mxfp8_weights(const moe_config* cfg, const void* W1, const void* W2, void* W1q, void* W1s,
+                                     void* W2q, void* W2s, moe_stream_t stream);
+size_t moe_workspace_size_mxfp8(const moe_config* cfg);
+moe_status moe_layer_forward_mxfp8(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                                   const void* W1q, const void* W1s, const void* W2q, const void* W2s, void* out,
+                                   moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Weight preparation (run once when the weights are loaded, not per forward):

@@ -22,7 +22,8 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_convert_bf16_to_f16", "moe_permute_static",
     "moe_expert_ffn_combine", "MOE_STATIC_SCRATCH_BYTES", "prepare_w2", "moe_aux_coef_update",
     "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_segments_scratch_size", "moe_expert_ffn_segments",
-    "moe_backward_workspace_size", "moe_layer_backward",
+    "moe_backward_workspace_size", "moe_layer_backward", "moe_mxfp8_weight_bytes", "moe_prepare_mxfp8_weights",
+    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8", "prepare_mxfp8",
     "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
     "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
@@ -39,7 +40,8 @@ EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size
                     "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine",
                     "moe_aux_coef_update", "moe_aux_coef_next", "moe_testing_set_expert_wait",
                     "moe_segments_scratch_size", "moe_expert_ffn_segments", "moe_backward_workspace_size",
-                    "moe_layer_backward"]
+                    "moe_layer_backward", "moe_mxfp8_weight_bytes", "moe_prepare_mxfp8_weights",
+                    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8"]
 MOE_STATIC_SCRATCH_BYTES = 2 << 20
 
 
@@ -104,13 +106,21 @@ def lib() -> ctypes.CDLL:
     L.moe_segments_scratch_size.argtypes = [cfgp, i32, i32]
     L.moe_segments_scratch_size.restype = ctypes.c_size_t
     L.moe_expert_ffn_segments.argtypes = [cfgp, i32, i32, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    sz = ctypes.POINTER(ctypes.c_size_t)
+    L.moe_mxfp8_weight_bytes.argtypes = [cfgp, sz, sz, sz, sz]
+    L.moe_mxfp8_weight_bytes.restype = ctypes.c_size_t
+    L.moe_prepare_mxfp8_weights.argtypes = [cfgp, P, P, P, P, P, P, P]
+    L.moe_workspace_size_mxfp8.argtypes = [cfgp]
+    L.moe_workspace_size_mxfp8.restype = ctypes.c_size_t
+    L.moe_layer_forward_mxfp8.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_backward_workspace_size.argtypes = [cfgp]
     L.moe_backward_workspace_size.restype = ctypes.c_size_t
     L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, f32, f32, P, ctypes.c_size_t, P, P, P, P, P, P, P, P,
                                      ctypes.c_size_t, P]
     for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
               "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine", "moe_aux_coef_update",
-              "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_expert_ffn_segments", "moe_layer_backward"]:
+              "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_expert_ffn_segments", "moe_layer_backward",
+              "moe_prepare_mxfp8_weights", "moe_layer_forward_mxfp8"]:
         getattr(L, n).restype = st
     _lib = L
     return L
@@ -252,6 +262,42 @@ def moe_testing_set_expert_wait(wait_ns: int, extra_dependency: int):
     """Test hook: limit of the one-launch expert kernel's waits (0 = default)
     and an amount added to its layer-2 dependency target (> 0: unreachable)."""
     _check("moe_testing_set_expert_wait", lib().moe_testing_set_expert_wait(wait_ns, extra_dependency))
+
+
+def moe_mxfp8_weight_bytes(cfg: moe_config):
+    """(total, (w1q, w1s, w2q, w2s)) bytes of the prepared FP8 weights (0 if unsupported)."""
+    v = [ctypes.c_size_t() for _ in range(4)]
+    n = lib().moe_mxfp8_weight_bytes(ctypes.byref(cfg), *[ctypes.byref(x) for x in v])
+    return n, tuple(x.value for x in v)
+
+
+def moe_prepare_mxfp8_weights(cfg, W1, W2, W1q, W1s, W2q, W2s, stream=None):
+    _check("moe_prepare_mxfp8_weights",
+           lib().moe_prepare_mxfp8_weights(ctypes.byref(cfg), _ptr(W1), _ptr(W2), _ptr(W1q), _ptr(W1s), _ptr(W2q),
+                                           _ptr(W2s), _stream(stream)))
+
+
+def prepare_mxfp8(cfg, W1, W2):
+    """Weight preparation for the FP8 layer: four new uint8 device tensors
+    (W1q, W1s, W2q, W2s) from bf16 W1, W2.  Run once at load time."""
+    import torch
+    n, sizes = moe_mxfp8_weight_bytes(cfg)
+    if n == 0:
+        raise MoeError("moe_mxfp8_weight_bytes", 2)
+    bufs = [torch.empty(max(sz, 16), dtype=torch.uint8, device=W1.device) for sz in sizes]
+    moe_prepare_mxfp8_weights(cfg, W1, W2, *bufs)
+    return tuple(bufs)
+
+
+def moe_workspace_size_mxfp8(cfg: moe_config) -> int:
+    return lib().moe_workspace_size_mxfp8(ctypes.byref(cfg))
+
+
+def moe_layer_forward_mxfp8(cfg, x, Wg, bg, W1q, W1s, W2q, W2s, out, stats, ws, stream=None):
+    _check("moe_layer_forward_mxfp8",
+           lib().moe_layer_forward_mxfp8(ctypes.byref(cfg), _ptr(x), _ptr(Wg), _ptr(bg), _ptr(W1q), _ptr(W1s),
+                                         _ptr(W2q), _ptr(W2s), _ptr(out), _ptr(stats), _ptr(ws), _nbytes(ws),
+                                         _stream(stream)))
 
 
 def moe_backward_workspace_size(cfg: moe_config) -> int:

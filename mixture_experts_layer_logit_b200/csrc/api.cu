@@ -220,8 +220,12 @@ moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* o
 struct BwdLayout {
   int rows;
   int nsplit, tok_per_split, col_tiles;
-  size_t pad_offsets, xp, dout_perm, wrow, u, du, hw, dwpart, dxp, z, dz, dwg_part, total;
+  size_t pad_offsets, xp, dout_perm, wrow, u, du, hw, dwpart, dxp, z, dz, dwg_part, amax, scale, w1h, total;
 };
+
+// The backward's GEMM operands are fp16 when the forward's hidden type is
+// fp16 (dout scaled into its range), else of the element type of x.
+bool bwd_f16(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.hidden_dtype == MOE_DTYPE_F16; }
 
 BwdLayout bwd_layout(const moe_config& c) {
   BwdLayout L{};
@@ -247,8 +251,42 @@ BwdLayout bwd_layout(const moe_config& c) {
   L.z = off;           off = align256(off + 4 * T * E);
   L.dz = off;          off = align256(off + 4 * T * E);
   L.dwg_part = off;    off = align256(off + 4 * (size_t)L.nsplit * E * (d + 1));
+  L.amax = off;        off = align256(off + 4);
+  L.scale = off;       off = align256(off + 8);
+  L.w1h = off;         off = align256(off + (bwd_f16(c) ? 2 * E * (size_t)F1 * d : 0));
   L.total = off;
   return L;
+}
+
+// The FP8 (MX) layer: the forward workspace, then its own regions.
+struct MxLayout {
+  moe_ws_layout base;
+  int rows_pad;
+  size_t pad, xq, xs, hq, hs, total;
+};
+
+MxLayout mx_layout(const moe_config& c) {
+  MxLayout L{};
+  L.base = layout_of(c);
+  const long long rows = (long long)c.T * c.k + (long long)(mx_pad_rows() - 1) * c.E;
+  L.rows_pad = (int)((rows + 127) / 128 * 128);
+  const size_t R = (size_t)L.rows_pad;
+  size_t off = L.base.total;
+  L.pad = off; off = align256(off + 4 * ((size_t)c.E + 1));
+  L.xq = off;  off = align256(off + R * (size_t)c.d);
+  L.xs = off;  off = align256(off + mx_scale_bytes(R, (size_t)c.d));
+  L.hq = off;  off = align256(off + R * (size_t)c.F);
+  L.hs = off;  off = align256(off + mx_scale_bytes(R, (size_t)c.F));
+  L.total = off;
+  return L;
+}
+
+moe_status check_mx_config(const moe_config* c) {
+  moe_status st = check_config(c);
+  if (st != MOE_OK) return st;
+  if (c->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (c->d % 128 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 }  // namespace
@@ -597,13 +635,22 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* 
   b.nsplit = BL.nsplit;
   b.tok_per_split = BL.tok_per_split;
   b.status = &stats->status;
+  b.f16 = bwd_f16(c);
+  b.amax = at<unsigned>(ws, BL.amax);
+  b.scale = at<float>(ws, BL.scale);
+  b.w1h = at<char>(ws, BL.w1h);
   // padded rows: x, dout and the gate weight of every kept assignment
   if (launch_bwd_front(c, x, dout, b, s) != cudaSuccess) return MOE_ERR_CUDA;
   // the first layer's pre-activation u = xp W1[e]^T, then the expert layers' gradients
   cudaError_t e;
   if (c.dtype == MOE_DTYPE_BF16) {
-    e = launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);
-    if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, W1, W2, dW1, dW2, s);
+    const void* w1 = W1;
+    if (b.f16) {   // fp16 operands: W1 converted once per call
+      if (launch_convert_bf16_f16(W1, b.w1h, (size_t)c.E * F1 * c.d, s) != cudaSuccess) return MOE_ERR_CUDA;
+      w1 = b.w1h;
+    }
+    e = launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u, b.status, b.f16, s);
+    if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, w1, W2, dW1, dW2, s);
   } else {
     e = launch_grouped_plain_simt(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);
     if (e == cudaSuccess) e = launch_expert_backward_simt(c, b, W1, W2, dW1, dW2, s);
@@ -611,6 +658,80 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* 
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // the gate: scores, logits, dx and dW_gate
   return cuda_status(launch_bwd_gate(c, x, Wg, bg, b, aux_coef, z_coef, dx, dWg, dbg, dw, s));
+}
+
+size_t moe_mxfp8_weight_bytes(const moe_config* cfg, size_t* w1q, size_t* w1s, size_t* w2q, size_t* w2s) {
+  if (check_mx_config(cfg) != MOE_OK) return 0;
+  const moe_config& c = *cfg;
+  const size_t F1 = c.act == MOE_ACT_SWIGLU ? 2 * (size_t)c.F : (size_t)c.F;
+  const size_t a = (size_t)c.E * F1 * c.d, b = mx_scale_bytes((size_t)c.E * F1, (size_t)c.d);
+  const size_t cq = (size_t)c.E * c.d * c.F, d = mx_scale_bytes((size_t)c.E * c.d, (size_t)c.F);
+  if (w1q) *w1q = a;
+  if (w1s) *w1s = b;
+  if (w2q) *w2q = cq;
+  if (w2s) *w2s = d;
+  return a + b + cq + d;
+}
+
+moe_status moe_prepare_mxfp8_weights(const moe_config* cfg, const void* W1, const void* W2, void* W1q, void* W1s,
+                                     void* W2q, void* W2s, moe_stream_t stream) {
+  moe_status st = check_mx_config(cfg);
+  if (st != MOE_OK) return st;
+  if (W1 == nullptr || W2 == nullptr || W1q == nullptr || W1s == nullptr || W2q == nullptr || W2s == nullptr)
+    return MOE_ERR_ARG;
+  if (!aligned16(W1) || !aligned16(W2) || !aligned16(W1q) || !aligned16(W1s) || !aligned16(W2q) || !aligned16(W2s))
+    return MOE_ERR_ARG;
+  if ((st = check_device(false)) != MOE_OK) return st;
+  return cuda_status(launch_mx_prepare_weights(*cfg, W1, W2, W1q, W1s, W2q, W2s,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_workspace_size_mxfp8(const moe_config* cfg) {
+  if (check_mx_config(cfg) != MOE_OK) return 0;
+  return mx_layout(*cfg).total;
+}
+
+moe_status moe_layer_forward_mxfp8(const moe_config* cfg, const void* x, const void* Wg, const float* bg,
+                                   const void* W1q, const void* W1s, const void* W2q, const void* W2s, void* out,
+                                   moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_mx_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (stats == nullptr) return MOE_ERR_ARG;
+  if (c.T > 0 && (x == nullptr || Wg == nullptr || W1q == nullptr || W1s == nullptr || W2q == nullptr ||
+                  W2s == nullptr || out == nullptr))
+    return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned4(bg) || !aligned16(W1q) || !aligned16(W1s) ||
+      !aligned16(W2q) || !aligned16(W2s) || !aligned16(out) || !aligned4(stats))
+    return MOE_ERR_ARG;
+  const MxLayout M = mx_layout(c);
+  const moe_ws_layout& L = M.base;
+  if ((st = check_ws(ws, ws_bytes, M.total)) != MOE_OK) return st;
+  if ((st = check_device(true)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scr = at<char>(ws, L.scratch);
+  const Scratch sc = scratch_layout(c);
+  int32_t* idx = at<int32_t>(ws, L.topk_idx);
+  float* w = at<float>(ws, L.topk_w);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  if (cudaMemsetAsync(&stats->status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  // steps 1-3 as the bf16 layer (the permuted rows in bf16, no fused combine)
+  cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
+                               at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), at<float>(scr, sc.zsum),
+                               &stats->status, at<char>(scr, sc.kslice), s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
+                         c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, c.T > 0 ? at<float>(scr, sc.zsum) : nullptr,
+                         at<int32_t>(ws, L.counts), at<int32_t>(ws, L.kept), offsets, row_of,
+                         at<int32_t>(ws, L.src_tok), at<char>(ws, L.xp), stats, sc, scr, s);
+  if (st != MOE_OK) return st;
+  // step 4 on the MX FP8 tensor cores, then step 5
+  MxBuffers b{offsets, at<int32_t>(ws, M.pad), at<char>(ws, L.xp), M.rows_pad, at<char>(ws, M.xq),
+              at<char>(ws, M.xs), at<char>(ws, M.hq), at<char>(ws, M.hs)};
+  float* yp = at<float>(ws, L.yp);
+  if (launch_mx_experts(c, b, W1q, W1s, W2q, W2s, yp, &stats->status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_combine(c, yp, row_of, w, out, s));
 }
 
 moe_status moe_testing_set_expert_wait(uint64_t wait_ns, int32_t extra_dependency) {

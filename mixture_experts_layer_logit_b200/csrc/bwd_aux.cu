@@ -14,16 +14,51 @@
 
 #include <math.h>
 
+#include <type_traits>
+
 namespace moe {
 namespace {
 
 constexpr int kPad = 64;   // rows of a backward segment: a multiple of the GEMMs' k-block
 
-// One warp: padded offsets, pad_offsets[e] = sum over e' < e of kept rounded up to 64.
-__global__ void bwd_prep_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad_offsets) {
+// max |dout| over the batch, as the bits of a non-negative float (their
+// integer order is the float order), for the fp16 operands' scale.
+__global__ void __launch_bounds__(256)
+dout_amax_kernel(const float* __restrict__ dout, size_t n, unsigned* __restrict__ amax) {
+  pdl_wait();
+  pdl_launch_dependents();
+  float m = 0.f;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 4; i += stride) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(dout) + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) atomicMax(amax, __float_as_uint(m));
+}
+
+// One warp: padded offsets, pad_offsets[e] = sum over e' < e of kept rounded
+// up to 64; and the scale of the fp16 operands: s = 2^(10 - ceil(log2 max|dout|)),
+// a power of two that brings max|s dout| into [512, 1024) (an all-zero or
+// non-finite dout keeps s = 1).
+__global__ void bwd_prep_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad_offsets,
+                                const unsigned* __restrict__ amax, float* __restrict__ scale) {
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x;
+  if (lane == 0) {
+    float s = 1.f;
+    if (amax != nullptr) {
+      const float a = __uint_as_float(*amax);
+      if (a > 0.f && isfinite(a)) {
+        int ex;
+        (void)frexpf(a, &ex);   // a = m 2^ex, m in [0.5, 1)
+        s = ldexpf(1.f, 10 - ex);
+      }
+    }
+    scale[0] = s;
+    scale[1] = 1.f / s;   // exact: s is a power of two
+  }
   constexpr int PER = kMaxExperts / 32;
   int loc[PER], sum = 0;
 #pragma unroll
@@ -69,15 +104,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 // One warp per padded row: the token of the row (kept rows of the forward's
 // permutation, each expert's segment moved to its padded start), its gate
-// weight, and the row's x and dout, the latter rounded to the element type of
-// the GEMMs.  Padding rows and rows past the last segment are zero.
-template <typename TX>
+// weight, and the row's x and s * dout in the GEMMs' operand type TG (bf16 or
+// fp16 on the bf16 path: fp16 saturates at +-65504 and sets MOE_DEV_RANGE;
+// fp32 on the fp32 path).  Padding rows and rows past the last segment are zero.
+template <typename TG> struct OpType;
+template <> struct OpType<__nv_bfloat16> {
+  __device__ __forceinline__ static uint32_t pack(float a, float b, bool&) { return pack_bf16x2(a, b); }
+};
+template <> struct OpType<__half> {
+  __device__ __forceinline__ static uint32_t pack(float a, float b, bool& over) {
+    const bool oa = fabsf(a) > 65504.f, ob = fabsf(b) > 65504.f;
+    over |= oa | ob;
+    __half2 h = __floats2half2_rn(oa ? copysignf(65504.f, a) : a, ob ? copysignf(65504.f, b) : b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+template <typename TX, typename TG>
 __global__ void __launch_bounds__(256)
 bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ pad_offsets, const int32_t* __restrict__ src_tok,
                   const int32_t* __restrict__ row_of, const float* __restrict__ topk_w, int E, int T, int k, int d,
-                  int rows_alloc, TX* __restrict__ xp, TX* __restrict__ dout_perm, float* __restrict__ wrow,
-                  uint32_t* __restrict__ status) {
+                  int rows_alloc, const float* __restrict__ scale, TG* __restrict__ xp, TG* __restrict__ dout_perm,
+                  float* __restrict__ wrow, uint32_t* __restrict__ status) {
   __shared__ int32_t s_off[kMaxExperts + 1], s_pad[kMaxExperts + 1];
   pdl_wait();
   pdl_launch_dependents();
@@ -89,6 +138,7 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
   const int lane = threadIdx.x & 31;
   const int pr = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (pr >= rows_alloc) return;
+  const float sc = scale[0];
   int t = -1;
   float w = 0.f;
   if (pr < s_pad[E]) {
@@ -107,21 +157,34 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
     }
   }
   if (lane == 0) wrow[pr] = w;
-  if (sizeof(TX) == 2) {
+  if constexpr (sizeof(TG) == 2) {
     const int nvec = d / 8;   // 8 elements = 16 bytes
     uint4* xo = reinterpret_cast<uint4*>(xp + (size_t)pr * d);
     uint4* go = reinterpret_cast<uint4*>(dout_perm + (size_t)pr * d);
+    bool over = false;
     for (int v = lane; v < nvec; v += 32) {
       uint4 xv = make_uint4(0u, 0u, 0u, 0u), gv = xv;
       if (t >= 0) {
         xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+        if constexpr (std::is_same<TG, __half>::value) {   // bf16 x -> fp16 (exact inside the fp16 range)
+          const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&xv);
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(b[q]);
+            o[q] = OpType<__half>::pack(f.x, f.y, over);
+          }
+          xv = make_uint4(o[0], o[1], o[2], o[3]);
+        }
         const float4 a = __ldg(reinterpret_cast<const float4*>(dout + (size_t)t * d) + 2 * v);
         const float4 b = __ldg(reinterpret_cast<const float4*>(dout + (size_t)t * d) + 2 * v + 1);
-        gv = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+        gv = make_uint4(OpType<TG>::pack(sc * a.x, sc * a.y, over), OpType<TG>::pack(sc * a.z, sc * a.w, over),
+                        OpType<TG>::pack(sc * b.x, sc * b.y, over), OpType<TG>::pack(sc * b.z, sc * b.w, over));
       }
       xo[v] = xv;
       go[v] = gv;
     }
+    if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(status, MOE_DEV_RANGE);
   } else {
     const int nvec = d / 4;
     float4* xo = reinterpret_cast<float4*>(xp + (size_t)pr * d);
@@ -131,6 +194,7 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
       if (t >= 0) {
         xv = __ldg(reinterpret_cast<const float4*>(x + (size_t)t * d) + v);
         gv = __ldg(reinterpret_cast<const float4*>(dout + (size_t)t * d) + v);
+        gv = make_float4(sc * gv.x, sc * gv.y, sc * gv.z, sc * gv.w);
       }
       xo[v] = xv;
       go[v] = gv;
@@ -419,15 +483,26 @@ __global__ void dwg_reduce_kernel(const float* __restrict__ part, int nsplit, in
   }
 }
 
-template <typename TX>
+template <typename TX, typename TG>
 cudaError_t launch_bwd_front_t(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                                cudaStream_t s) {
-  cudaError_t e = launch_pdl(bwd_prep_kernel, dim3(1), dim3(32), 0, s, st.offsets, c.E, st.pad_offsets);
+  cudaError_t e;
+  if (st.f16) {   // max |dout| for the scale of the fp16 operands
+    if ((e = cudaMemsetAsync(st.amax, 0, sizeof(unsigned), s)) != cudaSuccess) return e;
+    DeviceInfo di;
+    if ((e = device_info(&di)) != cudaSuccess) return e;
+    const size_t n = (size_t)c.T * c.d;   // d is a multiple of 16: whole float4 vectors
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>((n / 4 + 255) / 256, (size_t)di.sms * 4));
+    if ((e = launch_pdl(dout_amax_kernel, dim3(grid), dim3(256), 0, s, dout, n, st.amax)) != cudaSuccess) return e;
+  }
+  e = launch_pdl(bwd_prep_kernel, dim3(1), dim3(32), 0, s, st.offsets, c.E, st.pad_offsets,
+                 (const unsigned*)(st.f16 ? st.amax : nullptr), st.scale);
   if (e != cudaSuccess) return e;
   const int rows = st.rows_alloc;
-  return launch_pdl(bwd_gather_kernel<TX>, dim3((rows + 7) / 8), dim3(256), 0, s, static_cast<const TX*>(x), dout,
-                    st.offsets, (const int32_t*)st.pad_offsets, st.src_tok, st.row_of, st.topk_w, c.E, c.T, c.k,
-                    c.d, rows, static_cast<TX*>(st.xp), static_cast<TX*>(st.dout_perm), st.wrow, st.status);
+  return launch_pdl(bwd_gather_kernel<TX, TG>, dim3((rows + 7) / 8), dim3(256), 0, s, static_cast<const TX*>(x),
+                    dout, st.offsets, (const int32_t*)st.pad_offsets, st.src_tok, st.row_of, st.topk_w, c.E, c.T,
+                    c.k, c.d, rows, (const float*)st.scale, static_cast<TG*>(st.xp), static_cast<TG*>(st.dout_perm),
+                    st.wrow, st.status);
 }
 
 template <typename TX>
@@ -439,7 +514,9 @@ cudaError_t launch_bwd_gate_t(const moe_config& c, const void* x, const void* wg
   cudaError_t e = launch_pdl(logits_kernel<TX>, dim3((c.T + kLT - 1) / kLT), dim3(256), 0, s, X, WG, bg, c.T, c.d,
                              c.E, st.z);
   if (e != cudaSuccess) return e;
-  const int nt2 = (c.F + 255) / 256;
+  // column tiles of the dh GEMM, each of which left one partial of dw per row
+  const int col = c.dtype == MOE_DTYPE_BF16 ? bwd_tc_col_tile() : bwd_simt_col_tile();
+  const int nt2 = (c.F + col - 1) / col;
   e = launch_pdl(gate_bwd_kernel, dim3((c.T + 7) / 8), dim3(256), 0, s, (const float*)st.z, st.topk_idx,
                  st.topk_w, st.row_of, st.offsets, (const int32_t*)st.pad_offsets, st.counts,
                  (const float*)st.dwpart, nt2, st.rows_alloc, c.T, c.E, c.k, c.lambda, aux_coef, z_coef, st.dz,
@@ -462,8 +539,11 @@ int bwd_pad_rows() { return kPad; }
 
 cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                              cudaStream_t s) {
-  if (c.dtype == MOE_DTYPE_BF16) return launch_bwd_front_t<__nv_bfloat16>(c, x, dout, st, s);
-  return launch_bwd_front_t<float>(c, x, dout, st, s);
+  if (c.dtype == MOE_DTYPE_BF16) {
+    if (st.f16) return launch_bwd_front_t<__nv_bfloat16, __half>(c, x, dout, st, s);
+    return launch_bwd_front_t<__nv_bfloat16, __nv_bfloat16>(c, x, dout, st, s);
+  }
+  return launch_bwd_front_t<float, float>(c, x, dout, st, s);
 }
 
 cudaError_t launch_bwd_gate(const moe_config& c, const void* x, const void* wg, const float* bg, const BwdState& st,

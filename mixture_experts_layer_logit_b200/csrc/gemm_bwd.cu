@@ -70,11 +70,51 @@ struct BwdParams {
   // kDgradAct epilogue
   const float* u;           // [rows][F1] pre-activation
   const float* wrow;        // [rows] gate weight of each padded row (0 on padding)
-  __nv_bfloat16* du;        // [rows][F1]
-  __nv_bfloat16* hw;        // [rows][F]  w * h
+  void* du;                 // [rows][F1]  (operand type)
+  void* hw;                 // [rows][F]   w * h (operand type)
   float* dwpart;            // [nt][rows] per column tile: sum over its columns of dh/w * h
   int F, F1;
+  const float* scale;       // [2]: s, 1/s -- the operands hold s * dout; results linear in dout are scaled by 1/s
 };
+
+// Two fp32 values -> one 32-bit pair of the operand type (round to nearest
+// even); fp16 saturates at +-65504 and notes it in `over`.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_op(float a, float b, bool& over) {
+  return pack_hidden<F16>(a, b, over);
+}
+
+// An epilogue warp's 32 rows x BN fp32 columns from TMEM, times `scale`, into
+// out[rows][Nout] (columns from n0; rows [wrow0, wrow0 + nrows)), turned
+// around in shared memory so that the stores write whole 128-byte lines.
+__device__ __forceinline__ void store_scaled(float* out, int Nout, uint32_t tb, int wrow0, int nrows, int n0,
+                                             float scale, uint4* stg, int lane) {
+#pragma unroll 1
+  for (int blk = 0; blk < BN / 32; ++blk) {
+    uint32_t a[32];
+    tmem_ld32(tb + blk * 32, a);
+    tmem_wait_ld();
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = make_uint4(__float_as_uint(scale * __uint_as_float(a[4 * i])),
+                        __float_as_uint(scale * __uint_as_float(a[4 * i + 1])),
+                        __float_as_uint(scale * __uint_as_float(a[4 * i + 2])),
+                        __float_as_uint(scale * __uint_as_float(a[4 * i + 3])));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) stg[lane * 8 + (i ^ (lane & 7))] = v[i];
+    __syncwarp();
+    const int col0 = n0 + blk * 32;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = it * 4 + (lane >> 3), cc = lane & 7;
+      const int col = col0 + cc * 4;
+      if (rr < nrows && col < Nout)
+        *reinterpret_cast<uint4*>(out + (size_t)(wrow0 + rr) * Nout + col) = stg[rr * 8 + (cc ^ (rr & 7))];
+    }
+  }
+}
 
 struct BwdTile {
   int e, row0, rows, m0, n0, k0, nkb;
@@ -115,9 +155,9 @@ __device__ __forceinline__ BwdTile bwd_tile(const Tail* tail, const BwdParams& p
 // through shared memory 32 columns at a time), h = act(u), w the row's gate
 // weight: dh = w G, du = dh act'(u), hw = w h (the B operand of dW2), and the
 // row's sum of G h over these columns (its part of dw = <dout, y>).
-template <int ACT>
+template <int ACT, bool F16>
 __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t tb, int wrow0, int nrows, int n0,
-                                                  int nti, uint4* stg, int lane) {
+                                                  int nti, uint4* stg, int lane, float inv_s, bool& over) {
   const int row = wrow0 + lane;
   const bool live = lane < nrows;
   const float w = live ? p.wrow[row] : 0.f;
@@ -181,20 +221,18 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
         dv[j] = du_second;
         hh[j] = w * h;
       }
-      __nv_bfloat162 b;
-      b = __floats2bfloat162_rn(dg[0], dg[1]);
-      du_g[i / 2] = *reinterpret_cast<uint32_t*>(&b);
-      b = __floats2bfloat162_rn(dv[0], dv[1]);
-      du_v[i / 2] = *reinterpret_cast<uint32_t*>(&b);
-      b = __floats2bfloat162_rn(hh[0], hh[1]);
-      hwp[i / 2] = *reinterpret_cast<uint32_t*>(&b);
+      bool o = false;
+      du_g[i / 2] = pack_op<F16>(dg[0], dg[1], o);
+      du_v[i / 2] = pack_op<F16>(dv[0], dv[1], o);
+      hwp[i / 2] = pack_op<F16>(hh[0], hh[1], o);
+      over |= o && live && (f0 + i < p.F);
     }
     if (live) {
       // 32 bf16 = 64 bytes per row and block; F is a multiple of 16, so a
       // block ends at F on a 16-column boundary
       const int nv = min(4, (p.F - f0) / 8);
-      uint4* dg_row = reinterpret_cast<uint4*>(p.du + (size_t)row * p.F1 + f0);
-      uint4* hw_row = reinterpret_cast<uint4*>(p.hw + (size_t)row * p.F + f0);
+      uint4* dg_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du) + (size_t)row * p.F1 + f0);
+      uint4* hw_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.hw) + (size_t)row * p.F + f0);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (q < nv) {
@@ -203,21 +241,22 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
         }
       }
       if (ACT == kSwiglu) {
-        uint4* dv_row = reinterpret_cast<uint4*>(p.du + (size_t)row * p.F1 + p.F + f0);
+        uint4* dv_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du) + (size_t)row * p.F1 + p.F + f0);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (q < nv) dv_row[q] = make_uint4(du_v[4 * q], du_v[4 * q + 1], du_v[4 * q + 2], du_v[4 * q + 3]);
       }
     }
   }
-  if (live) p.dwpart[(size_t)nti * p.rows_alloc + row] = dwp;
+  if (live) p.dwpart[(size_t)nti * p.rows_alloc + row] = dwp * inv_s;
 }
 
-// A_MN / B_MN: the operand is MN-major in memory (rows along K).
-template <int MODE, int ACT, bool A_MN, bool B_MN>
+// A_MN / B_MN: the operand is MN-major in memory (rows along K).  F16: both
+// operands fp16 (else bf16).
+template <int MODE, int ACT, bool A_MN, bool B_MN, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const BwdParams p) {
-  constexpr uint32_t kIdesc = idesc_f16kind(BM, BN, false) | (A_MN ? kIdescAMN : 0u) | (B_MN ? kIdescBMN : 0u);
+  constexpr uint32_t kIdesc = idesc_f16kind(BM, BN, F16) | (A_MN ? kIdescAMN : 0u) | (B_MN ? kIdescBMN : 0u);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -358,8 +397,10 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)(warp - 2) * kStageWarpBytes);
+    const float inv_s = p.scale[1];
     int tl = 0;
     bool ok = true;
+    bool over = false;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tl) {
       const BwdTile t = bwd_tile<MODE>(tail, p, L);
       const int acc = tl & 1;
@@ -372,15 +413,9 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       if (MODE == kWgrad) {
         const int m0 = t.m0 + q * 32;
         const int nrows = max(0, min(32, p.M - m0));
-        Params po{};
-        po.out = p.out + (size_t)t.e * p.M * p.N;
-        po.Nout = p.N;
-        po.rows_alloc = p.M;
-        po.status = p.status;
-        bool over = false;
         if (nrows > 0) {
           if (t.nkb > 0) {
-            store_tile<kPlain, false>(po, tb, m0, nrows, t.n0, stg, lane, over);
+            store_scaled(p.out + (size_t)t.e * p.M * p.N, p.N, tb, m0, nrows, t.n0, inv_s, stg, lane);
           } else if (lane < nrows) {   // an expert without rows: its gradient is zero
             float* dst = p.out + (size_t)t.e * p.M * p.N + (size_t)(m0 + lane) * p.N;
             for (int c = t.n0; c < min(t.n0 + BN, p.N); c += 4)
@@ -395,23 +430,17 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           nrows = p.rows_alloc - wrow0;
         }
         if (nrows > 0) {
-          if (MODE == kDgradAct) {
-            act_backward_tile<ACT>(p, tb, wrow0, nrows, t.n0, t.n0 / BN, stg, lane);
-          } else {
-            Params po{};
-            po.out = p.out;
-            po.Nout = p.Nout;
-            po.rows_alloc = p.rows_alloc;
-            po.status = p.status;
-            bool over = false;
-            store_tile<kPlain, false>(po, tb, wrow0, nrows, t.n0, stg, lane, over);
-          }
+          if (MODE == kDgradAct)
+            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, t.n0 / BN, stg, lane, inv_s, over);
+          else
+            store_scaled(p.out, p.Nout, tb, wrow0, nrows, t.n0, inv_s, stg, lane);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
     }
+    if (F16 && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(p.status, MOE_DEV_RANGE);
     if (!ok && lane == 0) {
       atomicOr(p.status, MOE_DEV_TIMEOUT);
       tail->abort_flag = 1;
@@ -426,20 +455,16 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
-template <int MODE, int ACT, bool A_MN, bool B_MN>
+template <int MODE, int ACT, bool A_MN, bool B_MN, bool F16>
 cudaError_t launch_bwd(const CUtensorMap& ma, const CUtensorMap& mb, const BwdParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_bwd_gemm<MODE, ACT, A_MN, B_MN>>(kSmemBytes);
+  cudaError_t err = set_smem_once<tc_bwd_gemm<MODE, ACT, A_MN, B_MN, F16>>(kSmemBytes);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_bwd_gemm<MODE, ACT, A_MN, B_MN>, dim3(grid), dim3(kThreads), kSmemBytes, s, ma, mb, p);
+  return launch_pdl(tc_bwd_gemm<MODE, ACT, A_MN, B_MN, F16>, dim3(grid), dim3(kThreads), kSmemBytes, s, ma, mb, p);
 }
 
-}  // namespace
-
-cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
-                                      float* dw1, float* dw2, cudaStream_t s) {
-  DeviceInfo di;
-  cudaError_t err = device_info(&di);
-  if (err != cudaSuccess) return err;
+template <bool F16>
+cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const void* w1, const void* w2, float* dw1,
+                              float* dw2, int sms, cudaStream_t s) {
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
   const uint64_t R = (uint64_t)st.rows_alloc;
   const long long mt_max = (long long)(R / BM) + c.E;
@@ -449,57 +474,69 @@ cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, c
   p.E = c.E;
   p.rows_alloc = st.rows_alloc;
   p.status = st.status;
+  p.scale = st.scale;
+  cudaError_t err;
 
   // dh = dout_perm W2[e] (K = d), its activation backward in the epilogue
-  if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, false) ||
-      !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F, false, 64))
+  if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, F16) ||
+      !make_map(&mb, w2, (uint64_t)c.E * c.d, (uint64_t)c.F, F16, 64))
     return cudaErrorInvalidValue;
   p.K = c.d;
   p.Nout = c.F;
   p.b_krows = c.d;
   p.u = st.u;
   p.wrow = st.wrow;
-  p.du = static_cast<__nv_bfloat16*>(st.du);
-  p.hw = static_cast<__nv_bfloat16*>(st.hw);
+  p.du = st.du;
+  p.hw = st.hw;
   p.dwpart = st.dwpart;
   p.F = c.F;
   p.F1 = F1;
-  int grid = (int)std::min<long long>(mt_max * ((c.F + BN - 1) / BN), di.sms);
-  err = (c.act == MOE_ACT_SWIGLU) ? launch_bwd<kDgradAct, kSwiglu, false, true>(ma, mb, p, grid, s)
-                                  : launch_bwd<kDgradAct, kRelu, false, true>(ma, mb, p, grid, s);
+  int grid = (int)std::min<long long>(mt_max * ((c.F + BN - 1) / BN), sms);
+  err = (c.act == MOE_ACT_SWIGLU) ? launch_bwd<kDgradAct, kSwiglu, false, true, F16>(ma, mb, p, grid, s)
+                                  : launch_bwd<kDgradAct, kRelu, false, true, F16>(ma, mb, p, grid, s);
   if (err != cudaSuccess) return err;
 
   // dxp = du W1[e] (K = F1)
-  if (!make_map(&ma, st.du, R, (uint64_t)F1, false) ||
-      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false, 64))
+  if (!make_map(&ma, st.du, R, (uint64_t)F1, F16) ||
+      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, F16, 64))
     return cudaErrorInvalidValue;
   p.K = F1;
   p.Nout = c.d;
   p.b_krows = F1;
   p.out = st.dxp;
-  grid = (int)std::min<long long>(mt_max * ((c.d + BN - 1) / BN), di.sms);
-  if ((err = launch_bwd<kDgradPlain, kRelu, false, true>(ma, mb, p, grid, s)) != cudaSuccess) return err;
+  grid = (int)std::min<long long>(mt_max * ((c.d + BN - 1) / BN), sms);
+  if ((err = launch_bwd<kDgradPlain, kRelu, false, true, F16>(ma, mb, p, grid, s)) != cudaSuccess) return err;
 
   // dW2[e] = dout_perm_e^T (w h)_e: M = d, N = F, K = the expert's padded rows
-  if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, false, 64) ||
-      !make_map(&mb, st.hw, R, (uint64_t)c.F, false, 64))
+  if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, F16, 64) || !make_map(&mb, st.hw, R, (uint64_t)c.F, F16, 64))
     return cudaErrorInvalidValue;
   p.M = c.d;
   p.N = c.F;
   p.out = dw2;
   long long tiles = (long long)c.E * ((c.d + BM - 1) / BM) * ((c.F + BN - 1) / BN);
-  if ((err = launch_bwd<kWgrad, kRelu, true, true>(ma, mb, p, (int)std::min<long long>(tiles, di.sms), s)) !=
+  if ((err = launch_bwd<kWgrad, kRelu, true, true, F16>(ma, mb, p, (int)std::min<long long>(tiles, sms), s)) !=
       cudaSuccess)
     return err;
 
   // dW1[e] = du_e^T xp_e: M = F1, N = d
-  if (!make_map(&ma, st.du, R, (uint64_t)F1, false, 64) || !make_map(&mb, st.xp, R, (uint64_t)c.d, false, 64))
+  if (!make_map(&ma, st.du, R, (uint64_t)F1, F16, 64) || !make_map(&mb, st.xp, R, (uint64_t)c.d, F16, 64))
     return cudaErrorInvalidValue;
   p.M = F1;
   p.N = c.d;
   p.out = dw1;
   tiles = (long long)c.E * ((F1 + BM - 1) / BM) * ((c.d + BN - 1) / BN);
-  return launch_bwd<kWgrad, kRelu, true, true>(ma, mb, p, (int)std::min<long long>(tiles, di.sms), s);
+  return launch_bwd<kWgrad, kRelu, true, true, F16>(ma, mb, p, (int)std::min<long long>(tiles, sms), s);
+}
+
+}  // namespace
+
+cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
+                                      float* dw1, float* dw2, cudaStream_t s) {
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  return st.f16 ? launch_backward_t<true>(c, st, w1, w2, dw1, dw2, di.sms, s)
+                : launch_backward_t<false>(c, st, w1, w2, dw1, dw2, di.sms, s);
 }
 
 int bwd_tc_col_tile() { return BN; }

@@ -267,17 +267,20 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
 }  // namespace
 
 cudaError_t launch_grouped_plain_tc(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
-                                    const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s) {
+                                    const void* B, int K, int Nout, float* out, uint32_t* status, bool f16,
+                                    cudaStream_t s) {
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, (uint64_t)rows_alloc, (uint64_t)K, false) ||
-      !make_map(&mb, B, (uint64_t)c.E * Nout, (uint64_t)K, false))
+  if (!make_map(&ma, A, (uint64_t)rows_alloc, (uint64_t)K, f16) ||
+      !make_map(&mb, B, (uint64_t)c.E * Nout, (uint64_t)K, f16))
     return cudaErrorInvalidValue;
   Params p{offsets, out, c.E, K, Nout, Nout, 0, rows_alloc, status};
   const long long tiles = ((long long)rows_alloc / BM + c.E) * ((Nout + BN - 1) / BN);
-  return launch_one<kPlain, false>(ma, mb, p, (int)std::min<long long>(tiles, di.sms), s);
+  const int grid = (int)std::min<long long>(tiles, di.sms);
+  // kPlain takes the hidden type's operands: fp16 when F16
+  return f16 ? launch_one<kPlain, true>(ma, mb, p, grid, s) : launch_one<kPlain, false>(ma, mb, p, grid, s);
 }
 
 cudaError_t launch_expert_ffn_tc(const moe_config& c, const void* xp, const int32_t* offsets,

@@ -141,11 +141,20 @@ struct BwdState {
   float* dwg_part;           // [nsplit][E][d + 1]
   int nsplit, tok_per_split;
   uint32_t* status;
+  // fp16 GEMM operands (bf16 path with an fp16 hidden type): dout is scaled
+  // by a power of two s into the fp16 range, and every result linear in dout
+  // is scaled back by 1/s where it is written
+  bool f16;
+  unsigned* amax;            // max |dout| as float bits (zeroed before the amax kernel)
+  float* scale;              // [2]: s, 1/s (1, 1 without fp16 operands)
+  void* w1h;                 // fp16 copy of W1 (f16), else unused
 };
 int bwd_pad_rows();
 int bwd_tc_col_tile();     // columns of a tensor-core backward tile (the dw partials per row)
 int bwd_simt_col_tile();
-// prep (padded offsets) and gather (x, dout, gate weight of every padded row)
+// bf16 -> fp16 (round to nearest even, saturating at +-65504)
+cudaError_t launch_convert_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t s);
+// prep (padded offsets, the dout scale) and gather (x, dout, gate weight of every padded row)
 cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                              cudaStream_t s);
 // the expert layers' gradients: dh with the activation backward, dxp, dW2, dW1
@@ -153,15 +162,40 @@ cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, c
                                       float* dw1, float* dw2, cudaStream_t s);
 cudaError_t launch_expert_backward_simt(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
                                         float* dw1, float* dw2, cudaStream_t s);
-// out[rows][Nout] = A[rows][K] B_e[Nout][K]^T over the segments of offsets (E of them), fp32 out
+// out[rows][Nout] = A[rows][K] B_e[Nout][K]^T over the segments of offsets (E of them), fp32 out;
+// f16: both operands fp16 (else bf16)
 cudaError_t launch_grouped_plain_tc(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
-                                    const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s);
+                                    const void* B, int K, int Nout, float* out, uint32_t* status, bool f16,
+                                    cudaStream_t s);
 cudaError_t launch_grouped_plain_simt(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
                                       const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s);
 // the gate's gradient (logits recomputed), dx and dW_gate / db
 cudaError_t launch_bwd_gate(const moe_config& c, const void* x, const void* wg, const float* bg, const BwdState& st,
                             float aux_coef, float z_coef, float* dx, float* dwg, float* dbg, float* dw_out,
                             cudaStream_t s);
+
+// ------------------------------------------------------- MX FP8 experts
+// Buffers of the FP8 expert step: kept offsets from the permutation, padded
+// offsets (multiples of mx_pad_rows()), the padded E4M3 layer-1 input rows and
+// hidden activation with their scale atoms.
+struct MxBuffers {
+  const int32_t* offsets;   // [E+1] kept
+  int32_t* pad;             // [E+1]
+  const void* xp;           // [rows][d] bf16 permuted rows (from the permutation)
+  int rows_pad;
+  void* xq;                 // [rows_pad][d] E4M3
+  void* xs;                 // scale atoms of xq
+  void* hq;                 // [rows_pad][F] E4M3
+  void* hs;                 // scale atoms of hq
+};
+int mx_pad_rows();
+size_t mx_scale_bytes(size_t rows, size_t K);   // rows, K multiples of 128
+cudaError_t launch_mx_prepare_weights(const moe_config& c, const void* w1, const void* w2, void* w1q, void* w1s,
+                                      void* w2q, void* w2s, cudaStream_t s);
+// steps 4 of the FP8 layer: padded offsets, the quantised input rows, both
+// layers; yp [rows][d] fp32 at the kept rows
+cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const void* w1q, const void* w1s,
+                              const void* w2q, const void* w2s, float* yp, uint32_t* status, cudaStream_t s);
 
 // Combine.
 cudaError_t launch_combine(const moe_config& c, const void* yp, const int32_t* row_of,

@@ -103,6 +103,41 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Block-scaled MMA of E4M3 operands with UE8M0 scales (one per 32 elements of
+// K) held in TMEM: sfa_tmem / sfb_tmem carry the byte of the 32-bit TMEM word
+// in bits 31:30, which the instruction descriptor repeats.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Copies 32 rows x 16 bytes of shared memory (described by sdesc_rows16) to
+// TMEM columns [taddr, taddr + 4) of lanes 0-31, repeated in lanes 32-63,
+// 64-95 and 96-127.
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Shared-memory descriptor of rows of 16 bytes, no swizzle: 8-row groups 128
+// bytes apart.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128 >> 4) << 16;   // leading byte offset
+  d |= (uint64_t)(128 >> 4) << 32;   // stride byte offset: the next 8 rows
+  d |= (uint64_t)1 << 46;            // version; layout type 0 = no swizzle
+  return d;
+}
+// instruction descriptor of kind::mxf8f6f4 with block scales: D fp32, A and B
+// E4M3, both K-major, UE8M0 scales; sf_id picks the byte of the scale word
+// (the 32-element K block within a 128-element K stage)
+constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24) | (sf_id << 29);
+}
+
 // ---- flags between CTAs of one grid (global memory, GPU scope)
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -246,6 +281,20 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   });
   return fn;
+}
+
+// 2-D tensor map over a row-major [rows, cols] matrix of bytes (E4M3); box =
+// 128 columns (128 bytes) x box_rows rows, 128-byte swizzle, zero fill outside.
+inline bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = 128) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D tensor map over a row-major [rows, cols] matrix of 16-bit elements

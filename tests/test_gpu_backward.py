@@ -4,10 +4,27 @@ differences of the forward oracle.
 
 For each layer: the forward runs (moe_layer_forward), then the backward of
 L = <dout, out> + aux_coef * aux + z_coef * z_loss on the forward's workspace.
-Every gradient (dx, dW_gate, db, dW1, dW2 and the gate-weight gradient dw) is
-compared element by element: bf16 path max|err| <= 2e-2 * RMS(ref), fp32 path
-max|err| <= 1e-4 * max|ref|.  Near-tie tokens take the device's selection in
-the oracle (both selections are correct there)."""
+Every gradient is compared element by element with the oracle's:
+
+* fp32 path: max|err| <= 1e-4 * max|ref| for every tensor;
+* bf16 path with the default fp16 hidden type (fp16 GEMM operands, dout
+  scaled by a power of two): every gradient within 2e-2 * RMS(ref);
+* bf16 path, the expert weight gradients dW1 and dW2, in addition: each is a
+  contraction over the expert's rows of operands rounded once each (dout and
+  w*h for dW2; du, which carries the rounding of dout and its own, for dW1),
+  so each product is off by at most 2u relative (u = 2^-11 for fp16 operands,
+  2^-9 for bf16).  The bound is element by element:
+  |err| <= 4u * (the same contraction over absolute values) + 1e-6 max|ref|
+  (a factor 2 over the rounding model, for the fp32 accumulation).  A wrong
+  row, column or expert gives an error of the size of the gradient itself and
+  fails it.  With a bf16 hidden type (bf16 operands) this bound is the bar for
+  dW1 and dW2: on layers whose weight gradients have heavy tails the bf16
+  roundings alone put max|err| above 2e-2 RMS (reported, not asserted), and
+  the other gradients are held to 4e-2 RMS (two bf16 roundings, of dout and
+  of du, feed them: 8x those of the fp16 default, which meets 2e-2).
+
+Near-tie tokens take the device's selection in the oracle (both selections are
+correct there)."""
 import numpy as np
 import pytest
 import torch
@@ -35,13 +52,13 @@ LAYERS = [
 AUX, ZC = 0.05, 0.01
 
 
-def _close(got, ref, dtype, name):
+def _close(got, ref, dtype, name, bar=2e-2):
     if ref.size == 0:
         return 0.0
     err = float(np.max(np.abs(got - ref)))
     if dtype == mw.BF16:
         rms = float(np.sqrt(np.mean(ref ** 2)))
-        assert err <= 2e-2 * rms, f"{name}: max|err| {err:.3e} > 2e-2 * RMS {rms:.3e}"
+        assert err <= bar * rms, f"{name}: max|err| {err:.3e} > {bar} * RMS {rms:.3e}"
         return err / rms
     scale = float(np.max(np.abs(ref)))
     assert err <= 1e-4 * scale, f"{name}: max|err| {err:.3e} > 1e-4 * max|ref| {scale:.3e}"
@@ -50,12 +67,15 @@ def _close(got, ref, dtype, name):
 
 def run_backward(L: DeviceLayer, seed: int):
     w, cfg = L.w, L.cfg
+    # bf16 operands (a bf16 hidden type) round dout and du 8x coarser than fp16:
+    # their bar for the non-weight gradients is 4e-2 RMS (weight gradients: the rounding bound)
+    bar = 4e-2 if L.hidden == "bf16" else 2e-2
     res = L.forward()
     T, d, E, F, k = L.T, w.d, w.E, w.F, w.k
     F1 = F if w.act == mw.RELU else 2 * F
     rng = np.random.default_rng(seed)
     dout = rng.standard_normal((T, d)).astype(np.float32)
-    w2_bwd = mw.to_device(L.inp.w2)       # W2 in the element type of x (not the fp16 copy)
+    w2_bwd = L.w2                         # W2 in the hidden type, as the forward took it
     dev = "cuda"
     dx = torch.empty((max(T, 1), d), dtype=torch.float32, device=dev)
     dwg = torch.empty((E, d), dtype=torch.float32, device=dev)
@@ -79,15 +99,31 @@ def run_backward(L: DeviceLayer, seed: int):
     forced = r0.gap < 1e-4
     fw = om.forward(x, wg, L.inp.bias, w1, w2, lc, forced if forced.any() else None,
                     res["topk_idx"] if forced.any() else None)
-    g = ob.backward(x, wg, L.inp.bias, w1, w2, lc, dout.astype(np.float64), AUX, ZC, fw=fw)
+    g = ob.backward(x, wg, L.inp.bias, w1, w2, lc, dout.astype(np.float64), AUX, ZC, fw=fw,
+                    want_abs=w.dtype == mw.BF16)
     out = {}
-    out["dw"] = _close(dw.cpu().numpy().astype(np.float64)[:T], g.dw, w.dtype, "dw")
-    out["dW2"] = _close(to_np64(dw2), g.dw2, w.dtype, "dW2")
-    out["dW1"] = _close(to_np64(dw1), g.dw1, w.dtype, "dW1")
-    out["dx"] = _close(to_np64(dx[:T]), g.dx, w.dtype, "dx")
-    out["dWg"] = _close(to_np64(dwg), g.dwg, w.dtype, "dWg")
+    out["dw"] = _close(dw.cpu().numpy().astype(np.float64)[:T], g.dw, w.dtype, "dw", bar)
+    if w.dtype == mw.BF16:
+        f16 = L.hidden == "f16"
+        u = 2.0 ** -11 if f16 else 2.0 ** -9
+        for name, got, ref, A in [("dW2", dw2, g.dw2, g.abs_dw2), ("dW1", dw1, g.dw1, g.abs_dw1)]:
+            got = to_np64(got)
+            err = np.abs(got - ref)
+            bound = 4 * u * A + 1e-6 * float(np.max(np.abs(ref)))
+            worst = float(np.max(err / bound))
+            assert worst <= 1.0, f"{name}: |err| exceeds the rounding bound by {worst:.2f}x"
+            rms = float(np.sqrt(np.mean(ref ** 2)))
+            out[name] = float(np.max(err)) / rms
+            out[name + "_of_bound"] = worst
+            if f16:
+                assert out[name] <= 2e-2, f"{name}: max|err| {out[name]:.3e} RMS > 2e-2"
+    else:
+        out["dW2"] = _close(to_np64(dw2), g.dw2, w.dtype, "dW2")
+        out["dW1"] = _close(to_np64(dw1), g.dw1, w.dtype, "dW1")
+    out["dx"] = _close(to_np64(dx[:T]), g.dx, w.dtype, "dx", bar)
+    out["dWg"] = _close(to_np64(dwg), g.dwg, w.dtype, "dWg", bar)
     if L.inp.bias is not None:
-        out["db"] = _close(to_np64(dbg), g.dbias, w.dtype, "db")
+        out["db"] = _close(to_np64(dbg), g.dbias, w.dtype, "db", bar)
     return out
 
 
@@ -97,11 +133,40 @@ def test_backward_matches_oracle(w):
     print(w.name, {k: f"{v:.2e}" for k, v in rel.items()})
 
 
-def test_backward_bf16_hidden_config():
-    """A bf16 hidden activation in the forward changes nothing in the backward
-    (it recomputes u in fp32)."""
-    w = LAYERS[1]
-    run_backward(DeviceLayer(w, hidden="bf16"), 5)
+@pytest.mark.parametrize("name", ["b_relu_cap", "b_wide", "b_fine_top6"])
+def test_backward_bf16_hidden(name):
+    """A bf16 hidden type: the backward's GEMM operands are bf16 (no dout
+    scale); the weight gradients meet the bf16 rounding bound."""
+    w = next(x for x in LAYERS if x.name == name)
+    rel = run_backward(DeviceLayer(w, hidden="bf16"), 5)
+    print(name, "bf16 operands", {k: f"{v:.2e}" for k, v in rel.items()})
+
+
+def test_backward_scale_invariance():
+    """dout scaled by 2^-20 (far below the fp16 range) gives gradients scaled
+    by 2^-20 to within the same tolerance: the power-of-two scale of the fp16
+    operands follows dout's magnitude."""
+    w = LAYERS[0]
+    L = DeviceLayer(w)
+    res = L.forward()
+    T, d, E, F, k = L.T, w.d, w.E, w.F, w.k
+    F1 = F if w.act == mw.RELU else 2 * F
+    g0 = np.random.default_rng(9).standard_normal((T, d)).astype(np.float32)
+    outs = []
+    for sc in (1.0, 2.0 ** -20):
+        dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+        dwg = torch.empty((E, d), dtype=torch.float32, device="cuda")
+        dw1 = torch.empty((E, F1, d), dtype=torch.float32, device="cuda")
+        dw2 = torch.empty((E, d, F), dtype=torch.float32, device="cuda")
+        stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(moe.moe_backward_workspace_size(L.cfg), dtype=torch.uint8, device="cuda")
+        moe.moe_layer_backward(L.cfg, L.x, L.wg, L.bias, L.w1, L.w2, torch.from_numpy(g0 * np.float32(sc)).cuda(),
+                               0.0, 0.0, res["ws"], dx, dwg, None, dw1, dw2, None, stats, ws)
+        torch.cuda.synchronize()
+        assert moe.read_stats(stats)["status"] == 0
+        outs.append([t.double().cpu().numpy() / sc for t in (dx, dwg, dw1, dw2)])
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b), "the power-of-two scale must cancel exactly"
 
 
 def test_backward_no_tokens():

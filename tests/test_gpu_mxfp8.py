@@ -1,0 +1,133 @@
+"""The layer with MX FP8 expert weights (moe_prepare_mxfp8_weights,
+moe_layer_forward_mxfp8) against the float64 MX oracle (oracle/moe_fp8.py).
+
+* The prepared weights, decoded here from their bytes (E4M3 bit fields and
+  the UE8M0 scale atoms, SwiGLU rows de-interleaved), equal the oracle's
+  quantisation of the same bf16 weights exactly (both take the same integer
+  decisions: the block exponent and round-to-nearest-even to the E4M3 grid).
+* The forward matches the MX oracle within 2e-2 * RMS(out): the oracle
+  quantises the input rows and the hidden activation the same way, so what
+  differs is fp32 accumulation and the rare hidden value whose fp32 and
+  float64 values round to neighbouring E4M3 values.
+* Routing, permutation and statistics are the bf16 layer's, compared exactly
+  off near ties."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as mw
+import mixture_experts_layer_logit_b200 as moe
+import oracle
+from oracle import moe_oracle as om
+from oracle import moe_fp8 as mf
+from tests.gpu_harness import check_routing, check_out, to_np64
+
+pytestmark = pytest.mark.gpu
+
+W = mw.Workload
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    b = b.astype(np.int64)
+    s, e, m = b >> 7, (b >> 3) & 15, b & 7
+    v = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    return np.where(s == 1, -v, v)
+
+
+def decode_matrix(q: np.ndarray, sf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Dequantised [rows][K] from E4M3 bytes and the scale atoms."""
+    vals = e4m3_decode(q.reshape(rows, K))
+    r = np.arange(rows)[:, None]
+    kb = np.arange(K // 32)[None, :]
+    off = ((r // 128) * (K // 128) + kb // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + kb % 4
+    X = sf[off].astype(np.int64) - 127
+    return vals * np.repeat(np.exp2(X.astype(np.float64)), 32, axis=1)
+
+
+LAYERS = [
+    W("mx_decode_like", T=64, d=256, E=16, F=256, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True, seed=81),
+    W("mx_relu_cap", T=500, d=256, E=8, F=384, k=2, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.0, seed=82),
+    W("mx_swiglu_lam", T=700, d=384, E=6, F=256, k=2, act=mw.SWIGLU, dtype=mw.BF16, lam=1.0, zipf_bias=True,
+      seed=83),
+    W("mx_E1", T=130, d=128, E=1, F=128, k=1, act=mw.RELU, dtype=mw.BF16, seed=84),
+    W("mx_many_rows", T=1500, d=256, E=4, F=256, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=85),
+]
+
+
+def _prepare(w, inp):
+    cfg = moe.make_config(w.T, w.d, w.E, w.F, w.k, w.act, w.dtype, w.capacity_factor, w.lam)
+    w1, w2 = mw.to_device(inp.w1), mw.to_device(inp.w2)
+    return cfg, moe.prepare_mxfp8(cfg, w1, w2)
+
+
+@pytest.mark.parametrize("w", [LAYERS[0], LAYERS[1]], ids=["swiglu", "relu"])
+def test_prepared_weights_equal_the_oracle_quantisation(w):
+    inp = mw.generate(w)
+    cfg, (w1q, w1s, w2q, w2s) = _prepare(w, inp)
+    torch.cuda.synchronize()
+    F1 = w.F1
+    W1 = decode_matrix(w1q.cpu().numpy(), w1s.cpu().numpy(), w.E * F1, w.d).reshape(w.E, F1, w.d)
+    W2 = decode_matrix(w2q.cpu().numpy(), w2s.cpu().numpy(), w.E * w.d, w.F).reshape(w.E, w.d, w.F)
+    if w.act == mw.SWIGLU:   # undo the interleave: rows [128 b, +64) gate 64 b.., the next 64 up 64 b..
+        F = w.F
+        perm = np.empty(F1, dtype=np.int64)
+        for b in range(F // 64):
+            perm[128 * b:128 * b + 64] = np.arange(64 * b, 64 * b + 64)
+            perm[128 * b + 64:128 * b + 128] = F + np.arange(64 * b, 64 * b + 64)
+        W1u = np.empty_like(W1)
+        W1u[:, perm, :] = W1
+        W1 = W1u
+    for e in range(w.E):
+        assert np.array_equal(W1[e], mf.mxq(mw.to_f64(inp.w1[e]))), f"W1[{e}]"
+        assert np.array_equal(W2[e], mf.mxq(mw.to_f64(inp.w2[e]))), f"W2[{e}]"
+
+
+def run_mx(w, sample=0):
+    inp = mw.generate(w)
+    cfg, (w1q, w1s, w2q, w2s) = _prepare(w, inp)
+    x, wg, bias = mw.to_device(inp.x), mw.to_device(inp.wg), mw.to_device(inp.bias)
+    T = w.T
+    ws = torch.empty(moe.moe_workspace_size_mxfp8(cfg), dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)
+    out = torch.empty((T, w.d), dtype=torch.float32, device="cuda")
+    stats = torch.zeros(moe.STATS_BYTES, dtype=torch.uint8, device="cuda")
+    moe.moe_layer_forward_mxfp8(cfg, x, wg, bias, w1q, w1s, w2q, w2s, out, stats, ws)
+    torch.cuda.synchronize()
+    st = moe.read_stats(stats)
+    assert st["status"] == 0, st
+    n, lay = moe.moe_workspace_size(cfg)
+    idx = ws[lay.topk_idx:lay.topk_idx + 4 * T * w.k].view(torch.int32).view(T, w.k).cpu().numpy()
+    lc = oracle.LayerConfig.from_workload(w)
+    xx, wgg = mw.to_f64(inp.x), mw.to_f64(inp.wg)
+    r0 = om.route(xx, wgg, inp.bias, lc)
+    forced, n_tie = check_routing(idx, r0)
+    r = om.route(xx, wgg, inp.bias, lc, forced, idx) if n_tie else r0
+    d = om.dispatch(r.idx, lc, r.prob_mean)
+    assert st["drop_count"] == d.drop_count and st["rows_kept"] == int(d.offsets[-1])
+    w1, w2 = mw.F64Experts(inp.w1), mw.F64Experts(inp.w2)
+    if sample:
+        toks = np.unique(np.concatenate([np.random.default_rng(0).choice(T, sample, replace=False), [0, T - 1]]))
+        ref = mf.forward_tokens(xx, w1, w2, lc, r, d, toks)
+        return check_out(to_np64(out[torch.from_numpy(toks).cuda()]), ref, mw.BF16)
+    fw = mf.forward(xx, wgg, inp.bias, w1, w2, lc, forced if n_tie else None, idx if n_tie else None)
+    return check_out(to_np64(out), fw.out, mw.BF16)
+
+
+@pytest.mark.parametrize("w", LAYERS, ids=[w.name for w in LAYERS])
+def test_mxfp8_forward_matches_mx_oracle(w):
+    rel = run_mx(w)
+    print(w.name, f"max|err|/RMS {rel:.2e}")
+
+
+@pytest.mark.parametrize("name", ["fine_decode_dropless", "fine_decode_cap"])
+def test_mxfp8_decode_layer(name):
+    rel = run_mx(mw.WORKLOADS[name])
+    print(name, f"max|err|/RMS {rel:.2e}")
+
+
+def test_mxfp8_rejects_unsupported_shapes():
+    cfg = moe.make_config(64, 192, 4, 256, 2, "relu")      # d not a multiple of 128
+    assert moe.moe_workspace_size_mxfp8(cfg) == 0
+    assert moe.moe_mxfp8_weight_bytes(cfg)[0] == 0
+    cfg = moe.make_config(64, 256, 4, 256, 2, "relu", dtype="f32")
+    assert moe.moe_workspace_size_mxfp8(cfg) == 0
