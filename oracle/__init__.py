@@ -7,7 +7,7 @@ from .moe_oracle import (  # noqa: F401
     LayerConfig, Routing, Dispatch, Forward, RELU, SWIGLU,
     gate_logits, normalise_logits, softmax, top_k, route, capacity, dispatch,
     expert_hidden, expert_ffn, expert_segments, combine, forward, forward_tokens,
-    brute_force, log_partition, z_loss, adaptive_aux_coef,
+    brute_force, log_partition, z_loss, adaptive_aux_coef, shared_expert, forward_with_shared,
 )
 from .moe_backward import (  # noqa: F401
     Grads, loss, backward, expert_backward, normalise_backward, silu_grad, gate_weight_backward,

@@ -348,6 +348,24 @@ def forward_tokens(x, w1, w2, cfg: LayerConfig, r: Routing, dsp: Dispatch,
     return out
 
 
+# ------------------------------------------------------------ shared expert
+def shared_expert(x, w1s, w2s, act: str, F_shared: int) -> np.ndarray:
+    """A shared expert (the MoE survey page, "MoE未来重点研究方向", item 4:
+    DeepSeekMoE's shared experts): an expert every token goes through with
+    weight 1, outside the routing.  Several shared experts are one expert of
+    their summed hidden width (their W1 rows stacked -- for SwiGLU all gate
+    rows, then all up rows -- and their W2 columns side by side)."""
+    return expert_ffn(np.asarray(x, np.float64), w1s, w2s, act, F_shared)
+
+
+def forward_with_shared(x, wg, bias, w1, w2, w1s, w2s, F_shared: int, cfg: LayerConfig, forced_mask=None,
+                        forced_idx=None) -> Forward:
+    """The layer plus a shared expert: out = routed combine + shared_expert(x)."""
+    fw = forward(x, wg, bias, w1, w2, cfg, forced_mask, forced_idx)
+    fw.out = fw.out + shared_expert(x, w1s, w2s, cfg.act, F_shared)
+    return fw
+
+
 # ------------------------------------------------------------- brute force
 def brute_force(x, wg, bias, w1, w2, cfg: LayerConfig) -> np.ndarray:
     """Dense check of the whole layer for tiny inputs, written independently of

@@ -281,6 +281,35 @@ def test_special_cases():
     assert check_special_cases() == []
 
 
+def check_shared():
+    """Shared expert: every token through it with weight 1.  E = 1, k = 1 and
+    the shared expert equal to the routed one gives twice the routed output;
+    two shared experts stacked into one wide expert equal their sum."""
+    bad = []
+    rng = np.random.default_rng(11)
+    T, d, F = 12, 8, 6
+    x = rng.standard_normal((T, d))
+    w1 = rng.standard_normal((1, 2 * F, d)) / 3
+    w2 = rng.standard_normal((1, d, F)) / 3
+    cfg = oracle.LayerConfig(T=T, d=d, E=1, F=F, k=1, act=oracle.SWIGLU)
+    fw = om.forward_with_shared(x, np.zeros((1, d)), None, w1, w2, w1[0], w2[0], F, cfg)
+    dense = om.forward(x, np.zeros((1, d)), None, w1, w2, cfg).out
+    if not np.allclose(fw.out, 2 * dense, rtol=0, atol=1e-12):
+        bad.append("shared == routed expert: out != 2 * routed")
+    a1, a2 = rng.standard_normal((2 * F, d)), rng.standard_normal((d, F))
+    b1, b2 = rng.standard_normal((2 * F, d)), rng.standard_normal((d, F))
+    wide1 = np.concatenate([a1[:F], b1[:F], a1[F:], b1[F:]])      # gate rows, then up rows
+    wide2 = np.concatenate([a2, b2], axis=1)
+    two = om.shared_expert(x, a1, a2, oracle.SWIGLU, F) + om.shared_expert(x, b1, b2, oracle.SWIGLU, F)
+    if not np.allclose(om.shared_expert(x, wide1, wide2, oracle.SWIGLU, 2 * F), two, rtol=0, atol=1e-12):
+        bad.append("two shared experts != one wide shared expert")
+    return bad
+
+
+def test_shared_expert():
+    assert check_shared() == []
+
+
 def test_losses_closed_forms():
     assert check_losses() == []
 
@@ -336,7 +365,7 @@ def test_workload_generator_is_seeded_and_bf16_exact():
 # -------------------------------------------------- planted mistakes (CPU)
 def _all_pins():
     return (check_closed_forms() + check_brute_force() + check_invariants() + check_special_cases() +
-            check_losses())
+            check_losses() + check_shared())
 
 
 def _mut_sample_std(z, lam):
@@ -441,6 +470,10 @@ def _mut_coef_beta_swapped(alpha, drop_rate, beta, xi):
     return (1.0 - beta) * alpha + beta * xi * drop_rate
 
 
+def _mut_shared_gate_weighted(x, w1s, w2s, act, F_shared):
+    return 0.5 * om.expert_ffn(np.asarray(x, np.float64), w1s, w2s, act, F_shared)
+
+
 MUTATIONS = {
     "sample_std": ("normalise_logits", _mut_sample_std),
     "lambda_ignored": ("normalise_logits", _mut_no_scale),
@@ -456,6 +489,7 @@ MUTATIONS = {
     "z_loss_summed_over_tokens": ("z_loss", _mut_z_loss_summed),
     "log_partition_is_the_max": ("log_partition", _mut_log_partition_is_max),
     "coef_smoothing_swapped": ("adaptive_aux_coef", _mut_coef_beta_swapped),
+    "shared_expert_weighted": ("shared_expert", _mut_shared_gate_weighted),
 }
 
 
