@@ -312,6 +312,25 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* 
                               float* dw, moe_stats* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * The layer with a shared expert: every token also goes, with weight 1 and
+ * outside the routing, through one more expert whose output is added to the
+ * routed experts' sum (the MoE survey page, "MoE未来重点研究方向", item 4:
+ * DeepSeekMoE's shared experts).  Several shared experts are one shared expert
+ * of their summed hidden width F_shared (W1 rows stacked -- for SwiGLU all the
+ * gate rows, then all the up rows -- and W2 columns side by side).
+ *   W1_shared[F1s, d] (F1s = F_shared or 2 F_shared) in the element type of x,
+ *   W2_shared[d, F_shared] in hidden_dtype; everything else as
+ *   moe_layer_forward, whose workspace layout the first moe_workspace_size(cfg)
+ *   bytes of ws keep.  ws: at least moe_workspace_size_shared(cfg, F_shared)
+ *   bytes (0 when F_shared is not a supported width).
+ */
+size_t moe_workspace_size_shared(const moe_config* cfg, int32_t F_shared);
+moe_status moe_layer_forward_shared(const moe_config* cfg, int32_t F_shared, const void* x, const void* Wg,
+                                    const float* bg, const void* W1, const void* W2, const void* W1_shared,
+                                    const void* W2_shared, void* out, moe_stats* stats, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/*
  * The layer with FP8 expert weights.  The Skywork-MoE release serves its model
  * with FP8 weights (inference section: 146 GB on an 8 x 4090 server); the
  * pages fix no FP8 format.  This library takes the microscaled (MX) form the

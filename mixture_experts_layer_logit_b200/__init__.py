@@ -23,7 +23,8 @@ __all__ = [
     "moe_expert_ffn_combine", "MOE_STATIC_SCRATCH_BYTES", "prepare_w2", "moe_aux_coef_update",
     "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_segments_scratch_size", "moe_expert_ffn_segments",
     "moe_backward_workspace_size", "moe_layer_backward", "moe_mxfp8_weight_bytes", "moe_prepare_mxfp8_weights",
-    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8", "prepare_mxfp8",
+    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8", "prepare_mxfp8", "moe_workspace_size_shared",
+    "moe_layer_forward_shared",
     "read_stats", "STATS_BYTES", "MOE_ACT_RELU", "MOE_ACT_SWIGLU", "MOE_DTYPE_F32", "MOE_DTYPE_BF16",
     "MOE_DTYPE_F16", "MOE_DEV_TIMEOUT", "MOE_DEV_BOUNDS", "MOE_DEV_RANGE", "EXPORTED_SYMBOLS",
 ]
@@ -41,7 +42,8 @@ EXPORTED_SYMBOLS = ["moe_status_string", "moe_scratch_size", "moe_workspace_size
                     "moe_aux_coef_update", "moe_aux_coef_next", "moe_testing_set_expert_wait",
                     "moe_segments_scratch_size", "moe_expert_ffn_segments", "moe_backward_workspace_size",
                     "moe_layer_backward", "moe_mxfp8_weight_bytes", "moe_prepare_mxfp8_weights",
-                    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8"]
+                    "moe_workspace_size_mxfp8", "moe_layer_forward_mxfp8", "moe_workspace_size_shared",
+                    "moe_layer_forward_shared"]
 MOE_STATIC_SCRATCH_BYTES = 2 << 20
 
 
@@ -113,6 +115,9 @@ def lib() -> ctypes.CDLL:
     L.moe_workspace_size_mxfp8.argtypes = [cfgp]
     L.moe_workspace_size_mxfp8.restype = ctypes.c_size_t
     L.moe_layer_forward_mxfp8.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.moe_workspace_size_shared.argtypes = [cfgp, i32]
+    L.moe_workspace_size_shared.restype = ctypes.c_size_t
+    L.moe_layer_forward_shared.argtypes = [cfgp, i32, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     L.moe_backward_workspace_size.argtypes = [cfgp]
     L.moe_backward_workspace_size.restype = ctypes.c_size_t
     L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, f32, f32, P, ctypes.c_size_t, P, P, P, P, P, P, P, P,
@@ -120,7 +125,7 @@ def lib() -> ctypes.CDLL:
     for n in ["moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
               "moe_convert_bf16_to_f16", "moe_permute_static", "moe_expert_ffn_combine", "moe_aux_coef_update",
               "moe_aux_coef_next", "moe_testing_set_expert_wait", "moe_expert_ffn_segments", "moe_layer_backward",
-              "moe_prepare_mxfp8_weights", "moe_layer_forward_mxfp8"]:
+              "moe_prepare_mxfp8_weights", "moe_layer_forward_mxfp8", "moe_layer_forward_shared"]:
         getattr(L, n).restype = st
     _lib = L
     return L
@@ -262,6 +267,18 @@ def moe_testing_set_expert_wait(wait_ns: int, extra_dependency: int):
     """Test hook: limit of the one-launch expert kernel's waits (0 = default)
     and an amount added to its layer-2 dependency target (> 0: unreachable)."""
     _check("moe_testing_set_expert_wait", lib().moe_testing_set_expert_wait(wait_ns, extra_dependency))
+
+
+def moe_workspace_size_shared(cfg: moe_config, F_shared: int) -> int:
+    return lib().moe_workspace_size_shared(ctypes.byref(cfg), F_shared)
+
+
+def moe_layer_forward_shared(cfg, F_shared, x, Wg, bg, W1, W2, W1_shared, W2_shared, out, stats, ws, stream=None):
+    """The layer plus a shared expert of hidden width F_shared (every token, weight 1)."""
+    _check("moe_layer_forward_shared",
+           lib().moe_layer_forward_shared(ctypes.byref(cfg), F_shared, _ptr(x), _ptr(Wg), _ptr(bg), _ptr(W1),
+                                          _ptr(W2), _ptr(W1_shared), _ptr(W2_shared), _ptr(out), _ptr(stats),
+                                          _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def moe_mxfp8_weight_bytes(cfg: moe_config):

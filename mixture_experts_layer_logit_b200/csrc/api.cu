@@ -289,6 +289,32 @@ moe_status check_mx_config(const moe_config* c) {
   return MOE_OK;
 }
 
+// The layer with a shared expert: the forward workspace, then the shared
+// expert's regions (its config is the layer's with one expert of width Fs
+// over T rows, one row per token).
+struct SharedLayout {
+  moe_ws_layout base;
+  moe_config sc;
+  size_t seg, h, y, scratch, total;
+};
+
+SharedLayout shared_layout(const moe_config& c, int Fs) {
+  SharedLayout L{};
+  L.base = layout_of(c);
+  moe_config one = c;
+  one.E = 1;
+  one.F = Fs;
+  L.sc = segments_config(one, 1, c.T);
+  const size_t hs = c.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  size_t off = L.base.total;
+  L.seg = off;     off = align256(off + 8);
+  L.h = off;       off = align256(off + hs * (size_t)c.T * Fs);
+  L.y = off;       off = align256(off + 4 * (size_t)c.T * c.d);
+  L.scratch = off; off = align256(off + scratch_layout(L.sc).total);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -732,6 +758,51 @@ moe_status moe_layer_forward_mxfp8(const moe_config* cfg, const void* x, const v
   float* yp = at<float>(ws, L.yp);
   if (launch_mx_experts(c, b, W1q, W1s, W2q, W2s, yp, &stats->status, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));
+}
+
+size_t moe_workspace_size_shared(const moe_config* cfg, int32_t F_shared) {
+  if (check_config(cfg) != MOE_OK || F_shared < 1) return 0;
+  moe_config one = *cfg;
+  one.E = 1;
+  one.k = 1;
+  one.F = F_shared;
+  if (check_config(&one) != MOE_OK) return 0;
+  return shared_layout(*cfg, F_shared).total;
+}
+
+moe_status moe_layer_forward_shared(const moe_config* cfg, int32_t F_shared, const void* x, const void* Wg,
+                                    const float* bg, const void* W1, const void* W2, const void* W1_shared,
+                                    const void* W2_shared, void* out, moe_stats* stats, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (F_shared < 1) return MOE_ERR_ARG;
+  moe_config one = c;
+  one.E = 1;
+  one.k = 1;
+  one.F = F_shared;
+  if ((st = check_config(&one)) != MOE_OK) return st;
+  if (c.T > 0 && (W1_shared == nullptr || W2_shared == nullptr)) return MOE_ERR_ARG;
+  if (!aligned16(W1_shared) || !aligned16(W2_shared)) return MOE_ERR_ARG;
+  const SharedLayout L = shared_layout(c, F_shared);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return st;
+  // the routed experts into out, on the front of the workspace
+  if ((st = moe_layer_forward(cfg, x, Wg, bg, W1, W2, out, stats, ws, L.base.total, stream)) != MOE_OK) return st;
+  if (c.T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the shared expert over every token (one segment of T rows, x as the rows), then out += its output
+  int32_t* seg = at<int32_t>(ws, L.seg);
+  if (launch_fill_segment(seg, c.T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const moe_config& sc = L.sc;
+  void* scr = at<char>(ws, L.scratch);
+  if (one_launch_plain(sc))
+    st = expert_mlp_plain(sc, x, seg, W1_shared, W2_shared, at<char>(ws, L.h), at<char>(ws, L.y), stats,
+                          at<int>(scr, scratch_layout(sc).mlp), false, s, 1);
+  else
+    st = expert_ffn(sc, x, seg, W1_shared, W2_shared, at<char>(ws, L.h), at<char>(ws, L.y), stats, s, nullptr, 1);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_add_rows(static_cast<float*>(out), at<float>(ws, L.y), (size_t)c.T * c.d, s));
 }
 
 moe_status moe_testing_set_expert_wait(uint64_t wait_ns, int32_t extra_dependency) {

@@ -64,9 +64,17 @@ struct TileCoord {
   int e, row0, rows, n0;
 };
 
+// m-tiles per group of the second layer's tile order (see decode_tile).
+constexpr int kL2Group = 8;
+
 // Tile L of the table: expert, first permuted row, rows inside the expert's
 // segment (up to TM) and first output column.  Within an expert the m-tiles
-// of one n-tile are consecutive.
+// of one n-tile are consecutive, so the CTAs running at the same time share
+// a weight tile in L2.  For the second layer (K = F, long rows of h) the
+// expert's m-tiles go in groups of kL2Group: all n-tiles of a group before
+// the next group.  A wave of tiles then reads about as many h rows as weight
+// rows (a 2-D block of the output) instead of every h row of the expert for
+// a few weight tiles, and stays inside L2.
 template <int MODE, int TM>
 __device__ __forceinline__ TileCoord decode_tile(const int* tstart, const int32_t* offsets, int E, int L) {
   TileCoord c;
@@ -75,7 +83,18 @@ __device__ __forceinline__ TileCoord decode_tile(const int* tstart, const int32_
   const int M = offsets[c.e + 1] - seg0;
   const int mt = (M + TM - 1) / TM;
   const int local = L - tstart[c.e];
-  const int nti = local / mt, mti = local - nti * mt;
+  int nti, mti;
+  if ((MODE == kPlain || MODE == kCombine) && mt > kL2Group) {
+    const int nt = (tstart[c.e + 1] - tstart[c.e]) / mt;
+    const int grp = local / (kL2Group * nt);
+    const int gsize = min(kL2Group, mt - grp * kL2Group);
+    const int rem = local - grp * kL2Group * nt;
+    nti = rem / gsize;
+    mti = grp * kL2Group + (rem - nti * gsize);
+  } else {
+    nti = local / mt;
+    mti = local - nti * mt;
+  }
   c.row0 = seg0 + mti * TM;
   c.rows = min(TM, M - mti * TM);
   c.n0 = nti * (MODE == kSwiglu ? BN / 2 : BN);

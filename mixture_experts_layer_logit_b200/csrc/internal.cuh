@@ -57,6 +57,10 @@ cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, 
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
 // *z_loss = sum over chunks of zsum / T (fixed order).
 cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s);
+// seg[0] = 0, seg[1] = rows (the shared expert's single segment)
+cudaError_t launch_fill_segment(int32_t* seg, int rows, cudaStream_t s);
+// out[i] += add[i] for n floats (n a multiple of 4)
+cudaError_t launch_add_rows(float* out, const float* add, size_t n, cudaStream_t s);
 // *coef = beta * *coef + (1 - beta) * xi * stats->drop_rate (one thread).
 cudaError_t launch_aux_coef_update(const moe_stats* stats, float* coef, float beta, float xi, cudaStream_t s);
 // Histogram of topk_idx per chunk (+ near ties from gap when given).

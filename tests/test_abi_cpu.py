@@ -235,3 +235,23 @@ def test_adaptive_aux_coef_rejects_bad_values(L, args):
     assert L.moe_aux_coef_next(ctypes.c_float(0.1), ctypes.c_float(0.2), ctypes.c_float(0.9), ctypes.c_float(1.0),
                                None) == 1
     assert L.moe_aux_coef_update(None, None, ctypes.c_float(0.9), ctypes.c_float(1.0), None) == 1
+
+
+def test_shared_expert_workspace_sizes(L):
+    cfg = moe.make_config(64, 128, 4, 128, 2, "relu")
+    assert moe.moe_workspace_size_shared(cfg, 0) == 0
+    assert moe.moe_workspace_size_shared(cfg, 100) == 0          # not a multiple of 16 on the bf16 path
+    assert moe.moe_workspace_size_shared(cfg, 128) > moe.moe_workspace_size(cfg)[0]
+
+
+def test_mxfp8_shapes(L):
+    ok = moe.make_config(64, 2048, 64, 1408, 6, "swiglu")
+    n, (a, b, c, d) = moe.moe_mxfp8_weight_bytes(ok)
+    assert a == 64 * 2816 * 2048 and c == 64 * 2048 * 1408
+    assert b == a // 32 and d == c // 32 and n == a + b + c + d
+    assert moe.moe_workspace_size_mxfp8(ok) > moe.moe_workspace_size(ok)[0]
+    for bad in [moe.make_config(64, 192, 4, 256, 2, "relu"),               # d not a multiple of 128
+                moe.make_config(64, 256, 4, 192, 2, "relu"),               # F not a multiple of 128
+                moe.make_config(64, 256, 4, 256, 2, "relu", dtype="f32")]:
+        assert moe.moe_workspace_size_mxfp8(bad) == 0
+        assert moe.moe_mxfp8_weight_bytes(bad)[0] == 0
