@@ -77,6 +77,31 @@ def mxq(a: np.ndarray) -> np.ndarray:
     return mx_quantize(a)[0]
 
 
+def near_decisions(a: np.ndarray, rel: float = 1e-4) -> np.ndarray:
+    """Rows of `a` whose quantisation takes a decision within `rel` (relative)
+    of its boundary: a block maximum near 1.75 * 2^k (where the exponent X
+    changes) or an element near a rounding midpoint of the E4M3 grid.  An
+    fp32 computation of `a` may take the other side there (both are correct
+    roundings of nearly the same value); the parity tests count such rows
+    apart, as the routing tests do with near ties."""
+    a = np.asarray(a, np.float64)
+    R, n = a.shape
+    blocks = a.reshape(R, n // BLOCK, BLOCK)
+    amax = np.max(np.abs(blocks), axis=-1)
+    near = np.zeros(R, dtype=bool)
+    with np.errstate(divide="ignore"):
+        k = np.round(np.log2(np.where(amax > 0, amax / 1.75, 1.0)))
+    edge = 1.75 * np.exp2(k)
+    near |= np.any((amax > 0) & (np.abs(amax - edge) <= rel * amax), axis=1)
+    X = np.vectorize(mx_scale_exponent, otypes=[np.int64])(amax) if amax.size else amax.astype(np.int64)
+    y = np.abs(blocks) / np.exp2(X.astype(np.float64))[..., None]
+    e = np.maximum(np.floor(np.log2(np.where(y > 0, y, 1.0))), -6.0)
+    step = np.exp2(e - 3.0)
+    frac = y / step - np.floor(y / step)           # position inside a grid step; 0.5 is a midpoint
+    near |= np.any((y > 0) & (np.abs(frac - 0.5) * step <= rel * y), axis=(1, 2))
+    return near
+
+
 class MXExperts:
     """Lazy dequantised view of stacked expert weights (each row quantised
     along its last axis): ``a[e]`` is expert e's matrix after the round trip."""
@@ -100,18 +125,23 @@ def expert_ffn_mx(xe, w1qe, w2qe, act: str, F: int) -> np.ndarray:
 
 def forward(x, wg, bias, w1, w2, cfg: om.LayerConfig, forced_mask=None, forced_idx=None) -> om.Forward:
     """The layer with MX FP8 expert weights: routing and permutation as the
-    bf16 layer; each expert's MLP on quantised inputs, weights and hidden."""
+    bf16 layer; each expert's MLP on quantised inputs, weights and hidden.
+    The returned Forward's ``h`` holds, per permuted row, whether its hidden
+    activation's quantisation sits near a decision boundary (near_decisions)."""
     x = np.asarray(x, np.float64)
     r = om.route(x, wg, bias, cfg, forced_mask, forced_idx)
     dsp = om.dispatch(r.idx, cfg, r.prob_mean)
     yp = np.zeros((int(dsp.offsets[-1]), cfg.d))
+    near = np.zeros(int(dsp.offsets[-1]), dtype=bool)
     w1q, w2q = MXExperts(w1), MXExperts(w2)
     for e in range(cfg.E):
         a, b = int(dsp.offsets[e]), int(dsp.offsets[e + 1])
         if a < b:
-            yp[a:b] = expert_ffn_mx(x[dsp.src_tok[a:b]], w1q[e], w2q[e], cfg.act, cfg.F)
+            h = om.expert_hidden(mxq(x[dsp.src_tok[a:b]]), w1q[e], cfg.act, cfg.F)
+            near[a:b] = near_decisions(h)
+            yp[a:b] = mxq(h) @ np.asarray(w2q[e], np.float64).T
     out = om.combine(yp, dsp.row_of, r.w, cfg.T, cfg.d)
-    return om.Forward(routing=r, dispatch=dsp, out=out, yp=yp)
+    return om.Forward(routing=r, dispatch=dsp, out=out, yp=yp, h=near)
 
 
 def forward_tokens(x, w1, w2, cfg: om.LayerConfig, r: om.Routing, dsp: om.Dispatch, tokens) -> np.ndarray:

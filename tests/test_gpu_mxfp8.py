@@ -7,8 +7,11 @@ moe_layer_forward_mxfp8) against the float64 MX oracle (oracle/moe_fp8.py).
   decisions: the block exponent and round-to-nearest-even to the E4M3 grid).
 * The forward matches the MX oracle within 2e-2 * RMS(out): the oracle
   quantises the input rows and the hidden activation the same way, so what
-  differs is fp32 accumulation and the rare hidden value whose fp32 and
-  float64 values round to neighbouring E4M3 values.
+  differs is fp32 accumulation -- and, on a token whose hidden activation has
+  a value within 1e-4 (relative) of a quantisation boundary, possibly the
+  other (equally correct) rounding of it.  Such tokens are the FP8 path's
+  near ties: counted, held to 5 % of the tokens, and left out of the
+  element-wise comparison, as the routing tests do with near-tie scores.
 * Routing, permutation and statistics are the bf16 layer's, compared exactly
   off near ties."""
 import numpy as np
@@ -20,7 +23,7 @@ import mixture_experts_layer_logit_b200 as moe
 import oracle
 from oracle import moe_oracle as om
 from oracle import moe_fp8 as mf
-from tests.gpu_harness import check_routing, check_out, to_np64
+from tests.gpu_harness import check_routing, to_np64
 
 pytestmark = pytest.mark.gpu
 
@@ -82,7 +85,7 @@ def test_prepared_weights_equal_the_oracle_quantisation(w):
         assert np.array_equal(W2[e], mf.mxq(mw.to_f64(inp.w2[e]))), f"W2[{e}]"
 
 
-def run_mx(w, sample=0):
+def run_mx(w):
     inp = mw.generate(w)
     cfg, (w1q, w1s, w2q, w2s) = _prepare(w, inp)
     x, wg, bias = mw.to_device(inp.x), mw.to_device(inp.wg), mw.to_device(inp.bias)
@@ -105,12 +108,19 @@ def run_mx(w, sample=0):
     d = om.dispatch(r.idx, lc, r.prob_mean)
     assert st["drop_count"] == d.drop_count and st["rows_kept"] == int(d.offsets[-1])
     w1, w2 = mw.F64Experts(inp.w1), mw.F64Experts(inp.w2)
-    if sample:
-        toks = np.unique(np.concatenate([np.random.default_rng(0).choice(T, sample, replace=False), [0, T - 1]]))
-        ref = mf.forward_tokens(xx, w1, w2, lc, r, d, toks)
-        return check_out(to_np64(out[torch.from_numpy(toks).cuda()]), ref, mw.BF16)
     fw = mf.forward(xx, wgg, inp.bias, w1, w2, lc, forced if n_tie else None, idx if n_tie else None)
-    return check_out(to_np64(out), fw.out, mw.BF16)
+    near_rows = fw.h
+    near_tok = np.zeros(T, dtype=bool)
+    for j in range(w.k):
+        r_ = fw.dispatch.row_of[:, j]
+        near_tok |= (r_ >= 0) & near_rows[np.maximum(r_, 0)]
+    assert near_tok.sum() <= max(2, 0.05 * T), f"{near_tok.sum()} near-tie tokens"
+    keep = ~near_tok
+    o = to_np64(out)
+    rms = float(np.sqrt(np.mean(fw.out ** 2)))
+    err = float(np.max(np.abs(o[keep] - fw.out[keep]))) if keep.any() else 0.0
+    assert err <= 2e-2 * rms, f"max|err| {err:.3e} > 2e-2 * RMS {rms:.3e} ({near_tok.sum()} near-tie tokens out)"
+    return err / rms
 
 
 @pytest.mark.parametrize("w", LAYERS, ids=[w.name for w in LAYERS])

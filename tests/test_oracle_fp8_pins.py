@@ -116,6 +116,23 @@ def check_exact_layer():
     return bad
 
 
+def check_near_decisions():
+    """A value just off a rounding midpoint or a block maximum just off
+    1.75 * 2^k is flagged; a value on the grid is not."""
+    bad = []
+    base = np.full((3, 32), 1.0)
+    base[1, 5] = 1.0625 * (1 + 1e-6)     # a midpoint (between 1 and 1.125 at X = -8 scaled) ...
+    base[2, 0] = 1.75 * (1 - 1e-6)       # ... and a block maximum just under 1.75
+    got = mf.near_decisions(base * 1.0)
+    if got.tolist() != [False, True, True]:
+        bad.append(f"near_decisions {got.tolist()}")
+    return bad
+
+
+def test_near_decisions():
+    assert check_near_decisions() == []
+
+
 def _all():
     return check_grid() + check_scales() + check_blocks() + check_exact_layer()
 
