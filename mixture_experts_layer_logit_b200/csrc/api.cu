@@ -675,7 +675,11 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* 
       if (launch_convert_bf16_f16(W1, b.w1h, (size_t)c.E * F1 * c.d, s) != cudaSuccess) return MOE_ERR_CUDA;
       w1 = b.w1h;
     }
-    e = launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u, b.status, b.f16, s);
+    // the recomputed pre-activation on 2-SM pair tiles when the segments are long, as the forward's layer 1
+    e = pair_tiles(c) ? launch_grouped_plain_tc_pair(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u,
+                                                     b.status, b.f16, s)
+                      : launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u, b.status,
+                                                b.f16, s);
     if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, w1, W2, dW1, dW2, s);
   } else {
     e = launch_grouped_plain_simt(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);

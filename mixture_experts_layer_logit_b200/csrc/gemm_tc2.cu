@@ -270,6 +270,22 @@ cudaError_t launch_layers(const moe_config& c, const void* xp, const int32_t* of
 
 }  // namespace
 
+cudaError_t launch_grouped_plain_tc_pair(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                         const void* B, int K, int Nout, float* out, uint32_t* status, bool f16,
+                                         cudaStream_t s) {
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, (uint64_t)rows_alloc, (uint64_t)K, f16) ||
+      !make_map(&mb, B, (uint64_t)c.E * Nout, (uint64_t)K, f16))
+    return cudaErrorInvalidValue;
+  Params p{offsets, out, c.E, K, Nout, Nout, 0, rows_alloc, status};
+  const long long tiles = ((long long)rows_alloc / PM + c.E) * ((Nout + BN - 1) / BN);
+  const int pairs = (int)std::min<long long>(tiles, std::max(1, di.sms / 2));
+  return f16 ? launch_one<kPlain, true>(ma, mb, p, pairs, s) : launch_one<kPlain, false>(ma, mb, p, pairs, s);
+}
+
 cudaError_t launch_expert_ffn_tc_pair(const moe_config& c, const void* xp, const int32_t* offsets,
                                       const void* w1, const void* w2, void* h, void* yp,
                                       uint32_t* status, cudaStream_t s, const CombineOut* comb, int e_mod) {

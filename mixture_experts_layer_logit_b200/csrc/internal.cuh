@@ -171,6 +171,9 @@ cudaError_t launch_expert_backward_simt(const moe_config& c, const BwdState& st,
 cudaError_t launch_grouped_plain_tc(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
                                     const void* B, int K, int Nout, float* out, uint32_t* status, bool f16,
                                     cudaStream_t s);
+cudaError_t launch_grouped_plain_tc_pair(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
+                                         const void* B, int K, int Nout, float* out, uint32_t* status, bool f16,
+                                         cudaStream_t s);
 cudaError_t launch_grouped_plain_simt(const moe_config& c, const void* A, const int32_t* offsets, int rows_alloc,
                                       const void* B, int K, int Nout, float* out, uint32_t* status, cudaStream_t s);
 // the gate's gradient (logits recomputed), dx and dW_gate / db

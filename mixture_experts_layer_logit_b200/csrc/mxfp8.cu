@@ -92,12 +92,12 @@ struct RowMapSwiglu {   // destination row of an expert's interleaved W1 -> sour
     return e * F1 + (j < 64 ? 64 * b + j : F + 64 * b + (j - 64));
   }
 };
-struct RowMapPadded {   // padded activation row -> kept permuted row
+struct RowMapPadded {   // padded activation row -> kept permuted row (-1: padding; -2: past the last segment)
   const int32_t* offsets;
   const int32_t* pad;
   int E;
   __device__ int operator()(int r) const {
-    if (r >= pad[E]) return -1;
+    if (r >= pad[E]) return -2;
     int lo = 0, hi = E - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -119,6 +119,7 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map m
   for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += (size_t)gridDim.x * blockDim.x) {
     const int r = (int)(b / nb), kb = (int)(b - (size_t)r * nb);
     const int sr = map(r);
+    if (sr == -2) continue;   // no tile reads rows past the last segment
     float v[32];
     if (sr >= 0) {
       const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)sr * K + 32 * kb);
@@ -150,17 +151,34 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map m
   }
 }
 
-// Padded offsets: every expert's kept rows rounded up to a multiple of 128.
+// Padded offsets: every expert's kept rows rounded up to a multiple of 128
+// (one warp; 8 experts per lane, then a shuffle scan).
 __global__ void mx_pad_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad) {
   pdl_wait();
   pdl_launch_dependents();
-  if (threadIdx.x != 0) return;
-  int run = 0;
-  for (int e = 0; e < E; ++e) {
-    pad[e] = run;
-    run += (offsets[e + 1] - offsets[e] + kMxPad - 1) / kMxPad * kMxPad;
+  constexpr int PER = kMaxExperts / 32;
+  const int lane = threadIdx.x;
+  int loc[PER], sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    loc[i] = (e < E) ? (offsets[e + 1] - offsets[e] + kMxPad - 1) / kMxPad * kMxPad : 0;
+    sum += loc[i];
   }
-  pad[E] = run;
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane * PER + i;
+    if (e < E) pad[e] = run;
+    run += loc[i];
+  }
+  if (lane == 31) pad[E] = incl;
 }
 
 struct MxParams {

@@ -77,29 +77,52 @@ def mxq(a: np.ndarray) -> np.ndarray:
     return mx_quantize(a)[0]
 
 
-def near_decisions(a: np.ndarray, rel: float = 1e-4) -> np.ndarray:
-    """Rows of `a` whose quantisation takes a decision within `rel` (relative)
-    of its boundary: a block maximum near 1.75 * 2^k (where the exponent X
-    changes) or an element near a rounding midpoint of the E4M3 grid.  An
-    fp32 computation of `a` may take the other side there (both are correct
-    roundings of nearly the same value); the parity tests count such rows
-    apart, as the routing tests do with near ties."""
-    a = np.asarray(a, np.float64)
-    R, n = a.shape
-    blocks = a.reshape(R, n // BLOCK, BLOCK)
-    amax = np.max(np.abs(blocks), axis=-1)
-    near = np.zeros(R, dtype=bool)
-    with np.errstate(divide="ignore"):
-        k = np.round(np.log2(np.where(amax > 0, amax / 1.75, 1.0)))
-    edge = 1.75 * np.exp2(k)
-    near |= np.any((amax > 0) & (np.abs(amax - edge) <= rel * amax), axis=1)
-    X = np.vectorize(mx_scale_exponent, otypes=[np.int64])(amax) if amax.size else amax.astype(np.int64)
-    y = np.abs(blocks) / np.exp2(X.astype(np.float64))[..., None]
-    e = np.maximum(np.floor(np.log2(np.where(y > 0, y, 1.0))), -6.0)
-    step = np.exp2(e - 3.0)
-    frac = y / step - np.floor(y / step)           # position inside a grid step; 0.5 is a midpoint
-    near |= np.any((y > 0) & (np.abs(frac - 0.5) * step <= rel * y), axis=(1, 2))
-    return near
+def hidden_window(xq: np.ndarray, w1q: np.ndarray, act: str, F: int, rel: float) -> np.ndarray:
+    """How far a finite-precision evaluation of one expert's hidden activation
+    may sit from the exact one, per element, when each pre-activation carries
+    an absolute error of at most rel * sum_i |xq_i w1q_i| (a dot product
+    accumulated in floating point) and the activation itself a relative one
+    of rel.  ReLU is 1-Lipschitz; for SwiGLU h = silu(g) up, |silu'| <= 1.1,
+    so |dh| <= 1.1 dg (|up| + dup) + |silu(g)| dup (expert_hidden gives the
+    two activations)."""
+    xq = np.asarray(xq, np.float64)
+    w1q = np.asarray(w1q, np.float64)
+    u = xq @ w1q.T
+    du = rel * (np.abs(xq) @ np.abs(w1q).T)
+    h = om.expert_hidden(xq, w1q, act, F)
+    if act == om.RELU:
+        return du + rel * np.abs(h)
+    g, up = u[:, :F], u[:, F:2 * F]
+    dg, dup = du[:, :F], du[:, F:2 * F]
+    with np.errstate(over="ignore"):
+        s = g / (1.0 + np.exp(-g))
+    return 1.1 * dg * (np.abs(up) + dup) + np.abs(s) * dup + rel * np.abs(h)
+
+
+def admits(hd: np.ndarray, Xd: np.ndarray, h: np.ndarray, window: np.ndarray):
+    """Whether the MX values hd (blocks of 32 along the last axis, block
+    exponents Xd) are the quantisation of SOME h' with |h' - h| <= window
+    element-wise.  Both decisions are monotone in the value: the block
+    exponent in the block maximum, the E4M3 rounding in the element, so h'
+    ranges over an interval and hd must lie between the quantisations of its
+    ends.  Returns (admitted, differs): per element, whether hd is admitted
+    and whether it differs from the quantisation of h itself."""
+    hd = np.asarray(hd, np.float64)
+    h = np.asarray(h, np.float64)
+    w = np.asarray(window, np.float64)
+    R, n = h.shape
+    nb = n // BLOCK
+    hb, wb, db = (a.reshape(R, nb, BLOCK) for a in (h, w, hd))
+    lo = np.max(np.maximum(np.abs(hb) - wb, 0.0), axis=-1)
+    hi = np.max(np.abs(hb) + wb, axis=-1)
+    Xs = np.vectorize(mx_scale_exponent, otypes=[np.int64])
+    Xd = np.asarray(Xd, np.int64).reshape(R, nb)
+    block_ok = (Xs(lo) <= Xd) & (Xd <= Xs(hi))
+    sc = np.exp2(Xd.astype(np.float64))[..., None]
+    q = db / sc
+    el_ok = (e4m3_round((hb - wb) / sc) <= q) & (q <= e4m3_round((hb + wb) / sc))
+    admitted = (el_ok & block_ok[..., None]).reshape(R, n)
+    return admitted, hd != mxq(h)
 
 
 class MXExperts:
@@ -126,22 +149,35 @@ def expert_ffn_mx(xe, w1qe, w2qe, act: str, F: int) -> np.ndarray:
 def forward(x, wg, bias, w1, w2, cfg: om.LayerConfig, forced_mask=None, forced_idx=None) -> om.Forward:
     """The layer with MX FP8 expert weights: routing and permutation as the
     bf16 layer; each expert's MLP on quantised inputs, weights and hidden.
-    The returned Forward's ``h`` holds, per permuted row, whether its hidden
-    activation's quantisation sits near a decision boundary (near_decisions)."""
+    The returned Forward's ``h`` holds, per permuted row, the hidden
+    activation before its quantisation."""
     x = np.asarray(x, np.float64)
     r = om.route(x, wg, bias, cfg, forced_mask, forced_idx)
     dsp = om.dispatch(r.idx, cfg, r.prob_mean)
     yp = np.zeros((int(dsp.offsets[-1]), cfg.d))
-    near = np.zeros(int(dsp.offsets[-1]), dtype=bool)
+    hid = np.zeros((int(dsp.offsets[-1]), cfg.F))
     w1q, w2q = MXExperts(w1), MXExperts(w2)
     for e in range(cfg.E):
         a, b = int(dsp.offsets[e]), int(dsp.offsets[e + 1])
         if a < b:
             h = om.expert_hidden(mxq(x[dsp.src_tok[a:b]]), w1q[e], cfg.act, cfg.F)
-            near[a:b] = near_decisions(h)
+            hid[a:b] = h
             yp[a:b] = mxq(h) @ np.asarray(w2q[e], np.float64).T
     out = om.combine(yp, dsp.row_of, r.w, cfg.T, cfg.d)
-    return om.Forward(routing=r, dispatch=dsp, out=out, yp=yp, h=near)
+    return om.Forward(routing=r, dispatch=dsp, out=out, yp=yp, h=hid)
+
+
+def hidden_windows(x, w1, cfg: om.LayerConfig, dsp: om.Dispatch, rel: float) -> np.ndarray:
+    """hidden_window for every permuted row of the layer (rows grouped by
+    expert as dsp orders them)."""
+    x = np.asarray(x, np.float64)
+    out = np.zeros((int(dsp.offsets[-1]), cfg.F))
+    w1q = MXExperts(w1)
+    for e in range(cfg.E):
+        a, b = int(dsp.offsets[e]), int(dsp.offsets[e + 1])
+        if a < b:
+            out[a:b] = hidden_window(mxq(x[dsp.src_tok[a:b]]), w1q[e], cfg.act, cfg.F, rel)
+    return out
 
 
 def forward_tokens(x, w1, w2, cfg: om.LayerConfig, r: om.Routing, dsp: om.Dispatch, tokens) -> np.ndarray:

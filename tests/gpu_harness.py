@@ -180,13 +180,16 @@ def check_dispatch_exact(dev: dict, d: om.Dispatch, r: om.Routing, dev_idx: np.n
     assert key_dev == key_ref, "row_of / drop mask"
 
 
-def check_out(out_dev: np.ndarray, out_ref: np.ndarray, dtype: str):
+def check_out(out_dev: np.ndarray, out_ref: np.ndarray, dtype: str, tol=BF16_TOL):
+    """max|err| against the bar of the path's type: bf16 paths within tol *
+    RMS(out) (tol None: measured, not asserted), fp32 paths within F32_TOL *
+    max|out|.  Returns the error over the bar's scale."""
     if out_ref.size == 0:
         return 0.0
     err = np.max(np.abs(out_dev - out_ref))
     if dtype == mw.BF16:
         rms = float(np.sqrt(np.mean(out_ref ** 2)))
-        assert err <= BF16_TOL * rms, f"max|err| {err:.3e} > {BF16_TOL} * RMS {rms:.3e}"
+        assert tol is None or err <= tol * rms, f"max|err| {err:.3e} > {tol} * RMS {rms:.3e}"
         return err / rms
     scale = float(np.max(np.abs(out_ref)))
     assert err <= F32_TOL * scale, f"max|err| {err:.3e} > {F32_TOL} * max|ref| {scale:.3e}"

@@ -10,6 +10,11 @@
 * A layer whose inputs and weights are small integers, so that every
   quantised tensor is exactly representable, gives the bf16 oracle's output
   exactly.
+* The parity tests' admission of a device quantisation (admits): a value
+  just off a rounding midpoint admits both neighbours only when the window
+  covers the midpoint, never a value two steps away, and likewise the block
+  exponent at the 448 * 2^X edge; hidden_window bounds sampled perturbations
+  of the pre-activations and is reached to within a factor ~3.
 * Planted mistakes (ties away from zero, the saturating floor-based scale,
   blocks along the wrong axis) each fail a pin."""
 import math
@@ -116,25 +121,93 @@ def check_exact_layer():
     return bad
 
 
-def check_near_decisions():
-    """A value just off a rounding midpoint or a block maximum just off
-    1.75 * 2^k is flagged; a value on the grid is not."""
+def check_admits():
+    """The admission check of a device quantisation (admits): in a block with
+    maximum 1.75 (X = -8 exactly, 1.75 = 448 * 2^-8), 1.0625 is the midpoint
+    of the grid neighbours 1.0 and 1.125.  Just above it, a zero window admits
+    only 1.125; a window that covers the midpoint admits both, never a value
+    two steps away.  A block maximum just above 1.75 takes X = -7; a zero
+    window rejects X = -8, one that reaches below 1.75 admits it.  Signs are
+    symmetric."""
     bad = []
-    base = np.full((3, 32), 1.0)
-    base[1, 5] = 1.0625 * (1 + 1e-6)     # a midpoint (between 1 and 1.125 at X = -8 scaled) ...
-    base[2, 0] = 1.75 * (1 - 1e-6)       # ... and a block maximum just under 1.75
-    got = mf.near_decisions(base * 1.0)
-    if got.tolist() != [False, True, True]:
-        bad.append(f"near_decisions {got.tolist()}")
+    h = np.full((1, 32), 0.5)
+    h[0, 0] = 1.75
+    h[0, 1] = 1.0625 * (1 + 1e-6)
+    h[0, 2] = -1.0625 * (1 + 1e-6)
+    q, X = mf.mx_quantize(h)
+    if X.tolist() != [[-8]] or q[0, 1] != 1.125 or q[0, 2] != -1.125:
+        bad.append(f"admits setup {X.tolist()} {q[0, :3].tolist()}")
+    zero, wide = np.zeros_like(h), np.full_like(h, 1e-5)
+    ok, diff = mf.admits(q, X, h, zero)
+    if not ok.all() or diff.any():
+        bad.append("admits: the quantisation of h itself")
+    for col, alt in ((1, 1.0), (2, -1.0)):
+        other = q.copy()
+        other[0, col] = alt
+        ok0, _ = mf.admits(other, X, h, zero)
+        okw, dw = mf.admits(other, X, h, wide)
+        if ok0[0, col] or not okw[0, col] or not dw[0, col] or dw.sum() != 1:
+            bad.append(f"admits: other neighbour of the midpoint (col {col})")
+        far = q.copy()
+        far[0, col] = 1.25 if alt > 0 else -1.25
+        if mf.admits(far, X, h, wide)[0][0, col]:
+            bad.append(f"admits: two steps away (col {col})")
+    hb = h.copy()
+    hb[0, 0] = 1.75 * (1 + 1e-6)
+    qb, Xb = mf.mx_quantize(hb)
+    if Xb.tolist() != [[-7]]:
+        bad.append(f"admits: X just above the edge {Xb.tolist()}")
+    if not mf.admits(qb, Xb, hb, zero)[0].all():
+        bad.append("admits: X = -7 with a zero window")
+    q8 = np.clip(hb, -1.75, 1.75)
+    q8 = mf.e4m3_round(q8 / 2.0 ** -8) * 2.0 ** -8
+    if mf.admits(q8, np.array([[-8]]), hb, zero)[0].any():
+        bad.append("admits: X = -8 with a zero window")
+    if not mf.admits(q8, np.array([[-8]]), hb, wide)[0].all():
+        bad.append("admits: X = -8 with a window below the edge")
     return bad
 
 
-def test_near_decisions():
-    assert check_near_decisions() == []
+def check_hidden_window():
+    """hidden_window bounds the hidden activation of every perturbation of
+    the pre-activations within rel * sum |x w| (sampled at the corners, where
+    the bound is approached), for ReLU and SwiGLU; with rel = 0 it is 0."""
+    bad = []
+    rng = np.random.default_rng(7)
+    x = mf.mxq(rng.standard_normal((6, 64)))
+    for act, F1 in ((om.RELU, 32), (om.SWIGLU, 64)):
+        F = 32
+        w = mf.mxq(rng.standard_normal((F1, 64)) / 4)
+        rel = 1e-3
+        win = mf.hidden_window(x, w, act, F, rel)
+        if np.any(mf.hidden_window(x, w, act, F, 0.0) != 0):
+            bad.append(f"hidden_window {act}: rel = 0")
+        u = x @ w.T
+        du = rel * (np.abs(x) @ np.abs(w).T)
+        h = om.expert_hidden(x, w, act, F)
+        worst = 0.0
+        for _ in range(64):
+            sgn = rng.choice([-1.0, 1.0], size=u.shape)
+            up = u + sgn * du
+            hp = np.maximum(up, 0) if act == om.RELU else \
+                up[:, :F] / (1 + np.exp(-up[:, :F])) * up[:, F:]
+            worst = max(worst, float(np.max(np.abs(hp - h) / np.maximum(win, 1e-300))))
+        # the perturbation reaches a good part of the bound, never past it
+        if not 0.3 < worst <= 1.0:
+            bad.append(f"hidden_window {act}: worst ratio {worst:.3f}")
+    return bad
+
+
+def test_admits():
+    assert check_admits() == []
+
+
+def test_hidden_window():
+    assert check_hidden_window() == []
 
 
 def _all():
-    return check_grid() + check_scales() + check_blocks() + check_exact_layer()
+    return check_grid() + check_scales() + check_blocks() + check_exact_layer() + check_admits()
 
 
 def test_grid():
