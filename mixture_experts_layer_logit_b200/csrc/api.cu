@@ -262,7 +262,7 @@ BwdLayout bwd_layout(const moe_config& c) {
 struct MxLayout {
   moe_ws_layout base;
   int rows_pad;
-  size_t pad, xq, xs, hq, hs, total;
+  size_t pad, xq, xs, hq, hs, ctr, total;
 };
 
 MxLayout mx_layout(const moe_config& c) {
@@ -277,6 +277,7 @@ MxLayout mx_layout(const moe_config& c) {
   L.xs = off;  off = align256(off + mx_scale_bytes(R, (size_t)c.d));
   L.hq = off;  off = align256(off + R * (size_t)c.F);
   L.hs = off;  off = align256(off + mx_scale_bytes(R, (size_t)c.F));
+  L.ctr = off; off = align256(off + 4 * (1 + R / 128));
   L.total = off;
   return L;
 }
@@ -758,7 +759,7 @@ moe_status moe_layer_forward_mxfp8(const moe_config* cfg, const void* x, const v
   if (st != MOE_OK) return st;
   // step 4 on the MX FP8 tensor cores, then step 5
   MxBuffers b{offsets, at<int32_t>(ws, M.pad), at<char>(ws, L.xp), M.rows_pad, at<char>(ws, M.xq),
-              at<char>(ws, M.xs), at<char>(ws, M.hq), at<char>(ws, M.hs)};
+              at<char>(ws, M.xs), at<char>(ws, M.hq), at<char>(ws, M.hs), at<int>(ws, M.ctr)};
   float* yp = at<float>(ws, L.yp);
   if (launch_mx_experts(c, b, W1q, W1s, W2q, W2s, yp, &stats->status, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(launch_combine(c, yp, row_of, w, out, s));

@@ -194,6 +194,7 @@ struct MxBuffers {
   void* xs;                 // scale atoms of xq
   void* hq;                 // [rows_pad][F] E4M3
   void* hs;                 // scale atoms of hq
+  int* ctr;                 // [1 + rows_pad / 128] the expert kernel's tile and dependency counters
 };
 int mx_pad_rows();
 size_t mx_scale_bytes(size_t rows, size_t K);   // rows, K multiples of 128

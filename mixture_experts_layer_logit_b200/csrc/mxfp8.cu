@@ -42,21 +42,30 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = MB * MK, B_BYTES = MN * MK;   // 16 KB each
 constexpr int SF_BYTES = 512;                         // one scale atom per operand
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256;                     // scale columns after the two 128-column accumulators
 constexpr int kMxPad = 128;
+constexpr int kQueue = 4;                             // claimed tiles in flight between the roles
 
-enum { kMxRelu = 0, kMxSwiglu = 1, kMxOut = 2 };
+enum { kMxRelu = 0, kMxSwiglu = 1 };
 
 // Least X with amax <= 448 * 2^X (-127 for 0); the UE8M0 byte is X + 127.
+// From the bit fields: amax = 1.m 2^(E-127), and 448 = 1.75 2^8, so X = E - 135
+// when 1.m <= 1.75 (mantissa bits <= 0x600000), else E - 134.  A subnormal
+// amax (< 2^-126) gives an X below -127, clamped; no finite float gives more
+// than 120.
 __device__ __forceinline__ int mx_exponent(float amax) {
   if (!(amax > 0.f)) return -127;
-  int e;
-  const float m = frexpf(amax, &e);   // amax = m 2^e, m in [0.5, 1)
-  const int X = (2.f * m <= 1.75f) ? e - 9 : e - 8;
-  return max(-127, min(127, X));
+  const uint32_t b = __float_as_uint(amax);
+  const int E = (int)(b >> 23);
+  if (E == 0) return -127;
+  return min(127, E - 135 + ((b & 0x7fffffu) > 0x600000u ? 1 : 0));
 }
+
+// 2^-X as a float, for X in [-127, 120] (exponent field 127 - X in [7, 254]).
+__device__ __forceinline__ float mx_inv_scale(int X) { return __uint_as_float((uint32_t)(127 - X) << 23); }
 
 __device__ __forceinline__ size_t sf_offset(int r, int k, int K) {
   return ((size_t)(r / 128) * (K / 128) + k / 128) * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + (k / 32) % 4;
@@ -64,7 +73,7 @@ __device__ __forceinline__ size_t sf_offset(int r, int k, int K) {
 
 // 32 fp32 values -> 32 E4M3 bytes (scaled by 2^-X), round to nearest even.
 __device__ __forceinline__ void quantize32(const float (&v)[32], int X, uint4& lo, uint4& hi) {
-  const float s = ldexpf(1.f, -X);
+  const float s = mx_inv_scale(X);
   uint32_t w[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -78,33 +87,35 @@ __device__ __forceinline__ void quantize32(const float (&v)[32], int X, uint4& l
   hi = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// One thread per 32-element block of a bf16 matrix [rows][K]: E4M3 bytes and
-// the block's scale.  src_row(r) maps a destination row to its source row
-// (-1: a zero row).  Used for the weights (with the SwiGLU interleave) and
-// for the padded layer-1 input rows.
+// One thread per 32-element block of a bf16 matrix: E4M3 bytes and the
+// block's scale.  The map takes an item (a row index) to (destination row,
+// source row); a negative destination skips the item.  Used for the weights
+// (identity, or the SwiGLU interleave) and for the kept activation rows,
+// which go to their expert's padded segment.  Padding rows stay unwritten:
+// every row of an MMA tile is computed from its own A row only, and no
+// output of a padding row is ever stored as a kept row.
 struct RowMapIdentity {
-  __device__ int operator()(int r) const { return r; }
+  __device__ int2 operator()(int r) const { return make_int2(r, r); }
 };
-struct RowMapSwiglu {   // destination row of an expert's interleaved W1 -> source row
+struct RowMapSwiglu {   // destination row of an expert's interleaved W1 <- source row
   int F;
-  __device__ int operator()(int r) const {
+  __device__ int2 operator()(int r) const {
     const int F1 = 2 * F, e = r / F1, i = r - e * F1, b = i / 128, j = i % 128;
-    return e * F1 + (j < 64 ? 64 * b + j : F + 64 * b + (j - 64));
+    return make_int2(r, e * F1 + (j < 64 ? 64 * b + j : F + 64 * b + (j - 64)));
   }
 };
-struct RowMapPadded {   // padded activation row -> kept permuted row (-1: padding; -2: past the last segment)
+struct RowMapKept {     // kept permuted row i -> its padded row; items past offsets[E] skipped
   const int32_t* offsets;
   const int32_t* pad;
   int E;
-  __device__ int operator()(int r) const {
-    if (r >= pad[E]) return -2;
-    int lo = 0, hi = E - 1;
+  __device__ int2 operator()(int i) const {
+    if (i >= offsets[E]) return make_int2(-1, -1);
+    int lo = 0, hi = E - 1;   // the largest e with offsets[e] <= i holds row i
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (pad[mid] <= r) lo = mid; else hi = mid - 1;
+      if (offsets[mid] <= i) lo = mid; else hi = mid - 1;
     }
-    const int i = r - pad[lo];
-    return i < offsets[lo + 1] - offsets[lo] ? offsets[lo] + i : -1;
+    return make_int2(pad[lo] + (i - offsets[lo]), i);
   }
 };
 
@@ -117,26 +128,22 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map m
   const int nb = K / 32;
   const size_t nblk = (size_t)rows * nb;
   for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += (size_t)gridDim.x * blockDim.x) {
-    const int r = (int)(b / nb), kb = (int)(b - (size_t)r * nb);
-    const int sr = map(r);
-    if (sr == -2) continue;   // no tile reads rows past the last segment
+    const int it = (int)(b / nb), kb = (int)(b - (size_t)it * nb);
+    const int2 m = map(it);
+    if (m.x < 0) continue;
+    const int r = m.x;
     float v[32];
-    if (sr >= 0) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)sr * K + 32 * kb);
+    const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)m.y * K + 32 * kb);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = __ldg(p + i);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = __ldg(p + i);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(h[j]);
-          v[8 * i + 2 * j] = f.x;
-          v[8 * i + 2 * j + 1] = f.y;
-        }
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h[j]);
+        v[8 * i + 2 * j] = f.x;
+        v[8 * i + 2 * j + 1] = f.y;
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
     }
     float amax = 0.f;
 #pragma unroll
@@ -152,12 +159,15 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map m
 }
 
 // Padded offsets: every expert's kept rows rounded up to a multiple of 128
-// (one warp; 8 experts per lane, then a shuffle scan).
-__global__ void mx_pad_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad) {
+// (one warp; 8 experts per lane, then a shuffle scan).  It also zeroes the
+// expert kernel's tile counter and per-m-tile dependency counters.
+__global__ void mx_pad_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad,
+                              int* __restrict__ ctr, int nctr) {
   pdl_wait();
   pdl_launch_dependents();
   constexpr int PER = kMaxExperts / 32;
   const int lane = threadIdx.x;
+  for (int i = lane; i < nctr; i += 32) ctr[i] = 0;
   int loc[PER], sum = 0;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
@@ -183,34 +193,74 @@ __global__ void mx_pad_kernel(const int32_t* __restrict__ offsets, int E, int32_
 
 struct MxParams {
   const int32_t* pad;        // [E+1] padded segment offsets (multiples of 128)
-  const int32_t* offsets;    // [E+1] kept offsets (kMxOut: the unpadded row of each padded row)
-  int E, K, Nout;            // Nout: output columns (layer 1: h columns F; layer 2: d)
-  int b_rows;                // weight rows per expert (F1 or d)
+  const int32_t* offsets;    // [E+1] kept offsets
+  int E, d, F, F1;           // model width, hidden width, layer-1 weight rows per expert (F or 2F)
   int rows_pad;              // padded rows allocated
-  const uint8_t* sfa;        // A scales (activation rows, atoms over K)
-  const uint8_t* sfb;        // B scales (weight rows, atoms over K)
-  uint8_t* hq;               // layer 1: [rows_pad][F] E4M3 h
-  uint8_t* hs;               // layer 1: h scales (atoms over F)
-  float* out;                // kMxOut: yp [rows][d] fp32 at the kept (unpadded) rows
+  const uint8_t* xs;         // layer-1 A scales (the quantised input rows)
+  const uint8_t* w1s;        // layer-1 B scales
+  const uint8_t* w2s;        // layer-2 B scales
+  uint8_t* hq;               // [rows_pad][F] E4M3 h: layer-1 output, layer-2 A
+  uint8_t* hs;               // its scales
+  float* out;                // yp [rows][d] fp32 at the kept (unpadded) rows
   uint32_t* status;
+  int* sched;                // tile counter, zeroed beforehand
+  int* dep;                  // per padded m-tile: layer-1 epilogue warps done; zeroed beforehand
 };
 
 struct MxTail {
   unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  unsigned long long qfull[kQueue], qempty[kQueue];
   uint32_t tmem_base;
   int abort_flag;
-  int tstart[kMaxExperts + 1];
+  int queue[kQueue];
+  int tstart1[kMaxExperts + 1];   // layer-1 tile table
+  int tstart2[kMaxExperts + 1];   // layer-2 tile table
   int seg[kMaxExperts + 1];
+  int cnt[kMaxExperts + 1];       // kept rows of each expert (the rest of its padded segment is padding)
 };
 constexpr size_t kMxSmem = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)STAGES * 2 * SF_BYTES +
                            gemm::kStagingBytes + sizeof(MxTail);
 static_assert(kMxSmem <= 227 * 1024, "shared memory of one CTA");
 
-// MODE kMxRelu / kMxSwiglu: layer 1, h = act(xq W1q^T) quantised into hq/hs;
-// kMxOut: layer 2, yp = hq W2q^T in fp32 at the kept rows.
-template <int MODE>
+struct MxTile {
+  bool l2;
+  int e, row0, n0, m;   // expert, first padded row, first output column (layer 1: weight row), m-tile
+};
+
+// Tile L of the two tables (layer 1 first).  Within an expert the m-tiles of
+// one n-tile are consecutive, so CTAs running at the same time share a weight
+// tile in L2.
+__device__ __forceinline__ MxTile mx_tile(const MxTail* t, int E, int T1, int L) {
+  MxTile r;
+  r.l2 = L >= T1;
+  const int* ts = r.l2 ? t->tstart2 : t->tstart1;
+  const int Ll = r.l2 ? L - T1 : L;
+  r.e = tile_expert(ts, E, Ll);
+  const int mt = (t->seg[r.e + 1] - t->seg[r.e]) / MB;
+  const int local = Ll - ts[r.e];
+  const int nti = local / mt, mti = local - nti * mt;
+  r.row0 = t->seg[r.e] + mti * MB;
+  r.n0 = nti * MN;
+  r.m = r.row0 / MB;
+  return r;
+}
+
+// Both expert layers in one persistent launch, tiles drawn from one counter:
+// every layer-1 tile (h = act(xq W1q^T), quantised in the epilogue), then
+// every layer-2 tile (yp = hq W2q^T in fp32 at the kept rows).  A layer-2
+// tile needs its m-tile's h from every layer-1 n-tile: each epilogue warp of
+// a finished layer-1 tile adds 1 to the m-tile's counter (a release after
+// its stores), and the producer of a layer-2 tile waits for kEpiWarps x nt1
+// (acquire, then a proxy fence so that its TMA and bulk reads see them).
+// Tiles are claimed in increasing order, so a claimed layer-2 tile only
+// waits for layer-1 tiles already claimed by running CTAs, which never wait.
+// Roles: warp 0 claims tiles and issues the TMA and scale loads, warp 1 the
+// scale copies to TMEM and the MMAs, warps 2-9 the epilogue; the claimed
+// tiles pass between them through a 4-slot queue in shared memory.
+template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const MxParams p) {
+tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const MxParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -219,12 +269,12 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   unsigned char* staging = sbase + (size_t)STAGES * STAGE_BYTES + (size_t)STAGES * 2 * SF_BYTES;
   MxTail* tail = reinterpret_cast<MxTail*>(staging + gemm::kStagingBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = (p.b_rows == 0) ? 0 : ((MODE == kMxOut ? p.Nout : (MODE == kMxSwiglu ? 2 * p.Nout : p.Nout)) +
-                                        MN - 1) / MN;
-  const int nkb = p.K / MK;
+  const int nt1 = p.F1 / MN, nt2 = p.d / MN;
+  const int nkb1 = p.d / MK, nkb2 = p.F / MK;
 
   const uint32_t full0 = smem_u32(&tail->full[0]), empty0 = smem_u32(&tail->empty[0]);
   const uint32_t tfull0 = smem_u32(&tail->tfull[0]), tempty0 = smem_u32(&tail->tempty[0]);
+  const uint32_t qfull0 = smem_u32(&tail->qfull[0]), qempty0 = smem_u32(&tail->qempty[0]);
   const uint32_t drain = smem_u32(&tail->drain);
   const volatile int* abort_flag = &tail->abort_flag;
 
@@ -235,7 +285,11 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 4);
+      mbar_init(tempty0 + 8 * a, kEpiWarps);
+    }
+    for (int q = 0; q < kQueue; ++q) {
+      mbar_init(qfull0 + 8 * q, 1);
+      mbar_init(qempty0 + 8 * q, 1 + kEpiWarps);   // the MMA lane and the epilogue warps
     }
     mbar_init(drain, 1);
     tail->abort_flag = 0;
@@ -247,41 +301,54 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA1)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB1)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA2)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB2)) : "memory");
   }
-  pdl_wait();
+  pdl_wait();   // pad[], the quantised rows and the zeroed counters come from earlier kernels
   pdl_launch_dependents();
   if (warp == 0) {
-    if (!tile_table_warp(p.pad, p.E, MB, nt, p.rows_pad, tail->tstart, lane) && lane == 0 && blockIdx.x == 0)
-      atomicOr(p.status, MOE_DEV_BOUNDS);
+    const bool ok1 = tile_table_warp(p.pad, p.E, MB, nt1, p.rows_pad, tail->tstart1, lane);
+    const bool ok2 = tile_table_warp(p.pad, p.E, MB, nt2, p.rows_pad, tail->tstart2, lane);
+    if (!(ok1 && ok2) && lane == 0 && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
   }
-  for (int e = threadIdx.x; e <= p.E; e += kThreads) tail->seg[e] = p.pad[e];
+  for (int e = threadIdx.x; e <= p.E; e += kThreads) {
+    tail->seg[e] = p.pad[e];
+    tail->cnt[e] = (e < p.E) ? p.offsets[e + 1] - p.offsets[e] : 0;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
-  const int total = tail->tstart[p.E];
-
-  auto decode = [&](int L, int& e, int& row0, int& n0) {
-    e = tile_expert(tail->tstart, p.E, L);
-    const int M = tail->seg[e + 1] - tail->seg[e];
-    const int mt = (M + MB - 1) / MB;
-    const int local = L - tail->tstart[e];
-    const int nti = local / mt, mti = local - nti * mt;
-    row0 = tail->seg[e] + mti * MB;
-    n0 = nti * MN;   // weight-row offset inside the expert (SwiGLU: interleaved rows)
-  };
+  const int T1 = tail->tstart1[p.E];
+  const int total = T1 + tail->tstart2[p.E];
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------ TMA producer
+      // ---------------------------------------------- tile claimer + TMA producer
       int it = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        int e, row0, n0;
-        decode(L, e, row0, n0);
-        const int brow = e * p.b_rows + n0;
+      for (int n = 0; ok; ++n) {
+        const int q = n % kQueue;
+        const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
+        if (!mbar_wait(qempty0 + 8 * q, qph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+        int L = atomicAdd(p.sched, 1);
+        if (L >= total) L = -1;
+        tail->queue[q] = L;
+        mbar_arrive(qfull0 + 8 * q);
+        if (L < 0) break;
+        const MxTile t = mx_tile(tail, p.E, T1, L);
+        const CUtensorMap* mA = t.l2 ? &tmA2 : &tmA1;
+        const CUtensorMap* mB = t.l2 ? &tmB2 : &tmB1;
+        const uint8_t* sfa = t.l2 ? p.hs : p.xs;
+        const uint8_t* sfb = t.l2 ? p.w2s : p.w1s;
+        const int brow = t.e * (t.l2 ? p.d : p.F1) + t.n0;
+        const int nkb = t.l2 ? nkb2 : nkb1;
+        if (t.l2) {   // the h rows of this m-tile: every layer-1 n-tile, every epilogue warp
+          if (!wait_flag_geq(p.dep + t.m, kEpiWarps * nt1, abort_flag, kWaitNs)) { ok = false; break; }
+          fence_proxy_async_global();
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -289,10 +356,10 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           const uint32_t sa = base + (uint32_t)(s * STAGE_BYTES);
           const uint32_t sfs = sf_base + (uint32_t)(s * 2 * SF_BYTES);
           mbar_expect_tx(full0 + 8 * s, STAGE_BYTES + 2 * SF_BYTES);
-          tma_load_2d(sa, &tmA, full0 + 8 * s, kb * MK, row0);
-          tma_load_2d(sa + A_BYTES, &tmB, full0 + 8 * s, kb * MK, brow);
-          bulk_load(sfs, p.sfa + ((size_t)(row0 / 128) * nkb + kb) * SF_BYTES, SF_BYTES, full0 + 8 * s);
-          bulk_load(sfs + SF_BYTES, p.sfb + ((size_t)(brow / 128) * nkb + kb) * SF_BYTES, SF_BYTES, full0 + 8 * s);
+          tma_load_2d(sa, mA, full0 + 8 * s, kb * MK, t.row0);
+          tma_load_2d(sa + A_BYTES, mB, full0 + 8 * s, kb * MK, brow);
+          bulk_load(sfs, sfa + ((size_t)(t.row0 / 128) * nkb + kb) * SF_BYTES, SF_BYTES, full0 + 8 * s);
+          bulk_load(sfs + SF_BYTES, sfb + ((size_t)(brow / 128) * nkb + kb) * SF_BYTES, SF_BYTES, full0 + 8 * s);
           ++it;
         }
       }
@@ -300,7 +367,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         atomicOr(p.status, MOE_DEV_TIMEOUT);
         tail->abort_flag = 1;
       }
-      for (int i = max(0, it - STAGES); i < it; ++i)
+      for (int i = max(0, it - STAGES); i < it; ++i)   // loads still in flight
         mbar_wait(full0 + 8 * (i % STAGES), (uint32_t)(i / STAGES) & 1u, nullptr, kDrainNs);
     }
   } else if (warp == 1) {
@@ -308,7 +375,14 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
       // ------------------------------------------------------- MMA issuer
       int it = 0, tl = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++tl) {
+      for (int n = 0; ok; ++n) {
+        const int q = n % kQueue;
+        const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
+        if (!mbar_wait(qfull0 + 8 * q, qph, abort_flag, kWaitNs)) { ok = false; break; }
+        const int L = tail->queue[q];
+        mbar_arrive(qempty0 + 8 * q);
+        if (L < 0) break;
+        const int nkb = (L >= T1) ? nkb2 : nkb1;
         const int acc = tl & 1;
         const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
         if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
@@ -335,6 +409,7 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         }
         if (!ok) break;
         tc_commit(tfull0 + 8 * acc);
+        ++tl;
       }
       if (!ok) {
         atomicOr(p.status, MOE_DEV_TIMEOUT);
@@ -345,55 +420,74 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)(warp - 2) * gemm::kStageWarpBytes);
+    // Eight warps: warp w drains TMEM lane quadrant w % 4; the two warps of a
+    // quadrant split the tile's 32-column blocks.  A warp whose 32 rows are
+    // all padding only takes part in the barriers and the counters (padding
+    // rows are computed from their own A rows and never stored as kept rows).
+    const int qw = warp & 3, half = (warp - 2) >> 2;
+    uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)qw * gemm::kStageWarpBytes);
     int tl = 0;
     bool ok = true;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++tl) {
-      int e, row0, n0;
-      decode(L, e, row0, n0);
+    for (int n = 0;; ++n) {
+      const int q = n % kQueue;
+      const uint32_t qph = (uint32_t)(n / kQueue) & 1u;
+      ok = mbar_wait(qfull0 + 8 * q, qph, abort_flag, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int L = tail->queue[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qempty0 + 8 * q);
+      if (L < 0) break;
+      const MxTile t = mx_tile(tail, p.E, T1, L);
       const int acc = tl & 1;
       const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
       ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kWaitNs);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * MN);
-      const int prow = row0 + q * 32 + lane;   // this thread's padded row
-      if (MODE != kMxOut) {
-        // h columns of the tile: ReLU 128 from n0; SwiGLU 64 from n0 / 2 (gate then up in TMEM)
-        const int hcols = (MODE == kMxSwiglu) ? MN / 2 : MN;
-        const int h0 = (MODE == kMxSwiglu) ? n0 / 2 : n0;
+      const uint32_t tb = tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * MN);
+      const int local0 = t.row0 - tail->seg[t.e] + qw * 32;   // first row of this warp inside the expert
+      const bool live = local0 < tail->cnt[t.e];
+      const int prow = t.row0 + qw * 32 + lane;                // this thread's padded row
+      if (!t.l2) {
+        // h columns of the tile: ReLU 128 from n0 (4 blocks); SwiGLU 64 from
+        // n0 / 2 (2 blocks; gate columns, then the up columns MN / 2 further)
+        constexpr int kBlk = (ACT == kMxSwiglu) ? MN / 64 : MN / 32;
+        const int h0 = (ACT == kMxSwiglu) ? t.n0 / 2 : t.n0;
+        if (live) {
 #pragma unroll 1
-        for (int blk = 0; blk < hcols / 32; ++blk) {
-          uint32_t a[32], u[32];
-          tmem_ld32(tb + blk * 32, a);
-          if (MODE == kMxSwiglu) tmem_ld32(tb + MN / 2 + blk * 32, u);
-          tmem_wait_ld();
-          float h[32];
-          float amax = 0.f;
+          for (int blk = half; blk < kBlk; blk += 2) {
+            uint32_t a[32], u[32];
+            tmem_ld32(tb + blk * 32, a);
+            if (ACT == kMxSwiglu) tmem_ld32(tb + MN / 2 + blk * 32, u);
+            tmem_wait_ld();
+            float h[32];
+            float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(a[i]);
-            h[i] = (MODE == kMxSwiglu) ? g / (1.f + __expf(-g)) * __uint_as_float(u[i]) : fmaxf(g, 0.f);
-            amax = fmaxf(amax, fabsf(h[i]));
-          }
-          const int X = mx_exponent(amax);
-          uint4 lo, hi;
-          quantize32(h, X, lo, hi);
-          const int c = h0 + blk * 32;
-          if (c < p.Nout && prow < p.rows_pad) {
-            uint4* dst = reinterpret_cast<uint4*>(p.hq + (size_t)prow * p.Nout + c);
+            for (int i = 0; i < 32; ++i) {
+              const float g = __uint_as_float(a[i]);
+              h[i] = (ACT == kMxSwiglu) ? __fdividef(g, 1.f + __expf(-g)) * __uint_as_float(u[i]) : fmaxf(g, 0.f);
+              amax = fmaxf(amax, fabsf(h[i]));
+            }
+            const int X = mx_exponent(amax);
+            uint4 lo, hi;
+            quantize32(h, X, lo, hi);
+            const int c = h0 + blk * 32;
+            uint4* dst = reinterpret_cast<uint4*>(p.hq + (size_t)prow * p.F + c);
             dst[0] = lo;
             dst[1] = hi;
-            p.hs[sf_offset(prow, c, p.Nout)] = (uint8_t)(X + 127);
+            p.hs[sf_offset(prow, c, p.F)] = (uint8_t)(X + 127);
           }
         }
-      } else {
+        // this warp's share of the tile is written: count it for the m-tile
+        // (__syncwarp orders the lanes' stores before lane 0's release, which
+        // carries them to GPU scope)
+        __syncwarp();
+        if (lane == 0) red_release_gpu_add(p.dep + t.m, 1);
+      } else if (half == 0 && live) {
         // fp32 rows to the kept row each padded row came from (padding rows are dropped)
-        const int i = prow - tail->seg[e];
-        const int kept = p.offsets[e + 1] - p.offsets[e];
-        const int row = (i < kept) ? p.offsets[e] + i : -1;
+        const int i = prow - tail->seg[t.e];
+        const int row = (i < tail->cnt[t.e]) ? p.offsets[t.e] + i : -1;
 #pragma unroll 1
         for (int blk = 0; blk < MN / 32; ++blk) {
           uint32_t a[32];
@@ -404,20 +498,20 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
           for (int v = 0; v < 8; ++v)
             stg[lane * 8 + (v ^ (lane & 7))] = make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
           __syncwarp();
-          const int col0 = n0 + blk * 32;
+          const int col0 = t.n0 + blk * 32;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int rr = t * 4 + (lane >> 3), cc = lane & 7;
+          for (int r8 = 0; r8 < 8; ++r8) {
+            const int rr = r8 * 4 + (lane >> 3), cc = lane & 7;
             const int trow = __shfl_sync(0xffffffffu, row, rr);
-            const int col = col0 + cc * 4;
-            if (trow >= 0 && col < p.Nout)
-              *reinterpret_cast<uint4*>(p.out + (size_t)trow * p.Nout + col) = stg[rr * 8 + (cc ^ (rr & 7))];
+            if (trow >= 0)
+              *reinterpret_cast<uint4*>(p.out + (size_t)trow * p.d + col0 + cc * 4) = stg[rr * 8 + (cc ^ (rr & 7))];
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);   // accumulator free again
+      ++tl;
     }
     if (!ok && lane == 0) {
       atomicOr(p.status, MOE_DEV_TIMEOUT);
@@ -433,11 +527,12 @@ tc_mx_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
   }
 }
 
-template <int MODE>
-cudaError_t launch_mx(const CUtensorMap& ma, const CUtensorMap& mb, const MxParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_mx_gemm<MODE>>(kMxSmem);
+template <int ACT>
+cudaError_t launch_mx(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2, const CUtensorMap& b2,
+                      const MxParams& p, int grid, cudaStream_t s) {
+  cudaError_t err = set_smem_once<tc_mx_mlp<ACT>>(kMxSmem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_mx_gemm<MODE>, dim3(grid), dim3(kThreads), kMxSmem, s, ma, mb, p);
+  return launch_pdl(tc_mx_mlp<ACT>, dim3(grid), dim3(kThreads), kMxSmem, s, a1, b1, a2, b2, p);
 }
 
 template <typename Map>
@@ -479,47 +574,43 @@ cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const voi
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
   const int F1 = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
-  // padded rows and the layer-1 input rows in E4M3
-  if ((err = launch_pdl(mx_pad_kernel, dim3(1), dim3(32), 0, s, b.offsets, c.E, b.pad)) != cudaSuccess) return err;
-  if ((err = launch_quantize(static_cast<const __nv_bfloat16*>(b.xp), b.rows_pad, c.d,
-                             RowMapPadded{b.offsets, b.pad, c.E}, static_cast<uint8_t*>(b.xq),
+  const int mt_max = b.rows_pad / MB;
+  // padded rows (and zeroed counters), then the kept layer-1 input rows in E4M3
+  if ((err = launch_pdl(mx_pad_kernel, dim3(1), dim3(32), 0, s, b.offsets, c.E, b.pad, b.ctr, 1 + mt_max)) !=
+      cudaSuccess)
+    return err;
+  if ((err = launch_quantize(static_cast<const __nv_bfloat16*>(b.xp), c.T * c.k, c.d,
+                             RowMapKept{b.offsets, b.pad, c.E}, static_cast<uint8_t*>(b.xq),
                              static_cast<uint8_t*>(b.xs), s)) != cudaSuccess)
     return err;
-  const long long mt_max = b.rows_pad / MB;
-  CUtensorMap ma, mb;
+  // both layers in one launch: h = act(xq W1q^T) quantised in the epilogue,
+  // then yp = hq W2q^T (fp32) at the kept rows
+  CUtensorMap a1, b1, a2, b2;
+  if (!make_map_u8(&a1, b.xq, (uint64_t)b.rows_pad, (uint64_t)c.d) ||
+      !make_map_u8(&b1, w1q, (uint64_t)c.E * F1, (uint64_t)c.d) ||
+      !make_map_u8(&a2, b.hq, (uint64_t)b.rows_pad, (uint64_t)c.F) ||
+      !make_map_u8(&b2, w2q, (uint64_t)c.E * c.d, (uint64_t)c.F))
+    return cudaErrorInvalidValue;
   MxParams p{};
   p.pad = b.pad;
   p.offsets = b.offsets;
   p.E = c.E;
+  p.d = c.d;
+  p.F = c.F;
+  p.F1 = F1;
   p.rows_pad = b.rows_pad;
-  p.status = status;
-  // layer 1: h = act(xq W1q^T), quantised in the epilogue
-  if (!make_map_u8(&ma, b.xq, (uint64_t)b.rows_pad, (uint64_t)c.d) ||
-      !make_map_u8(&mb, w1q, (uint64_t)c.E * F1, (uint64_t)c.d))
-    return cudaErrorInvalidValue;
-  p.K = c.d;
-  p.Nout = c.F;
-  p.b_rows = F1;
-  p.sfa = static_cast<const uint8_t*>(b.xs);
-  p.sfb = static_cast<const uint8_t*>(w1s);
+  p.xs = static_cast<const uint8_t*>(b.xs);
+  p.w1s = static_cast<const uint8_t*>(w1s);
+  p.w2s = static_cast<const uint8_t*>(w2s);
   p.hq = static_cast<uint8_t*>(b.hq);
   p.hs = static_cast<uint8_t*>(b.hs);
-  int grid = (int)std::min<long long>(mt_max * ((F1 + MN - 1) / MN), di.sms);
-  err = (c.act == MOE_ACT_SWIGLU) ? launch_mx<kMxSwiglu>(ma, mb, p, std::max(grid, 1), s)
-                                  : launch_mx<kMxRelu>(ma, mb, p, std::max(grid, 1), s);
-  if (err != cudaSuccess) return err;
-  // layer 2: yp = hq W2q^T (fp32), written at the kept rows
-  if (!make_map_u8(&ma, b.hq, (uint64_t)b.rows_pad, (uint64_t)c.F) ||
-      !make_map_u8(&mb, w2q, (uint64_t)c.E * c.d, (uint64_t)c.F))
-    return cudaErrorInvalidValue;
-  p.K = c.F;
-  p.Nout = c.d;
-  p.b_rows = c.d;
-  p.sfa = static_cast<const uint8_t*>(b.hs);
-  p.sfb = static_cast<const uint8_t*>(w2s);
   p.out = yp;
-  grid = (int)std::min<long long>(mt_max * ((c.d + MN - 1) / MN), di.sms);
-  return launch_mx<kMxOut>(ma, mb, p, std::max(grid, 1), s);
+  p.status = status;
+  p.sched = b.ctr;
+  p.dep = b.ctr + 1;
+  const int grid = (int)std::max<long long>(1, std::min<long long>((long long)mt_max * (F1 / MN + c.d / MN), di.sms));
+  return (c.act == MOE_ACT_SWIGLU) ? launch_mx<kMxSwiglu>(a1, b1, a2, b2, p, grid, s)
+                                   : launch_mx<kMxRelu>(a1, b1, a2, b2, p, grid, s);
 }
 
 }  // namespace moe

@@ -103,15 +103,17 @@ def _align256(n):
 
 def mx_regions(cfg, w):
     """Byte offsets of the MX forward's own workspace regions, which follow
-    the bf16 forward's: padded offsets, xq, xs, hq, hs (the layout of
-    moe_workspace_size_mxfp8, checked against its total)."""
+    the bf16 forward's: padded offsets, xq, xs, hq, hs and the expert
+    kernel's counters (the layout of moe_workspace_size_mxfp8, checked
+    against its total)."""
     _, lay = moe.moe_workspace_size(cfg)
     rows = w.T * w.k + 127 * w.E
     R = (rows + 127) // 128 * 128
     sb = lambda K: (R // 128) * (K // 128) * 512
     off = lay.total
     reg = {}
-    for name, n in (("pad", 4 * (w.E + 1)), ("xq", R * w.d), ("xs", sb(w.d)), ("hq", R * w.F), ("hs", sb(w.F))):
+    for name, n in (("pad", 4 * (w.E + 1)), ("xq", R * w.d), ("xs", sb(w.d)), ("hq", R * w.F), ("hs", sb(w.F)),
+                    ("ctr", 4 * (1 + R // 128))):
         reg[name] = off
         off = _align256(off + n)
     assert off == moe.moe_workspace_size_mxfp8(cfg)
