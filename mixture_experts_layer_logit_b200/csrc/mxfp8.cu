@@ -87,38 +87,47 @@ __device__ __forceinline__ void quantize32(const float (&v)[32], int X, uint4& l
   hi = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// One thread per 32-element block of a bf16 matrix: E4M3 bytes and the
-// block's scale.  The map takes an item (a row index) to (destination row,
-// source row); a negative destination skips the item.  Used for the weights
-// (identity, or the SwiGLU interleave) and for the kept activation rows,
-// which go to their expert's padded segment.  Padding rows stay unwritten:
-// every row of an MMA tile is computed from its own A row only, and no
-// output of a padding row is ever stored as a kept row.
+// One 32-element block of a bf16 row -> 32 E4M3 bytes at q and the block's
+// scale byte at sf (row r of the destination, block kb of K / 32).
+__device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__ src, int r, int kb, int K,
+                                               uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  float v[32];
+  const uint4* p = reinterpret_cast<const uint4*>(src + 32 * kb);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(p + i);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * i + 2 * j] = f.x;
+      v[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int X = mx_exponent(amax);
+  uint4 lo, hi;
+  quantize32(v, X, lo, hi);
+  uint4* qo = reinterpret_cast<uint4*>(q + (size_t)r * K + 32 * kb);
+  qo[0] = lo;
+  qo[1] = hi;
+  sf[sf_offset(r, 32 * kb, K)] = (uint8_t)(X + 127);
+}
+
+// The weights, once: one thread per 32-element block.  The map takes a
+// destination row to its source row (identity, or the SwiGLU interleave).
 struct RowMapIdentity {
-  __device__ int2 operator()(int r) const { return make_int2(r, r); }
+  __device__ int operator()(int r) const { return r; }
 };
 struct RowMapSwiglu {   // destination row of an expert's interleaved W1 <- source row
   int F;
-  __device__ int2 operator()(int r) const {
+  __device__ int operator()(int r) const {
     const int F1 = 2 * F, e = r / F1, i = r - e * F1, b = i / 128, j = i % 128;
-    return make_int2(r, e * F1 + (j < 64 ? 64 * b + j : F + 64 * b + (j - 64)));
+    return e * F1 + (j < 64 ? 64 * b + j : F + 64 * b + (j - 64));
   }
 };
-struct RowMapKept {     // kept permuted row i -> its padded row; items past offsets[E] skipped
-  const int32_t* offsets;
-  const int32_t* pad;
-  int E;
-  __device__ int2 operator()(int i) const {
-    if (i >= offsets[E]) return make_int2(-1, -1);
-    int lo = 0, hi = E - 1;   // the largest e with offsets[e] <= i holds row i
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (offsets[mid] <= i) lo = mid; else hi = mid - 1;
-    }
-    return make_int2(pad[lo] + (i - offsets[lo]), i);
-  }
-};
-
 template <typename Map>
 __global__ void __launch_bounds__(256)
 mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map map, uint8_t* __restrict__ q,
@@ -128,67 +137,71 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, Map m
   const int nb = K / 32;
   const size_t nblk = (size_t)rows * nb;
   for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += (size_t)gridDim.x * blockDim.x) {
-    const int it = (int)(b / nb), kb = (int)(b - (size_t)it * nb);
-    const int2 m = map(it);
-    if (m.x < 0) continue;
-    const int r = m.x;
-    float v[32];
-    const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)m.y * K + 32 * kb);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(p + i);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(h[j]);
-        v[8 * i + 2 * j] = f.x;
-        v[8 * i + 2 * j + 1] = f.y;
-      }
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const int X = mx_exponent(amax);
-    uint4 lo, hi;
-    quantize32(v, X, lo, hi);
-    uint4* qo = reinterpret_cast<uint4*>(q + (size_t)r * K + 32 * kb);
-    qo[0] = lo;
-    qo[1] = hi;
-    sf[sf_offset(r, 32 * kb, K)] = (uint8_t)(X + 127);
+    const int r = (int)(b / nb), kb = (int)(b - (size_t)r * nb);
+    quantize_block(src + (size_t)map(r) * K, r, kb, K, q, sf);
   }
 }
 
-// Padded offsets: every expert's kept rows rounded up to a multiple of 128
-// (one warp; 8 experts per lane, then a shuffle scan).  It also zeroes the
-// expert kernel's tile counter and per-m-tile dependency counters.
-__global__ void mx_pad_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad,
-                              int* __restrict__ ctr, int nctr) {
+// The layer-1 input rows, per call: every CTA first derives the padded
+// segment offsets (each expert's kept rows rounded up to a multiple of 128;
+// one warp, 8 experts per lane and a shuffle scan); CTA 0 publishes them and
+// zeroes the expert kernel's tile and dependency counters.  Then one thread
+// per 32-element block of a kept row, written at its row of the expert's
+// padded segment.  Padding rows stay unwritten: every row of an MMA tile is
+// computed from its own A row only, and no output of a padding row is
+// stored as a kept row.
+__global__ void __launch_bounds__(256)
+mx_quantize_rows_kernel(const __nv_bfloat16* __restrict__ xp, int rows_max, int rows_pad, int K,
+                        const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pad_out,
+                        int* __restrict__ ctr, int nctr, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  __shared__ int s_off[kMaxExperts + 1], s_pad[kMaxExperts + 1];
   pdl_wait();
   pdl_launch_dependents();
-  constexpr int PER = kMaxExperts / 32;
-  const int lane = threadIdx.x;
-  for (int i = lane; i < nctr; i += 32) ctr[i] = 0;
-  int loc[PER], sum = 0;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    constexpr int PER = kMaxExperts / 32;
+    const int lane = threadIdx.x;
+    int loc[PER], sum = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane * PER + i;
-    loc[i] = (e < E) ? (offsets[e + 1] - offsets[e] + kMxPad - 1) / kMxPad * kMxPad : 0;
-    sum += loc[i];
-  }
-  int incl = sum;
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      loc[i] = (e < E) ? (s_off[e + 1] - s_off[e] + kMxPad - 1) / kMxPad * kMxPad : 0;
+      sum += loc[i];
+    }
+    int incl = sum;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  int run = incl - sum;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    int run = incl - sum;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane * PER + i;
-    if (e < E) pad[e] = run;
-    run += loc[i];
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      if (e < E) s_pad[e] = run;
+      run += loc[i];
+    }
+    if (lane == 31) s_pad[E] = incl;
   }
-  if (lane == 31) pad[E] = incl;
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) pad_out[e] = s_pad[e];
+    for (int i = threadIdx.x; i < nctr; i += blockDim.x) ctr[i] = 0;
+  }
+  const int nb = K / 32;
+  const int kept = min(s_off[E], rows_max);
+  const size_t nblk = (size_t)kept * nb;
+  for (size_t b = (size_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += (size_t)gridDim.x * blockDim.x) {
+    const int i = (int)(b / nb), kb = (int)(b - (size_t)i * nb);
+    int lo = 0, hi = E - 1;   // the largest e with offsets[e] <= i holds row i
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int r = s_pad[lo] + (i - s_off[lo]);
+    if ((unsigned)r < (unsigned)rows_pad) quantize_block(xp + (size_t)i * K, r, kb, K, q, sf);
+  }
 }
 
 struct MxParams {
@@ -575,14 +588,17 @@ cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const voi
   if (err != cudaSuccess) return err;
   const int F1 = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   const int mt_max = b.rows_pad / MB;
-  // padded rows (and zeroed counters), then the kept layer-1 input rows in E4M3
-  if ((err = launch_pdl(mx_pad_kernel, dim3(1), dim3(32), 0, s, b.offsets, c.E, b.pad, b.ctr, 1 + mt_max)) !=
-      cudaSuccess)
-    return err;
-  if ((err = launch_quantize(static_cast<const __nv_bfloat16*>(b.xp), c.T * c.k, c.d,
-                             RowMapKept{b.offsets, b.pad, c.E}, static_cast<uint8_t*>(b.xq),
-                             static_cast<uint8_t*>(b.xs), s)) != cudaSuccess)
-    return err;
+  // the padded segments (and zeroed counters), the kept layer-1 input rows in E4M3
+  {
+    const int rows_max = c.T * c.k;
+    const size_t nblk = (size_t)rows_max * (c.d / 32);
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>((nblk + 255) / 256, (size_t)di.sms * 8));
+    err = launch_pdl(mx_quantize_rows_kernel, dim3(grid), dim3(256), 0, s,
+                     static_cast<const __nv_bfloat16*>(b.xp), rows_max, b.rows_pad, c.d, b.offsets, c.E, b.pad,
+                     b.ctr,
+                     1 + mt_max, static_cast<uint8_t*>(b.xq), static_cast<uint8_t*>(b.xs));
+    if (err != cudaSuccess) return err;
+  }
   // both layers in one launch: h = act(xq W1q^T) quantised in the epilogue,
   // then yp = hq W2q^T (fp32) at the kept rows
   CUtensorMap a1, b1, a2, b2;
