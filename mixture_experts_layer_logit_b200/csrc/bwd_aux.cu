@@ -14,6 +14,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 #include <type_traits>
 
 namespace moe {
@@ -126,7 +128,7 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
                   const int32_t* __restrict__ pad_offsets, const int32_t* __restrict__ src_tok,
                   const int32_t* __restrict__ row_of, const float* __restrict__ topk_w, int E, int T, int k, int d,
                   int rows_alloc, const float* __restrict__ scale, TG* __restrict__ xp, TG* __restrict__ dout_perm,
-                  float* __restrict__ wrow, uint32_t* __restrict__ status) {
+                  TX* __restrict__ xp_raw, float* __restrict__ wrow, uint32_t* __restrict__ status) {
   __shared__ int32_t s_off[kMaxExperts + 1], s_pad[kMaxExperts + 1];
   pdl_wait();
   pdl_launch_dependents();
@@ -161,11 +163,13 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
     const int nvec = d / 8;   // 8 elements = 16 bytes
     uint4* xo = reinterpret_cast<uint4*>(xp + (size_t)pr * d);
     uint4* go = reinterpret_cast<uint4*>(dout_perm + (size_t)pr * d);
+    uint4* ro = xp_raw != nullptr ? reinterpret_cast<uint4*>(xp_raw + (size_t)pr * d) : nullptr;
     bool over = false;
     for (int v = lane; v < nvec; v += 32) {
       uint4 xv = make_uint4(0u, 0u, 0u, 0u), gv = xv;
       if (t >= 0) {
         xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+        if (ro != nullptr) ro[v] = xv;
         if constexpr (std::is_same<TG, __half>::value) {   // bf16 x -> fp16 (exact inside the fp16 range)
           const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&xv);
           uint32_t o[4];
@@ -181,6 +185,7 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
         gv = make_uint4(OpType<TG>::pack(sc * a.x, sc * a.y, over), OpType<TG>::pack(sc * a.z, sc * a.w, over),
                         OpType<TG>::pack(sc * b.x, sc * b.y, over), OpType<TG>::pack(sc * b.z, sc * b.w, over));
       }
+      if (t < 0 && ro != nullptr) ro[v] = xv;
       xo[v] = xv;
       go[v] = gv;
     }
@@ -202,51 +207,52 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
   }
 }
 
-// Gate logits z[T, E] = x W_gate^T (+ b) in fp32 (the forward keeps them on
-// chip only): 32 tokens per block, model width staged 32 at a time.
-constexpr int kLT = 32, kLK = 32;
+// Gate logits in fp32 (the forward keeps them on chip only), as partial sums
+// over slices of the model width: zpart[s][t][e] = sum over slice s of
+// x[t, c] W_gate[e, c].  The reader adds the bias and the slices in slice
+// order.  A block computes 32 tokens x 16 experts (two per thread), the
+// slice staged 32 columns at a time; the slices (blockIdx.z) put enough
+// blocks in flight when T is small.
+constexpr int kLT = 32, kLK = 32, kLE = 16;
 template <typename TX>
 __global__ void __launch_bounds__(256)
-logits_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* __restrict__ bg, int T, int d, int E,
-              float* __restrict__ z) {
+logits_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, int T, int d, int E, int kslice,
+              float* __restrict__ zpart) {
   __shared__ float xs[kLT][kLK + 1];
-  __shared__ float ws[kMaxExperts][kLK + 1];
+  __shared__ float ws[kLE][kLK + 1];
   pdl_wait();
   pdl_launch_dependents();
-  const int t0 = blockIdx.x * kLT;
+  const int t0 = blockIdx.x * kLT, e0 = blockIdx.y * kLE;
+  const int ks = blockIdx.z;
+  const int kbeg = ks * kslice, kend = min(d, kbeg + kslice);
   const int tid = threadIdx.x;
-  // thread (tt, eg): token tt = tid % 32, experts eg, eg + 8, ...
+  // thread (tt, eg): token t0 + tt, experts e0 + eg and e0 + eg + 8
   const int tt = tid & 31, eg = tid >> 5;
-  float acc[kMaxExperts / 8];
+  float acc0 = 0.f, acc1 = 0.f;
+  for (int k0 = kbeg; k0 < kend; k0 += kLK) {
 #pragma unroll
-  for (int i = 0; i < kMaxExperts / 8; ++i) acc[i] = 0.f;
-  for (int k0 = 0; k0 < d; k0 += kLK) {
     for (int i = tid; i < kLT * kLK; i += 256) {
       const int r = i / kLK, c = i % kLK;
-      xs[r][c] = (t0 + r < T && k0 + c < d) ? to_float(x[(size_t)(t0 + r) * d + k0 + c]) : 0.f;
+      xs[r][c] = (t0 + r < T && k0 + c < kend) ? to_float(x[(size_t)(t0 + r) * d + k0 + c]) : 0.f;
     }
-    for (int i = tid; i < E * kLK; i += 256) {
+#pragma unroll
+    for (int i = tid; i < kLE * kLK; i += 256) {
       const int r = i / kLK, c = i % kLK;
-      ws[r][c] = (k0 + c < d) ? to_float(wg[(size_t)r * d + k0 + c]) : 0.f;
+      ws[r][c] = (e0 + r < E && k0 + c < kend) ? to_float(wg[(size_t)(e0 + r) * d + k0 + c]) : 0.f;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
     for (int c = 0; c < kLK; ++c) {
       const float xv = xs[tt][c];
-#pragma unroll
-      for (int i = 0; i < kMaxExperts / 8; ++i) {
-        const int e = eg + 8 * i;
-        if (e < E) acc[i] = fmaf(xv, ws[e][c], acc[i]);
-      }
+      acc0 = fmaf(xv, ws[eg][c], acc0);
+      acc1 = fmaf(xv, ws[eg + 8][c], acc1);
     }
     __syncthreads();
   }
   if (t0 + tt < T) {
-#pragma unroll
-    for (int i = 0; i < kMaxExperts / 8; ++i) {
-      const int e = eg + 8 * i;
-      if (e < E) z[(size_t)(t0 + tt) * E + e] = acc[i] + (bg != nullptr ? bg[e] : 0.f);
-    }
+    float* zs = zpart + ((size_t)ks * T + t0 + tt) * E;
+    if (e0 + eg < E) zs[e0 + eg] = acc0;
+    if (e0 + eg + 8 < E) zs[e0 + eg + 8] = acc1;
   }
 }
 
@@ -261,7 +267,8 @@ logits_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* 
 // The softmax is recomputed from the fp32 logits the way the route kernel
 // computes it.  Lanes hold experts lane + 32 i.
 __global__ void __launch_bounds__(256)
-gate_bwd_kernel(const float* __restrict__ z, const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
+gate_bwd_kernel(const float* __restrict__ zpart, int nks, const float* __restrict__ bg,
+                const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
                 const int32_t* __restrict__ row_of, const int32_t* __restrict__ offsets,
                 const int32_t* __restrict__ pad_offsets, const int32_t* __restrict__ counts,
                 const float* __restrict__ dwpart, int nt2, int rows_alloc, int T, int E, int k, float lam,
@@ -278,7 +285,12 @@ gate_bwd_kernel(const float* __restrict__ z, const int32_t* __restrict__ topk_id
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     ok[i] = e < E;
-    zv[i] = ok[i] ? z[(size_t)t * E + e] : 0.f;
+    float zz = 0.f;
+    if (ok[i]) {
+      zz = (bg != nullptr) ? bg[e] : 0.f;
+      for (int sl = 0; sl < nks; ++sl) zz += zpart[((size_t)sl * T + t) * E + e];
+    }
+    zv[i] = zz;
   }
   float mu = 0.f, sd = 0.f;
   if (lam > 0.f) {
@@ -386,45 +398,88 @@ gate_bwd_kernel(const float* __restrict__ z, const int32_t* __restrict__ topk_id
 }
 
 // dx[t, c] = sum over kept slots (slot order) of dxp[padded row, c]
-//          + sum_e dz[t, e] W_gate[e, c];  32 tokens x 128 columns per block.
+//          + sum_e dz[t, e] W_gate[e, c];  16 tokens x 512 columns per block
+// (4 consecutive columns per thread when d is a multiple of 4).  The padded
+// rows of the block's slots are found once, into shared memory, so that the
+// row loads of different tokens are independent.
 template <typename TX>
 __global__ void __launch_bounds__(128)
 dx_kernel(const float* __restrict__ dxp, const float* __restrict__ dz, const TX* __restrict__ wg,
           const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ row_of,
           const int32_t* __restrict__ offsets, const int32_t* __restrict__ pad_offsets, int T, int E, int k, int d,
           int rows_alloc, float* __restrict__ dx) {
-  constexpr int TT = 32;
+  constexpr int TT = 16, V = 4;
   __shared__ float dzs[TT][kMaxExperts + 1];
+  __shared__ int prow[TT * kMaxExperts];
   pdl_wait();
   pdl_launch_dependents();
   const int t0 = blockIdx.x * TT;
-  const int c = blockIdx.y * 128 + threadIdx.x;
-  for (int i = threadIdx.x; i < TT * E; i += 128) {
+  for (int i = threadIdx.x; i < TT * E; i += blockDim.x) {
     const int r = i / E, e = i % E;
     dzs[r][e] = (t0 + r < T) ? dz[(size_t)(t0 + r) * E + e] : 0.f;
   }
-  __syncthreads();
-  if (c >= d) return;
-  float acc[TT];
-#pragma unroll
-  for (int r = 0; r < TT; ++r) acc[r] = 0.f;
-  for (int e = 0; e < E; ++e) {
-    const float wv = to_float(wg[(size_t)e * d + c]);
-#pragma unroll
-    for (int r = 0; r < TT; ++r) acc[r] = fmaf(dzs[r][e], wv, acc[r]);
-  }
-  for (int r = 0; r < TT; ++r) {
-    const int t = t0 + r;
-    if (t >= T) break;
-    float v = 0.f;
-    for (int j = 0; j < k; ++j) {
+  for (int i = threadIdx.x; i < TT * k; i += blockDim.x) {
+    const int r = i / k, j = i % k, t = t0 + r;
+    int pr = -1;
+    if (t < T) {
       const int row = row_of[(size_t)t * k + j];
       const int e = topk_idx[(size_t)t * k + j];
-      if (row < 0 || (unsigned)e >= (unsigned)E) continue;
-      const int pr = pad_offsets[e] + (row - offsets[e]);
-      if ((unsigned)pr < (unsigned)rows_alloc) v += dxp[(size_t)pr * d + c];
+      if (row >= 0 && (unsigned)e < (unsigned)E) {
+        pr = pad_offsets[e] + (row - offsets[e]);
+        if ((unsigned)pr >= (unsigned)rows_alloc) pr = -1;
+      }
     }
-    dx[(size_t)t * d + c] = v + acc[r];
+    prow[i] = pr;
+  }
+  __syncthreads();
+  const int nt = min(TT, T - t0);
+  if ((d & (V - 1)) == 0) {
+    const int c = (blockIdx.y * blockDim.x + threadIdx.x) * V;
+    if (c >= d) return;
+    float4 acc[TT];
+#pragma unroll
+    for (int r = 0; r < TT; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < E; ++e) {
+      const float w0 = to_float(wg[(size_t)e * d + c]), w1 = to_float(wg[(size_t)e * d + c + 1]);
+      const float w2 = to_float(wg[(size_t)e * d + c + 2]), w3 = to_float(wg[(size_t)e * d + c + 3]);
+#pragma unroll
+      for (int r = 0; r < TT; ++r) {
+        const float zv = dzs[r][e];
+        acc[r].x = fmaf(zv, w0, acc[r].x);
+        acc[r].y = fmaf(zv, w1, acc[r].y);
+        acc[r].z = fmaf(zv, w2, acc[r].z);
+        acc[r].w = fmaf(zv, w3, acc[r].w);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < TT; ++r) {
+      if (r >= nt) continue;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < k; ++j) {
+        const int pr = prow[r * k + j];
+        if (pr < 0) continue;
+        const float4 a = __ldcs(reinterpret_cast<const float4*>(dxp + (size_t)pr * d + c));
+        v.x += a.x;
+        v.y += a.y;
+        v.z += a.z;
+        v.w += a.w;
+      }
+      __stcs(reinterpret_cast<float4*>(dx + (size_t)(t0 + r) * d + c),
+             make_float4(v.x + acc[r].x, v.y + acc[r].y, v.z + acc[r].z, v.w + acc[r].w));
+    }
+  } else {
+    for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * V, cend = min(d, c + V); c < cend; ++c) {
+      for (int r = 0; r < nt; ++r) {
+        float a = 0.f;
+        for (int e = 0; e < E; ++e) a = fmaf(dzs[r][e], to_float(wg[(size_t)e * d + c]), a);
+        float v = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int pr = prow[r * k + j];
+          if (pr >= 0) v += dxp[(size_t)pr * d + c];
+        }
+        dx[(size_t)(t0 + r) * d + c] = v + a;
+      }
+    }
   }
 }
 
@@ -502,7 +557,7 @@ cudaError_t launch_bwd_front_t(const moe_config& c, const void* x, const float* 
   return launch_pdl(bwd_gather_kernel<TX, TG>, dim3((rows + 7) / 8), dim3(256), 0, s, static_cast<const TX*>(x),
                     dout, st.offsets, (const int32_t*)st.pad_offsets, st.src_tok, st.row_of, st.topk_w, c.E, c.T,
                     c.k, c.d, rows, (const float*)st.scale, static_cast<TG*>(st.xp), static_cast<TG*>(st.dout_perm),
-                    st.wrow, st.status);
+                    static_cast<TX*>(st.f16 ? st.xp_b : nullptr), st.wrow, st.status);
 }
 
 template <typename TX>
@@ -511,18 +566,20 @@ cudaError_t launch_bwd_gate_t(const moe_config& c, const void* x, const void* wg
                               float* dw_out, cudaStream_t s) {
   const TX* X = static_cast<const TX*>(x);
   const TX* WG = static_cast<const TX*>(wg);
-  cudaError_t e = launch_pdl(logits_kernel<TX>, dim3((c.T + kLT - 1) / kLT), dim3(256), 0, s, X, WG, bg, c.T, c.d,
-                             c.E, st.z);
+  const int nks = bwd_logit_slices(c);
+  const int kslice = (c.d + nks - 1) / nks;
+  cudaError_t e = launch_pdl(logits_kernel<TX>, dim3((c.T + kLT - 1) / kLT, (c.E + kLE - 1) / kLE, nks), dim3(256),
+                             0, s, X, WG, c.T, c.d, c.E, kslice, st.z);
   if (e != cudaSuccess) return e;
   // column tiles of the dh GEMM, each of which left one partial of dw per row
   const int col = c.dtype == MOE_DTYPE_BF16 ? bwd_tc_col_tile() : bwd_simt_col_tile();
   const int nt2 = (c.F + col - 1) / col;
-  e = launch_pdl(gate_bwd_kernel, dim3((c.T + 7) / 8), dim3(256), 0, s, (const float*)st.z, st.topk_idx,
+  e = launch_pdl(gate_bwd_kernel, dim3((c.T + 7) / 8), dim3(256), 0, s, (const float*)st.z, nks, bg, st.topk_idx,
                  st.topk_w, st.row_of, st.offsets, (const int32_t*)st.pad_offsets, st.counts,
                  (const float*)st.dwpart, nt2, st.rows_alloc, c.T, c.E, c.k, c.lambda, aux_coef, z_coef, st.dz,
                  dw_out);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(dx_kernel<TX>, dim3((c.T + 31) / 32, (c.d + 127) / 128), dim3(128), 0, s, (const float*)st.dxp,
+  e = launch_pdl(dx_kernel<TX>, dim3((c.T + 15) / 16, (c.d + 511) / 512), dim3(128), 0, s, (const float*)st.dxp,
                  (const float*)st.dz, WG, st.topk_idx, st.row_of, st.offsets, (const int32_t*)st.pad_offsets, c.T,
                  c.E, c.k, c.d, st.rows_alloc, dx);
   if (e != cudaSuccess) return e;
@@ -536,6 +593,14 @@ cudaError_t launch_bwd_gate_t(const moe_config& c, const void* x, const void* wg
 }  // namespace
 
 int bwd_pad_rows() { return kPad; }
+
+// Model-width slices of the logits recompute: enough 32 x 16 blocks for
+// about four waves of 148 SMs, at most 8, each slice at least 32 columns.
+int bwd_logit_slices(const moe_config& c) {
+  const int blocks = ((c.T + kLT - 1) / kLT) * ((c.E + kLE - 1) / kLE);
+  const int want = blocks > 0 ? (4 * 148 + blocks - 1) / blocks : 1;
+  return std::max(1, std::min({want, 8, (c.d + kLK - 1) / kLK}));
+}
 
 cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                              cudaStream_t s) {

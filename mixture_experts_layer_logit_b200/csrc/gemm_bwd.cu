@@ -71,6 +71,7 @@ struct BwdParams {
   const float* u;           // [rows][F1] pre-activation
   const float* wrow;        // [rows] gate weight of each padded row (0 on padding)
   void* du;                 // [rows][F1]  (operand type)
+  void* du_b;               // [rows][F1]  bf16 copy of du for the bf16 dxp GEMM (fp16 operands only; else null)
   void* hw;                 // [rows][F]   w * h (operand type)
   float* dwpart;            // [nt][rows] per column tile: sum over its columns of dh/w * h
   int F, F1;
@@ -195,7 +196,7 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
         dst[4 * i + 3] = __uint_as_float(v.w);
       }
     }
-    uint32_t du_g[16], du_v[16], hwp[16];
+    uint32_t du_g[16], du_v[16], hwp[16], db_g[16], db_v[16];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
       float dg[2], dv[2], hh[2];
@@ -225,6 +226,11 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
       du_g[i / 2] = pack_op<F16>(dg[0], dg[1], o);
       du_v[i / 2] = pack_op<F16>(dv[0], dv[1], o);
       hwp[i / 2] = pack_op<F16>(hh[0], hh[1], o);
+      if (F16) {
+        bool ob = false;   // bf16 does not overflow where fp16 did not
+        db_g[i / 2] = pack_op<false>(dg[0], dg[1], ob);
+        db_v[i / 2] = pack_op<false>(dv[0], dv[1], ob);
+      }
       over |= o && live && (f0 + i < p.F);
     }
     if (live) {
@@ -245,6 +251,18 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (q < nv) dv_row[q] = make_uint4(du_v[4 * q], du_v[4 * q + 1], du_v[4 * q + 2], du_v[4 * q + 3]);
+      }
+      if (F16 && p.du_b != nullptr) {
+        uint4* bg_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du_b) + (size_t)row * p.F1 + f0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nv) bg_row[q] = make_uint4(db_g[4 * q], db_g[4 * q + 1], db_g[4 * q + 2], db_g[4 * q + 3]);
+        if (ACT == kSwiglu) {
+          uint4* bv_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du_b) + (size_t)row * p.F1 + p.F + f0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < nv) bv_row[q] = make_uint4(db_v[4 * q], db_v[4 * q + 1], db_v[4 * q + 2], db_v[4 * q + 3]);
+        }
       }
     }
   }
@@ -487,6 +505,7 @@ cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const voi
   p.u = st.u;
   p.wrow = st.wrow;
   p.du = st.du;
+  p.du_b = F16 ? st.du_b : nullptr;
   p.hw = st.hw;
   p.dwpart = st.dwpart;
   p.F = c.F;
@@ -496,16 +515,17 @@ cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const voi
                                   : launch_bwd<kDgradAct, kRelu, false, true, F16>(ma, mb, p, grid, s);
   if (err != cudaSuccess) return err;
 
-  // dxp = du W1[e] (K = F1)
-  if (!make_map(&ma, st.du, R, (uint64_t)F1, F16) ||
-      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, F16, 64))
+  // dxp = du W1[e] (K = F1), on the weights' own type: with fp16 operands du
+  // goes in its bf16 copy (still scaled by s), so W1 needs no fp16 copy
+  if (!make_map(&ma, F16 ? st.du_b : st.du, R, (uint64_t)F1, false) ||
+      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false, 64))
     return cudaErrorInvalidValue;
   p.K = F1;
   p.Nout = c.d;
   p.b_krows = F1;
   p.out = st.dxp;
   grid = (int)std::min<long long>(mt_max * ((c.d + BN - 1) / BN), sms);
-  if ((err = launch_bwd<kDgradPlain, kRelu, false, true, F16>(ma, mb, p, grid, s)) != cudaSuccess) return err;
+  if ((err = launch_bwd<kDgradPlain, kRelu, false, true, false>(ma, mb, p, grid, s)) != cudaSuccess) return err;
 
   // dW2[e] = dout_perm_e^T (w h)_e: M = d, N = F, K = the expert's padded rows
   if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, F16, 64) || !make_map(&mb, st.hw, R, (uint64_t)c.F, F16, 64))

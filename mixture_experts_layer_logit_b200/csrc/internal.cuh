@@ -140,7 +140,7 @@ struct BwdState {
   void* hw;                  // [rows][F]   w * h (element type of the path)
   float* dwpart;             // [column tiles of F][rows]
   float* dxp;                // [rows][d]
-  float* z;                  // [T][E] logits
+  float* z;                  // [slices][T][E] partial logits (bwd_logit_slices)
   float* dz;                 // [T][E]
   float* dwg_part;           // [nsplit][E][d + 1]
   int nsplit, tok_per_split;
@@ -151,13 +151,14 @@ struct BwdState {
   bool f16;
   unsigned* amax;            // max |dout| as float bits (zeroed before the amax kernel)
   float* scale;              // [2]: s, 1/s (1, 1 without fp16 operands)
-  void* w1h;                 // fp16 copy of W1 (f16), else unused
+  void* xp_b;                // [rows][d]   bf16 x of each padded row (f16 only: the recomputed u in bf16)
+  void* du_b;                // [rows][F1]  bf16 copy of the scaled du (f16 only: the dxp GEMM in bf16)
 };
 int bwd_pad_rows();
+int bwd_logit_slices(const moe_config& c);
 int bwd_tc_col_tile();     // columns of a tensor-core backward tile (the dw partials per row)
 int bwd_simt_col_tile();
 // bf16 -> fp16 (round to nearest even, saturating at +-65504)
-cudaError_t launch_convert_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t s);
 // prep (padded offsets, the dout scale) and gather (x, dout, gate weight of every padded row)
 cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                              cudaStream_t s);
