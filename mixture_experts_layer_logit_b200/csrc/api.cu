@@ -220,7 +220,7 @@ moe_status experts_combine(const moe_config& c, const void* xp, const int32_t* o
 struct BwdLayout {
   int rows;
   int nsplit, tok_per_split, col_tiles;
-  size_t pad_offsets, xp, dout_perm, wrow, u, du, hw, dwpart, dxp, z, dz, dwg_part, amax, scale, xp_b, du_b, total;
+  size_t pad_offsets, xp, dout_perm, wrow, u, du, hw, dwpart, dxp, z, dz, dwg_part, amax, scale, w1h, total;
 };
 
 // The backward's GEMM operands are fp16 when the forward's hidden type is
@@ -253,8 +253,7 @@ BwdLayout bwd_layout(const moe_config& c) {
   L.dwg_part = off;    off = align256(off + 4 * (size_t)L.nsplit * E * (d + 1));
   L.amax = off;        off = align256(off + 4);
   L.scale = off;       off = align256(off + 8);
-  L.xp_b = off;        off = align256(off + (bwd_f16(c) ? 2 * R * d : 0));
-  L.du_b = off;        off = align256(off + (bwd_f16(c) ? 2 * R * (size_t)F1 : 0));
+  L.w1h = off;         off = align256(off + (bwd_f16(c) ? 2 * E * (size_t)F1 * d : 0));
   L.total = off;
   return L;
 }
@@ -666,22 +665,23 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* x, const void* 
   b.f16 = bwd_f16(c);
   b.amax = at<unsigned>(ws, BL.amax);
   b.scale = at<float>(ws, BL.scale);
-  b.xp_b = at<char>(ws, BL.xp_b);
-  b.du_b = at<char>(ws, BL.du_b);
+  b.w1h = at<char>(ws, BL.w1h);
   // padded rows: x, dout and the gate weight of every kept assignment
   if (launch_bwd_front(c, x, dout, b, s) != cudaSuccess) return MOE_ERR_CUDA;
   // the first layer's pre-activation u = xp W1[e]^T, then the expert layers' gradients
   cudaError_t e;
   if (c.dtype == MOE_DTYPE_BF16) {
-    // u from the bf16 rows and W1 exactly as the forward's layer 1 (with fp16
-    // operands the gather also keeps a bf16 copy of the rows), on 2-SM pair
-    // tiles when the segments are long
-    const void* xb = b.f16 ? b.xp_b : b.xp;
-    e = pair_tiles(c) ? launch_grouped_plain_tc_pair(c, xb, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u,
-                                                     b.status, false, s)
-                      : launch_grouped_plain_tc(c, xb, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status,
-                                                false, s);
-    if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, W1, W2, dW1, dW2, s);
+    const void* w1 = W1;
+    if (b.f16) {   // fp16 operands: W1 converted once per call (kind::f16 takes one type for A and B)
+      if (launch_convert_bf16_f16(W1, b.w1h, (size_t)c.E * F1 * c.d, s) != cudaSuccess) return MOE_ERR_CUDA;
+      w1 = b.w1h;
+    }
+    // the recomputed pre-activation on 2-SM pair tiles when the segments are long, as the forward's layer 1
+    e = pair_tiles(c) ? launch_grouped_plain_tc_pair(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u,
+                                                     b.status, b.f16, s)
+                      : launch_grouped_plain_tc(c, b.xp, b.pad_offsets, b.rows_alloc, w1, c.d, F1, b.u, b.status,
+                                                b.f16, s);
+    if (e == cudaSuccess) e = launch_expert_backward_tc(c, b, w1, W2, dW1, dW2, pair_tiles(c), s);
   } else {
     e = launch_grouped_plain_simt(c, b.xp, b.pad_offsets, b.rows_alloc, W1, c.d, F1, b.u, b.status, s);
     if (e == cudaSuccess) e = launch_expert_backward_simt(c, b, W1, W2, dW1, dW2, s);

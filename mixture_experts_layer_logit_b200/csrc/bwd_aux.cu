@@ -128,7 +128,7 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
                   const int32_t* __restrict__ pad_offsets, const int32_t* __restrict__ src_tok,
                   const int32_t* __restrict__ row_of, const float* __restrict__ topk_w, int E, int T, int k, int d,
                   int rows_alloc, const float* __restrict__ scale, TG* __restrict__ xp, TG* __restrict__ dout_perm,
-                  TX* __restrict__ xp_raw, float* __restrict__ wrow, uint32_t* __restrict__ status) {
+                  float* __restrict__ wrow, uint32_t* __restrict__ status) {
   __shared__ int32_t s_off[kMaxExperts + 1], s_pad[kMaxExperts + 1];
   pdl_wait();
   pdl_launch_dependents();
@@ -163,13 +163,11 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
     const int nvec = d / 8;   // 8 elements = 16 bytes
     uint4* xo = reinterpret_cast<uint4*>(xp + (size_t)pr * d);
     uint4* go = reinterpret_cast<uint4*>(dout_perm + (size_t)pr * d);
-    uint4* ro = xp_raw != nullptr ? reinterpret_cast<uint4*>(xp_raw + (size_t)pr * d) : nullptr;
     bool over = false;
     for (int v = lane; v < nvec; v += 32) {
       uint4 xv = make_uint4(0u, 0u, 0u, 0u), gv = xv;
       if (t >= 0) {
         xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
-        if (ro != nullptr) ro[v] = xv;
         if constexpr (std::is_same<TG, __half>::value) {   // bf16 x -> fp16 (exact inside the fp16 range)
           const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&xv);
           uint32_t o[4];
@@ -185,7 +183,6 @@ bwd_gather_kernel(const TX* __restrict__ x, const float* __restrict__ dout, cons
         gv = make_uint4(OpType<TG>::pack(sc * a.x, sc * a.y, over), OpType<TG>::pack(sc * a.z, sc * a.w, over),
                         OpType<TG>::pack(sc * b.x, sc * b.y, over), OpType<TG>::pack(sc * b.z, sc * b.w, over));
       }
-      if (t < 0 && ro != nullptr) ro[v] = xv;
       xo[v] = xv;
       go[v] = gv;
     }
@@ -557,7 +554,7 @@ cudaError_t launch_bwd_front_t(const moe_config& c, const void* x, const float* 
   return launch_pdl(bwd_gather_kernel<TX, TG>, dim3((rows + 7) / 8), dim3(256), 0, s, static_cast<const TX*>(x),
                     dout, st.offsets, (const int32_t*)st.pad_offsets, st.src_tok, st.row_of, st.topk_w, c.E, c.T,
                     c.k, c.d, rows, (const float*)st.scale, static_cast<TG*>(st.xp), static_cast<TG*>(st.dout_perm),
-                    static_cast<TX*>(st.f16 ? st.xp_b : nullptr), st.wrow, st.status);
+                    st.wrow, st.status);
 }
 
 template <typename TX>

@@ -30,6 +30,18 @@ __global__ void convert_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 
 }  // namespace
 
+namespace moe {
+cudaError_t launch_convert_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  const size_t want = (n / 8 + 255) / 256;
+  const int grid = (int)std::max<size_t>(1, std::min<size_t>(want, (size_t)di.sms * 8));
+  convert_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n);
+  return cudaGetLastError();
+}
+}  // namespace moe
 
 extern "C" moe_status moe_convert_bf16_to_f16(const void* src, void* dst, size_t n, moe_stream_t stream) {
   if (n == 0) return MOE_OK;

@@ -71,7 +71,6 @@ struct BwdParams {
   const float* u;           // [rows][F1] pre-activation
   const float* wrow;        // [rows] gate weight of each padded row (0 on padding)
   void* du;                 // [rows][F1]  (operand type)
-  void* du_b;               // [rows][F1]  bf16 copy of du for the bf16 dxp GEMM (fp16 operands only; else null)
   void* hw;                 // [rows][F]   w * h (operand type)
   float* dwpart;            // [nt][rows] per column tile: sum over its columns of dh/w * h
   int F, F1;
@@ -196,7 +195,7 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
         dst[4 * i + 3] = __uint_as_float(v.w);
       }
     }
-    uint32_t du_g[16], du_v[16], hwp[16], db_g[16], db_v[16];
+    uint32_t du_g[16], du_v[16], hwp[16];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
       float dg[2], dv[2], hh[2];
@@ -226,11 +225,6 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
       du_g[i / 2] = pack_op<F16>(dg[0], dg[1], o);
       du_v[i / 2] = pack_op<F16>(dv[0], dv[1], o);
       hwp[i / 2] = pack_op<F16>(hh[0], hh[1], o);
-      if (F16) {
-        bool ob = false;   // bf16 does not overflow where fp16 did not
-        db_g[i / 2] = pack_op<false>(dg[0], dg[1], ob);
-        db_v[i / 2] = pack_op<false>(dv[0], dv[1], ob);
-      }
       over |= o && live && (f0 + i < p.F);
     }
     if (live) {
@@ -251,18 +245,6 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (q < nv) dv_row[q] = make_uint4(du_v[4 * q], du_v[4 * q + 1], du_v[4 * q + 2], du_v[4 * q + 3]);
-      }
-      if (F16 && p.du_b != nullptr) {
-        uint4* bg_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du_b) + (size_t)row * p.F1 + f0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q < nv) bg_row[q] = make_uint4(db_g[4 * q], db_g[4 * q + 1], db_g[4 * q + 2], db_g[4 * q + 3]);
-        if (ACT == kSwiglu) {
-          uint4* bv_row = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.du_b) + (size_t)row * p.F1 + p.F + f0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q < nv) bv_row[q] = make_uint4(db_v[4 * q], db_v[4 * q + 1], db_v[4 * q + 2], db_v[4 * q + 3]);
-        }
       }
     }
   }
@@ -473,6 +455,283 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
+// ------------------------------------------------------------ 2-SM pair tiles
+// The same GEMMs on tiles of 256 x 256 computed by a pair of CTAs on two SMs
+// of one cluster (tcgen05.mma.cta_group::2), as the forward's pair kernel:
+// CTA r of the pair loads its half of the A tile (kDgrad*: rows
+// [128 r, 128 r + 128) of the tile's activation rows; kWgrad: output rows
+// [m0 + 128 r, +128), MN-major) and its half of the B tile (N columns
+// [n0 + 128 r, +128), MN-major), to the same shared-memory offsets; the even
+// CTA issues the MMA (M = 256, N = 256, K = 16) and each CTA's TMEM receives
+// its 128 rows x 256 columns.  Per SM and k-block this loads 32 KB for
+// 128 x 256 x 64 multiply-adds where the 1-SM tile loads 48 KB: the 1-SM
+// kernels are bound by how fast an SM takes in its loads, not by the tensor
+// pipe.  Barriers, aborts and teardown as in the forward's pair kernel.
+constexpr int PM = 256, HM = PM / 2, HN = BN / 2;
+constexpr int PSTAGES = 6;
+constexpr int PA_BYTES = HM * BK * 2;              // 16 KB
+constexpr int PB_BYTES = HN * BK * 2;              // 16 KB
+constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+
+struct PTail {
+  unsigned long long full[PSTAGES], empty[PSTAGES], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int tstart[kMaxExperts + 1];
+  int seg[kMaxExperts + 1];
+};
+constexpr size_t kPairSmemBytes = 1024 + (size_t)PSTAGES * PSTAGE_BYTES + kStagingBytes + sizeof(PTail);
+static_assert(kPairSmemBytes <= 227 * 1024, "shared memory of one CTA");
+
+// Tile L of the pair kernels (256-row / 256-column tiles).
+template <int MODE>
+__device__ __forceinline__ BwdTile bwd_tile_pair(const PTail* tail, const BwdParams& p, int L) {
+  BwdTile t;
+  if (MODE == kWgrad) {
+    const int mt = (p.M + PM - 1) / PM, nt = (p.N + BN - 1) / BN;
+    t.e = L / (mt * nt);
+    const int r = L - t.e * mt * nt;
+    const int ni = r / mt, mi = r - ni * mt;
+    t.m0 = mi * PM;
+    t.n0 = ni * BN;
+    t.row0 = t.m0;
+    t.rows = min(PM, p.M - t.m0);
+    t.k0 = tail->seg[t.e];
+    t.nkb = (tail->seg[t.e + 1] - t.k0) / BK;
+  } else {
+    const TileCoord c = decode_tile<kPlain, PM>(tail->tstart, tail->seg, p.E, L);
+    t.e = c.e;
+    t.row0 = c.row0;
+    t.rows = c.rows;
+    t.m0 = 0;
+    t.n0 = c.n0;
+    t.k0 = 0;
+    t.nkb = (p.K + BK - 1) / BK;
+  }
+  return t;
+}
+
+template <int MODE, int ACT, bool A_MN, bool F16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const BwdParams p) {
+  constexpr uint32_t kIdesc = idesc_f16kind(PM, BN, F16) | (A_MN ? kIdescAMN : 0u) | kIdescBMN;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;   // the same offset in both CTAs
+  unsigned char* staging = smem_raw + (base - raw) + (size_t)PSTAGES * PSTAGE_BYTES;
+  PTail* tail = reinterpret_cast<PTail*>(staging + kStagingBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = (int)cluster_id(), npairs = (int)cluster_count();
+  const int ncols = (MODE == kWgrad) ? p.N : p.Nout;
+  const int nt = (ncols + BN - 1) / BN;
+
+  const uint32_t full0 = smem_u32(&tail->full[0]), empty0 = smem_u32(&tail->empty[0]);
+  const uint32_t tfull0 = smem_u32(&tail->tfull[0]), tempty0 = smem_u32(&tail->tempty[0]);
+  const uint32_t drain = smem_u32(&tail->drain);
+  const volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 8);
+    }
+    mbar_init(drain, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {   // the same warp in both CTAs allocates the pair's TMEM
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&tail->tmem_base)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (warp == 0) {
+    bool table_ok = true;
+    if (MODE == kWgrad) {
+      // every expert's segment must be a whole number of k-blocks inside the buffer
+      bool ok = true;
+      for (int e = lane; e < p.E; e += 32) {
+        const int a = p.offsets[e], b = p.offsets[e + 1];
+        ok &= a >= 0 && b >= a && b <= p.rows_alloc && (a % BK) == 0 && (b % BK) == 0;
+      }
+      table_ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) tail->tstart[p.E] = table_ok ? p.E * ((p.M + PM - 1) / PM) * nt : 0;
+    } else {
+      table_ok = tile_table_warp(p.offsets, p.E, PM, nt, p.rows_alloc, tail->tstart, lane);
+    }
+    if (!table_ok && lane == 0 && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
+  }
+  for (int e = threadIdx.x; e <= p.E; e += kThreads) tail->seg[e] = p.offsets[e];
+  tc_fence_before();
+  cluster_sync();              // both CTAs: barriers initialised, TMEM allocated, tile tables built
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+  const int total = tail->tstart[p.E];
+  // the even CTA's barriers and the peer's abort flag, as cluster addresses
+  const uint32_t full0_lead = cluster_addr(full0, 0), tempty0_lead = cluster_addr(tempty0, 0);
+  const uint32_t abort_peer = cluster_addr(smem_u32(&tail->abort_flag), rank ^ 1u);
+  auto give_up = [&]() {
+    atomicOr(p.status, MOE_DEV_TIMEOUT);
+    tail->abort_flag = 1;
+    st_cluster_u32(abort_peer, 1u);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int it = 0;
+      bool ok = true;
+      for (int L = pair; L < total && ok; L += npairs) {
+        const BwdTile t = bwd_tile_pair<MODE>(tail, p, L);
+        const int ncol = t.n0 + HN * (int)rank;
+        for (int kb = 0; kb < t.nkb; ++kb) {
+          const int s = it % PSTAGES;
+          const uint32_t ph = (uint32_t)(it / PSTAGES) & 1u;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+          const uint32_t sa = base + (uint32_t)(s * PSTAGE_BYTES);
+          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * PSTAGE_BYTES);   // both halves
+          if (A_MN) {   // this CTA's 128 M columns, rows along K: two 64-column boxes
+            const int krow = t.k0 + kb * BK, mcol = t.m0 + HM * (int)rank;
+            tma_load_2d_pair(sa, &tmA, full0_lead + 8 * s, mcol, krow);
+            tma_load_2d_pair(sa + kMNBox, &tmA, full0_lead + 8 * s, mcol + 64, krow);
+          } else {
+            tma_load_2d_pair(sa, &tmA, full0_lead + 8 * s, kb * BK, t.row0 + HM * (int)rank);
+          }
+          // B, MN-major: this CTA's 128 of the 256 N columns
+          const int brow = (MODE == kWgrad) ? t.k0 + kb * BK : t.e * p.b_krows + kb * BK;
+          tma_load_2d_pair(sa + PA_BYTES, &tmB, full0_lead + 8 * s, ncol, brow);
+          tma_load_2d_pair(sa + PA_BYTES + kMNBox, &tmB, full0_lead + 8 * s, ncol + 64, brow);
+          ++it;
+        }
+      }
+      if (!ok) give_up();
+      if (rank == 0) {
+        // the loads still in flight (of both CTAs) complete on these barriers
+        for (int i = max(0, it - PSTAGES); i < it; ++i)
+          mbar_wait(full0 + 8 * (i % PSTAGES), (uint32_t)(i / PSTAGES) & 1u, nullptr, kDrainNs);
+      } else if (!ok) {
+        // loads of this CTA whose phase the even CTA never armed: give them
+        // time to land before the shared memory can be released
+        const unsigned long long t0 = now_ns();
+        while (now_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------- MMA issuer
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int L = pair; L < total && ok; L += npairs, ++tl) {
+        const BwdTile t = bwd_tile_pair<MODE>(tail, p, L);
+        const int acc = tl & 1;
+        const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
+        if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < t.nkb; ++kb) {
+          const int s = it % PSTAGES;
+          const uint32_t ph = (uint32_t)(it / PSTAGES) & 1u;
+          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kWaitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + (uint32_t)(s * PSTAGE_BYTES);
+          const uint64_t ad = A_MN ? sdesc_mn(sa, kMNBox) : sdesc(sa);
+          const uint64_t bd = sdesc_mn(sa + PA_BYTES, kMNBox);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t astep = A_MN ? (uint64_t)(128 * kk) : (uint64_t)(2 * kk);
+            tc_mma_pair(d_tmem, ad + astep, bd + (uint64_t)(128 * kk), kIdesc, (kb | kk) != 0);
+          }
+          tc_commit_pair(empty0 + 8 * s, 0x3);   // stage s free again in both CTAs
+          ++it;
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull0 + 8 * acc, 0x3);   // accumulator ready in both CTAs
+      }
+      if (!ok) give_up();
+      tc_commit_pair(drain, 0x1);                // every MMA issued above has completed
+      mbar_wait(drain, 0, nullptr, kDrainNs);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)(warp - 2) * kStageWarpBytes);
+    const float inv_s = p.scale[1];
+    int tl = 0;
+    bool ok = true;
+    bool over = false;
+    for (int L = pair; L < total; L += npairs, ++tl) {
+      const BwdTile t = bwd_tile_pair<MODE>(tail, p, L);
+      const int acc = tl & 1;
+      const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
+      ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (MODE == kWgrad) {
+        const int m0 = t.m0 + HM * (int)rank + q * 32;
+        const int nrows = max(0, min(32, p.M - m0));
+        if (nrows > 0) {
+          if (t.nkb > 0) {
+            store_scaled(p.out + (size_t)t.e * p.M * p.N, p.N, tb, m0, nrows, t.n0, inv_s, stg, lane);
+          } else if (lane < nrows) {   // an expert without rows: its gradient is zero
+            float* dst = p.out + (size_t)t.e * p.M * p.N + (size_t)(m0 + lane) * p.N;
+            for (int c = t.n0; c < min(t.n0 + BN, p.N); c += 4)
+              *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      } else {
+        const int wrow0 = t.row0 + HM * (int)rank + q * 32;
+        int nrows = min(32, t.rows - HM * (int)rank - q * 32);
+        if (nrows > 0 && wrow0 + nrows > p.rows_alloc) {
+          if (lane == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
+          nrows = p.rows_alloc - wrow0;
+        }
+        if (nrows > 0) {
+          if (MODE == kDgradAct)
+            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, t.n0 / BN, stg, lane, inv_s, over);
+          else
+            store_scaled(p.out, p.Nout, tb, wrow0, nrows, t.n0, inv_s, stg, lane);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0_lead + 8 * acc);   // accumulator free again
+    }
+    if (F16 && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(p.status, MOE_DEV_RANGE);
+    if (!ok && lane == 0) give_up();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();              // the pair's MMAs and loads are done with both CTAs' shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+template <int MODE, int ACT, bool A_MN, bool F16>
+cudaError_t launch_bwd_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdParams& p, int pairs,
+                            cudaStream_t s) {
+  cudaError_t err = set_smem_once<tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>>(kPairSmemBytes);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>, dim3(2 * pairs), dim3(kThreads), kPairSmemBytes, s, ma,
+                    mb, p);
+}
+
 template <int MODE, int ACT, bool A_MN, bool B_MN, bool F16>
 cudaError_t launch_bwd(const CUtensorMap& ma, const CUtensorMap& mb, const BwdParams& p, int grid, cudaStream_t s) {
   cudaError_t err = set_smem_once<tc_bwd_gemm<MODE, ACT, A_MN, B_MN, F16>>(kSmemBytes);
@@ -482,7 +741,8 @@ cudaError_t launch_bwd(const CUtensorMap& ma, const CUtensorMap& mb, const BwdPa
 
 template <bool F16>
 cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const void* w1, const void* w2, float* dw1,
-                              float* dw2, int sms, cudaStream_t s) {
+                              float* dw2, int sms, bool pair, cudaStream_t s) {
+  const int max_pairs = std::max(1, sms / 2);
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
   const uint64_t R = (uint64_t)st.rows_alloc;
   const long long mt_max = (long long)(R / BM) + c.E;
@@ -505,27 +765,35 @@ cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const voi
   p.u = st.u;
   p.wrow = st.wrow;
   p.du = st.du;
-  p.du_b = F16 ? st.du_b : nullptr;
   p.hw = st.hw;
   p.dwpart = st.dwpart;
   p.F = c.F;
   p.F1 = F1;
-  int grid = (int)std::min<long long>(mt_max * ((c.F + BN - 1) / BN), sms);
-  err = (c.act == MOE_ACT_SWIGLU) ? launch_bwd<kDgradAct, kSwiglu, false, true, F16>(ma, mb, p, grid, s)
-                                  : launch_bwd<kDgradAct, kRelu, false, true, F16>(ma, mb, p, grid, s);
+  const long long pt_max = (long long)(R / PM) + c.E;   // pair m-tiles at most
+  if (pair) {
+    const int pairs = (int)std::min<long long>(pt_max * ((c.F + BN - 1) / BN), max_pairs);
+    err = (c.act == MOE_ACT_SWIGLU) ? launch_bwd_pair<kDgradAct, kSwiglu, false, F16>(ma, mb, p, pairs, s)
+                                    : launch_bwd_pair<kDgradAct, kRelu, false, F16>(ma, mb, p, pairs, s);
+  } else {
+    const int grid = (int)std::min<long long>(mt_max * ((c.F + BN - 1) / BN), sms);
+    err = (c.act == MOE_ACT_SWIGLU) ? launch_bwd<kDgradAct, kSwiglu, false, true, F16>(ma, mb, p, grid, s)
+                                    : launch_bwd<kDgradAct, kRelu, false, true, F16>(ma, mb, p, grid, s);
+  }
   if (err != cudaSuccess) return err;
 
-  // dxp = du W1[e] (K = F1), on the weights' own type: with fp16 operands du
-  // goes in its bf16 copy (still scaled by s), so W1 needs no fp16 copy
-  if (!make_map(&ma, F16 ? st.du_b : st.du, R, (uint64_t)F1, false) ||
-      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, false, 64))
+  // dxp = du W1[e] (K = F1)
+  if (!make_map(&ma, st.du, R, (uint64_t)F1, F16) ||
+      !make_map(&mb, w1, (uint64_t)c.E * F1, (uint64_t)c.d, F16, 64))
     return cudaErrorInvalidValue;
   p.K = F1;
   p.Nout = c.d;
   p.b_krows = F1;
   p.out = st.dxp;
-  grid = (int)std::min<long long>(mt_max * ((c.d + BN - 1) / BN), sms);
-  if ((err = launch_bwd<kDgradPlain, kRelu, false, true, false>(ma, mb, p, grid, s)) != cudaSuccess) return err;
+  err = pair ? launch_bwd_pair<kDgradPlain, kRelu, false, F16>(
+                   ma, mb, p, (int)std::min<long long>(pt_max * ((c.d + BN - 1) / BN), max_pairs), s)
+             : launch_bwd<kDgradPlain, kRelu, false, true, F16>(
+                   ma, mb, p, (int)std::min<long long>(mt_max * ((c.d + BN - 1) / BN), sms), s);
+  if (err != cudaSuccess) return err;
 
   // dW2[e] = dout_perm_e^T (w h)_e: M = d, N = F, K = the expert's padded rows
   if (!make_map(&ma, st.dout_perm, R, (uint64_t)c.d, F16, 64) || !make_map(&mb, st.hw, R, (uint64_t)c.F, F16, 64))
@@ -533,10 +801,15 @@ cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const voi
   p.M = c.d;
   p.N = c.F;
   p.out = dw2;
-  long long tiles = (long long)c.E * ((c.d + BM - 1) / BM) * ((c.F + BN - 1) / BN);
-  if ((err = launch_bwd<kWgrad, kRelu, true, true, F16>(ma, mb, p, (int)std::min<long long>(tiles, sms), s)) !=
-      cudaSuccess)
-    return err;
+  if (pair)
+    err = launch_bwd_pair<kWgrad, kRelu, true, F16>(
+        ma, mb, p,
+        (int)std::min<long long>((long long)c.E * ((c.d + PM - 1) / PM) * ((c.F + BN - 1) / BN), max_pairs), s);
+  else
+    err = launch_bwd<kWgrad, kRelu, true, true, F16>(
+        ma, mb, p, (int)std::min<long long>((long long)c.E * ((c.d + BM - 1) / BM) * ((c.F + BN - 1) / BN), sms),
+        s);
+  if (err != cudaSuccess) return err;
 
   // dW1[e] = du_e^T xp_e: M = F1, N = d
   if (!make_map(&ma, st.du, R, (uint64_t)F1, F16, 64) || !make_map(&mb, st.xp, R, (uint64_t)c.d, F16, 64))
@@ -544,19 +817,23 @@ cudaError_t launch_backward_t(const moe_config& c, const BwdState& st, const voi
   p.M = F1;
   p.N = c.d;
   p.out = dw1;
-  tiles = (long long)c.E * ((F1 + BM - 1) / BM) * ((c.d + BN - 1) / BN);
-  return launch_bwd<kWgrad, kRelu, true, true, F16>(ma, mb, p, (int)std::min<long long>(tiles, sms), s);
+  if (pair)
+    return launch_bwd_pair<kWgrad, kRelu, true, F16>(
+        ma, mb, p, (int)std::min<long long>((long long)c.E * ((F1 + PM - 1) / PM) * ((c.d + BN - 1) / BN), max_pairs),
+        s);
+  return launch_bwd<kWgrad, kRelu, true, true, F16>(
+      ma, mb, p, (int)std::min<long long>((long long)c.E * ((F1 + BM - 1) / BM) * ((c.d + BN - 1) / BN), sms), s);
 }
 
 }  // namespace
 
 cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
-                                      float* dw1, float* dw2, cudaStream_t s) {
+                                      float* dw1, float* dw2, bool pair, cudaStream_t s) {
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  return st.f16 ? launch_backward_t<true>(c, st, w1, w2, dw1, dw2, di.sms, s)
-                : launch_backward_t<false>(c, st, w1, w2, dw1, dw2, di.sms, s);
+  return st.f16 ? launch_backward_t<true>(c, st, w1, w2, dw1, dw2, di.sms, pair, s)
+                : launch_backward_t<false>(c, st, w1, w2, dw1, dw2, di.sms, pair, s);
 }
 
 int bwd_tc_col_tile() { return BN; }

@@ -151,20 +151,21 @@ struct BwdState {
   bool f16;
   unsigned* amax;            // max |dout| as float bits (zeroed before the amax kernel)
   float* scale;              // [2]: s, 1/s (1, 1 without fp16 operands)
-  void* xp_b;                // [rows][d]   bf16 x of each padded row (f16 only: the recomputed u in bf16)
-  void* du_b;                // [rows][F1]  bf16 copy of the scaled du (f16 only: the dxp GEMM in bf16)
+  void* w1h;                 // fp16 copy of W1 (f16), else unused
 };
 int bwd_pad_rows();
 int bwd_logit_slices(const moe_config& c);
 int bwd_tc_col_tile();     // columns of a tensor-core backward tile (the dw partials per row)
 int bwd_simt_col_tile();
 // bf16 -> fp16 (round to nearest even, saturating at +-65504)
+cudaError_t launch_convert_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t s);
 // prep (padded offsets, the dout scale) and gather (x, dout, gate weight of every padded row)
 cudaError_t launch_bwd_front(const moe_config& c, const void* x, const float* dout, const BwdState& st,
                              cudaStream_t s);
 // the expert layers' gradients: dh with the activation backward, dxp, dW2, dW1
+// pair: 2-SM pair tiles (256 x 256) for every GEMM, else 1-SM tiles (128 x 256)
 cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
-                                      float* dw1, float* dw2, cudaStream_t s);
+                                      float* dw1, float* dw2, bool pair, cudaStream_t s);
 cudaError_t launch_expert_backward_simt(const moe_config& c, const BwdState& st, const void* w1, const void* w2,
                                         float* dw1, float* dw2, cudaStream_t s);
 // out[rows][Nout] = A[rows][K] B_e[Nout][K]^T over the segments of offsets (E of them), fp32 out;

@@ -48,6 +48,11 @@ LAYERS = [
     W("b_E1", T=130, d=64, E=1, F=64, k=1, act=mw.RELU, dtype=mw.BF16, seed=75),
     W("b_fp32_relu", T=300, d=64, E=5, F=96, k=2, act=mw.RELU, dtype=mw.F32, capacity_factor=1.0, seed=76),
     W("b_fp32_swiglu", T=257, d=32, E=6, F=40, k=3, act=mw.SWIGLU, dtype=mw.F32, lam=0.5, seed=77),
+    # T*k >= 512*E: every expert GEMM of the backward on 2-SM pair tiles
+    # (ragged: F and F1 not multiples of 256, segments not multiples of 256)
+    W("b_pair_swiglu", T=1300, d=256, E=4, F=320, k=2, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True, seed=78),
+    W("b_pair_relu_cap", T=2600, d=192, E=8, F=448, k=2, act=mw.RELU, dtype=mw.BF16, capacity_factor=1.1,
+      seed=79),
 ]
 AUX, ZC = 0.05, 0.01
 
@@ -133,7 +138,7 @@ def test_backward_matches_oracle(w):
     print(w.name, {k: f"{v:.2e}" for k, v in rel.items()})
 
 
-@pytest.mark.parametrize("name", ["b_relu_cap", "b_wide", "b_fine_top6"])
+@pytest.mark.parametrize("name", ["b_relu_cap", "b_wide", "b_fine_top6", "b_pair_swiglu"])
 def test_backward_bf16_hidden(name):
     """A bf16 hidden type: the backward's GEMM operands are bf16 (no dout
     scale); the weight gradients meet the bf16 rounding bound."""
