@@ -46,6 +46,7 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 
 enum { kDgradAct = 0, kDgradPlain = 1, kWgrad = 2 };
+constexpr int kDwCols = 128;   // columns of F per partial of dw (half a 256-column tile)
 
 struct Tail {
   unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -150,22 +151,26 @@ __device__ __forceinline__ BwdTile bwd_tile(const Tail* tail, const BwdParams& p
   return t;
 }
 
-// The activation backward of one epilogue warp on its 32 rows x 256 columns
-// of G = dout_perm W2[e] (fp32 in TMEM): with u the pre-activation (staged
-// through shared memory 32 columns at a time), h = act(u), w the row's gate
-// weight: dh = w G, du = dh act'(u), hw = w h (the B operand of dW2), and the
-// row's sum of G h over these columns (its part of dw = <dout, y>).
+// The activation backward of one epilogue warp on its 32 rows and the
+// 32-column blocks [blk0, blk1) of a 256-column tile of G = dout_perm W2[e]
+// (fp32 in TMEM): with u the pre-activation (staged through shared memory 32
+// columns at a time), h = act(u), w the row's gate weight: dh = w G,
+// du = dh act'(u), hw = w h (the B operand of dW2), and the row's sums of
+// G h over each 128-column half of the tile (its parts of dw = <dout, y>,
+// one partial per 128 columns of F).  [blk0, blk1) is a whole number of halves.
 template <int ACT, bool F16>
 __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t tb, int wrow0, int nrows, int n0,
-                                                  int nti, uint4* stg, int lane, float inv_s, bool& over) {
+                                                  int blk0, int blk1, uint4* stg, int lane, float inv_s,
+                                                  bool& over) {
   const int row = wrow0 + lane;
   const bool live = lane < nrows;
   const float w = live ? p.wrow[row] : 0.f;
+  const int nhalf = (p.F + kDwCols - 1) / kDwCols;
   float dwp = 0.f;
 #pragma unroll 1
-  for (int blk = 0; blk < BN / 32; ++blk) {
+  for (int blk = blk0; blk < blk1; ++blk) {
     const int f0 = n0 + blk * 32;
-    if (f0 >= p.F) break;
+    if (f0 < p.F) {
     uint32_t g[32];
     tmem_ld32(tb + blk * 32, g);
     tmem_wait_ld();
@@ -247,8 +252,13 @@ __device__ __forceinline__ void act_backward_tile(const BwdParams& p, uint32_t t
           if (q < nv) dv_row[q] = make_uint4(du_v[4 * q], du_v[4 * q + 1], du_v[4 * q + 2], du_v[4 * q + 3]);
       }
     }
+    }
+    if ((blk & 3) == 3) {   // end of a 128-column half: its partial of dw
+      const int hi = n0 / kDwCols + blk / 4;
+      if (live && hi < nhalf) p.dwpart[(size_t)hi * p.rows_alloc + row] = dwp * inv_s;
+      dwp = 0.f;
+    }
   }
-  if (live) p.dwpart[(size_t)nti * p.rows_alloc + row] = dwp * inv_s;
 }
 
 // A_MN / B_MN: the operand is MN-major in memory (rows along K).  F16: both
@@ -431,7 +441,7 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         if (nrows > 0) {
           if (MODE == kDgradAct)
-            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, t.n0 / BN, stg, lane, inv_s, over);
+            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, 0, BN / 32, stg, lane, inv_s, over);
           else
             store_scaled(p.out, p.Nout, tb, wrow0, nrows, t.n0, inv_s, stg, lane);
         }
@@ -480,8 +490,19 @@ struct PTail {
   int tstart[kMaxExperts + 1];
   int seg[kMaxExperts + 1];
 };
-constexpr size_t kPairSmemBytes = 1024 + (size_t)PSTAGES * PSTAGE_BYTES + kStagingBytes + sizeof(PTail);
-static_assert(kPairSmemBytes <= 227 * 1024, "shared memory of one CTA");
+// The dh GEMM's epilogue (the activation backward, reading u and writing du
+// and w h) is the heaviest: it runs on eight warps, two per TMEM lane
+// quadrant, each taking one 128-column half of the tile, with five stages so
+// that their staging fits; the other modes keep four warps and six stages.
+__host__ __device__ constexpr int pair_epi_warps(int mode) { return mode == kDgradAct ? 8 : 4; }
+__host__ __device__ constexpr int pair_threads(int mode) { return 64 + 32 * pair_epi_warps(mode); }
+__host__ __device__ constexpr int pair_stages(int mode) { return mode == kDgradAct ? 5 : PSTAGES; }
+constexpr size_t pair_smem_bytes(int mode) {
+  return 1024 + (size_t)pair_stages(mode) * PSTAGE_BYTES + (size_t)pair_epi_warps(mode) * kStageWarpBytes +
+         sizeof(PTail);
+}
+static_assert(pair_smem_bytes(kDgradAct) <= 227 * 1024 && pair_smem_bytes(kWgrad) <= 227 * 1024,
+              "shared memory of one CTA");
 
 // Tile L of the pair kernels (256-row / 256-column tiles).
 template <int MODE>
@@ -512,15 +533,16 @@ __device__ __forceinline__ BwdTile bwd_tile_pair(const PTail* tail, const BwdPar
 }
 
 template <int MODE, int ACT, bool A_MN, bool F16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(MODE), 1)
 tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const BwdParams p) {
   constexpr uint32_t kIdesc = idesc_f16kind(PM, BN, F16) | (A_MN ? kIdescAMN : 0u) | kIdescBMN;
+  constexpr int kEpi = pair_epi_warps(MODE), kPT = pair_threads(MODE), kST = pair_stages(MODE);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;   // the same offset in both CTAs
-  unsigned char* staging = smem_raw + (base - raw) + (size_t)PSTAGES * PSTAGE_BYTES;
-  PTail* tail = reinterpret_cast<PTail*>(staging + kStagingBytes);
+  unsigned char* staging = smem_raw + (base - raw) + (size_t)kST * PSTAGE_BYTES;
+  PTail* tail = reinterpret_cast<PTail*>(staging + (size_t)kEpi * kStageWarpBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int pair = (int)cluster_id(), npairs = (int)cluster_count();
@@ -533,13 +555,13 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const volatile int* abort_flag = &tail->abort_flag;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PSTAGES; ++s) {
+    for (int s = 0; s < kST; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 8);
+      mbar_init(tempty0 + 8 * a, 2 * kEpi);
     }
     mbar_init(drain, 1);
     tail->abort_flag = 0;
@@ -572,7 +594,7 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     if (!table_ok && lane == 0 && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
   }
-  for (int e = threadIdx.x; e <= p.E; e += kThreads) tail->seg[e] = p.offsets[e];
+  for (int e = threadIdx.x; e <= p.E; e += kPT) tail->seg[e] = p.offsets[e];
   tc_fence_before();
   cluster_sync();              // both CTAs: barriers initialised, TMEM allocated, tile tables built
   tc_fence_after();
@@ -596,8 +618,8 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const BwdTile t = bwd_tile_pair<MODE>(tail, p, L);
         const int ncol = t.n0 + HN * (int)rank;
         for (int kb = 0; kb < t.nkb; ++kb) {
-          const int s = it % PSTAGES;
-          const uint32_t ph = (uint32_t)(it / PSTAGES) & 1u;
+          const int s = it % kST;
+          const uint32_t ph = (uint32_t)(it / kST) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, kWaitNs)) { ok = false; break; }
           const uint32_t sa = base + (uint32_t)(s * PSTAGE_BYTES);
           if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * PSTAGE_BYTES);   // both halves
@@ -618,8 +640,8 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (!ok) give_up();
       if (rank == 0) {
         // the loads still in flight (of both CTAs) complete on these barriers
-        for (int i = max(0, it - PSTAGES); i < it; ++i)
-          mbar_wait(full0 + 8 * (i % PSTAGES), (uint32_t)(i / PSTAGES) & 1u, nullptr, kDrainNs);
+        for (int i = max(0, it - kST); i < it; ++i)
+          mbar_wait(full0 + 8 * (i % kST), (uint32_t)(i / kST) & 1u, nullptr, kDrainNs);
       } else if (!ok) {
         // loads of this CTA whose phase the even CTA never armed: give them
         // time to land before the shared memory can be released
@@ -641,8 +663,8 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < t.nkb; ++kb) {
-          const int s = it % PSTAGES;
-          const uint32_t ph = (uint32_t)(it / PSTAGES) & 1u;
+          const int s = it % kST;
+          const uint32_t ph = (uint32_t)(it / kST) & 1u;
           if (!mbar_wait(full0 + 8 * s, ph, abort_flag, kWaitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + (uint32_t)(s * PSTAGE_BYTES);
@@ -665,7 +687,7 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3, half = (warp - 2) >> 2;   // half: 0, or 1 for the dh GEMM's second four warps
     uint4* stg = reinterpret_cast<uint4*>(staging + (size_t)(warp - 2) * kStageWarpBytes);
     const float inv_s = p.scale[1];
     int tl = 0;
@@ -701,7 +723,8 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         if (nrows > 0) {
           if (MODE == kDgradAct)
-            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, t.n0 / BN, stg, lane, inv_s, over);
+            act_backward_tile<ACT, F16>(p, tb, wrow0, nrows, t.n0, 4 * half, 4 * half + 4, stg, lane, inv_s,
+                                        over);
           else
             store_scaled(p.out, p.Nout, tb, wrow0, nrows, t.n0, inv_s, stg, lane);
         }
@@ -726,9 +749,10 @@ tc_bwd_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 template <int MODE, int ACT, bool A_MN, bool F16>
 cudaError_t launch_bwd_pair(const CUtensorMap& ma, const CUtensorMap& mb, const BwdParams& p, int pairs,
                             cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>>(kPairSmemBytes);
+  constexpr size_t smem = pair_smem_bytes(MODE);
+  cudaError_t err = set_smem_once<tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>>(smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>, dim3(2 * pairs), dim3(kThreads), kPairSmemBytes, s, ma,
+  return launch_pdl(tc_bwd_gemm_pair<MODE, ACT, A_MN, F16>, dim3(2 * pairs), dim3(pair_threads(MODE)), smem, s, ma,
                     mb, p);
 }
 
@@ -836,6 +860,6 @@ cudaError_t launch_expert_backward_tc(const moe_config& c, const BwdState& st, c
                 : launch_backward_t<false>(c, st, w1, w2, dw1, dw2, di.sms, pair, s);
 }
 
-int bwd_tc_col_tile() { return BN; }
+int bwd_tc_col_tile() { return kDwCols; }
 
 }  // namespace moe
