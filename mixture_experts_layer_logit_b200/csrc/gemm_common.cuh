@@ -161,8 +161,10 @@ __device__ __forceinline__ void store_tile(const Params& p, uint32_t tb, int wro
               a1 = fmaxf(a1, 0.f);
             } else {
               const float u0 = __uint_as_float(u[8 * i + 2 * j]), u1 = __uint_as_float(u[8 * i + 2 * j + 1]);
-              a0 = a0 / (1.f + __expf(-a0)) * u0;
-              a1 = a1 / (1.f + __expf(-a1)) * u1;
+              // silu(a) = a / (1 + e^-a) with the fast division (a few ulp; the
+              // denominator overflows to +inf only where silu is -0 anyway)
+              a0 = __fdividef(a0, 1.f + __expf(-a0)) * u0;
+              a1 = __fdividef(a1, 1.f + __expf(-a1)) * u1;
             }
             pk[j] = pack_hidden<F16>(a0, a1, row_over);
           }
