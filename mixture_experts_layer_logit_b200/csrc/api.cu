@@ -48,7 +48,6 @@ Scratch scratch_layout(const moe_config& c) {
   s.zsum = off;  off = align256(off + sizeof(float) * nch);
   s.status = off; off = align256(off + sizeof(uint32_t));
   s.mlp = off;    off = align256(off + (c.dtype == MOE_DTYPE_BF16 ? sizeof(int) * expert_mlp_counters(c) : 0));
-  s.kslice = off; off = align256(off + route_tc_scratch_bytes(c));
   s.total = off > 0 ? off : 256;
   return s;
 }
@@ -360,7 +359,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route(c, x, Wg, bg, topk_idx, topk_w, gap, at<int32_t>(ws, sc.hist),
                                at<float>(ws, sc.psum), at<int32_t>(ws, sc.ntie), at<float>(ws, sc.zsum),
-                               at<uint32_t>(ws, sc.status), at<char>(ws, sc.kslice), s);
+                               at<uint32_t>(ws, sc.status), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (c.T == 0) {   // empty batch: P_e and the z-loss are not defined
     if (prob_mean != nullptr && cudaMemsetAsync(prob_mean, 0xff, sizeof(float) * (size_t)c.E, s) != cudaSuccess)
@@ -500,7 +499,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* x, const void* W
   // histograms (the scatter scans them itself)
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
                                at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), at<float>(scr, sc.zsum),
-                               &stats->status, at<char>(scr, sc.kslice), s);
+                               &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   float* row_w = at<float>(ws, L.row_w);
   float* out_f = static_cast<float*>(out);
@@ -750,7 +749,7 @@ moe_status moe_layer_forward_mxfp8(const moe_config* cfg, const void* x, const v
   // steps 1-3 as the bf16 layer (the permuted rows in bf16, no fused combine)
   cudaError_t e = launch_route(c, x, Wg, bg, idx, w, at<float>(ws, L.gap), at<int32_t>(scr, sc.hist),
                                at<float>(scr, sc.psum), at<int32_t>(scr, sc.ntie), at<float>(scr, sc.zsum),
-                               &stats->status, at<char>(scr, sc.kslice), s);
+                               &stats->status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   st = permute_from_hist(c, x, idx, nullptr, c.T > 0 ? at<float>(scr, sc.psum) : nullptr,
                          c.T > 0 ? at<int32_t>(scr, sc.ntie) : nullptr, c.T > 0 ? at<float>(scr, sc.zsum) : nullptr,

@@ -26,7 +26,6 @@ struct Scratch {
   size_t zsum;      // float [nchunks]      per-chunk sums of squared log-partitions (router z-loss)
   size_t status;    // uint32               device error bits of a standalone moe_route
   size_t mlp;       // int32 [expert_mlp_counters] tile queue of the one-launch expert kernel (bf16)
-  size_t kslice;    // the route's K-slice arrival counters and partial logits (may be empty); last
   size_t total;
 };
 
@@ -40,19 +39,15 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Route: logits, normalisation, softmax, top-k; per-chunk histogram, probability
 // sums, near-tie counts and z-loss sums into scratch.  TX = float or __nv_bfloat16.
-// kscratch: route_tc_scratch_bytes(c) bytes (or NULL: no K-slice split).
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
                          int32_t* hist, float* psum, int32_t* ntie, float* zsum, uint32_t* status,
-                         void* kscratch, cudaStream_t s);
+                         cudaStream_t s);
 // The same on tcgen05 tensor cores (bf16, k <= 8).
 bool route_tc_supported(const moe_config& c);
-// Scratch bytes of the tensor-core route's model-width split (0 when it never
-// splits this layer): per-chunk arrival counters, then the partial logits.
-size_t route_tc_scratch_bytes(const moe_config& c);
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, float* zsum, uint32_t* status, void* kscratch, cudaStream_t s);
+                            int32_t* ntie, float* zsum, uint32_t* status, cudaStream_t s);
 // prob_mean[e] = sum over chunks of psum / T (fixed order).
 cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
 // *z_loss = sum over chunks of zsum / T (fixed order).

@@ -330,10 +330,10 @@ cudaError_t launch_route_t(const moe_config& c, const void* x, const void* wg, c
 cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, const float* bg,
                          int32_t* topk_idx, float* topk_w, float* gap,
                          int32_t* hist, float* psum, int32_t* ntie, float* zsum, uint32_t* status,
-                         void* kscratch, cudaStream_t s) {
+                         cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   if (route_tc_supported(c))
-    return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, kscratch, s);
+    return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s);
   if (c.dtype == MOE_DTYPE_BF16)
     return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);
   return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);

@@ -23,13 +23,13 @@
 // log-partitions (the router z-loss, Megatron-Core best-practice page,
 // "Megatron-Core MoE的关键特性") for the permutation step.
 //
-// A small batch with a wide model (decode: one chunk, d = 2048) would leave
-// the reduction to one SM, one ring of loads after another.  There the model
-// width is cut into up to 8 slices, one CTA each.  Every CTA writes its
-// partial logits to the scratch workspace and takes a ticket.  The last CTA
-// of the chunk to arrive adds the partials in slice order (the same sum
-// whichever CTA comes last) and runs the epilogue.  Nothing waits on another
-// CTA, so the split cannot stall.
+// A small batch would leave most SMs idle and each chunk's loads to one SM
+// (decode: one chunk, d = 2048).  There the model width is cut into up to 8
+// slices, one CTA each, and a chunk's slices run as one thread-block cluster:
+// each keeps its partial logits in its own shared memory, the CTAs add a
+// share of the rows over the slices in slice order through distributed
+// shared memory into CTA 0, and CTA 0 runs the epilogue.  The CTAs of a
+// cluster are co-scheduled, so the two cluster barriers cannot stall.
 #include "tc_ptx.cuh"
 
 #include <math.h>
@@ -48,7 +48,6 @@ constexpr int kThreads = RM * kSplit;
 constexpr int kMaxKeep = 9;        // top-(k+1) list length for k <= 8
 constexpr int kMaxKSlices = 8;     // CTAs that may share one chunk's model width
 constexpr int kKSliceMaxChunks = 74;           // only batches of at most this many chunks split
-constexpr size_t kKSliceBudget = 1u << 20;     // bytes of partial logits at most
 static_assert(RM == kChunk, "one CTA per routing chunk");
 
 struct RTail {
@@ -56,7 +55,6 @@ struct RTail {
   uint32_t tmem_base;
   int abort_flag;
   int ntie;
-  int ticket;                      // arrival order of this CTA among its chunk's slices
   int hist[kMaxExperts];
   float bias[kMaxExperts];
   float part[kSplit][4][RM];       // per quarter: sum, squares, max, exp-sum of each row
@@ -149,9 +147,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
                 int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-                float* __restrict__ zsum_out, int nch, uint32_t* __restrict__ status, int lists_off,
-                float* __restrict__ kpart,
-                int* __restrict__ karrive, int nks) {
+                float* __restrict__ zsum_out, int nch, uint32_t* __restrict__ status, int lists_off, int nks) {
   constexpr int k = KB;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -272,51 +268,24 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   __syncthreads();
   bool lead = true;   // this CTA finishes the chunk
   if (nks > 1) {
-    // partials [chunk][slice][row][expert] in fp32 (RM * E is a multiple of 4:
-    // 16-byte vectors); fence, then the ticket
-    const int nv = RM * E / 4;
-    float4* mine = reinterpret_cast<float4*>(kpart + ((size_t)chunk * nks + ks) * RM * E);
-    for (int v = tid; v < nv; v += kThreads) {
-      float z[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = 4 * v + u, r = i / E;
-        z[u] = Zall[(size_t)r * ldz + (i - r * E)];
-      }
-      mine[v] = make_float4(z[0], z[1], z[2], z[3]);
+    // The chunk's slices are one thread-block cluster, each slice's partial
+    // logits in its own shared memory.  CTA ks sums rows [r0, r1) of the
+    // chunk's real tokens over the slices, in slice order, adds the bias and
+    // stores them into CTA 0's rows; CTA 0 then runs the epilogue.
+    cluster_sync();   // every slice's partials are written
+    const int nrows = min(RM, T - t0);
+    const int r0 = (nrows * ks) / nks, r1 = (nrows * (ks + 1)) / nks;
+    const uint32_t zl = smem_u32(Zall);
+    const uint32_t zdst = cluster_addr(zl, 0);
+    for (int i = tid; i < (r1 - r0) * E; i += kThreads) {
+      const int rr = i / E, e = i - rr * E;
+      const uint32_t off = (uint32_t)(((r0 + rr) * ldz + e) * 4);
+      float z = 0.f;
+      for (int sl = 0; sl < nks; ++sl) z += ld_cluster_f32(cluster_addr(zl, (uint32_t)sl) + off);
+      st_cluster_f32(zdst + off, z + tail->bias[e]);
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) tail->ticket = atomicAdd(&karrive[chunk], 1);
-    __syncthreads();
-    lead = tail->ticket == nks - 1;
-    if (lead) {
-      __threadfence();
-      // every slice's vector is loaded before any is added, so the loads
-      // overlap; the additions run in slice order
-      const float4* c0 = reinterpret_cast<const float4*>(kpart + (size_t)chunk * nks * RM * E);
-      for (int v = tid; v < nv; v += kThreads) {
-        float4 p[kMaxKSlices];
-#pragma unroll
-        for (int sl = 0; sl < kMaxKSlices; ++sl)
-          if (sl < nks) p[sl] = __ldcg(c0 + (size_t)sl * nv + v);
-        float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int sl = 0; sl < kMaxKSlices; ++sl)
-          if (sl < nks) {
-            z[0] += p[sl].x;
-            z[1] += p[sl].y;
-            z[2] += p[sl].z;
-            z[3] += p[sl].w;
-          }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = 4 * v + u, r = i / E, e = i - r * E;
-          Zall[(size_t)r * ldz + e] = z[u] + tail->bias[e];
-        }
-      }
-    }
-    __syncthreads();
+    cluster_sync();   // CTA 0 holds the sums; no CTA reads a peer's memory any more
+    lead = ks == 0;
   }
   if (lead) {
     const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
@@ -435,24 +404,23 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 
 // Slices of the model width per chunk: doubled while the reduction takes more
 // than one round of the stage ring, each slice keeps at least half a ring of
-// k-blocks, the grid stays within one CTA per SM and the partials within the
-// budget.
+// k-blocks and the grid stays within one CTA per SM; only batches of at most
+// 74 chunks split.  A chunk's slices form one cluster of at most 8 CTAs.  (A
+// split of the FastMoE layer's one-ring reduction over pairs ran 6 us slower:
+// its epilogue, not its loads, sets the kernel's time.)
 int kslices(const moe_config& c, long long sms) {
   const int EP = ((c.E + 15) / 16) * 16;
   const int nch = num_chunks(c.T), nkb = (c.d + RK - 1) / RK, nst = num_stages(EP);
   if (nkb <= nst || nch > kKSliceMaxChunks) return 1;
   int n = 1;
-  while (n < kMaxKSlices && (long long)nch * n * 2 <= sms && nkb / (n * 2) >= nst / 2 &&
-         (size_t)nch * n * 2 * RM * c.E * sizeof(float) <= kKSliceBudget)
-    n *= 2;
+  while (n < kMaxKSlices && (long long)nch * n * 2 <= sms && nkb / (n * 2) >= nst / 2) n *= 2;
   return n;
 }
-size_t karrive_bytes(int nch) { return ((size_t)nch * sizeof(int) + 255) & ~(size_t)255; }
 
 template <int KB>
 cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
                       int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
-                      float* zsum, uint32_t* status, void* kscratch, cudaStream_t s) {
+                      float* zsum, uint32_t* status, cudaStream_t s) {
   // the most any E <= kMaxExperts needs, so one attribute serves every launch
   static const size_t kMaxSmem = [] {
     size_t m = 0;
@@ -464,30 +432,33 @@ cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensor
   DeviceInfo di;
   if ((err = device_info(&di)) != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
-  const int nks = kscratch != nullptr ? kslices(c, di.sms) : 1;
-  int* karrive = static_cast<int*>(kscratch);
-  float* kpart = nks > 1 ? reinterpret_cast<float*>(static_cast<char*>(kscratch) + karrive_bytes(nch)) : nullptr;
-  if (nks > 1 && (err = cudaMemsetAsync(karrive, 0, sizeof(int) * (size_t)nch, s)) != cudaSuccess) return err;
-  return launch_pdl(route_tc_kernel<KB>, dim3(nch * nks), dim3(kThreads), smem_bytes(c.E, EP), s, mx, mw, bg, c.T,
-                    c.d, c.E, EP, num_stages(EP), c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch, status,
-                    (int)lists_offset(c.E, EP), kpart, karrive, nks);
+  const int nks = kslices(c, di.sms);
+  // PDL, and a chunk's slices as one cluster (nks consecutive CTAs)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nch * nks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes(c.E, EP);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)nks;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, route_tc_kernel<KB>, mx, mw, bg, c.T, c.d, c.E, EP, num_stages(EP), c.lambda, idx,
+                            w, gap, hist, psum, ntie, zsum, nch, status, (int)lists_offset(c.E, EP), nks);
 }
 
 }  // namespace
 
 bool route_tc_supported(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 && c.k <= 8; }
 
-size_t route_tc_scratch_bytes(const moe_config& c) {
-  if (!route_tc_supported(c) || c.T <= 0) return 0;
-  const int n = kslices(c, 1LL << 30);   // the most any device could choose
-  if (n == 1) return 0;
-  const int nch = num_chunks(c.T);
-  return karrive_bytes(nch) + (size_t)nch * n * RM * c.E * sizeof(float);
-}
-
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, float* zsum, uint32_t* status, void* kscratch, cudaStream_t s) {
+                            int32_t* ntie, float* zsum, uint32_t* status, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const int EP = ((c.E + 15) / 16) * 16;
   CUtensorMap mx, mw;
@@ -495,7 +466,7 @@ cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, 
       !make_map(&mw, wg, (uint64_t)c.E, (uint64_t)c.d, false, (uint32_t)EP))
     return cudaErrorInvalidValue;
 #define MOE_ROUTE_K(K) \
-  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, kscratch, s)
+  case K: return launch_kb<K>(c, mx, mw, EP, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s)
   switch (c.k) {
     MOE_ROUTE_K(1); MOE_ROUTE_K(2); MOE_ROUTE_K(3); MOE_ROUTE_K(4);
     MOE_ROUTE_K(5); MOE_ROUTE_K(6); MOE_ROUTE_K(7); MOE_ROUTE_K(8);

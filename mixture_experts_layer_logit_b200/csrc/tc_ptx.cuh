@@ -193,6 +193,14 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr_, uint32_t 
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr_) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr_) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr_, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr_), "f"(v) : "memory");
+}
 __device__ __forceinline__ void fence_mbar_init_cluster() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

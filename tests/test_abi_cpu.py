@@ -186,24 +186,19 @@ def test_static_scratch_limit_as_documented(L):
     assert abs(t_f32 - 345_000) < 1_000, t_f32
 
 
-def test_route_split_scratch_only_for_wide_layers_on_few_chunks(L):
-    # the gate GEMM is cut over the model width (partial logits in scratch)
-    # only when its reduction needs more than one ring of loads and the batch
-    # has at most 74 chunks of 128 tokens: decode (d = 2048, one chunk) splits
-    # 8 ways, 8 x 128 x 64 fp32 partials; FastMoE (d = 512) and a batch of
-    # 128 chunks do not
-    decode = moe.moe_scratch_size(cfg(T=64, d=2048, E=64, F=1408, k=6, act="swiglu"))
-    assert decode >= 8 * 128 * 64 * 4
-    fastmoe = moe.moe_scratch_size(cfg(T=8192, d=512, E=64, F=1024, k=2))
-    wide_many = moe.moe_scratch_size(cfg(T=16384, d=2048, E=64, F=1408, k=6, act="swiglu"))
-    narrow = moe.moe_scratch_size(cfg(T=64, d=512, E=64, F=1408, k=6, act="swiglu"))
-    assert narrow < 8 * 128 * 64 * 4
-    # no partials: every byte is accounted for by the per-chunk tables and the
-    # tile-queue counters (a few 256-byte alignment pads aside)
-    for s, T, k in ((fastmoe, 8192, 2), (wide_many, 16384, 6)):
+def test_route_scratch_holds_no_partial_logits(L):
+    # the gate GEMM's model-width split (decode: 8 slices of one chunk) sums
+    # its partial logits inside a thread-block cluster, through distributed
+    # shared memory, so the scratch is the per-chunk tables and the
+    # tile-queue counters alone (a few 256-byte alignment pads aside) on
+    # every layer, split or not
+    for T, d, F, k, act in ((64, 2048, 1408, 6, "swiglu"), (8192, 512, 1024, 2, "relu"),
+                            (16384, 2048, 1408, 6, "swiglu"), (64, 512, 1408, 6, "swiglu")):
+        s = moe.moe_scratch_size(cfg(T=T, d=d, E=64, F=F, k=k, act=act))
         nch = (T + 127) // 128
         tables = 4 * (3 * 64 * nch + nch + 1) + 4 * (2 + T * k // 128 + 64)
-        assert s <= tables + 8 * 256, (s, tables)
+        assert s <= tables + 8 * 256, (T, d, s, tables)
+    assert moe.moe_scratch_size(cfg(T=64, d=2048, E=64, F=1408, k=6, act="swiglu")) < 8 * 128 * 64 * 4
 
 
 def test_adaptive_aux_coef_on_the_host_follows_the_oracle(L):
