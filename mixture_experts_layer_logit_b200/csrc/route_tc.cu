@@ -130,8 +130,15 @@ __device__ __forceinline__ float topk_range(TopList<KB>& top, const float* Z, in
 }
 template <int N, int KB>
 __device__ __forceinline__ void topk_merge(TopList<KB>& top, const float (*lv)[RM], const int (*li)[RM], int row) {
+  // the later list is sorted best first and its experts all have higher
+  // indices: once a pair fails to beat the kept N-th score (strictly), so do
+  // all after it
 #pragma unroll
-  for (int j = 0; j < N; ++j) top.template insert<N>(lv[j][row], li[j][row]);
+  for (int j = 0; j < N; ++j) {
+    const float sc = lv[j][row];
+    if (!(sc > top.v[N - 1])) break;
+    top.template insert<N>(sc, li[j][row]);
+  }
 }
 
 // Score the top-k is taken on: the biased logit, or its normalised value.
