@@ -563,8 +563,9 @@ scatter_generic_kernel(const TX* __restrict__ x, const int32_t* __restrict__ top
 // blocks per SM), every block stages its slice of x in shared memory before
 // it waits for the routing kernel (slices of up to kSliceVec 16-byte vectors,
 // 64 KB for a 128-token chunk), so the reads overlap that kernel.  Otherwise
-// blocks read x directly, and rows are cut into slices of at least 32 vectors
-// until there are about two blocks per SM.
+// blocks read x directly, and rows are cut into as many slices (of at least
+// 32 vectors) as keep the grid within one wave of two blocks per SM: a
+// second, partly filled wave cost more than the longer rows per block.
 constexpr int kSliceVec = 32;
 
 inline bool scatter_staged(int nch, int nvec, int sms) {
@@ -576,7 +577,7 @@ inline int scatter_slices(int nch, int nvec, bool staged, int sms, int* slice_ve
   if (staged) {
     S = (nvec + kSliceVec - 1) / kSliceVec;
   } else {
-    S = (2 * sms + nch - 1) / nch;
+    S = (2 * sms) / nch;
     S = std::min(S, nvec / 32);
   }
   S = std::max(S, 1);

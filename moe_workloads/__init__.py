@@ -113,7 +113,7 @@ WORKLOADS: Dict[str, Workload] = {
 # one GPU (Mixtral-8x7B shape, 11.5 TFLOP of expert GEMMs per forward).
 BENCH_WORKLOAD = "mixtral_8x7b"
 # Further workloads the bench times on the device and reports beside it.
-BENCH_EXTRA_WORKLOADS = ("fastmoe_txl", "fine_decode_dropless")
+BENCH_EXTRA_WORKLOADS = ("fastmoe_txl", "fine_decode_dropless", "fine_large_dropless")
 
 
 # ---------------------------------------------------------------- bf16 helpers
