@@ -537,10 +537,13 @@ def mxfp8_measure(moe, name: str, a, flush, pk, dev):
     touched = int(np.sum(np.diff(offs) > 0))
     F1 = w.F1
     wbytes = touched * (F1 * w.d + w.d * w.F) * (1 + 1 / 32)   # E4M3 elements + one scale byte per 32
+    kept = int(offs[-1])
+    flops = 2.0 * kept * w.d * (F1 + w.F)
     res = {"value": w.T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "workload": name,
            "weights": "MX FP8 (E4M3, UE8M0 scale per 32 along K), both expert layers",
            "touched_expert_weight_bytes": wbytes,
-           "weight_stream_gbs_over_whole_forward": wbytes / (ms * 1e-3) / 1e9}
+           "weight_stream_gbs_over_whole_forward": wbytes / (ms * 1e-3) / 1e9,
+           "expert_flops": flops, "tflops_over_whole_forward": flops / (ms * 1e-3) / 1e12}
     del g, L, ws, w1q, w1s, w2q, w2s
     torch.cuda.empty_cache()
     return res
@@ -726,6 +729,8 @@ def main():
 
     if world == 1 and not a.no_fp8:
         extra["fine_decode_dropless_mxfp8"] = mxfp8_measure(moe, "fine_decode_dropless", a, flush, pk, dev)
+        if a.workload != "fine_decode_dropless":
+            extra[a.workload + "_mxfp8"] = mxfp8_measure(moe, a.workload, a, flush, pk, dev)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
