@@ -152,7 +152,11 @@ size_t moe_workspace_size(const moe_config* cfg, moe_ws_layout* layout);
  * "图4" (top-2 gate: the two highest-scoring experts are activated).
  *   x[T, d], Wg[E, d] (cfg dtype); bg[E] fp32 or NULL (no bias).
  *   topk_idx[T, k] int32: selected experts, best first; equal scores resolve
- *     to the lower expert index.
+ *     to the lower expert index.  A NaN or -inf score is never selected: a
+ *     token with fewer than k scores above -inf (NaN logits) keeps 2^31 - 1
+ *     in its remaining slots, which the permutation drops; in
+ *     moe_layer_forward such a token sets MOE_DEV_BOUNDS and its output row
+ *     is 0.
  *   topk_w[T, k] fp32: softmax probabilities of the selected experts divided
  *     by their sum (they sum to 1).
  *   gap[T] fp32: k-th minus (k+1)-th largest score (z_hat or z), +inf if k == E.

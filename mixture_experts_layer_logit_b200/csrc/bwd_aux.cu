@@ -303,7 +303,7 @@ gate_bwd_kernel(const float* __restrict__ zpart, int nks, const float* __restric
     }
     sd = sqrtf(warp_sum(q) / (float)E);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) s[i] = (sd > 0.f) ? lam * (zv[i] - mu) / sd : 0.f;
+    for (int i = 0; i < PER; ++i) s[i] = (sd == 0.f) ? 0.f : lam * (zv[i] - mu) / sd;   // as the forward
   } else {
 #pragma unroll
     for (int i = 0; i < PER; ++i) s[i] = zv[i];
@@ -369,7 +369,7 @@ gate_bwd_kernel(const float* __restrict__ zpart, int nks, const float* __restric
 #pragma unroll
   for (int i = 0; i < PER; ++i) ds[i] = ok[i] ? p[i] * (dp[i] - dpp) + zs * p[i] : 0.f;
   if (lam > 0.f) {
-    if (sd > 0.f) {
+    if (sd != 0.f) {
       float a = 0.f, b = 0.f;
 #pragma unroll
       for (int i = 0; i < PER; ++i) {

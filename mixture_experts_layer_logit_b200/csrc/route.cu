@@ -67,7 +67,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
              int T, int d, int E, int k, float lam,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, float* __restrict__ gap_out,
              int32_t* __restrict__ hist_out, float* __restrict__ psum_out, int32_t* __restrict__ ntie_out,
-             float* __restrict__ zsum_out, int nch) {
+             float* __restrict__ zsum_out, int nch, uint32_t* __restrict__ status) {
   using L = RouteSmem<NJ>;
   constexpr int EP = L::EP;
   constexpr int V = VecLoad<TX>::N;
@@ -181,7 +181,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
       }
       const float sd = sqrtf(warp_sum(q) / (float)E);
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) v[i] = (sd > 0.f) ? lam * (v[i] - mu) / sd : 0.f;
+      for (int i = 0; i < EPL; ++i) v[i] = (sd == 0.f) ? 0.f : lam * (v[i] - mu) / sd;   // NaN spread stays NaN
     }
     float m = -INFINITY;
 #pragma unroll
@@ -203,7 +203,10 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
       pacc[i] += p[i];
     }
 
-    // top-k by repeated warp argmax; equal scores -> lower expert index
+    // top-k by repeated warp argmax; equal scores -> lower expert index; a NaN
+    // or -inf score is never taken, so a row with fewer than k scores above
+    // -inf keeps empty slots (out of range: dropped by the permutation, and
+    // flagged)
     unsigned taken = 0u;
     float kth = 0.f, gap = INFINITY;
     const int rounds = (k < E) ? k + 1 : k;
@@ -212,7 +215,7 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
       int bi = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
-        if (ok[i] && !((taken >> i) & 1u) && (v[i] > bv || bi == 0x7fffffff)) {
+        if (ok[i] && !((taken >> i) & 1u) && v[i] > bv) {
           bv = v[i];
           bi = lane + 32 * i;
         }
@@ -244,7 +247,8 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
       const int e = seli[warp][j];
       topk_idx[(size_t)t * k + j] = e;
       topk_w[(size_t)t * k + j] = selp[warp][j] * rs;
-      atomicAdd(&shist[e], 1);
+      if ((unsigned)e < (unsigned)E) atomicAdd(&shist[e], 1);
+      else atomicOr(status, MOE_DEV_BOUNDS);
     }
     if (lane == 0) {
       gap_out[t] = gap;
@@ -303,26 +307,27 @@ __global__ void prob_mean_kernel(const float* __restrict__ psum, int nch, int E,
 template <int NJ, typename TX>
 cudaError_t launch_route_nj(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* idx, float* w, float* gap, int32_t* hist, float* psum,
-                            int32_t* ntie, float* zsum, cudaStream_t s) {
+                            int32_t* ntie, float* zsum, uint32_t* status, cudaStream_t s) {
   const size_t smem = RouteSmem<NJ>::total;
   auto kern = route_kernel<NJ, TX>;
   cudaError_t err = set_smem_once<route_kernel<NJ, TX>>(smem);
   if (err != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
   kern<<<nch, kThreads, smem, s>>>(static_cast<const TX*>(x), static_cast<const TX*>(wg), bg,
-                                   c.T, c.d, c.E, c.k, c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch);
+                                   c.T, c.d, c.E, c.k, c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch,
+                                   status);
   return cudaGetLastError();
 }
 
 template <typename TX>
 cudaError_t launch_route_t(const moe_config& c, const void* x, const void* wg, const float* bg,
                            int32_t* idx, float* w, float* gap, int32_t* hist, float* psum,
-                           int32_t* ntie, float* zsum, cudaStream_t s) {
-  if (c.E <= 16) return launch_route_nj<1, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
-  if (c.E <= 32) return launch_route_nj<2, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
-  if (c.E <= 64) return launch_route_nj<4, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
-  if (c.E <= 128) return launch_route_nj<8, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
-  return launch_route_nj<16, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, s);
+                           int32_t* ntie, float* zsum, uint32_t* status, cudaStream_t s) {
+  if (c.E <= 16) return launch_route_nj<1, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, status, s);
+  if (c.E <= 32) return launch_route_nj<2, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, status, s);
+  if (c.E <= 64) return launch_route_nj<4, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, status, s);
+  if (c.E <= 128) return launch_route_nj<8, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, status, s);
+  return launch_route_nj<16, TX>(c, x, wg, bg, idx, w, gap, hist, psum, ntie, zsum, status, s);
 }
 
 }  // namespace
@@ -335,8 +340,8 @@ cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, con
   if (route_tc_supported(c))
     return launch_route_tc(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s);
   if (c.dtype == MOE_DTYPE_BF16)
-    return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);
-  return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, s);
+    return launch_route_t<__nv_bfloat16>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s);
+  return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s);
 }
 
 cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s) {

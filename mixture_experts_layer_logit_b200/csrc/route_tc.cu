@@ -23,12 +23,15 @@
 // log-partitions (the router z-loss, Megatron-Core best-practice page,
 // "Megatron-Core MoE的关键特性") for the permutation step.
 //
-// A small batch would leave most SMs idle and each chunk's loads to one SM
-// (decode: one chunk, d = 2048).  There the model width is cut into up to 8
-// slices, one CTA each, and a chunk's slices run as one thread-block cluster:
-// each keeps its partial logits in its own shared memory, the CTAs add a
-// share of the rows over the slices in slice order through distributed
-// shared memory into CTA 0, and CTA 0 runs the epilogue.  The CTAs of a
+// A small batch would leave most SMs idle and each chunk's loads and gating
+// to one SM (decode: one chunk, d = 2048).  There the model width is cut into
+// up to 8 slices, one CTA each, and a chunk's slices run as one thread-block
+// cluster: each keeps its partial logits in its own shared memory, and each
+// CTA adds its share of the chunk's rows over the slices, in slice order,
+// through distributed shared memory.  It then gates those rows itself, one
+// warp per token: butterfly reductions for the row statistics and k + 1
+// rounds of a warp-wide arg-max (shuffles) for the top-(k+1).  The CTAs'
+// histograms and sums meet in CTA 0, added in slice order.  The CTAs of a
 // cluster are co-scheduled, so the two cluster barriers cannot stall.
 #include "tc_ptx.cuh"
 
@@ -141,9 +144,118 @@ __device__ __forceinline__ void topk_merge(TopList<KB>& top, const float (*lv)[R
   }
 }
 
-// Score the top-k is taken on: the biased logit, or its normalised value.
+// Score the top-k is taken on: the biased logit, or its normalised value
+// (zero spread -> 0; a NaN spread, from a NaN logit, leaves NaN scores).
 __device__ __forceinline__ float gate_score(float zb, float lam, float mu, float sd) {
-  return lam > 0.f ? (sd > 0.f ? lam * (zb - mu) / sd : 0.f) : zb;
+  return lam > 0.f ? (sd == 0.f ? 0.f : lam * (zb - mu) / sd) : zb;
+}
+
+// The partial results of each CTA of a cluster, gathered in CTA 0 (they live
+// where the quarter lists would: the split epilogue has none).
+struct RSlots {
+  float psum[kMaxKSlices][kMaxExperts];
+  int hist[kMaxKSlices][kMaxExperts];
+  int ntie[kMaxKSlices];
+  float zsum[kMaxKSlices];
+};
+static_assert(sizeof(RSlots) <= sizeof(RLists), "the slots reuse the lists' space");
+
+// One warp gates one token row Z[0, E) (biased logits, in shared memory) on
+// its own: lane l owns experts l, l + 32, ...  Mean, spread and the softmax
+// sum are butterfly reductions (every lane ends with the same value); the
+// top-(k+1) comes from k + 1 rounds of a warp-wide arg-max over the lanes'
+// sorted local lists, ordered by score and then by the lower index, so the
+// lowest index wins equal scores, and the first round's winner is the row's
+// maximum.  Afterwards Z holds the row's softmax probabilities (zeros for an
+// invalid row); lane j < k writes slot j.
+template <int KB>
+__device__ __forceinline__ void gate_row_warp(float* Z, int E, float lam, int t, bool valid, int lane,
+                                              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                              float* __restrict__ gap_out, int* hist, int* ntie, float* zrow,
+                                              uint32_t* status) {
+  constexpr int k = KB;
+  if (lam > 0.f) {   // z_hat = lambda (z - mean) / std, written over z
+    float s = 0.f;
+    for (int e = lane; e < E; e += 32) s += Z[e];
+    const float mu = warp_sum(s) / (float)E;
+    float qq = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      const float dv = Z[e] - mu;
+      qq += dv * dv;
+    }
+    const float sd = sqrtf(warp_sum(qq) / (float)E);
+    for (int e = lane; e < E; e += 32) Z[e] = gate_score(Z[e], lam, mu, sd);
+  }
+  TopList<KB> top;
+  top.init();
+  for (int e = lane; e < E; e += 32) top.template insert<KB + 1>(Z[e], e);
+  // k + 1 rounds: the best head of the 32 local lists, then its owner pops it
+  float wv[KB + 1];
+  int wi[KB + 1];
+#pragma unroll
+  for (int r = 0; r <= KB; ++r) {
+    float cv = top.v[0];
+    int ci = top.i[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, cv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, ci, o);
+      const bool take = ov > cv || (ov == cv && oi < ci);
+      cv = take ? ov : cv;
+      ci = take ? oi : ci;
+    }
+    wv[r] = cv;
+    wi[r] = ci;
+    const bool pop = top.i[0] == ci;
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      top.v[j] = pop ? top.v[j + 1] : top.v[j];
+      top.i[j] = pop ? top.i[j + 1] : top.i[j];
+    }
+    top.v[KB] = pop ? -INFINITY : top.v[KB];
+    top.i[KB] = pop ? TopList<KB>::kEmpty : top.i[KB];
+  }
+  // the first winner is the row's largest score (-inf when no score is a
+  // number above -inf, as the maximum over the row would be)
+  const float m = wv[0];
+  float Sh = 0.f;
+  for (int e = lane; e < E; e += 32) {   // unnormalised probabilities over the scores
+    const float pe = __expf(Z[e] - m);
+    Z[e] = pe;
+    Sh += pe;
+  }
+  const float S = warp_sum(Sh);
+  const float invS = 1.f / S;
+  float psel[KB], sel = 0.f;
+#pragma unroll
+  for (int j = 0; j < KB; ++j) {
+    psel[j] = __expf(wv[j] - m) * invS;
+    sel += psel[j];                     // slot order
+  }
+  const float rs = 1.f / sel;
+  const float gap = (k < E) ? wv[k - 1] - wv[k] : INFINITY;
+  if (valid) {
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      if (lane == j) {
+        topk_idx[(size_t)t * k + j] = wi[j];
+        topk_w[(size_t)t * k + j] = psel[j] * rs;
+        // a row with fewer than k scores above -inf (NaN logits) keeps empty
+        // slots: out of range, dropped by the permutation, and flagged
+        if ((unsigned)wi[j] < (unsigned)E) atomicAdd(&hist[wi[j]], 1);
+        else atomicOr(status, MOE_DEV_BOUNDS);
+      }
+    }
+    if (lane == 0) {
+      gap_out[t] = gap;
+      if (gap < MOE_NEAR_TIE_GAP) atomicAdd(ntie, 1);
+    }
+  }
+  if (lane == 0) {
+    const float lse = m + logf(S);   // log sum_e exp(score): the router z-loss term of this row
+    *zrow = valid ? lse * lse : 0.f;
+  }
+  for (int e = lane; e < E; e += 32) Z[e] = valid ? Z[e] * invS : 0.f;
 }
 
 // KB is the exact number of experts per token, so that every index into the
@@ -261,7 +373,9 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   float* Zall = reinterpret_cast<float*>(sbase);   // [RM][ldz]
   float* Z = Zall + (size_t)row * ldz;
   const int nch32 = (E + 31) / 32;
-  for (int c = qtr; c < nch32; c += kSplit) {
+  // a split chunk's rows past the batch are never read: their warps skip the copy
+  const int ncopy = (nks == 1 || q * 32 < T - t0) ? nch32 : 0;
+  for (int c = qtr; c < ncopy; c += kSplit) {
     uint32_t r[32];
     tmem_ld32(tb + c * 32, r);
     tmem_wait_ld();
@@ -273,27 +387,103 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
-  bool lead = true;   // this CTA finishes the chunk
   if (nks > 1) {
     // The chunk's slices are one thread-block cluster, each slice's partial
     // logits in its own shared memory.  CTA ks sums rows [r0, r1) of the
-    // chunk's real tokens over the slices, in slice order, adds the bias and
-    // stores them into CTA 0's rows; CTA 0 then runs the epilogue.
+    // chunk's real tokens over the slices, in slice order, adds the bias,
+    // keeps them in its own rows and gates them, one warp per row.  Its
+    // histogram, probability sums, near-tie count and z-loss sum go into CTA
+    // 0's slots, which CTA 0 adds in slice order.
     cluster_sync();   // every slice's partials are written
     const int nrows = min(RM, T - t0);
     const int r0 = (nrows * ks) / nks, r1 = (nrows * (ks + 1)) / nks;
-    const uint32_t zl = smem_u32(Zall);
-    const uint32_t zdst = cluster_addr(zl, 0);
-    for (int i = tid; i < (r1 - r0) * E; i += kThreads) {
-      const int rr = i / E, e = i - rr * E;
-      const uint32_t off = (uint32_t)(((r0 + rr) * ldz + e) * 4);
-      float z = 0.f;
-      for (int sl = 0; sl < nks; ++sl) z += ld_cluster_f32(cluster_addr(zl, (uint32_t)sl) + off);
-      st_cluster_f32(zdst + off, z + tail->bias[e]);
+    uint32_t zsl[kMaxKSlices];   // Zall in each slice's shared memory
+#pragma unroll
+    for (int sl = 0; sl < kMaxKSlices; ++sl) zsl[sl] = sl < nks ? cluster_addr(smem_u32(Zall), (uint32_t)sl) : 0u;
+    // up to four elements per pass, all their loads issued before the first sum
+    constexpr int kU = 4;
+    const int nel = (r1 - r0) * E;
+    for (int i0 = tid; i0 < nel; i0 += kU * kThreads) {
+      float v[kU][kMaxKSlices];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * kThreads;
+        const int rr = i / E, e = i - rr * E;
+        const uint32_t off = (uint32_t)(((r0 + rr) * ldz + e) * 4);
+#pragma unroll
+        for (int sl = 0; sl < kMaxKSlices; ++sl) v[u][sl] = (sl < nks && i < nel) ? ld_cluster_f32(zsl[sl] + off) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i >= nel) break;
+        const int rr = i / E, e = i - rr * E;
+        float z = 0.f;
+#pragma unroll
+        for (int sl = 0; sl < kMaxKSlices; ++sl)
+          if (sl < nks) z += v[u][sl];
+        Zall[(size_t)(r0 + rr) * ldz + e] = z + tail->bias[e];   // a row only this CTA reads
+      }
     }
-    cluster_sync();   // CTA 0 holds the sums; no CTA reads a peer's memory any more
-    lead = ks == 0;
+    __syncthreads();
+    for (int r = r0 + warp; r < r1; r += kThreads / 32)
+      gate_row_warp<KB>(Zall + (size_t)r * ldz, E, lam, t0 + r, ok, lane, topk_idx, topk_w, gap_out, tail->hist,
+                        &tail->ntie, &tail->zrow[r], status);
+    __syncthreads();
+    // this CTA's probability sums over its rows: nG groups of rows, the group
+    // partials added in group order
+    float* colpart = &tail->part[0][0][0];
+    const int nG = kThreads / E;
+    const int R = (r1 - r0 + nG - 1) / nG;
+    if (tid < nG * E) {
+      const int e = tid % E, g = tid / E;
+      float sum = 0.f;
+      const int ra = r0 + g * R, rb = min(r1, ra + R);
+      for (int rr = ra; rr < rb; ++rr) sum += Zall[(size_t)rr * ldz + e];
+      colpart[g * E + e] = sum;
+    }
+    __syncthreads();
+    RSlots* slots = reinterpret_cast<RSlots*>(lists);
+    for (int e = tid; e < E; e += kThreads) {
+      float sum = 0.f;
+      for (int g = 0; g < nG; ++g) sum += colpart[g * E + e];
+      st_cluster_f32(cluster_addr(smem_u32(&slots->psum[ks][e]), 0), sum);
+      st_cluster_u32(cluster_addr(smem_u32(&slots->hist[ks][e]), 0), (uint32_t)tail->hist[e]);
+    }
+    if (warp == 0) {   // the z-loss sum of this CTA's rows, in a fixed order
+      float z = 0.f;
+      for (int r = r0 + lane; r < r1; r += 32) z += tail->zrow[r];
+      z = warp_sum(z);
+      if (lane == 0) {
+        st_cluster_f32(cluster_addr(smem_u32(&slots->zsum[ks]), 0), z);
+        st_cluster_u32(cluster_addr(smem_u32(&slots->ntie[ks]), 0), (uint32_t)tail->ntie);
+      }
+    }
+    cluster_sync();   // the slots of CTA 0 are filled; no CTA touches a peer's memory any more
+    if (ks == 0) {
+      for (int e = tid; e < E; e += kThreads) {
+        float ps = 0.f;
+        int hs = 0;
+        for (int sl = 0; sl < nks; ++sl) {
+          ps += slots->psum[sl][e];
+          hs += slots->hist[sl][e];
+        }
+        psum_out[(size_t)chunk * E + e] = ps;
+        hist_out[(size_t)e * nch + chunk] = hs;
+      }
+      if (tid == 0) {
+        float z = 0.f;
+        int nt = 0;
+        for (int sl = 0; sl < nks; ++sl) {
+          z += slots->zsum[sl];
+          nt += slots->ntie[sl];
+        }
+        zsum_out[chunk] = z;
+        ntie_out[chunk] = nt;
+      }
+    }
   }
+  const bool lead = nks == 1;   // the quarter epilogue: this CTA gates the whole chunk
   if (lead) {
     const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
     float (*part)[4][RM] = tail->part;
@@ -365,7 +555,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         for (int j = 0; j < KB; ++j) {
           topk_idx[(size_t)t * k + j] = top.i[j];
           topk_w[(size_t)t * k + j] = psel[j] * rs;
-          atomicAdd(&tail->hist[top.i[j]], 1);
+          // a row with fewer than k scores above -inf (NaN logits) keeps empty
+          // slots: out of range, dropped by the permutation, and flagged
+          if ((unsigned)top.i[j] < (unsigned)E) atomicAdd(&tail->hist[top.i[j]], 1);
+          else atomicOr(status, MOE_DEV_BOUNDS);
         }
         gap_out[t] = gap;
         if (gap < MOE_NEAR_TIE_GAP) atomicAdd(&tail->ntie, 1);
@@ -412,9 +605,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 // Slices of the model width per chunk: doubled while the reduction takes more
 // than one round of the stage ring, each slice keeps at least half a ring of
 // k-blocks and the grid stays within one CTA per SM; only batches of at most
-// 74 chunks split.  A chunk's slices form one cluster of at most 8 CTAs.  (A
-// split of the FastMoE layer's one-ring reduction over pairs ran 6 us slower:
-// its epilogue, not its loads, sets the kernel's time.)
+// 74 chunks split.  A chunk's slices form one cluster of at most 8 CTAs, and
+// each CTA gates its share of the chunk's rows.  (Splitting the FastMoE
+// layer's one-ring reduction over pairs made its route 8 us slower and its
+// forward 14 us slower.)
 int kslices(const moe_config& c, long long sms) {
   const int EP = ((c.E + 15) / 16) * 16;
   const int nch = num_chunks(c.T), nkb = (c.d + RK - 1) / RK, nst = num_stages(EP);

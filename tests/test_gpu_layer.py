@@ -6,6 +6,8 @@
   drop mask over all tokens, outputs on sampled tokens the oracle evaluates one
   by one (the FastMoE layer is small enough to check in full);
 * edge cases: no tokens, one token, k = E, one expert, determinism."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -189,6 +191,47 @@ def test_layer_deterministic():
     b = L.forward()
     assert torch.equal(a["out"], b["out"])
     assert a["stats"] == b["stats"]
+
+
+# dropless layers for a token with a NaN in its row: the tensor-core route with
+# four threads per token (and the fused combine), the same route cut over the
+# model width (one cluster of 4 slices per chunk, a warp per token), top-6
+# with the separate combine, and the fp32 route on CUDA cores
+NAN_LAYERS = {
+    "nan_quarter": W("nan_quarter", T=300, d=256, E=16, F=64, k=2, act=mw.RELU, dtype=mw.BF16, seed=41),
+    "nan_split": W("nan_split", T=200, d=1024, E=16, F=64, k=2, act=mw.SWIGLU, dtype=mw.BF16, lam=1.0, seed=42),
+    "nan_k6": W("nan_k6", T=500, d=128, E=64, F=176, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True, seed=43),
+    "nan_fp32": W("nan_fp32", T=300, d=64, E=5, F=96, k=2, act=mw.RELU, dtype=mw.F32, seed=44),
+}
+
+
+@pytest.mark.parametrize("name", sorted(NAN_LAYERS))
+def test_nan_token_is_dropped_and_flagged(name):
+    """A token whose row of x holds a NaN has no score above -inf: its k slots
+    stay empty (outside [0, E)), it adds nothing to the histogram, the forward
+    sets MOE_DEV_BOUNDS and the token's output row is zero.  Every other
+    token's selection, gate weights and output are bit-identical to those of
+    the same forward without the NaN (routing is per token, and a row's
+    expert outputs do not depend on its position in the segment)."""
+    w = NAN_LAYERS[name]
+    inp = mw.generate(w)
+    clean = DeviceLayer(w, inp).forward()
+    assert clean["stats"]["status"] == 0
+    bad = 37
+    x = inp.x.copy()
+    x[bad, 3] = 0x7FC0 if w.dtype == mw.BF16 else np.float32(np.nan)   # bf16 bits of a quiet NaN
+    r = DeviceLayer(w, dataclasses.replace(inp, x=x)).forward()
+    assert r["stats"]["status"] == moe.MOE_DEV_BOUNDS
+    assert np.all((r["topk_idx"][bad] < 0) | (r["topk_idx"][bad] >= w.E))
+    assert np.all(r["row_of"][bad] == -1)
+    others = np.arange(w.T) != bad
+    assert np.array_equal(r["topk_idx"][others], clean["topk_idx"][others])
+    assert np.array_equal(r["topk_w"][others].view(np.uint32), clean["topk_w"][others].view(np.uint32))
+    assert np.array_equal(r["counts"], np.bincount(clean["topk_idx"][others].ravel(), minlength=w.E))
+    assert r["stats"]["rows_kept"] == (w.T - 1) * w.k
+    out, ref = r["out"].cpu(), clean["out"].cpu()
+    assert torch.all(out[bad] == 0)
+    assert torch.equal(out[torch.from_numpy(others)], ref[torch.from_numpy(others)])
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "fastmoe_txl", "fine_decode_dropless", "fine_decode_cap"])

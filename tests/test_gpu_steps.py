@@ -37,8 +37,9 @@ MEDIUM = {
                             lam=1.0, seed=20),
     # model widths of more than one ring of gate loads on few chunks: the gate
     # GEMM is cut over the model width (4 slices here, the last one 5 k-blocks
-    # with a zero-filled tail, d = 1072), partials summed by the last CTA;
-    # E = 24 is not a multiple of 16, with normalisation and a gate bias
+    # with a zero-filled tail, d = 1072), one cluster per chunk whose CTAs each
+    # sum and gate a share of the rows; E = 24 is not a multiple of 16, with
+    # normalisation and a gate bias
     "ksplit_lambda_bias": W("ksplit_lambda_bias", T=300, d=1072, E=24, F=64, k=3, act=mw.SWIGLU, dtype=mw.BF16,
                             capacity_factor=1.0, lam=1.0, zipf_bias=True, seed=33),
     # one chunk, the largest expert count and k (4 slices of 2 k-blocks)
