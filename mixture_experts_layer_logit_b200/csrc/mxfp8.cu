@@ -38,10 +38,25 @@ namespace {
 using namespace tc;
 
 constexpr int MB = 128, MN = 128, MK = 128;   // tile rows, columns, K elements (bytes) per stage
-constexpr int STAGES = 6;
-constexpr int A_BYTES = MB * MK, B_BYTES = MN * MK;   // 16 KB each
+constexpr int B_BYTES = MN * MK;                      // 16 KB
 constexpr int SF_BYTES = 512;                         // one scale atom per operand
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int kMaxStages = 8;
+
+// Stage layouts.  Wide: A and B tiles of 128 rows (16 KB each), 6 stages.
+// Narrow, for batches of at most 64 tokens (a token takes an expert at most
+// once, so no expert has more than 64 kept rows): A holds 64 rows (8 KB) and
+// 8 stages keep 128 KB of weight tiles in flight per SM instead of 96 KB.  The
+// MMA still reads 128 A rows, the last 64 from the stage's own B tile: those
+// rows of the accumulator are computed and never stored (their epilogue warps
+// are not live).
+template <bool NARROW>
+struct MxLayout {
+  static constexpr int kARows = NARROW ? 64 : MB;
+  static constexpr int kABytes = kARows * MK;
+  static constexpr int kStages = NARROW ? 8 : 6;
+  static constexpr int kStageBytes = kABytes + B_BYTES;
+  static_assert(kStages <= kMaxStages && kStageBytes % 1024 == 0, "stages of 1 KB-aligned tiles");
+};
 constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -221,7 +236,7 @@ struct MxParams {
 };
 
 struct MxTail {
-  unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  unsigned long long full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2], drain;
   unsigned long long qfull[kQueue], qempty[kQueue];
   uint32_t tmem_base;
   int abort_flag;
@@ -231,9 +246,13 @@ struct MxTail {
   int seg[kMaxExperts + 1];
   int cnt[kMaxExperts + 1];       // kept rows of each expert (the rest of its padded segment is padding)
 };
-constexpr size_t kMxSmem = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)STAGES * 2 * SF_BYTES +
-                           gemm::kStagingBytes + sizeof(MxTail);
-static_assert(kMxSmem <= 227 * 1024, "shared memory of one CTA");
+template <bool NARROW>
+constexpr size_t mx_smem() {
+  using Lay = MxLayout<NARROW>;
+  return 1024 + (size_t)Lay::kStages * Lay::kStageBytes + (size_t)Lay::kStages * 2 * SF_BYTES +
+         gemm::kStagingBytes + sizeof(MxTail);
+}
+static_assert(mx_smem<false>() <= 227 * 1024 && mx_smem<true>() <= 227 * 1024, "shared memory of one CTA");
 
 struct MxTile {
   bool l2;
@@ -270,10 +289,13 @@ __device__ __forceinline__ MxTile mx_tile(const MxTail* t, int E, int T1, int L)
 // Roles: warp 0 claims tiles and issues the TMA and scale loads, warp 1 the
 // scale copies to TMEM and the MMAs, warps 2-9 the epilogue; the claimed
 // tiles pass between them through a 4-slot queue in shared memory.
-template <int ACT>
+template <int ACT, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const MxParams p) {
+  constexpr int STAGES = MxLayout<NARROW>::kStages;
+  constexpr int STAGE_BYTES = MxLayout<NARROW>::kStageBytes;
+  constexpr int A_BYTES = MxLayout<NARROW>::kABytes;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -329,6 +351,10 @@ tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
   for (int e = threadIdx.x; e <= p.E; e += kThreads) {
     tail->seg[e] = p.pad[e];
     tail->cnt[e] = (e < p.E) ? p.offsets[e + 1] - p.offsets[e] : 0;
+    // the narrow layout holds 64 A rows: more kept rows than that would be
+    // computed from the B tile, so the launch is flagged (the host picks it
+    // only when no expert can have more)
+    if (NARROW && tail->cnt[e] > MxLayout<true>::kARows && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
   }
   tc_fence_before();
   __syncthreads();
@@ -540,12 +566,13 @@ tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
   }
 }
 
-template <int ACT>
+template <int ACT, bool NARROW>
 cudaError_t launch_mx(const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2, const CUtensorMap& b2,
                       const MxParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_mx_mlp<ACT>>(kMxSmem);
+  constexpr size_t smem = mx_smem<NARROW>();
+  cudaError_t err = set_smem_once<tc_mx_mlp<ACT, NARROW>>(smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_mx_mlp<ACT>, dim3(grid), dim3(kThreads), kMxSmem, s, a1, b1, a2, b2, p);
+  return launch_pdl(tc_mx_mlp<ACT, NARROW>, dim3(grid), dim3(kThreads), smem, s, a1, b1, a2, b2, p);
 }
 
 template <typename Map>
@@ -601,10 +628,12 @@ cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const voi
   }
   // both layers in one launch: h = act(xq W1q^T) quantised in the epilogue,
   // then yp = hq W2q^T (fp32) at the kept rows
+  const bool narrow = c.T <= MxLayout<true>::kARows;
+  const uint32_t a_rows = narrow ? MxLayout<true>::kARows : MxLayout<false>::kARows;
   CUtensorMap a1, b1, a2, b2;
-  if (!make_map_u8(&a1, b.xq, (uint64_t)b.rows_pad, (uint64_t)c.d) ||
+  if (!make_map_u8(&a1, b.xq, (uint64_t)b.rows_pad, (uint64_t)c.d, a_rows) ||
       !make_map_u8(&b1, w1q, (uint64_t)c.E * F1, (uint64_t)c.d) ||
-      !make_map_u8(&a2, b.hq, (uint64_t)b.rows_pad, (uint64_t)c.F) ||
+      !make_map_u8(&a2, b.hq, (uint64_t)b.rows_pad, (uint64_t)c.F, a_rows) ||
       !make_map_u8(&b2, w2q, (uint64_t)c.E * c.d, (uint64_t)c.F))
     return cudaErrorInvalidValue;
   MxParams p{};
@@ -625,8 +654,11 @@ cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const voi
   p.sched = b.ctr;
   p.dep = b.ctr + 1;
   const int grid = (int)std::max<long long>(1, std::min<long long>((long long)mt_max * (F1 / MN + c.d / MN), di.sms));
-  return (c.act == MOE_ACT_SWIGLU) ? launch_mx<kMxSwiglu>(a1, b1, a2, b2, p, grid, s)
-                                   : launch_mx<kMxRelu>(a1, b1, a2, b2, p, grid, s);
+  if (narrow)
+    return (c.act == MOE_ACT_SWIGLU) ? launch_mx<kMxSwiglu, true>(a1, b1, a2, b2, p, grid, s)
+                                     : launch_mx<kMxRelu, true>(a1, b1, a2, b2, p, grid, s);
+  return (c.act == MOE_ACT_SWIGLU) ? launch_mx<kMxSwiglu, false>(a1, b1, a2, b2, p, grid, s)
+                                   : launch_mx<kMxRelu, false>(a1, b1, a2, b2, p, grid, s);
 }
 
 }  // namespace moe
