@@ -25,6 +25,9 @@
 // order, so a claimed layer-2 tile only waits for layer-1 tiles already
 // claimed by running CTAs, which never wait themselves.
 //
+// Batches of at most 64 tokens (decode) take m-tiles of 64 rows and one more
+// stage of weight tiles in flight (MlpLayout).
+//
 // Roles as in the 1-SM grouped GEMM (warp 0 TMA producer and tile claimer,
 // warp 1 MMA issuer, warps 2-5 epilogue); the producer passes each claimed
 // tile to the other roles through a 4-slot queue in shared memory.  Every
@@ -41,17 +44,31 @@ namespace {
 using namespace tc;
 using namespace gemm;
 
-constexpr int BM = 128;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;              // 16 KB
+constexpr int BM = 128;                           // MMA rows
 constexpr int B_BYTES = BN * BK * 2;              // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int kMaxStages = 5;
+constexpr int kNarrowRows = 64;
+
+// Stage layouts.  Wide: m-tiles of 128 rows, A 16 KB + B 32 KB, 4 stages.
+// Narrow, for batches of at most 64 tokens: m-tiles of 64 rows (a decode
+// expert has at most 64), A 8 KB, and 5 stages keep 160 KB of weight tiles
+// in flight per SM instead of 128 KB.  The MMA still reads 128 A rows, the
+// last 64 from the stage's own B tile; those accumulator rows are computed
+// and never stored (a tile's rows end at 64).
+template <bool NARROW>
+struct MlpLayout {
+  static constexpr int kTileRows = NARROW ? kNarrowRows : BM;
+  static constexpr int kABytes = kTileRows * BK * 2;
+  static constexpr int kStages = NARROW ? 5 : 4;
+  static constexpr int kStageBytes = kABytes + B_BYTES;
+  static_assert(kStages <= kMaxStages && kStageBytes % 1024 == 0, "stages of 1 KB-aligned tiles");
+};
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kQueue = 4;                         // claimed tiles in flight between the roles
 
 struct Tail {
-  unsigned long long full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  unsigned long long full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2], drain;
   unsigned long long qfull[kQueue], qempty[kQueue];
   uint32_t tmem_base;
   int abort_flag;
@@ -61,8 +78,11 @@ struct Tail {
   int mstart[kMaxExperts + 1];    // first m-tile of each expert (dependency counters)
   int seg[kMaxExperts + 1];       // copy of offsets[]
 };
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + kStagingBytes + sizeof(Tail);
-static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
+template <bool NARROW>
+constexpr size_t mlp_smem() {
+  return 1024 + (size_t)MlpLayout<NARROW>::kStages * MlpLayout<NARROW>::kStageBytes + kStagingBytes + sizeof(Tail);
+}
+static_assert(mlp_smem<false>() <= 227 * 1024 && mlp_smem<true>() <= 227 * 1024, "shared memory of one CTA");
 
 struct MlpParams {
   const int32_t* offsets;
@@ -89,21 +109,25 @@ struct MlpTile {
   int m;
 };
 
-template <int ACT>
+template <int ACT, int TM>
 __device__ __forceinline__ MlpTile mlp_tile(const Tail* tail, int E, int T1, int L) {
   MlpTile t;
   t.l2 = L >= T1;
-  t.c = t.l2 ? decode_tile<kCombine, BM>(tail->tstart2, tail->seg, E, L - T1)
-             : decode_tile<ACT, BM>(tail->tstart1, tail->seg, E, L);
-  t.m = tail->mstart[t.c.e] + (t.c.row0 - tail->seg[t.c.e]) / BM;
+  t.c = t.l2 ? decode_tile<kCombine, TM>(tail->tstart2, tail->seg, E, L - T1)
+             : decode_tile<ACT, TM>(tail->tstart1, tail->seg, E, L);
+  t.m = tail->mstart[t.c.e] + (t.c.row0 - tail->seg[t.c.e]) / TM;
   return t;
 }
 
-template <int ACT, bool F16, bool COMB>
+template <int ACT, bool F16, bool COMB, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
               const MlpParams p) {
+  constexpr int TM = MlpLayout<NARROW>::kTileRows;
+  constexpr int STAGES = MlpLayout<NARROW>::kStages;
+  constexpr int A_BYTES = MlpLayout<NARROW>::kABytes;
+  constexpr int STAGE_BYTES = MlpLayout<NARROW>::kStageBytes;
   constexpr uint32_t kIdesc1 = idesc_f16kind(BM, BN, false);   // xp, W1: bf16
   constexpr uint32_t kIdesc2 = idesc_f16kind(BM, BN, F16);     // h, W2: the hidden type
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -154,9 +178,9 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
   pdl_launch_dependents();
   bool table_ok = true;
   if (warp == 0) {
-    table_ok = tile_table_warp(p.offsets, p.E, BM, nt1, p.rows_alloc, tail->tstart1, lane);
-    table_ok &= tile_table_warp(p.offsets, p.E, BM, nt2, p.rows_alloc, tail->tstart2, lane);
-    table_ok &= tile_table_warp(p.offsets, p.E, BM, 1, p.rows_alloc, tail->mstart, lane);
+    table_ok = tile_table_warp(p.offsets, p.E, TM, nt1, p.rows_alloc, tail->tstart1, lane);
+    table_ok &= tile_table_warp(p.offsets, p.E, TM, nt2, p.rows_alloc, tail->tstart2, lane);
+    table_ok &= tile_table_warp(p.offsets, p.E, TM, 1, p.rows_alloc, tail->mstart, lane);
     if (!table_ok && lane == 0 && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
   }
   for (int e = threadIdx.x; e <= p.E; e += kThreads) tail->seg[e] = p.offsets[e];
@@ -184,7 +208,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         tail->queue[q] = L;
         mbar_arrive(qfull0 + 8 * q);
         if (L < 0) break;
-        const MlpTile t = mlp_tile<ACT>(tail, p.E, T1, L);
+        const MlpTile t = mlp_tile<ACT, TM>(tail, p.E, T1, L);
         const CUtensorMap* mA = t.l2 ? &tmA2 : &tmA1;
         const CUtensorMap* mB = t.l2 ? &tmB2 : &tmB1;
         int b0, b1;
@@ -279,7 +303,7 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty0 + 8 * q);
       if (L < 0) break;
-      const MlpTile t = mlp_tile<ACT>(tail, p.E, T1, L);
+      const MlpTile t = mlp_tile<ACT, TM>(tail, p.E, T1, L);
       const int acc = tl & 1;
       const uint32_t aph = (uint32_t)(tl >> 1) & 1u;
       ok = mbar_wait(tfull0 + 8 * acc, aph, abort_flag, p.wait_ns);
@@ -321,16 +345,22 @@ tc_expert_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
   }
 }
 
-template <int ACT, bool F16, bool COMB>
+template <int ACT, bool F16, bool COMB, bool NARROW>
 cudaError_t launch_t(const CUtensorMap (&maps)[4], const MlpParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = set_smem_once<tc_expert_mlp<ACT, F16, COMB>>(kSmemBytes);
+  constexpr size_t smem = mlp_smem<NARROW>();
+  cudaError_t err = set_smem_once<tc_expert_mlp<ACT, F16, COMB, NARROW>>(smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(tc_expert_mlp<ACT, F16, COMB>, dim3(grid), dim3(kThreads), kSmemBytes, s, maps[0], maps[1],
+  return launch_pdl(tc_expert_mlp<ACT, F16, COMB, NARROW>, dim3(grid), dim3(kThreads), smem, s, maps[0], maps[1],
                     maps[2], maps[3], p);
 }
+template <int ACT, bool F16, bool NARROW>
+cudaError_t launch_n(const CUtensorMap (&maps)[4], const MlpParams& p, bool comb, int grid, cudaStream_t s) {
+  return comb ? launch_t<ACT, F16, true, NARROW>(maps, p, grid, s) : launch_t<ACT, F16, false, NARROW>(maps, p, grid, s);
+}
 template <int ACT, bool F16>
-cudaError_t launch_c(const CUtensorMap (&maps)[4], const MlpParams& p, bool comb, int grid, cudaStream_t s) {
-  return comb ? launch_t<ACT, F16, true>(maps, p, grid, s) : launch_t<ACT, F16, false>(maps, p, grid, s);
+cudaError_t launch_c(const CUtensorMap (&maps)[4], const MlpParams& p, bool comb, bool narrow, int grid,
+                     cudaStream_t s) {
+  return narrow ? launch_n<ACT, F16, true>(maps, p, comb, grid, s) : launch_n<ACT, F16, false>(maps, p, comb, grid, s);
 }
 
 std::atomic<unsigned long long> g_wait_ns{kWaitNs};
@@ -344,7 +374,8 @@ void set_expert_mlp_test_hooks(unsigned long long wait_ns, int dep_extra) {
 }
 
 size_t expert_mlp_counters(const moe_config& c) {
-  return 1 + (size_t)c.T * c.k / BM + (size_t)c.E + 1;
+  const int tm = c.T <= kNarrowRows ? kNarrowRows : BM;   // the m-tile height the launch takes
+  return 1 + (size_t)c.T * c.k / tm + (size_t)c.E + 1;
 }
 
 cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t* offsets, const void* w1,
@@ -359,23 +390,29 @@ cudaError_t launch_expert_mlp(const moe_config& c, const void* xp, const int32_t
   const uint64_t rows = (uint64_t)c.T * (uint64_t)c.k;
   const int F1 = (c.act == MOE_ACT_SWIGLU) ? 2 * c.F : c.F;
   const int EW = e_mod > 0 ? e_mod : c.E;   // experts whose weights are given
+  // narrow tiles where no routed expert can have more than 64 rows (any
+  // segment stays correct: it is cut into 64-row m-tiles); the counters'
+  // count (expert_mlp_counters) follows the same rule
+  const bool narrow = c.T <= kNarrowRows;
+  const uint32_t tm = narrow ? kNarrowRows : BM;
   CUtensorMap maps[4];
-  if (!make_map(&maps[0], xp, rows, (uint64_t)c.d, false) ||
+  if (!make_map(&maps[0], xp, rows, (uint64_t)c.d, false, tm) ||
       !make_map(&maps[1], w1, (uint64_t)EW * F1, (uint64_t)c.d, false) ||
-      !make_map(&maps[2], h, rows, (uint64_t)c.F, f16) ||
+      !make_map(&maps[2], h, rows, (uint64_t)c.F, f16, tm) ||
       !make_map(&maps[3], w2, (uint64_t)EW * c.d, (uint64_t)c.F, f16))
     return cudaErrorInvalidValue;
   MlpParams p{offsets, h, comb ? comb->out : yp, comb ? comb->src_tok : nullptr, comb ? comb->row_w : nullptr,
               c.E, c.d, c.F, F1, comb ? comb->T : 0, (int)rows, counters, counters + 1, status,
               g_wait_ns.load(), g_dep_extra.load(), EW};
   const bool cb = comb != nullptr;
-  const long long mt_max = (long long)(rows / BM) + c.E;
+  const long long mt_max = (long long)(rows / tm) + c.E;
   const long long nt = (c.act == MOE_ACT_SWIGLU ? (c.F + BN / 2 - 1) / (BN / 2) : (c.F + BN - 1) / BN) +
                        (c.d + BN - 1) / BN;
   const int grid = (int)std::min<long long>(mt_max * nt, di.sms);
   if (c.act == MOE_ACT_SWIGLU)
-    return f16 ? launch_c<kSwiglu, true>(maps, p, cb, grid, s) : launch_c<kSwiglu, false>(maps, p, cb, grid, s);
-  return f16 ? launch_c<kRelu, true>(maps, p, cb, grid, s) : launch_c<kRelu, false>(maps, p, cb, grid, s);
+    return f16 ? launch_c<kSwiglu, true>(maps, p, cb, narrow, grid, s)
+               : launch_c<kSwiglu, false>(maps, p, cb, narrow, grid, s);
+  return f16 ? launch_c<kRelu, true>(maps, p, cb, narrow, grid, s) : launch_c<kRelu, false>(maps, p, cb, narrow, grid, s);
 }
 
 }  // namespace moe

@@ -334,6 +334,28 @@ def test_expert_ffn_short_layer_any_segment(offsets):
     check_out(to_np64(yp[:n]), yp_ref, w.dtype)
 
 
+def test_expert_ffn_small_batch_long_segment():
+    """A batch of at most 64 tokens takes 64-row m-tiles (the narrow stage
+    layout); a caller-made segment of 700 rows then spans 11 of them, more
+    than one group of the second layer's tile order, next to a ragged short
+    segment and empty ones."""
+    w = W("narrow_long", T=64, d=64, E=16, F=96, k=12, act=mw.SWIGLU, dtype=mw.BF16, seed=36)
+    L = DeviceLayer(w)
+    _, _, _, w1, w2 = oracle_inputs(L)
+    cfg = lcfg_of(w, L.T)
+    A = L.T * w.k
+    offsets = [0, 0, 700, 700, 733] + [733] * 11 + [768]
+    assert len(offsets) == w.E + 1 and offsets[-1] == A
+    g = torch.Generator().manual_seed(9)
+    xp = torch.randn((A, w.d), generator=g).to(torch.bfloat16).cuda()
+    h, yp, stats = L.expert_ffn(xp, torch.tensor(offsets, dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    assert moe.read_stats(stats)["status"] == 0
+    xp64 = xp.float().cpu().numpy().astype(np.float64)
+    _, yp_ref = om.expert_segments(xp64, np.array(offsets), w1, w2, cfg)
+    check_out(to_np64(yp), yp_ref, w.dtype)
+
+
 def test_adaptive_aux_coef_on_the_device_follows_the_oracle():
     """moe_aux_coef_update, chained on the stream over scripted drop rates
     written into a device moe_stats, against the oracle's coefficient step."""
