@@ -259,8 +259,10 @@ __device__ __forceinline__ void gate_row_warp(float* Z, int E, float lam, int t,
 }
 
 // KB is the exact number of experts per token, so that every index into the
-// top-k registers is a compile-time constant.
-template <int KB>
+// top-k registers is a compile-time constant.  SPLIT: the chunk's model width
+// is cut over a cluster of nks > 1 CTAs (a separate instantiation, so the
+// unsplit kernel carries none of the exchange's registers).
+template <int KB, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                 const float* __restrict__ bg, int T, int d, int E, int EP, int nst, float lam,
@@ -374,7 +376,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   float* Z = Zall + (size_t)row * ldz;
   const int nch32 = (E + 31) / 32;
   // a split chunk's rows past the batch are never read: their warps skip the copy
-  const int ncopy = (nks == 1 || q * 32 < T - t0) ? nch32 : 0;
+  const int ncopy = (!SPLIT || q * 32 < T - t0) ? nch32 : 0;
   for (int c = qtr; c < ncopy; c += kSplit) {
     uint32_t r[32];
     tmem_ld32(tb + c * 32, r);
@@ -382,12 +384,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int e = c * 32 + i;
-      if (e < E) Z[e] = __uint_as_float(r[i]) + (nks == 1 ? tail->bias[e] : 0.f);
+      if (e < E) Z[e] = __uint_as_float(r[i]) + (SPLIT ? 0.f : tail->bias[e]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (nks > 1) {
+  if constexpr (SPLIT) {
     // The chunk's slices are one thread-block cluster, each slice's partial
     // logits in its own shared memory.  CTA ks sums rows [r0, r1) of the
     // chunk's real tokens over the slices, in slice order, adds the bias,
@@ -483,7 +485,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       }
     }
   }
-  const bool lead = nks == 1;   // the quarter epilogue: this CTA gates the whole chunk
+  constexpr bool lead = !SPLIT;   // the quarter epilogue: this CTA gates the whole chunk
   if (lead) {
     const int lo = (E * qtr) / kSplit, hi = (E * (qtr + 1)) / kSplit;
     float (*part)[4][RM] = tail->part;
@@ -618,22 +620,19 @@ int kslices(const moe_config& c, long long sms) {
   return n;
 }
 
-template <int KB>
-cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
+template <int KB, bool SPLIT>
+cudaError_t launch_ks(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
                       int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
-                      float* zsum, uint32_t* status, cudaStream_t s) {
+                      float* zsum, uint32_t* status, int nks, cudaStream_t s) {
   // the most any E <= kMaxExperts needs, so one attribute serves every launch
   static const size_t kMaxSmem = [] {
     size_t m = 0;
     for (int e = 1; e <= kMaxExperts; ++e) m = std::max(m, smem_bytes(e, ((e + 15) / 16) * 16));
     return m;
   }();
-  cudaError_t err = set_smem_once<route_tc_kernel<KB>>(kMaxSmem);
+  cudaError_t err = set_smem_once<route_tc_kernel<KB, SPLIT>>(kMaxSmem);
   if (err != cudaSuccess) return err;
-  DeviceInfo di;
-  if ((err = device_info(&di)) != cudaSuccess) return err;
   const int nch = num_chunks(c.T);
-  const int nks = kslices(c, di.sms);
   // PDL, and a chunk's slices as one cluster (nks consecutive CTAs)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nch * nks);
@@ -649,8 +648,21 @@ cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensor
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, route_tc_kernel<KB>, mx, mw, bg, c.T, c.d, c.E, EP, num_stages(EP), c.lambda, idx,
-                            w, gap, hist, psum, ntie, zsum, nch, status, (int)lists_offset(c.E, EP), nks);
+  return cudaLaunchKernelEx(&cfg, route_tc_kernel<KB, SPLIT>, mx, mw, bg, c.T, c.d, c.E, EP, num_stages(EP),
+                            c.lambda, idx, w, gap, hist, psum, ntie, zsum, nch, status, (int)lists_offset(c.E, EP),
+                            nks);
+}
+
+template <int KB>
+cudaError_t launch_kb(const moe_config& c, const CUtensorMap& mx, const CUtensorMap& mw, int EP, const float* bg,
+                      int32_t* idx, float* w, float* gap, int32_t* hist, float* psum, int32_t* ntie,
+                      float* zsum, uint32_t* status, cudaStream_t s) {
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const int nks = kslices(c, di.sms);
+  return nks > 1 ? launch_ks<KB, true>(c, mx, mw, EP, bg, idx, w, gap, hist, psum, ntie, zsum, status, nks, s)
+                 : launch_ks<KB, false>(c, mx, mw, EP, bg, idx, w, gap, hist, psum, ntie, zsum, status, 1, s);
 }
 
 }  // namespace
