@@ -367,10 +367,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* Wg, const
     if (z_loss != nullptr && cudaMemsetAsync(z_loss, 0xff, sizeof(float), s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  if (prob_mean != nullptr && (e = launch_prob_mean(c, at<float>(ws, sc.psum), prob_mean, s)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (z_loss != nullptr) e = launch_z_loss(c, at<float>(ws, sc.zsum), z_loss, s);
-  return cuda_status(e);
+  return cuda_status(launch_route_totals(c, at<float>(ws, sc.psum), at<float>(ws, sc.zsum), prob_mean, z_loss, s));
 }
 
 moe_status moe_permute(const moe_config* cfg, const void* x, const int32_t* topk_idx,

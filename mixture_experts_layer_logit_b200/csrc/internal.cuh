@@ -48,10 +48,10 @@ bool route_tc_supported(const moe_config& c);
 cudaError_t launch_route_tc(const moe_config& c, const void* x, const void* wg, const float* bg,
                             int32_t* topk_idx, float* topk_w, float* gap, int32_t* hist, float* psum,
                             int32_t* ntie, float* zsum, uint32_t* status, cudaStream_t s);
-// prob_mean[e] = sum over chunks of psum / T (fixed order).
-cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s);
-// *z_loss = sum over chunks of zsum / T (fixed order).
-cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s);
+// One launch: prob_mean[e] = sum over chunks of psum / T and *z_loss = sum over
+// chunks of zsum / T, both in a fixed order; either output may be NULL.
+cudaError_t launch_route_totals(const moe_config& c, const float* psum, const float* zsum, float* prob_mean,
+                                float* z_loss, cudaStream_t s);
 // seg[0] = 0, seg[1] = rows (the shared expert's single segment)
 cudaError_t launch_fill_segment(int32_t* seg, int rows, cudaStream_t s);
 // out[i] += add[i] for n floats (n a multiple of 4)

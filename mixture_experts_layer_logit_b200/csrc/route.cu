@@ -281,23 +281,28 @@ route_kernel(const TX* __restrict__ x, const TX* __restrict__ wg, const float* _
   }
 }
 
-// Router z-loss of a standalone route: sum of the per-chunk sums / T.
-__global__ void z_loss_kernel(const float* __restrict__ zsum, int nch, int T, float* __restrict__ z_loss) {
-  const int lane = threadIdx.x;
-  double s = 0.0;
-  for (int c = lane; c < nch; c += 32) s += (double)zsum[c];
+// The totals of a standalone route, in one launch: P_e = sum over chunks of
+// psum / T, one warp per expert (lanes stride over the chunks, then a
+// fixed-order butterfly sum: deterministic); with z_loss, the last block's
+// first warp adds the chunks' squared log-partitions (double) and divides by
+// T.  Launched with programmatic dependent launch: it waits here for the
+// route kernel's results.
+__global__ void route_totals_kernel(const float* __restrict__ psum, const float* __restrict__ zsum, int nch,
+                                    int E, int T, float* __restrict__ prob_mean, float* __restrict__ z_loss) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (z_loss != nullptr && blockIdx.x == gridDim.x - 1) {
+    if (warp != 0) return;
+    double s = 0.0;
+    for (int c = lane; c < nch; c += 32) s += (double)zsum[c];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) *z_loss = (float)(s / (double)T);
-}
-
-// One warp per expert: lanes stride over the chunks, then a fixed-order
-// butterfly sum (deterministic).
-__global__ void prob_mean_kernel(const float* __restrict__ psum, int nch, int E, int T,
-                                 float* __restrict__ prob_mean) {
-  const int e = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (e >= E) return;
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) *z_loss = (float)(s / (double)T);
+    return;
+  }
+  const int e = blockIdx.x * (blockDim.x / 32) + warp;
+  if (prob_mean == nullptr || e >= E) return;
   float s = 0.f;
   for (int c = lane; c < nch; c += 32) s += psum[(size_t)c * E + e];
   s = warp_sum(s);
@@ -344,14 +349,12 @@ cudaError_t launch_route(const moe_config& c, const void* x, const void* wg, con
   return launch_route_t<float>(c, x, wg, bg, topk_idx, topk_w, gap, hist, psum, ntie, zsum, status, s);
 }
 
-cudaError_t launch_z_loss(const moe_config& c, const float* zsum, float* z_loss, cudaStream_t s) {
-  z_loss_kernel<<<1, 32, 0, s>>>(zsum, num_chunks(c.T), c.T, z_loss);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_prob_mean(const moe_config& c, const float* psum, float* prob_mean, cudaStream_t s) {
-  prob_mean_kernel<<<(c.E + 7) / 8, 256, 0, s>>>(psum, num_chunks(c.T), c.E, c.T, prob_mean);
-  return cudaGetLastError();
+cudaError_t launch_route_totals(const moe_config& c, const float* psum, const float* zsum, float* prob_mean,
+                                float* z_loss, cudaStream_t s) {
+  if (prob_mean == nullptr && z_loss == nullptr) return cudaSuccess;
+  const int blocks = (prob_mean != nullptr ? (c.E + 7) / 8 : 0) + (z_loss != nullptr ? 1 : 0);
+  return launch_pdl(route_totals_kernel, dim3(blocks), dim3(256), 0, s, psum, zsum, num_chunks(c.T), c.E, c.T,
+                    prob_mean, z_loss);
 }
 
 }  // namespace moe
