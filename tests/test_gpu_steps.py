@@ -44,6 +44,11 @@ MEDIUM = {
                             capacity_factor=1.0, lam=1.0, zipf_bias=True, seed=33),
     # one chunk, the largest expert count and k (4 slices of 2 k-blocks)
     "ksplit_E256_k8": W("ksplit_E256_k8", T=64, d=512, E=256, F=32, k=8, act=mw.RELU, dtype=mw.BF16, seed=34),
+    # 8 slices of one chunk that holds fewer tokens than slices: one token
+    # (seven CTAs gate no row), and nine (one or two rows per CTA)
+    "ksplit_T1": W("ksplit_T1", T=1, d=2048, E=64, F=64, k=6, act=mw.SWIGLU, dtype=mw.BF16, zipf_bias=True,
+                   seed=37),
+    "ksplit_T9": W("ksplit_T9", T=9, d=2048, E=40, F=64, k=4, act=mw.RELU, dtype=mw.BF16, lam=1.0, seed=38),
 }
 
 
