@@ -8,7 +8,8 @@
 // (FastMoE announcement, "1. MoE 设计" and "图4").  Normalisation
 // (Skywork-MoE release, "Gating Logits归一化操作"; slides, slide 6):
 // z_hat = lambda (z - mean) / std over the experts, population std, zero
-// spread -> 0.  Equal scores: the lower expert index wins.
+// spread -> 0.  Equal scores: the lower expert index wins; a NaN or -inf
+// score is never selected (a token with NaN logits keeps empty slots).
 //
 // Layout: x [T, d] and W_gate [E, d] are K-major bf16 and go through TMA
 // (128-byte swizzle) into a ring of up to 8 stages (enough for the whole
@@ -17,8 +18,9 @@
 // accumulates the 128 x N logits in fp32 in TMEM.  The epilogue copies them to
 // shared memory and gives every token four threads, each owning a quarter
 // of the experts: partial sums, maxima and top-(k+1) lists are merged through
-// shared memory in quarter order.  Each CTA is one routing chunk of 128 tokens: it also writes the
-// chunk's per-expert histogram, per-expert sum of softmax probabilities
+// shared memory in quarter order.  Each routing chunk of 128 tokens (one
+// CTA, or one cluster below) also writes the chunk's per-expert histogram,
+// per-expert sum of softmax probabilities
 // (summed in a fixed order), near-tie count and sum of squared
 // log-partitions (the router z-loss, Megatron-Core best-practice page,
 // "Megatron-Core MoE的关键特性") for the permutation step.
