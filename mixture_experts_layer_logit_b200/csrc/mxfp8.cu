@@ -50,7 +50,7 @@ constexpr int kMaxStages = 8;
 // rows of the accumulator are computed and never stored (their epilogue warps
 // are not live).
 template <bool NARROW>
-struct MxLayout {
+struct MxStages {
   static constexpr int kARows = NARROW ? 64 : MB;
   static constexpr int kABytes = kARows * MK;
   static constexpr int kStages = NARROW ? 8 : 6;
@@ -248,7 +248,7 @@ struct MxTail {
 };
 template <bool NARROW>
 constexpr size_t mx_smem() {
-  using Lay = MxLayout<NARROW>;
+  using Lay = MxStages<NARROW>;
   return 1024 + (size_t)Lay::kStages * Lay::kStageBytes + (size_t)Lay::kStages * 2 * SF_BYTES +
          gemm::kStagingBytes + sizeof(MxTail);
 }
@@ -293,9 +293,9 @@ template <int ACT, bool NARROW>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const MxParams p) {
-  constexpr int STAGES = MxLayout<NARROW>::kStages;
-  constexpr int STAGE_BYTES = MxLayout<NARROW>::kStageBytes;
-  constexpr int A_BYTES = MxLayout<NARROW>::kABytes;
+  constexpr int STAGES = MxStages<NARROW>::kStages;
+  constexpr int STAGE_BYTES = MxStages<NARROW>::kStageBytes;
+  constexpr int A_BYTES = MxStages<NARROW>::kABytes;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -354,7 +354,7 @@ tc_mx_mlp(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
     // the narrow layout holds 64 A rows: more kept rows than that would be
     // computed from the B tile, so the launch is flagged (the host picks it
     // only when no expert can have more)
-    if (NARROW && tail->cnt[e] > MxLayout<true>::kARows && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
+    if (NARROW && tail->cnt[e] > MxStages<true>::kARows && blockIdx.x == 0) atomicOr(p.status, MOE_DEV_BOUNDS);
   }
   tc_fence_before();
   __syncthreads();
@@ -628,8 +628,8 @@ cudaError_t launch_mx_experts(const moe_config& c, const MxBuffers& b, const voi
   }
   // both layers in one launch: h = act(xq W1q^T) quantised in the epilogue,
   // then yp = hq W2q^T (fp32) at the kept rows
-  const bool narrow = c.T <= MxLayout<true>::kARows;
-  const uint32_t a_rows = narrow ? MxLayout<true>::kARows : MxLayout<false>::kARows;
+  const bool narrow = c.T <= MxStages<true>::kARows;
+  const uint32_t a_rows = narrow ? MxStages<true>::kARows : MxStages<false>::kARows;
   CUtensorMap a1, b1, a2, b2;
   if (!make_map_u8(&a1, b.xq, (uint64_t)b.rows_pad, (uint64_t)c.d, a_rows) ||
       !make_map_u8(&b1, w1q, (uint64_t)c.E * F1, (uint64_t)c.d) ||
