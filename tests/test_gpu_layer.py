@@ -193,6 +193,21 @@ def test_layer_deterministic():
     assert a["stats"] == b["stats"]
 
 
+@pytest.mark.parametrize("name", ["m_ksplit", "fine_decode_dropless"])
+def test_layer_deterministic_split_route(name):
+    """The width-split route (partial logits summed over a cluster, rows gated
+    per CTA, the chunk's sums gathered in CTA 0) and, on the decode layer, the
+    narrow expert tiles give bit-identical results run to run."""
+    w = next((m for m in MEDIUM if m.name == name), None) or mw.WORKLOADS[name]
+    L = DeviceLayer(w)
+    a = L.forward()
+    b = L.forward()
+    for key in ("topk_idx", "topk_w", "gap", "counts", "row_of"):
+        assert np.array_equal(a[key], b[key]), key
+    assert torch.equal(a["out"], b["out"])
+    assert a["stats"] == b["stats"]
+
+
 # dropless layers for a token with a NaN in its row: the tensor-core route with
 # four threads per token (and the fused combine), the same route cut over the
 # model width (one cluster of 4 slices per chunk, a warp per token), top-6
