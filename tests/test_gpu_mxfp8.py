@@ -59,6 +59,9 @@ LAYERS = [
       seed=83),
     W("mx_E1", T=130, d=128, E=1, F=128, k=1, act=mw.RELU, dtype=mw.BF16, seed=84),
     W("mx_many_rows", T=1500, d=256, E=4, F=256, k=2, act=mw.SWIGLU, dtype=mw.BF16, seed=85),
+    # at most 64 tokens with ReLU: the narrow stage layout's other activation,
+    # and one expert holding every token (k = E = 2)
+    W("mx_relu_narrow", T=40, d=256, E=2, F=384, k=2, act=mw.RELU, dtype=mw.BF16, seed=86),
 ]
 
 
